@@ -1,0 +1,375 @@
+"""Pins of the CPU oracle against things other than itself.
+
+Each test ties one step of the oracle to a closed form, a library routine, a
+brute-force search or an invariant of "Prism: Spectral-Aware Block-Sparse
+Attention", so that a dropped term, a wrong sign, a wrong index or a
+transposed operand in the oracle fails at least one of them.
+"""
+
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import prism_oracle as po
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "dirichlet_factors.txt")
+
+
+def _golden_rows():
+    rows = []
+    with open(GOLDEN) as f:
+        for line in f:
+            if line.startswith("#") or not line.strip():
+                continue
+            base, d, m, beta, theta, D = line.split()
+            rows.append((float(base), int(d), int(m), int(beta), float(theta), float(D)))
+    return rows
+
+
+# ---------------------------------------------------------------------------
+# §2: amplitude collapse of mean pooling under RoPE (closed-form Dirichlet factor)
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("row", _golden_rows())
+def test_pooled_pair_amplitude_is_dirichlet_factor(row):
+    base, d, m, beta, theta, D = row
+    L = 4 * beta
+    cos, sin = po.rope_tables(base, L, d)
+    x = np.zeros((L, d))
+    x[:, m] = 1.0                       # constant pair (1, 0) rotated at theta_m
+    xr = po.apply_rope(x, cos, sin)
+    xbar = po.pool_blocks(xr, beta)
+    amp = np.hypot(xbar[:, m], xbar[:, m + d // 2])
+    # every block keeps the same amplitude (a block offset only rotates the mean)
+    np.testing.assert_allclose(amp, D, rtol=0, atol=3e-6)
+    # and the oracle's frequency formula gives the golden theta
+    assert po.rope_frequencies(base, d)[m] == pytest.approx(theta, rel=1e-15)
+
+
+def test_retained_amplitude_closed_form_multi_pair():
+    base, d, beta, L, bs = 1e4, 32, 16, 128, 5
+    cos, sin = po.rope_tables(base, L, d)
+    rng = np.random.default_rng(7)
+    vec = rng.normal(size=d)
+    xr = po.apply_rope(np.broadcast_to(vec, (L, d)).copy(), cos, sin)
+    xbar = po.pool_blocks(xr, beta)
+    theta = po.rope_frequencies(base, d)
+    Dm = np.abs(np.sin(beta * theta / 2)) / (beta * np.abs(np.sin(theta / 2)))
+    pair_e = vec[: d // 2] ** 2 + vec[d // 2:] ** 2
+    high, low = po.band_masks(d, bs)
+    for band, pairs in ((high, np.arange(bs)), (low, np.arange(bs, d // 2))):
+        expect = math.sqrt((pair_e[pairs] * Dm[pairs] ** 2).sum() / pair_e[pairs].sum())
+        got = po.retained_amplitude(xr, xbar, band)
+        assert got == pytest.approx(expect, rel=2e-6)
+
+
+# ---------------------------------------------------------------------------
+# §3.2: the energy temperature undoes the pooling attenuation exactly for a
+# single rotary pair: calibrated block logit == token logit at block starts.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("beta,rtol", [(8, 2e-6), (16, 2e-5)])
+def test_single_pair_calibration_identity(beta, rtol):
+    d, L, base = 16, 8 * beta, 1e4
+    cos, sin = po.rope_tables(base, L, d)
+    rng = np.random.default_rng(3)
+    q = np.zeros(d)
+    k = np.zeros(d)
+    q[[0, d // 2]] = rng.normal(size=2)
+    k[[0, d // 2]] = rng.normal(size=2)
+    Q = np.broadcast_to(q, (1, 1, L, d)).copy()
+    K = np.broadcast_to(k, (1, 1, L, d)).copy()
+    sc = po.prism_scores(Q, K, beta, band_split=1, flags=0, rope=(cos, sin))
+    qr = po.apply_rope(Q, cos, sin)[0, 0]
+    kr = po.apply_rope(K, cos, sin)[0, 0]
+    nb = L // beta
+    tok = np.array([[qr[i * beta] @ kr[j * beta] for j in range(nb)] for i in range(nb)]) / math.sqrt(d)
+    scale = np.abs(q).max() * np.abs(k).max() * 2 / math.sqrt(d)
+    np.testing.assert_allclose(sc.logits[0, 0], tok, rtol=0, atol=rtol * scale * 10)
+    # the same logits without calibration are attenuated by D^2
+    raw = po.prism_scores(Q, K, beta, band_split=1, flags=po.FLAG_NO_CALIB, rope=(cos, sin))
+    D = abs(math.sin(beta / 2)) / (beta * abs(math.sin(0.5)))
+    np.testing.assert_allclose(raw.logits[0, 0], tok * D * D, rtol=0, atol=rtol * scale * 10)
+    assert sc.tau[0, 0, 0] == pytest.approx(D * D, rel=1e-5)
+
+
+def test_tau_is_product_of_q_and_k_ratios_gqa():
+    base, d, beta, L, bs = 1e4, 16, 8, 64, 3
+    cos, sin = po.rope_tables(base, L, d)
+    rng = np.random.default_rng(11)
+    qv = rng.normal(size=(1, 4, 1, d))
+    kv = rng.normal(size=(1, 2, 1, d))
+    Q = np.broadcast_to(qv, (1, 4, L, d)).copy()
+    K = np.broadcast_to(kv, (1, 2, L, d)).copy()
+    sc = po.prism_scores(Q, K, beta, bs, 0, (cos, sin))
+    theta = po.rope_frequencies(base, d)
+    Dm = np.abs(np.sin(beta * theta / 2)) / (beta * np.abs(np.sin(theta / 2)))
+
+    def rho(v, pairs):
+        e = v[pairs] ** 2 + v[pairs + d // 2] ** 2
+        return math.sqrt((e * Dm[pairs] ** 2).sum() / e.sum())
+
+    for h in range(4):
+        g = h // 2
+        for bi, pairs in enumerate((np.arange(bs), np.arange(bs, d // 2))):
+            expect = rho(qv[0, h, 0], pairs) * rho(kv[0, g, 0], pairs)
+            assert sc.tau[0, h, bi] == pytest.approx(expect, rel=5e-6)
+
+
+# ---------------------------------------------------------------------------
+# RoPE convention against the transformers Llama rotary routine.
+# ---------------------------------------------------------------------------
+def test_rope_matches_transformers_llama_rotary():
+    from transformers.models.llama.modeling_llama import apply_rotary_pos_emb
+    L, d = 37, 16
+    cos, sin = po.rope_tables(5e5, L, d)
+    rng = np.random.default_rng(0)
+    q = rng.normal(size=(1, 2, L, d))
+    k = rng.normal(size=(1, 1, L, d))
+    c = torch.from_numpy(np.concatenate([cos, cos], -1).astype(np.float64))[None]
+    s = torch.from_numpy(np.concatenate([sin, sin], -1).astype(np.float64))[None]
+    qe, ke = apply_rotary_pos_emb(torch.from_numpy(q), torch.from_numpy(k), c, s)
+    np.testing.assert_allclose(po.apply_rope(q, cos, sin), qe.numpy(), rtol=0, atol=1e-14)
+    np.testing.assert_allclose(po.apply_rope(k, cos, sin), ke.numpy(), rtol=0, atol=1e-14)
+
+
+def test_rope_invariants():
+    L, d = 300, 32
+    cos, sin = po.rope_tables(1e4, L, d)
+    rng = np.random.default_rng(1)
+    x = rng.normal(size=(L, d))
+    xr = po.apply_rope(x, cos, sin)
+    np.testing.assert_array_equal(xr[0], x[0])                 # position 0 is the identity
+    n0 = x[:, : d // 2] ** 2 + x[:, d // 2:] ** 2
+    n1 = xr[:, : d // 2] ** 2 + xr[:, d // 2:] ** 2
+    np.testing.assert_allclose(n1, n0, rtol=3e-7)              # pair norms kept (fp32 table)
+    q = np.broadcast_to(rng.normal(size=d), (L, d)).copy()
+    k = np.broadcast_to(rng.normal(size=d), (L, d)).copy()
+    qr = po.apply_rope(q, cos, sin)
+    kr = po.apply_rope(k, cos, sin)
+    for a, b, delta in [(5, 2, 100), (40, 40, 17), (10, 90, 150)]:
+        assert qr[a] @ kr[b] == pytest.approx(qr[a + delta] @ kr[b + delta], abs=2e-5)
+    # energies per band are the same before and after rotation
+    e_pre = po.block_token_energy(x[None], 10, 5, 0)
+    e_post = po.block_token_energy(xr[None], 10, 5, 0)
+    np.testing.assert_allclose(e_post, e_pre, rtol=3e-7)
+
+
+# ---------------------------------------------------------------------------
+# Block size 1: pooling is the identity, tau == 1, probabilities are the
+# token-level causal softmax (computed here with torch's rotary + softmax).
+# ---------------------------------------------------------------------------
+def _torch_rotate(x, cos, sin):
+    from transformers.models.llama.modeling_llama import rotate_half
+    c = torch.from_numpy(np.concatenate([cos, cos], -1).astype(np.float64))
+    s = torch.from_numpy(np.concatenate([sin, sin], -1).astype(np.float64))
+    t = torch.from_numpy(np.asarray(x, dtype=np.float64))
+    return t * c + rotate_half(t) * s
+
+
+def test_block_one_equals_token_causal_softmax():
+    B, Hq, Hkv, L, d = 2, 4, 2, 12, 8
+    cos, sin = po.rope_tables(1e4, L, d)
+    rng = np.random.default_rng(5)
+    Q = rng.normal(size=(B, Hq, L, d))
+    K = rng.normal(size=(B, Hkv, L, d))
+    sc = po.prism_scores(Q, K, 1, 2, 0, (cos, sin))
+    np.testing.assert_allclose(sc.tau, 1.0, rtol=1e-12)
+    qt = _torch_rotate(Q, cos, sin)
+    kt = torch.repeat_interleave(_torch_rotate(K, cos, sin), Hq // Hkv, dim=1)
+    logits = qt @ kt.transpose(-1, -2) / math.sqrt(d)
+    mask = torch.ones(L, L, dtype=torch.bool).tril()
+    ref = torch.softmax(logits.masked_fill(~mask, float("-inf")), dim=-1)
+    np.testing.assert_allclose(sc.probs, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_no_calib_is_plain_mean_pool_matmul():
+    B, Hq, Hkv, L, d, beta = 1, 4, 1, 96, 16, 8
+    cos, sin = po.rope_tables(1e4, L, d)
+    rng = np.random.default_rng(9)
+    Q = rng.normal(size=(B, Hq, L, d))
+    K = rng.normal(size=(B, Hkv, L, d))
+    sc = po.prism_scores(Q, K, beta, 4, po.FLAG_NO_CALIB, (cos, sin))
+    pool = torch.nn.functional.avg_pool1d
+    qt = _torch_rotate(Q, cos, sin).reshape(B * Hq, L, d).transpose(1, 2)
+    kt = _torch_rotate(K, cos, sin).reshape(B * Hkv, L, d).transpose(1, 2)
+    qb = pool(qt, beta).transpose(1, 2).reshape(B, Hq, L // beta, d)
+    kb = pool(kt, beta).transpose(1, 2).reshape(B, Hkv, L // beta, d)
+    kb = torch.repeat_interleave(kb, Hq // Hkv, dim=1)
+    s = qb @ kb.transpose(-1, -2) / math.sqrt(d)
+    nb = L // beta
+    mask = torch.ones(nb, nb, dtype=torch.bool).tril()
+    ref = torch.softmax(s.masked_fill(~mask, float("-inf")), -1)
+    np.testing.assert_allclose(sc.qbar, qb.numpy(), rtol=0, atol=1e-13)
+    np.testing.assert_allclose(sc.probs, ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_band_bookkeeping_equivalences():
+    B, Hq, Hkv, L, d, beta = 1, 2, 1, 64, 16, 8
+    cos, sin = po.rope_tables(1e4, L, d)
+    rng = np.random.default_rng(2)
+    Q = rng.normal(size=(B, Hq, L, d))
+    K = rng.normal(size=(B, Hkv, L, d))
+    single = po.prism_scores(Q, K, beta, 3, po.FLAG_SINGLE_BAND, (cos, sin))
+    all_low = po.prism_scores(Q, K, beta, 0, 0, (cos, sin))      # band H empty
+    all_high = po.prism_scores(Q, K, beta, d // 2, 0, (cos, sin))  # band L empty
+    np.testing.assert_allclose(all_low.probs, single.probs, rtol=0, atol=1e-13)
+    np.testing.assert_allclose(all_high.probs, single.probs, rtol=0, atol=1e-13)
+    # a real split differs from the single band (the two temperatures differ)
+    split = po.prism_scores(Q, K, beta, 3, 0, (cos, sin))
+    assert not np.allclose(split.tau[..., 0], split.tau[..., 1])
+    assert np.abs(split.probs - single.probs).max() > 1e-6
+    # high-band dims are pairs m < bs and their partners m + d/2
+    hm = po.high_band_mask(d, 3)
+    assert list(np.nonzero(hm)[0]) == [0, 1, 2, 8, 9, 10]
+
+
+# ---------------------------------------------------------------------------
+# Selection: brute force over subsets on tiny rows.
+# ---------------------------------------------------------------------------
+def _dominates(pa, a, pb, b):
+    return pa > pb or (pa == pb and a < b)
+
+
+def _brute_topk(p, cand, n):
+    found = []
+    for S in itertools.combinations(cand, n):
+        rest = [c for c in cand if c not in S]
+        if all(_dominates(p[a], a, p[b], b) for a in S for b in rest):
+            found.append(set(S))
+    assert len(found) == 1
+    best = max(sum(p[j] for j in S) for S in itertools.combinations(cand, n)) if n else 0.0
+    assert sum(p[j] for j in found[0]) == best
+    return found[0]
+
+
+@pytest.mark.parametrize("seed", range(6))
+@pytest.mark.parametrize("flags", [0, po.FLAG_KEEP_SINK])
+def test_selection_matches_bruteforce(seed, flags):
+    rng = np.random.default_rng(seed)
+    nb = 9
+    # dyadic values with many exact ties: sums are exact in float64
+    P = rng.integers(0, 6, size=(nb, nb)).astype(np.float64) / 64.0
+    for i in range(nb):
+        forced = po.forced_blocks(i, flags)
+        cand = [j for j in range(i + 1) if j not in forced]
+        for k in range(0, nb + 1):
+            r = po.select_row(P[i], i, flags, k=k)
+            S = _brute_topk(P[i], cand, min(k, len(cand)))
+            assert set(r.kept.tolist()) == S | set(forced)
+            assert list(r.kept) == sorted(r.kept)
+        for mass in (0.0, 3 / 64, 0.25, 0.5, 0.9, 1.0, 5.0):
+            r = po.select_row(P[i], i, flags, mass=mass)
+            base = sum(P[i][j] for j in forced)
+            n_need = len(cand)
+            for n in range(len(cand) + 1):
+                best = max(sum(P[i][j] for j in S) for S in itertools.combinations(cand, n)) if n else 0.0
+                if base + best >= mass:
+                    n_need = n
+                    break
+            S = _brute_topk(P[i], cand, n_need)
+            assert r.n_taken == n_need
+            assert set(r.kept.tolist()) == S | set(forced)
+
+
+def test_selection_invariants_on_softmax_rows():
+    rng = np.random.default_rng(4)
+    nb = 20
+    s = rng.normal(size=(1, 1, nb, nb)) * 3
+    p = po.causal_block_softmax(s)
+    np.testing.assert_allclose(p.sum(-1), 1.0, rtol=1e-12)
+    assert np.all(np.triu(p[0, 0], 1) == 0)
+    for flags in (0, po.FLAG_KEEP_SINK):
+        sel0 = po.select_blocks(p, flags, k=0)
+        all1 = po.select_blocks(p, flags, mass=1.0)
+        for i in range(nb):
+            assert set(sel0[0][0][i].kept.tolist()) == set(po.forced_blocks(i, flags))
+            assert list(all1[0][0][i].kept) == list(range(i + 1))
+            for kk in (1, 3, 50):
+                r = po.select_row(p[0, 0, i], i, flags, k=kk)
+                assert i in r.kept
+                assert len(r.kept) == min(i + 1, kk + len(po.forced_blocks(i, flags)))
+
+
+# ---------------------------------------------------------------------------
+# Attention: exact over kept blocks (§1) against torch SDPA and brute force.
+# ---------------------------------------------------------------------------
+def _sdpa(Q, K, V, causal):
+    group = Q.shape[1] // K.shape[1]
+    k = torch.repeat_interleave(torch.from_numpy(K), group, dim=1)
+    v = torch.repeat_interleave(torch.from_numpy(V), group, dim=1)
+    return torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(Q), k, v, is_causal=causal).numpy()
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_all_blocks_kept_equals_dense_attention(causal):
+    B, Hq, Hkv, L, d, beta = 1, 4, 2, 64, 8, 16
+    rng = np.random.default_rng(6)
+    Q, K, V = (rng.normal(size=(B, h, L, d)) for h in (Hq, Hkv, Hkv))
+    nb = L // beta
+    kept = [[[np.arange(nb if not causal else i + 1) for i in range(nb)] for _ in range(Hq)]
+            for _ in range(B)]
+    O, lse = po.sparse_attention(Q, K, V, kept, beta, causal=causal)
+    np.testing.assert_allclose(O, _sdpa(Q, K, V, causal), rtol=0, atol=1e-12)
+    if causal:
+        np.testing.assert_allclose(O, po.dense_causal_attention_bruteforce(Q, K, V), rtol=0, atol=1e-12)
+    from scipy.special import logsumexp
+    g = Hq // Hkv
+    for h in range(Hq):
+        s = Q[0, h] @ K[0, h // g].T / math.sqrt(d)
+        if causal:
+            s = np.where(np.tril(np.ones((L, L), bool)), s, -np.inf)
+        np.testing.assert_allclose(lse[0, h], logsumexp(s, axis=1), rtol=0, atol=1e-12)
+
+
+def test_diagonal_only_is_blockwise_local_attention():
+    B, Hq, Hkv, L, d, beta = 1, 2, 1, 48, 8, 16
+    rng = np.random.default_rng(8)
+    Q, K, V = (rng.normal(size=(B, h, L, d)) for h in (Hq, Hkv, Hkv))
+    nb = L // beta
+    kept = [[[np.array([i]) for i in range(nb)] for _ in range(Hq)]]
+    O, _ = po.sparse_attention(Q, K, V, kept, beta)
+    for i in range(nb):
+        sl = slice(i * beta, (i + 1) * beta)
+        ref = po.dense_causal_attention_bruteforce(Q[:, :, sl], K[:, :, sl], V[:, :, sl])
+        np.testing.assert_allclose(O[:, :, sl], ref, rtol=0, atol=1e-12)
+
+
+def test_attention_special_cases():
+    rng = np.random.default_rng(10)
+    Q, K, V = (rng.normal(size=(1, 1, 1, 4)) for _ in range(3))
+    O, lse = po.sparse_attention(Q, K, V, [[[np.array([0])]]], 1)
+    np.testing.assert_allclose(O[0, 0, 0], V[0, 0, 0], rtol=0, atol=0)   # a single key: o = v0
+    Q, K, V = (rng.normal(size=(1, 1, 8, 4)) for _ in range(3))
+    O, lse = po.sparse_attention(Q, K, V, [[[np.array([], dtype=np.int64), np.array([0, 1])]]], 4)
+    assert np.all(O[0, 0, :4] == 0) and np.all(np.isneginf(lse[0, 0, :4]))
+    np.testing.assert_allclose(O[0, 0, 0 + 4 * 0], 0.0)
+    O2, _ = po.sparse_attention(Q, K, V, [[[np.array([0]), np.array([0, 1])]]], 4)
+    np.testing.assert_allclose(O2[0, 0, 0], V[0, 0, 0], atol=1e-15)       # first token sees itself
+
+
+def test_bf16_rounding_matches_torch():
+    rng = np.random.default_rng(12)
+    x = (rng.normal(size=100000) * np.exp(rng.normal(size=100000) * 4)).astype(np.float32)
+    ours = po.round_to_bf16(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.bfloat16).to(torch.float64).numpy()
+    np.testing.assert_array_equal(ours, ref)
+
+
+def test_tiny_path_structure():
+    from block_sparse_long_dual_b200.workloads import TINY
+    from block_sparse_long_dual_b200.synthetic import make_inputs
+    w = TINY.scaled(seq_len=512)
+    Q, K, V = (t.numpy() for t in make_inputs(w))
+    cos, sin = po.rope_tables(w.rope_base, w.seq_len, w.head_dim)
+    r = po.prism_path(Q, K, V, block=w.block, band_split=w.band_split, flags=w.flags, k=w.k,
+                      rope=(cos, sin), dtype="f32")
+    nb = w.nb
+    for i in range(nb):
+        kept = r.selection[0][0][i].kept
+        assert i in kept and (i == 0 or 0 in kept)
+        assert len(kept) == min(i + 1, w.k + (2 if i else 1))
+    assert np.all(np.isfinite(r.out))
