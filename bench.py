@@ -1,0 +1,367 @@
+"""Benchmark of the Prism block-sparse attention path (one prefill attention layer).
+
+A step is one pass of the whole path over one layer of synthetic input already
+resident in HBM: sfa_block_scores (RoPE + dual-band pooling + energy
+temperature + block scores), sfa_select, sfa_block_sparse_attn.
+
+    python bench.py [--gpus N --steps K --warmup W] [--workload NAME] [--impl ours|reference]
+
+One process per GPU (torchrun for N > 1).  Every rank runs an independent
+replica of the layer (the path has no exchange step between layers' units;
+"scaling": "weak").  Rank 0 prints one JSON line.
+
+value  = attention FLOPs over the kept blocks (causal diagonal counted half),
+         summed over ranks, / the slowest rank's device time for K steps -> TFLOP/s.
+e2e    = the same metric through PrismAttention.run_host from pinned host
+         tensors: H2D of Q, K, V and D2H of O inside every timed step.
+--impl reference times the CPU oracle (the slow fp64 restatement) on a
+bounded sample of the same workload (see cpu_baseline.sample).
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from block_sparse_long_dual_b200 import workloads as wl  # noqa: E402
+from block_sparse_long_dual_b200.synthetic import make_inputs  # noqa: E402
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_STEP = 5  # rope_pool_energy, band_temperature, block_score_softmax, select, attention
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=wl.LLAMA_128K.name, choices=sorted(wl.ALL))
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=None)
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def attention_flops(counts: np.ndarray, block: int, d: int) -> float:
+    """4*d*(block^2 per off-diagonal kept block + block(block+1)/2 per diagonal block), summed."""
+    n = counts.astype(np.float64)
+    diag = (n > 0).astype(np.float64)  # the diagonal block is always in the selection
+    return float(4.0 * d * (block * block * (n - diag) + block * (block + 1) / 2.0 * diag).sum())
+
+
+def scoring_bytes(w: wl.Workload) -> float:
+    """Algorithmic HBM bytes of sfa_block_scores: read Q, K; write Q_r, K_r; read the cos/sin
+    table once; write the block means; write probs [B, Hq, nb, nb]."""
+    e = 2 if w.dtype == "bf16" else 4
+    qk = w.batch * (w.heads_q + w.heads_kv) * w.seq_len * w.head_dim * e
+    table = 2 * w.seq_len * (w.head_dim // 2) * 4
+    means = w.batch * (w.heads_q + w.heads_kv) * w.nb * w.head_dim * 4
+    probs = w.batch * w.heads_q * w.nb * w.nb * 4
+    return float(2 * qk + table + means + probs)
+
+
+def select_bytes(w: wl.Workload, kmax: int) -> float:
+    """Read the causal triangle of probs, write counts and idx."""
+    tri = w.batch * w.heads_q * w.nb * (w.nb + 1) / 2 * 4
+    return float(tri + w.batch * w.heads_q * w.nb * (1 + kmax) * 4)
+
+
+def traffic_record(kernel_file: str):
+    """ncu DRAM bytes per launch of the attention kernel, if captured for the current source."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        rec = json.load(f)
+    h = hashlib.sha256()
+    for fn in rec.get("sources", []):
+        with open(os.path.join(ROOT, fn), "rb") as f:
+            h.update(f.read())
+    if rec.get("sha256") != h.hexdigest():
+        return None
+    return rec
+
+
+class ClockSampler:
+    """Samples SM clock and throttle reasons through NVML while the timed region runs."""
+
+    def __init__(self, index: int, period_s: float = 0.005):
+        self.samples, self.reasons = [], set()
+        self.period, self.index = period_s, index
+        self.ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "sw_power_cap": getattr(nv, "nvmlClocksEventReasonSwPowerCap", 0x4),
+            "hw_slowdown": getattr(nv, "nvmlClocksEventReasonHwSlowdown", 0x8),
+            "sw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonSwThermalSlowdown", 0x20),
+            "hw_thermal_slowdown": getattr(nv, "nvmlClocksEventReasonHwThermalSlowdown", 0x40),
+            "hw_power_brake_slowdown": getattr(nv, "nvmlClocksEventReasonHwPowerBrakeSlowdown", 0x80),
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in names.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        if self.ok:
+            self._stop.set()
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def oracle_head_sample(w: wl.Workload, Q, K, V, h: int = 0, attn_blocks: int | None = None):
+    """Time the CPU oracle on one (batch 0, Q head h) unit of the workload.
+
+    Runs the estimate, the selection of every row and exact attention over
+    ``attn_blocks`` evenly spaced query blocks (all when None); the attention
+    time is scaled to all query blocks of the head.  Returns (TFLOP/s, seconds, sample text)."""
+    from oracle import prism_oracle as po
+    g = h // w.group
+    Qh = Q[0:1, h:h + 1].to(torch.float64).numpy()
+    Kh = K[0:1, g:g + 1].to(torch.float64).numpy()
+    Vh = V[0:1, g:g + 1].to(torch.float64).numpy()
+    mass = None if w.mass is None else float(np.float32(w.mass))
+    t0 = time.perf_counter()
+    cos, sin = po.rope_tables(w.rope_base, w.seq_len, w.head_dim)
+    sc = po.prism_scores(Qh, Kh, w.block, w.band_split, w.flags, (cos, sin))
+    sel = po.select_blocks(sc.probs, w.flags, k=w.k, mass=mass)
+    qa = po.round_to_dtype(sc.q_rot, w.dtype)
+    ka = po.round_to_dtype(sc.k_rot, w.dtype)
+    t1 = time.perf_counter()
+    nb = w.nb
+    rows = list(range(nb)) if attn_blocks is None or attn_blocks >= nb else \
+        sorted(set(np.linspace(0, nb - 1, attn_blocks).astype(int).tolist()))
+    keep = set(rows)
+    kept = [[[sel[0][0][i].kept if i in keep else np.zeros(0, np.int64) for i in range(nb)]]]
+    po.sparse_attention(qa, ka, Vh, kept, w.block)
+    t2 = time.perf_counter()
+    counts = np.array([sel[0][0][i].kept.size for i in range(nb)])
+    flops = attention_flops(counts, w.block, w.head_dim)
+    secs = (t1 - t0) + (t2 - t1) * nb / len(rows)
+    text = (f"batch 0, Q head {h} of {w.heads_q}: RoPE tables, estimate and selection over the full "
+            f"{w.seq_len}-token head, exact attention on {len(rows)} of {nb} query blocks"
+            + ("" if len(rows) == nb else f" (attention time scaled by {nb}/{len(rows)})"))
+    return flops / secs / 1e12, secs, text
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i["num_threads"] for i in threadpool_info()] or [1])
+    except Exception:
+        return None
+
+
+def run_reference(args, w, rank, world):
+    """The reference arm: the CPU oracle as it stands, on host cores, bounded sample per step."""
+    if rank != 0:
+        return
+    Q, K, V = make_inputs(w.scaled(batch=1), seed=0)
+    per_step = []
+    blocks = max(4, min(64, w.nb // 16))
+    text = ""
+    for s in range(args.warmup + args.steps):
+        v, secs, text = oracle_head_sample(w, Q, K, V, h=s % w.heads_q, attn_blocks=blocks)
+        if s >= args.warmup:
+            per_step.append((v, secs))
+    value = float(np.mean([v for v, _ in per_step]))
+    ms = float(np.mean([s for _, s in per_step]) * 1e3)
+    cores = len(os.sched_getaffinity(0))
+    line = {"metric": "prefill attention effective TFLOP/s over kept blocks (whole path)", "value": value,
+            "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": w.name, "layer": f"B={w.batch} Hq={w.heads_q} Hkv={w.heads_kv} "
+                       f"L={w.seq_len} d={w.head_dim} block={w.block}"},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads() or cores,
+                             "kind": "oracle", "sample": text},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    w = wl.ALL[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+
+    from block_sparse_long_dual_b200 import sfa
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    Q, K, V = make_inputs(w, seed=rank)
+    model = sfa.PrismAttention(batch=w.batch, heads_q=w.heads_q, heads_kv=w.heads_kv, seq_len=w.seq_len,
+                               head_dim=w.head_dim, dtype=w.dtype, block=w.block, rope_base=w.rope_base,
+                               band_split=w.band_split, k=w.k, mass=w.mass, flags=w.flags, device=dev)
+    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        model(Qd, Kd, Vd)
+    torch.cuda.synchronize(dev)
+    if int(model.status.item()) != 0:
+        raise RuntimeError(f"device status {int(model.status.item())}")
+
+    K_ = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for s in range(K_):
+            ev[s][0].record(stream)
+            model.scores(Qd, Kd)
+            ev[s][1].record(stream)
+            model.select()
+            ev[s][2].record(stream)
+            model.attend(Vd)
+            ev[s][3].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    total_ms = start.elapsed_time(stop)
+    t_scores = [ev[s][0].elapsed_time(ev[s][1]) for s in range(K_)]
+    t_select = [ev[s][1].elapsed_time(ev[s][2]) for s in range(K_)]
+    t_attn = [ev[s][2].elapsed_time(ev[s][3]) for s in range(K_)]
+
+    counts = model.counts.cpu().numpy()
+    flops_step = attention_flops(counts, w.block, w.head_dim)
+    kept_frac = float(counts.sum()) / (w.batch * w.heads_q * w.nb * (w.nb + 1) / 2)
+
+    # e2e: the public API from pinned host buffers, copies inside the timed region
+    e2e_steps = args.e2e_steps or K_
+    Qh, Kh, Vh = (t.pin_memory() for t in (Q, K, V))
+    Oh = torch.empty(model.O.shape, dtype=model.O.dtype).pin_memory()
+    dev_in = (torch.empty_like(Qd), torch.empty_like(Kd), torch.empty_like(Vd))
+    model.run_host(Qh, Kh, Vh, Oh, dev_in=dev_in)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        model.run_host(Qh, Kh, Vh, Oh, dev_in=dev_in)
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh))
+    d2h = Oh.numel() * Oh.element_size()
+
+    vals = torch.tensor([total_ms, e2e_ms, float(np.mean(t_attn)), float(np.mean(t_scores)),
+                         float(np.mean(t_select))], dtype=torch.float64, device=dev)
+    fl = torch.tensor([flops_step], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+        dist.all_reduce(fl, op=dist.ReduceOp.SUM)
+    total_ms, e2e_ms, attn_ms, scores_ms, select_ms = vals.tolist()
+    flops_all = fl.item()
+
+    if rank == 0:
+        pk, pk_src = peaks()
+        value = flops_all * K_ / (total_ms * 1e-3) / 1e12
+        e2e_value = flops_all * e2e_steps / (e2e_ms * 1e-3) / 1e12
+        achieved = flops_step / (attn_ms * 1e-3) / 1e12
+        peak = float(pk["bf16_tflops"])
+        tr = traffic_record("block_sparse_long_dual_b200/csrc/attn_tc.cu")
+        sb, selb = scoring_bytes(w), select_bytes(w, model.kmax)
+        line = {
+            "metric": "prefill attention effective TFLOP/s over kept blocks (whole path)",
+            "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K_, "warmup": args.warmup,
+            "ms_per_step": total_ms / K_, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": w.dtype, "data": "synthetic",
+            "config": {"workload": w.name,
+                       "layer": f"B={w.batch} Hq={w.heads_q} Hkv={w.heads_kv} L={w.seq_len} d={w.head_dim} "
+                                f"block={w.block} rope_base={w.rope_base:g} band_split={w.band_split}",
+                       "budget": (f"top-{w.k} + diagonal" if w.k is not None else f"mass {w.mass}"),
+                       "kept_fraction": round(kept_frac, 5), "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (Q 1.07 GB, K 0.27 GB, V 0.27 GB at 128K); no flush"},
+            "stages_ms": {"block_scores": scores_ms, "select": select_ms, "attention": attn_ms},
+            "scoring": {"bytes": sb + selb, "GB_s": (sb + selb) / ((scores_ms + select_ms) * 1e-3) / 1e9,
+                        "frac_hbm": (sb + selb) / ((scores_ms + select_ms) * 1e-3) / 1e9 / float(pk["hbm_gbs"])},
+            "roofline": {"kernel": "attn_tc_kernel (sfa_block_sparse_attn)", "bound": "tensor",
+                         "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+                         "peak_source": f"{pk_src} bf16 burst",
+                         "traffic": (tr["bytes_per_launch"] * (flops_step / tr["flops_per_launch"])
+                                     if tr else None),
+                         "flops_per_launch": flops_step},
+            "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
+            "gpu_launches": KERNELS_PER_STEP * K_,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, secs, text = oracle_head_sample(w, Q, K, V, h=0)
+            line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s",
+                                    "cores": blas_threads() or len(os.sched_getaffinity(0)),
+                                    "kind": "oracle", "sample": text, "seconds": secs}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

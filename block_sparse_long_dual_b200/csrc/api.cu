@@ -1,0 +1,262 @@
+// C-ABI host layer: argument validation, workspace layout, tensor maps and
+// kernel launches on the caller's stream.  Declarations and the contract of
+// every entry point are in include/sfa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdlib.h>
+#include <string.h>
+
+#include <mutex>
+#include <vector>
+
+#include "kernels.h"
+#include "sfa.h"
+
+using namespace sfa;
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxBlocks = 2048;
+constexpr unsigned kKnownFlags = SFA_KEEP_SINK | SFA_NO_CALIB | SFA_SINGLE_BAND;
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+size_t align256(size_t x) { return (x + 255) & ~(size_t)255; }
+
+// Common shape checks; nb_out receives L / block.
+sfa_status check_shape(const sfa_shape* s, int block, int* nb_out) {
+  if (s == nullptr) return SFA_ERR_INVALID_ARG;
+  if (s->dtype != SFA_F32 && s->dtype != SFA_BF16) return SFA_ERR_DTYPE;
+  if (s->batch < 1 || s->heads_q < 1 || s->heads_kv < 1 || s->seq_len < 1) return SFA_ERR_SHAPE;
+  if (s->head_dim != 64 && s->head_dim != 128) return SFA_ERR_SHAPE;
+  if (block != 64 && block != 128) return SFA_ERR_SHAPE;
+  if (s->heads_q % s->heads_kv != 0) return SFA_ERR_SHAPE;
+  if (s->seq_len % block != 0) return SFA_ERR_SHAPE;
+  const int nb = s->seq_len / block;
+  if (nb > kMaxBlocks) return SFA_ERR_UNSUPPORTED;
+  // Row indices of the [B*H*L, d] views and tile ids must fit in int32.
+  const long long rows = (long long)s->batch * s->heads_q * s->seq_len;
+  if (rows >= (1LL << 31)) return SFA_ERR_UNSUPPORTED;
+  if (nb_out) *nb_out = nb;
+  return SFA_OK;
+}
+
+struct WsLayout {
+  size_t off[4];
+  size_t total;
+};
+
+WsLayout ws_layout(const sfa_shape* s, int nb) {
+  WsLayout w;
+  const size_t d = s->head_dim;
+  size_t o = 0;
+  w.off[0] = o;
+  o = align256(o + (size_t)s->batch * s->heads_q * nb * d * sizeof(float));
+  w.off[1] = o;
+  o = align256(o + (size_t)s->batch * s->heads_kv * nb * d * sizeof(float));
+  w.off[2] = o;
+  o = align256(o + (size_t)s->batch * (s->heads_q + s->heads_kv) * nb * 4 * sizeof(float));
+  w.off[3] = o;
+  o = align256(o + (size_t)s->batch * s->heads_q * 2 * sizeof(double));
+  w.total = o;
+  return w;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda link).
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::once_flag once;
+  static EncodeTiledFn fn = nullptr;
+  std::call_once(once, [] {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  });
+  return fn;
+}
+
+// 2D bf16 view [rows, 128] with 64 x 128 boxes and 128-byte swizzle.
+bool make_tile_map(CUtensorMap* m, const void* base, uint64_t rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t dims[2] = {128, rows};
+  const cuuint64_t strides[1] = {128 * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+sfa_status cuda_status(cudaError_t e) { return e == cudaSuccess ? SFA_OK : SFA_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int sfa_version(void) { return kVersion; }
+
+const char* sfa_status_string(sfa_status status) {
+  switch (status) {
+    case SFA_OK: return "ok";
+    case SFA_ERR_INVALID_ARG: return "invalid argument";
+    case SFA_ERR_SHAPE: return "invalid shape";
+    case SFA_ERR_DTYPE: return "unsupported dtype";
+    case SFA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case SFA_ERR_WORKSPACE: return "workspace missing or too small";
+    case SFA_ERR_CUDA: return "CUDA error";
+    case SFA_ERR_TIMEOUT: return "device wait timed out";
+    case SFA_ERR_INDEX: return "invalid block index list";
+  }
+  return "unknown status";
+}
+
+sfa_status sfa_rope_table(double base, int seq_len, int head_dim, float* cos_out, float* sin_out,
+                          void* stream) {
+  if (cos_out == nullptr || sin_out == nullptr || !(base > 0.0)) return SFA_ERR_INVALID_ARG;
+  if (seq_len < 1 || head_dim < 2 || (head_dim & 1)) return SFA_ERR_SHAPE;
+  const int half = head_dim / 2;
+  const size_t n = (size_t)seq_len * half;
+  std::vector<float> c(n), s(n);
+  std::vector<double> theta(half);
+  for (int m = 0; m < half; ++m) theta[m] = pow(base, -2.0 * m / head_dim);
+  for (int p = 0; p < seq_len; ++p) {
+    for (int m = 0; m < half; ++m) {
+      const double a = (double)p * theta[m];
+      c[(size_t)p * half + m] = (float)cos(a);
+      s[(size_t)p * half + m] = (float)sin(a);
+    }
+  }
+  cudaStream_t st = as_stream(stream);
+  // Pageable source: the call returns once the host data has been staged.
+  if (cudaMemcpyAsync(cos_out, c.data(), n * sizeof(float), cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return SFA_ERR_CUDA;
+  if (cudaMemcpyAsync(sin_out, s.data(), n * sizeof(float), cudaMemcpyHostToDevice, st) != cudaSuccess)
+    return SFA_ERR_CUDA;
+  return SFA_OK;
+}
+
+size_t sfa_block_scores_workspace(const sfa_shape* shape, int block) {
+  int nb = 0;
+  if (check_shape(shape, block, &nb) != SFA_OK) return 0;
+  return ws_layout(shape, nb).total;
+}
+
+sfa_status sfa_workspace_layout(const sfa_shape* shape, int block, size_t offsets[4]) {
+  int nb = 0;
+  const sfa_status st = check_shape(shape, block, &nb);
+  if (st != SFA_OK) return st;
+  if (offsets == nullptr) return SFA_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(shape, nb);
+  for (int q = 0; q < 4; ++q) offsets[q] = w.off[q];
+  return SFA_OK;
+}
+
+sfa_status sfa_block_scores(const sfa_shape* shape, const void* Q, const void* K, const sfa_rope* rope,
+                            int band_split, int block, unsigned flags, void* Q_rot, void* K_rot, float* probs,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  int nb = 0;
+  sfa_status st = check_shape(shape, block, &nb);
+  if (st != SFA_OK) return st;
+  const int D = shape->head_dim;
+  if (Q == nullptr || K == nullptr || rope == nullptr || probs == nullptr) return SFA_ERR_INVALID_ARG;
+  if (flags & ~kKnownFlags) return SFA_ERR_INVALID_ARG;
+  if (band_split < 0 || band_split > D / 2) return SFA_ERR_INVALID_ARG;
+  if (rope->apply && (rope->cos == nullptr || rope->sin == nullptr || Q_rot == nullptr || K_rot == nullptr))
+    return SFA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || (rope->apply && (!aligned16(Q_rot) || !aligned16(K_rot) ||
+                                                         !aligned16(rope->cos) || !aligned16(rope->sin))))
+    return SFA_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(shape, nb);
+  if (workspace == nullptr || workspace_bytes < w.total || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return SFA_ERR_WORKSPACE;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  cudaStream_t cs = as_stream(stream);
+  const int band_pairs = (flags & SFA_SINGLE_BAND) ? D / 2 : band_split;
+
+  RopePoolParams rp;
+  rp.Q = Q; rp.K = K; rp.Qr = Q_rot; rp.Kr = K_rot;
+  rp.cos = rope->cos; rp.sin = rope->sin;
+  rp.apply = rope->apply ? 1 : 0;
+  rp.write_rot = rope->apply ? 1 : 0;
+  rp.qbar = reinterpret_cast<float*>(ws + w.off[0]);
+  rp.kbar = reinterpret_cast<float*>(ws + w.off[1]);
+  rp.energy = reinterpret_cast<float*>(ws + w.off[2]);
+  rp.B = shape->batch; rp.Hq = shape->heads_q; rp.Hkv = shape->heads_kv;
+  rp.L = shape->seq_len; rp.block = block; rp.nb = nb; rp.band_pairs = band_pairs;
+  st = cuda_status(launch_rope_pool_energy(rp, shape->dtype, D, cs));
+  if (st != SFA_OK) return st;
+
+  TauParams tp;
+  tp.energy = rp.energy;
+  tp.tau = reinterpret_cast<double*>(ws + w.off[3]);
+  tp.B = rp.B; tp.Hq = rp.Hq; tp.Hkv = rp.Hkv; tp.L = rp.L; tp.nb = nb; tp.flags = flags;
+  st = cuda_status(launch_band_temperature(tp, cs));
+  if (st != SFA_OK) return st;
+
+  ScoreParams sp;
+  sp.qbar = rp.qbar; sp.kbar = rp.kbar; sp.tau = tp.tau; sp.probs = probs;
+  sp.B = rp.B; sp.Hq = rp.Hq; sp.Hkv = rp.Hkv; sp.nb = nb; sp.band_pairs = band_pairs;
+  return cuda_status(launch_block_score_softmax(sp, D, cs));
+}
+
+sfa_status sfa_select(const sfa_shape* shape, int block, const float* probs, int k, float mass, unsigned flags,
+                      int* counts, int* idx, int kmax, void* stream) {
+  int nb = 0;
+  sfa_status st = check_shape(shape, block, &nb);
+  if (st != SFA_OK) return st;
+  if (probs == nullptr || counts == nullptr || idx == nullptr) return SFA_ERR_INVALID_ARG;
+  if (flags & ~kKnownFlags) return SFA_ERR_INVALID_ARG;
+  const int nforced = (flags & SFA_KEEP_SINK) && nb > 1 ? 2 : 1;
+  int need;
+  if (k >= 0) {
+    need = k + nforced < nb ? k + nforced : nb;
+  } else {
+    if (!(mass > 0.f && mass <= 1.f)) return SFA_ERR_INVALID_ARG;
+    need = nb;
+  }
+  if (kmax < need || kmax < 1) return SFA_ERR_INVALID_ARG;
+  SelectParams p;
+  p.probs = probs; p.counts = counts; p.idx = idx;
+  p.B = shape->batch; p.Hq = shape->heads_q; p.nb = nb; p.kmax = kmax;
+  p.k = k; p.mass = (double)mass; p.flags = flags;
+  return cuda_status(launch_select(p, as_stream(stream)));
+}
+
+sfa_status sfa_block_sparse_attn(const sfa_shape* shape, int block, const void* Q, const void* K, const void* V,
+                                 const int* counts, const int* idx, int kmax, int causal, float scale, void* O,
+                                 float* lse, int* status_word, void* stream) {
+  int nb = 0;
+  sfa_status st = check_shape(shape, block, &nb);
+  if (st != SFA_OK) return st;
+  if (Q == nullptr || K == nullptr || V == nullptr || counts == nullptr || idx == nullptr || O == nullptr)
+    return SFA_ERR_INVALID_ARG;
+  if (kmax < 1 || !(isfinite(scale))) return SFA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SFA_ERR_INVALID_ARG;
+  const int D = shape->head_dim;
+  AttnParams p;
+  p.Q = Q; p.K = K; p.V = V; p.counts = counts; p.idx = idx; p.O = O; p.lse = lse; p.status = status_word;
+  p.B = shape->batch; p.Hq = shape->heads_q; p.Hkv = shape->heads_kv; p.L = shape->seq_len;
+  p.block = block; p.nb = nb; p.kmax = kmax; p.causal = causal ? 1 : 0;
+  p.scale = scale > 0.f ? scale : (float)(1.0 / sqrt((double)D));
+  cudaStream_t cs = as_stream(stream);
+  if (shape->dtype == SFA_BF16 && block == 128 && D == 128) {
+    CUtensorMap tq, tk, tv;
+    const uint64_t rq = (uint64_t)p.B * p.Hq * p.L, rkv = (uint64_t)p.B * p.Hkv * p.L;
+    if (!make_tile_map(&tq, Q, rq) || !make_tile_map(&tk, K, rkv) || !make_tile_map(&tv, V, rkv))
+      return SFA_ERR_CUDA;
+    return cuda_status(launch_attn_tcgen05(p, tq, tk, tv, cs));
+  }
+  return cuda_status(launch_attn_simt(p, shape->dtype, D, cs));
+}
+
+}  // extern "C"

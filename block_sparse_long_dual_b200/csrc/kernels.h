@@ -1,0 +1,76 @@
+// Internal launch interface between the C-ABI host layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace sfa {
+
+struct RopePoolParams {
+  const void* Q;
+  const void* K;
+  void* Qr;
+  void* Kr;
+  const float* cos;
+  const float* sin;
+  int apply;      // rotate (else Q, K are already rotated)
+  int write_rot;  // write the rotated copies
+  float* qbar;
+  float* kbar;
+  float* energy;
+  int B, Hq, Hkv, L, block, nb;
+  int band_pairs;  // rotary pairs in band H (d/2 with a single band)
+};
+
+struct TauParams {
+  const float* energy;
+  double* tau;
+  int B, Hq, Hkv, L, nb;
+  unsigned flags;
+};
+
+struct ScoreParams {
+  const float* qbar;
+  const float* kbar;
+  const double* tau;
+  float* probs;
+  int B, Hq, Hkv, nb;
+  int band_pairs;
+};
+
+struct SelectParams {
+  const float* probs;
+  int* counts;
+  int* idx;
+  int B, Hq, nb, kmax;
+  int k;        // >= 0: top-k; < 0: mass
+  double mass;
+  unsigned flags;
+};
+
+struct AttnParams {
+  const void* Q;
+  const void* K;
+  const void* V;
+  const int* counts;
+  const int* idx;
+  void* O;
+  float* lse;
+  int* status;
+  int B, Hq, Hkv, L, block, nb, kmax;
+  int causal;
+  float scale;  // softmax scale (natural-log units)
+};
+
+cudaError_t launch_rope_pool_energy(const RopePoolParams& p, int dtype, int D, cudaStream_t st);
+cudaError_t launch_band_temperature(const TauParams& p, cudaStream_t st);
+cudaError_t launch_block_score_softmax(const ScoreParams& p, int D, cudaStream_t st);
+size_t score_smem_bytes(int nb, int D);
+cudaError_t launch_select(const SelectParams& p, cudaStream_t st);
+cudaError_t launch_attn_simt(const AttnParams& p, int dtype, int D, cudaStream_t st);
+cudaError_t launch_attn_tcgen05(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                const CUtensorMap& tmV, cudaStream_t st);
+
+}  // namespace sfa

@@ -1,0 +1,274 @@
+"""Python binding of the C-ABI library ``libsfa.so`` (argument marshalling only).
+
+Every step of the path runs in the library's CUDA kernels; this module only
+checks tensor shapes / dtypes / devices, allocates outputs with PyTorch and
+passes raw device pointers plus the current CUDA stream.  If the library is
+missing it raises: there is no fallback.
+
+Names follow include/sfa.h: ``rope_table``, ``block_scores``, ``select``,
+``block_sparse_attn``; ``PrismAttention`` chains the three calls of the
+estimate -> select -> attend path of "Prism: Spectral-Aware Block-Sparse
+Attention" for one fixed layer shape with preallocated buffers.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from ctypes import POINTER, c_double, c_float, c_int, c_int32, c_size_t, c_uint, c_void_p
+
+import torch
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsfa.so")
+
+F32, BF16 = 0, 1
+KEEP_SINK, NO_CALIB, SINGLE_BAND = 1, 2, 4
+STATUS = {0: "SFA_OK", 1: "SFA_ERR_INVALID_ARG", 2: "SFA_ERR_SHAPE", 3: "SFA_ERR_DTYPE",
+          4: "SFA_ERR_UNSUPPORTED", 5: "SFA_ERR_WORKSPACE", 6: "SFA_ERR_CUDA", 7: "SFA_ERR_TIMEOUT",
+          8: "SFA_ERR_INDEX"}
+
+
+class SfaError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what}: {STATUS.get(code, code)}")
+        self.code = code
+
+
+class Shape(ctypes.Structure):
+    _fields_ = [("batch", c_int32), ("heads_q", c_int32), ("heads_kv", c_int32),
+                ("seq_len", c_int32), ("head_dim", c_int32), ("dtype", c_int32)]
+
+
+class Rope(ctypes.Structure):
+    _fields_ = [("cos", c_void_p), ("sin", c_void_p), ("apply", c_int32)]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libsfa.so (built by ``block_sparse_long_dual_b200.build``); raise if it is missing."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} not found: build it with `python -m block_sparse_long_dual_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    lib.sfa_version.restype = c_int
+    lib.sfa_status_string.restype = ctypes.c_char_p
+    lib.sfa_status_string.argtypes = [c_int]
+    lib.sfa_rope_table.restype = c_int
+    lib.sfa_rope_table.argtypes = [c_double, c_int, c_int, c_void_p, c_void_p, c_void_p]
+    lib.sfa_block_scores_workspace.restype = c_size_t
+    lib.sfa_block_scores_workspace.argtypes = [POINTER(Shape), c_int]
+    lib.sfa_workspace_layout.restype = c_int
+    lib.sfa_workspace_layout.argtypes = [POINTER(Shape), c_int, POINTER(c_size_t)]
+    lib.sfa_block_scores.restype = c_int
+    lib.sfa_block_scores.argtypes = [POINTER(Shape), c_void_p, c_void_p, POINTER(Rope), c_int, c_int, c_uint,
+                                     c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]
+    lib.sfa_select.restype = c_int
+    lib.sfa_select.argtypes = [POINTER(Shape), c_int, c_void_p, c_int, c_float, c_uint, c_void_p, c_void_p,
+                               c_int, c_void_p]
+    lib.sfa_block_sparse_attn.restype = c_int
+    lib.sfa_block_sparse_attn.argtypes = [POINTER(Shape), c_int, c_void_p, c_void_p, c_void_p, c_void_p,
+                                          c_void_p, c_int, c_int, c_float, c_void_p, c_void_p, c_void_p,
+                                          c_void_p]
+    _lib = lib
+    return lib
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise SfaError(code, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _cuda(t: torch.Tensor, name: str):
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def make_shape(Q: torch.Tensor, K: torch.Tensor) -> Shape:
+    if Q.dim() != 4 or K.dim() != 4:
+        raise ValueError("Q and K must be [B, H, L, d]")
+    B, Hq, L, d = Q.shape
+    if K.shape[0] != B or K.shape[2] != L or K.shape[3] != d or K.dtype != Q.dtype:
+        raise ValueError("K must be [B, Hkv, L, d] with the dtype of Q")
+    return Shape(B, Hq, K.shape[1], L, d, _dtype_code(Q))
+
+
+def rope_table(base: float, seq_len: int, head_dim: int, device="cuda", stream=None):
+    """cos/sin tables [seq_len, head_dim/2] float32 on ``device`` (sfa_rope_table)."""
+    lib = load()
+    cos = torch.empty((seq_len, head_dim // 2), dtype=torch.float32, device=device)
+    sin = torch.empty_like(cos)
+    _check(lib.sfa_rope_table(float(base), seq_len, head_dim, _ptr(cos), _ptr(sin), _stream(stream)),
+           "sfa_rope_table")
+    return cos, sin
+
+
+def workspace_bytes(shape: Shape, block: int) -> int:
+    return int(load().sfa_block_scores_workspace(ctypes.byref(shape), block))
+
+
+def workspace_layout(shape: Shape, block: int):
+    off = (c_size_t * 4)()
+    _check(load().sfa_workspace_layout(ctypes.byref(shape), block, off), "sfa_workspace_layout")
+    return [int(x) for x in off]
+
+
+def workspace_views(ws: torch.Tensor, shape: Shape, block: int):
+    """Qbar, Kbar, energy, tau views of a workspace buffer (see include/sfa.h)."""
+    off = workspace_layout(shape, block)
+    nb = shape.seq_len // block
+    B, Hq, Hkv, d = shape.batch, shape.heads_q, shape.heads_kv, shape.head_dim
+
+    def view(i, n, dt, shp):
+        nbytes = n * torch.tensor([], dtype=dt).element_size()
+        return ws[off[i]:off[i] + nbytes].view(dt).view(*shp)
+
+    return (view(0, B * Hq * nb * d, torch.float32, (B, Hq, nb, d)),
+            view(1, B * Hkv * nb * d, torch.float32, (B, Hkv, nb, d)),
+            view(2, B * (Hq + Hkv) * nb * 4, torch.float32, (B, Hq + Hkv, nb, 4)),
+            view(3, B * Hq * 2, torch.float64, (B, Hq, 2)))
+
+
+def block_scores(Q, K, cos, sin, *, band_split: int, block: int, flags: int = 0, apply_rope: bool = True,
+                 Q_rot=None, K_rot=None, probs=None, workspace=None, stream=None):
+    """sfa_block_scores: returns (Q_rot, K_rot, probs, workspace)."""
+    lib = load()
+    _cuda(Q, "Q"); _cuda(K, "K")
+    shape = make_shape(Q, K)
+    nb = shape.seq_len // block if block > 0 else 0
+    if apply_rope:
+        Q_rot = torch.empty_like(Q) if Q_rot is None else Q_rot
+        K_rot = torch.empty_like(K) if K_rot is None else K_rot
+        _cuda(cos, "cos"); _cuda(sin, "sin")
+    if probs is None:
+        probs = torch.empty((shape.batch, shape.heads_q, nb, nb), dtype=torch.float32, device=Q.device)
+    if workspace is None:
+        workspace = torch.empty(max(workspace_bytes(shape, block), 256), dtype=torch.uint8, device=Q.device)
+    rope = Rope(cos.data_ptr() if apply_rope else None, sin.data_ptr() if apply_rope else None,
+                1 if apply_rope else 0)
+    _check(lib.sfa_block_scores(ctypes.byref(shape), _ptr(Q), _ptr(K), ctypes.byref(rope), band_split, block,
+                                flags, _ptr(Q_rot) if apply_rope else None, _ptr(K_rot) if apply_rope else None,
+                                _ptr(probs), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "sfa_block_scores")
+    return (Q_rot if apply_rope else Q), (K_rot if apply_rope else K), probs, workspace
+
+
+def kmax_for(nb: int, k: int | None, flags: int) -> int:
+    if k is None:
+        return nb
+    nforced = 2 if (flags & KEEP_SINK) and nb > 1 else 1
+    return min(nb, k + nforced)
+
+
+def select(probs, shape: Shape, *, block: int, k: int | None = None, mass: float | None = None,
+           flags: int = 0, kmax: int | None = None, counts=None, idx=None, stream=None):
+    """sfa_select: returns (counts [B,Hq,nb] int32, idx [B,Hq,nb,kmax] int32)."""
+    lib = load()
+    _cuda(probs, "probs")
+    if (k is None) == (mass is None):
+        raise ValueError("give exactly one of k / mass")
+    nb = shape.seq_len // block
+    kmax = kmax_for(nb, k, flags) if kmax is None else kmax
+    if counts is None:
+        counts = torch.empty((shape.batch, shape.heads_q, nb), dtype=torch.int32, device=probs.device)
+    if idx is None:
+        idx = torch.empty((shape.batch, shape.heads_q, nb, kmax), dtype=torch.int32, device=probs.device)
+    _check(lib.sfa_select(ctypes.byref(shape), block, _ptr(probs), -1 if k is None else int(k),
+                          0.0 if mass is None else float(mass), flags, _ptr(counts), _ptr(idx), kmax,
+                          _stream(stream)), "sfa_select")
+    return counts, idx
+
+
+def block_sparse_attn(Q, K, V, counts, idx, *, block: int, causal: bool = True, scale: float = 0.0,
+                      O=None, lse=None, status=None, stream=None):
+    """sfa_block_sparse_attn: returns O (and writes lse / status when given)."""
+    lib = load()
+    for t, n in ((Q, "Q"), (K, "K"), (V, "V"), (counts, "counts"), (idx, "idx")):
+        _cuda(t, n)
+    shape = make_shape(Q, K)
+    if V.shape != K.shape or V.dtype != K.dtype:
+        raise ValueError("V must match K")
+    O = torch.empty_like(Q) if O is None else O
+    _check(lib.sfa_block_sparse_attn(ctypes.byref(shape), block, _ptr(Q), _ptr(K), _ptr(V), _ptr(counts),
+                                     _ptr(idx), idx.shape[-1], 1 if causal else 0, float(scale), _ptr(O),
+                                     _ptr(lse), _ptr(status), _stream(stream)), "sfa_block_sparse_attn")
+    return O
+
+
+class PrismAttention:
+    """The whole path for one layer shape: estimate -> select -> exact sparse attention.
+
+    Buffers (rotated Q/K, probabilities, workspace, index lists, output) are
+    allocated once here; ``__call__`` only launches the library's kernels."""
+
+    def __init__(self, *, batch, heads_q, heads_kv, seq_len, head_dim, dtype, block, rope_base, band_split,
+                 k=None, mass=None, flags=0, causal=True, device="cuda", with_lse=False):
+        tdt = torch.bfloat16 if dtype in ("bf16", torch.bfloat16) else torch.float32
+        self.block, self.band_split, self.k, self.mass, self.flags, self.causal = (
+            block, band_split, k, mass, flags, causal)
+        self.shape = Shape(batch, heads_q, heads_kv, seq_len, head_dim, BF16 if tdt == torch.bfloat16 else F32)
+        nb = seq_len // block
+        self.nb = nb
+        self.kmax = kmax_for(nb, k, flags)
+        dev = torch.device(device)
+        self.cos, self.sin = rope_table(rope_base, seq_len, head_dim, device=dev)
+        self.Q_rot = torch.empty((batch, heads_q, seq_len, head_dim), dtype=tdt, device=dev)
+        self.K_rot = torch.empty((batch, heads_kv, seq_len, head_dim), dtype=tdt, device=dev)
+        self.probs = torch.empty((batch, heads_q, nb, nb), dtype=torch.float32, device=dev)
+        self.workspace = torch.empty(workspace_bytes(self.shape, block), dtype=torch.uint8, device=dev)
+        self.counts = torch.empty((batch, heads_q, nb), dtype=torch.int32, device=dev)
+        self.idx = torch.empty((batch, heads_q, nb, self.kmax), dtype=torch.int32, device=dev)
+        self.O = torch.empty((batch, heads_q, seq_len, head_dim), dtype=tdt, device=dev)
+        self.lse = torch.empty((batch, heads_q, seq_len), dtype=torch.float32, device=dev) if with_lse else None
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def scores(self, Q, K, stream=None):
+        block_scores(Q, K, self.cos, self.sin, band_split=self.band_split, block=self.block, flags=self.flags,
+                     Q_rot=self.Q_rot, K_rot=self.K_rot, probs=self.probs, workspace=self.workspace,
+                     stream=stream)
+
+    def select(self, stream=None):
+        select(self.probs, self.shape, block=self.block, k=self.k, mass=self.mass, flags=self.flags,
+               kmax=self.kmax, counts=self.counts, idx=self.idx, stream=stream)
+
+    def attend(self, V, stream=None):
+        block_sparse_attn(self.Q_rot, self.K_rot, V, self.counts, self.idx, block=self.block,
+                          causal=self.causal, O=self.O, lse=self.lse, status=self.status, stream=stream)
+
+    def __call__(self, Q, K, V, stream=None):
+        self.scores(Q, K, stream)
+        self.select(stream)
+        self.attend(V, stream)
+        return self.O
+
+    def run_host(self, Q_host, K_host, V_host, O_host, dev_in=None, stream=None):
+        """End to end from pinned host tensors: H2D copies, the path, D2H copy of O."""
+        if dev_in is None:
+            dev_in = tuple(torch.empty(t.shape, dtype=t.dtype, device=self.O.device) for t in (Q_host, K_host, V_host))
+        for d, h in zip(dev_in, (Q_host, K_host, V_host)):
+            d.copy_(h, non_blocking=True)
+        self(*dev_in, stream=stream)
+        O_host.copy_(self.O, non_blocking=True)
+        return O_host

@@ -1,0 +1,181 @@
+/*
+ * sfa.h - C ABI of the B200 (sm_100a) importance-scored block-sparse attention library.
+ *
+ * The library computes, on one GPU, the two stages described in
+ * "Prism: Spectral-Aware Block-Sparse Attention":
+ *   1. a block-importance estimate from RoPE-applied Q/K that are mean-pooled
+ *      per block, split into a high- and a low-frequency band and calibrated
+ *      by an energy (RMS) temperature, followed by a block-level score matrix
+ *      and a per-query-block selection (§1, §2, §3.1, §3.2, §5);
+ *   2. exact softmax attention over the kept key blocks only (§1).
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are contiguous, row-major, layout [B, H, L, d] (batch, head,
+ *     token, head dim).  Q has heads_q heads, K and V have heads_kv heads;
+ *     Q head h reads KV head h / (heads_q / heads_kv) (grouped-query attention).
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The
+ *     library never allocates or frees device memory and never synchronises
+ *     the stream; every launch goes on `stream` (a cudaStream_t passed as
+ *     void*, NULL = legacy default stream).
+ *   - Arguments are validated on the host before anything is launched; a
+ *     validation failure returns an error status and launches nothing.  A
+ *     failed launch returns SFA_ERR_CUDA.  Faults detected on the device
+ *     (bounded waits that ran out, bad index lists) are written into the
+ *     optional `status_word` (a device int, first error wins; 0 = ok) and the
+ *     kernel returns without hanging.  No C++ exception crosses this ABI.
+ *   - Sizes: L % block == 0; block in {64, 128}; d in {64, 128};
+ *     heads_q % heads_kv == 0; nb = L / block <= 2048.
+ */
+#ifndef SFA_H_
+#define SFA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SFA_OK = 0,
+  SFA_ERR_INVALID_ARG = 1,  /* null pointer, bad k / mass / flags / scale */
+  SFA_ERR_SHAPE = 2,        /* sizes violate the rules above */
+  SFA_ERR_DTYPE = 3,        /* unknown dtype code */
+  SFA_ERR_UNSUPPORTED = 4,  /* valid but not implemented (e.g. nb > 2048) */
+  SFA_ERR_WORKSPACE = 5,    /* workspace missing or too small */
+  SFA_ERR_CUDA = 6,         /* a CUDA runtime / driver call failed */
+  SFA_ERR_TIMEOUT = 7,      /* device: a bounded wait ran out (status_word only) */
+  SFA_ERR_INDEX = 8         /* device: an index list entry out of range / not ascending */
+} sfa_status;
+
+typedef enum { SFA_F32 = 0, SFA_BF16 = 1 } sfa_dtype;
+
+/* Problem shape.  dtype is the element type of Q, K, V, Q_rot, K_rot and O. */
+typedef struct {
+  int32_t batch, heads_q, heads_kv, seq_len, head_dim;
+  int32_t dtype; /* sfa_dtype */
+} sfa_shape;
+
+/* RoPE tables: cos/sin of angle p * base^(-2m/d), [L, d/2] float32, device.
+ * apply = 0 means Q and K are already rotated (tables ignored, may be NULL). */
+typedef struct {
+  const float* cos;
+  const float* sin;
+  int32_t apply;
+} sfa_rope;
+
+/* Flags for sfa_block_scores / sfa_select. */
+enum {
+  SFA_KEEP_SINK = 1,   /* select: also force key block 0 into every row */
+  SFA_NO_CALIB = 2,    /* scores: temperature tau = 1 (plain mean pooling) */
+  SFA_SINGLE_BAND = 4  /* scores: all d dims form one band (one tau) */
+};
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+int sfa_version(void);
+
+/* Human-readable text for a status code (static storage, never NULL). */
+const char* sfa_status_string(sfa_status status);
+
+/*
+ * RoPE tables (Prism §2 names RoPE; the rotate-half convention of the Llama
+ * and Qwen models of §5).  cos[p, m] = cos(p * base^(-2m/d)) and likewise
+ * sin, computed on the host in double precision and rounded to float32, then
+ * copied to the device arrays `cos` and `sin` ([seq_len, head_dim/2] each,
+ * caller-owned) on `stream`.  Uses a temporary host buffer; returns after the
+ * copies are enqueued.  Errors: SFA_ERR_INVALID_ARG for null pointers or
+ * base <= 0; SFA_ERR_SHAPE for seq_len < 1 or an odd / non-positive head_dim.
+ */
+sfa_status sfa_rope_table(double base, int seq_len, int head_dim, float* cos, float* sin,
+                          void* stream);
+
+/*
+ * Bytes of workspace sfa_block_scores needs for this shape and block size
+ * (0 if the shape is invalid).  The workspace holds, each at a 256-byte
+ * aligned offset given by sfa_workspace_layout:
+ *   [0] Qbar   [B, heads_q,  nb, d] float32  block means of rotated Q
+ *   [1] Kbar   [B, heads_kv, nb, d] float32  block means of rotated K
+ *   [2] energy [B, heads_q + heads_kv, nb, 4] float32 per block:
+ *              sum_t ||x_t^H||^2, sum_t ||x_t^L||^2, ||xbar^H||^2, ||xbar^L||^2
+ *              (Q heads first, then KV heads)
+ *   [3] tau    [B, heads_q, 2] float64  (band H, band L)
+ */
+size_t sfa_block_scores_workspace(const sfa_shape* shape, int block);
+
+/* Byte offsets of the four workspace arrays above.  Errors as sfa_block_scores. */
+sfa_status sfa_workspace_layout(const sfa_shape* shape, int block, size_t offsets[4]);
+
+/*
+ * Block-importance estimate (Prism §2, §3.1, §3.2, §5).
+ *
+ * Q [B, heads_q, L, d], K [B, heads_kv, L, d] (dtype of shape): pre-RoPE values
+ * when rope->apply, else already rotated.  With rope->apply the rotated
+ * tensors are written to Q_rot / K_rot (same shape and dtype, rounded to
+ * nearest even); they are the Q and K the attention call should read.
+ *
+ * Per (batch, Q head, band b in {H, L}), with band H = rotary pairs
+ * m < band_split (dims m and m + d/2), band L = the other dims:
+ *   xbar_j  = mean of the rotated vectors of block j (float32)
+ *   rho^b   = sqrt(mean_j ||xbar_j^b||^2 / mean_t ||x_t^b||^2)   (1 if the band is empty)
+ *   tau^b   = max(rho^b(Q_h) * rho^b(K_g), 1e-6)   (1 with SFA_NO_CALIB)
+ *   s_ij    = sum_b (qbar_i^b . kbar_j^b) / (tau^b * sqrt(d)),  j <= i
+ *   probs_ij = exp(s_ij) / sum_{j' <= i} exp(s_ij'), and 0 for j > i.
+ * probs [B, heads_q, nb, nb] float32.  SFA_SINGLE_BAND puts all dims in band H.
+ * The logits are accumulated with float64 partial sums and the softmax is
+ * evaluated in float64, then rounded once to float32.
+ *
+ * workspace: device buffer of at least sfa_block_scores_workspace() bytes,
+ * 256-byte aligned; its contents are documented above and may be read back.
+ * Errors: SFA_ERR_INVALID_ARG (null pointers, band_split outside [0, d/2],
+ * unknown flags), SFA_ERR_SHAPE, SFA_ERR_DTYPE, SFA_ERR_UNSUPPORTED,
+ * SFA_ERR_WORKSPACE, SFA_ERR_CUDA.  Launches 3 kernels.
+ */
+sfa_status sfa_block_scores(const sfa_shape* shape, const void* Q, const void* K,
+                            const sfa_rope* rope, int band_split, int block, unsigned flags,
+                            void* Q_rot, void* K_rot, float* probs, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
+/*
+ * Block selection (Prism §1: attention runs over a chosen subset of key blocks).
+ * For every row (b, h, i) of probs [B, heads_q, nb, nb]:
+ *   forced F_i = {i}, plus {0} with SFA_KEEP_SINK;
+ *   candidates {0..i} \ F_i ordered by (probability desc, index asc);
+ *   top-k (k >= 0, mass ignored): keep F_i and the first min(k, |C_i|);
+ *   mass (k < 0, 0 < mass <= 1): keep F_i, then add candidates in order while
+ *     the running sum of kept probabilities (forced blocks included,
+ *     accumulated in float64) is below mass.
+ * Writes counts [B, heads_q, nb] int32 and idx [B, heads_q, nb, kmax] int32:
+ * the kept indices ascending, padded with -1.  kmax must be >= the largest
+ * possible count: min(nb, k + |F|) for top-k, nb for mass.
+ * Errors: SFA_ERR_INVALID_ARG (nulls, mass outside (0, 1], kmax too small,
+ * unknown flags), SFA_ERR_SHAPE, SFA_ERR_UNSUPPORTED, SFA_ERR_CUDA.
+ */
+sfa_status sfa_select(const sfa_shape* shape, int block, const float* probs, int k, float mass,
+                      unsigned flags, int* counts, int* idx, int kmax, void* stream);
+
+/*
+ * Exact attention over the kept blocks (Prism §1).  For each query token t
+ * of query block i, over the tokens s of the blocks idx[b, h, i, 0..count)
+ * (with s <= t when causal):
+ *   O_t = sum_s softmax_s(scale * q_t . k_s) v_s,   lse_t = log sum_s exp(scale * q_t . k_s)
+ * Q [B, heads_q, L, d]; K, V [B, heads_kv, L, d]; O like Q; lse [B, heads_q, L]
+ * float32 (natural log; optional, may be NULL).  An empty row gives O = 0 and
+ * lse = -inf.  Each idx row must be ascending with entries in [0, nb) (and
+ * <= i when causal); a violation found on the device sets status_word to
+ * SFA_ERR_INDEX and that tile is skipped.
+ * scale <= 0 selects 1/sqrt(d).
+ * bf16 with block = 128 and d = 128 runs on the tcgen05 tensor cores (TMA
+ * tiles fetched through the index list, accumulators in tensor memory);
+ * every other case (float32, block 64, d 64) runs a float32 CUDA-core kernel.
+ * Errors: SFA_ERR_INVALID_ARG, SFA_ERR_SHAPE, SFA_ERR_DTYPE, SFA_ERR_CUDA.
+ */
+sfa_status sfa_block_sparse_attn(const sfa_shape* shape, int block, const void* Q, const void* K,
+                                 const void* V, const int* counts, const int* idx, int kmax,
+                                 int causal, float scale, void* O, float* lse, int* status_word,
+                                 void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SFA_H_ */

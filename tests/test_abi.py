@@ -1,0 +1,133 @@
+"""The C-ABI library loads, exports every declared entry point, and rejects bad
+arguments on the host before touching the GPU (these run without a GPU)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from block_sparse_long_dual_b200 import build as sfa_build
+from block_sparse_long_dual_b200 import sfa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    sfa_build.build()
+    return sfa.load()
+
+
+def declared_functions():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for fn in sorted(os.listdir(inc)):
+        if fn.endswith(".h"):
+            text = open(os.path.join(inc, fn)).read()
+            text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+            names += re.findall(r"^\s*(?:[A-Za-z_][\w\s\*]*?[\s\*])(sfa_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("sfa_block_scores", "sfa_select", "sfa_block_sparse_attn", "sfa_rope_table",
+                     "sfa_block_scores_workspace", "sfa_workspace_layout", "sfa_status_string", "sfa_version"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_version_and_status_strings(lib):
+    assert lib.sfa_version() >= 100
+    for code in range(9):
+        assert lib.sfa_status_string(code)
+    assert lib.sfa_status_string(99) == b"unknown status"
+
+
+def S(B=1, Hq=4, Hkv=2, L=1024, d=128, dt=sfa.BF16):
+    return sfa.Shape(B, Hq, Hkv, L, d, dt)
+
+
+@pytest.mark.parametrize("shape,block,code", [
+    (S(L=1000), 128, 2),           # L not a multiple of the block
+    (S(), 96, 2),                  # block not 64 / 128
+    (S(d=96), 128, 2),             # head dim
+    (S(Hq=6, Hkv=4), 128, 2),      # heads_q % heads_kv
+    (S(dt=7), 128, 3),             # dtype
+    (S(L=128 * 4096), 128, 4),     # nb > 2048
+    (S(B=0), 128, 2),
+])
+def test_shape_validation(lib, shape, block, code):
+    assert lib.sfa_block_scores_workspace(ctypes.byref(shape), block) == 0
+    off = (ctypes.c_size_t * 4)()
+    assert lib.sfa_workspace_layout(ctypes.byref(shape), block, off) == code
+    rope = sfa.Rope(None, None, 0)
+    dummy = ctypes.c_void_p(256)
+    assert lib.sfa_block_scores(ctypes.byref(shape), dummy, dummy, ctypes.byref(rope), 16, block, 0, None, None,
+                                dummy, dummy, 1 << 30, None) == code
+    assert lib.sfa_select(ctypes.byref(shape), block, dummy, 4, 0.0, 0, dummy, dummy, 64, None) == code
+    assert lib.sfa_block_sparse_attn(ctypes.byref(shape), block, dummy, dummy, dummy, dummy, dummy, 8, 1, 0.0,
+                                     dummy, None, None, None) == code
+
+
+def test_workspace_layout_matches_documented_sizes(lib):
+    shape = S(B=2, Hq=4, Hkv=2, L=2048, d=128)
+    nb = 16
+    off = sfa.workspace_layout(shape, 128)
+    assert off[0] == 0
+    assert off[1] >= 2 * 4 * nb * 128 * 4 and off[1] % 256 == 0
+    assert off[2] >= off[1] + 2 * 2 * nb * 128 * 4 and off[2] % 256 == 0
+    assert off[3] >= off[2] + 2 * 6 * nb * 4 * 4 and off[3] % 256 == 0
+    total = lib.sfa_block_scores_workspace(ctypes.byref(shape), 128)
+    assert total >= off[3] + 2 * 4 * 2 * 8
+
+
+def test_argument_validation_before_launch(lib):
+    shape = S()
+    d = ctypes.c_void_p(1 << 20)
+    rope = sfa.Rope(d, d, 1)
+    ws = lib.sfa_block_scores_workspace(ctypes.byref(shape), 128)
+    bs = lib.sfa_block_scores
+    # null Q / probs, band_split out of range, unknown flags, rope without rotated outputs
+    assert bs(ctypes.byref(shape), None, d, ctypes.byref(rope), 16, 128, 0, d, d, d, d, ws, None) == 1
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 0, d, d, None, d, ws, None) == 1
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 65, 128, 0, d, d, d, d, ws, None) == 1
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), -1, 128, 0, d, d, d, d, ws, None) == 1
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 8, d, d, d, d, ws, None) == 1
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 0, None, d, d, d, ws, None) == 1
+    # misaligned pointers
+    assert bs(ctypes.byref(shape), ctypes.c_void_p((1 << 20) + 2), d, ctypes.byref(rope), 16, 128, 0, d, d, d, d,
+              ws, None) == 1
+    # workspace too small / missing / misaligned
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 0, d, d, d, d, ws - 1, None) == 5
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 0, d, d, d, None, ws, None) == 5
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 0, d, d, d, ctypes.c_void_p((1 << 20) + 16),
+              ws, None) == 5
+    sel = lib.sfa_select
+    nb = 8
+    assert sel(ctypes.byref(shape), 128, d, -1, 0.0, 0, d, d, nb, None) == 1     # mass 0
+    assert sel(ctypes.byref(shape), 128, d, -1, 1.5, 0, d, d, nb, None) == 1     # mass > 1
+    assert sel(ctypes.byref(shape), 128, d, -1, 0.9, 0, d, d, nb - 1, None) == 1  # kmax < nb for mass
+    assert sel(ctypes.byref(shape), 128, d, 3, 0.0, 0, d, d, 3, None) == 1       # kmax < k + 1
+    assert sel(ctypes.byref(shape), 128, d, 3, 0.0, 1, d, d, 4, None) == 1       # kmax < k + 2 with sink
+    assert sel(ctypes.byref(shape), 128, None, 3, 0.0, 0, d, d, 4, None) == 1
+    assert sel(ctypes.byref(shape), 128, d, 3, 0.0, 16, d, d, 4, None) == 1      # unknown flag
+    at = lib.sfa_block_sparse_attn
+    assert at(ctypes.byref(shape), 128, d, d, d, d, d, 0, 1, 0.0, d, None, None, None) == 1  # kmax 0
+    assert at(ctypes.byref(shape), 128, d, None, d, d, d, 4, 1, 0.0, d, None, None, None) == 1
+    assert at(ctypes.byref(shape), 128, d, d, d, d, d, 4, 1, float("nan"), d, None, None, None) == 1
+    assert lib.sfa_rope_table(0.0, 16, 64, d, d, None) == 1
+    assert lib.sfa_rope_table(1e4, 16, 63, d, d, None) == 2
+    assert lib.sfa_rope_table(1e4, 0, 64, d, d, None) == 2
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(sfa, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(sfa, "_lib", None)
+    with pytest.raises(ImportError):
+        sfa.load()
