@@ -53,11 +53,11 @@ WsLayout ws_layout(const sfa_shape* s, int nb) {
   const size_t d = s->head_dim;
   size_t o = 0;
   w.off[0] = o;
-  o = align256(o + (size_t)s->batch * s->heads_q * nb * d * sizeof(float));
+  o = align256(o + (size_t)s->batch * s->heads_q * nb * d * sizeof(double));
   w.off[1] = o;
-  o = align256(o + (size_t)s->batch * s->heads_kv * nb * d * sizeof(float));
+  o = align256(o + (size_t)s->batch * s->heads_kv * nb * d * sizeof(double));
   w.off[2] = o;
-  o = align256(o + (size_t)s->batch * (s->heads_q + s->heads_kv) * nb * 4 * sizeof(float));
+  o = align256(o + (size_t)s->batch * (s->heads_q + s->heads_kv) * nb * 4 * sizeof(double));
   w.off[3] = o;
   o = align256(o + (size_t)s->batch * s->heads_q * 2 * sizeof(double));
   w.total = o;
@@ -188,9 +188,9 @@ sfa_status sfa_block_scores(const sfa_shape* shape, const void* Q, const void* K
   rp.cos = rope->cos; rp.sin = rope->sin;
   rp.apply = rope->apply ? 1 : 0;
   rp.write_rot = rope->apply ? 1 : 0;
-  rp.qbar = reinterpret_cast<float*>(ws + w.off[0]);
-  rp.kbar = reinterpret_cast<float*>(ws + w.off[1]);
-  rp.energy = reinterpret_cast<float*>(ws + w.off[2]);
+  rp.qbar = reinterpret_cast<double*>(ws + w.off[0]);
+  rp.kbar = reinterpret_cast<double*>(ws + w.off[1]);
+  rp.energy = reinterpret_cast<double*>(ws + w.off[2]);
   rp.B = shape->batch; rp.Hq = shape->heads_q; rp.Hkv = shape->heads_kv;
   rp.L = shape->seq_len; rp.block = block; rp.nb = nb; rp.band_pairs = band_pairs;
   st = cuda_status(launch_rope_pool_energy(rp, shape->dtype, D, cs));

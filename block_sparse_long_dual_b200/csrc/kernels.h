@@ -17,23 +17,23 @@ struct RopePoolParams {
   const float* sin;
   int apply;      // rotate (else Q, K are already rotated)
   int write_rot;  // write the rotated copies
-  float* qbar;
-  float* kbar;
-  float* energy;
+  double* qbar;
+  double* kbar;
+  double* energy;
   int B, Hq, Hkv, L, block, nb;
   int band_pairs;  // rotary pairs in band H (d/2 with a single band)
 };
 
 struct TauParams {
-  const float* energy;
+  const double* energy;
   double* tau;
   int B, Hq, Hkv, L, nb;
   unsigned flags;
 };
 
 struct ScoreParams {
-  const float* qbar;
-  const float* kbar;
+  const double* qbar;
+  const double* kbar;
   const double* tau;
   float* probs;
   int B, Hq, Hkv, nb;

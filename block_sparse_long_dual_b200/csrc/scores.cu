@@ -7,8 +7,8 @@
 //                     mean vectors and per-band energies (one CTA per block
 //                     and head).
 //   band_temperature  per (batch, Q head): reduce the energies to tau^H, tau^L.
-//   block_score_softmax  calibrated block logits (float32 products, float64
-//                     partial sums) and the causal row softmax in float64.
+//   block_score_softmax  calibrated block logits and the causal row softmax,
+//                     both in float64.
 #include <math.h>
 
 #include "common.cuh"
@@ -51,7 +51,7 @@ __global__ void __launch_bounds__(256) rope_pool_energy_kernel(RopePoolParams p)
   float slo[8], shi[8];
 #pragma unroll
   for (int e = 0; e < 8; ++e) slo[e] = shi[e] = 0.f;
-  float eh = 0.f, el = 0.f;
+  double eh = 0.0, el = 0.0;
 
   const int passes = p.block / TPP;
   for (int ps = 0; ps < passes; ++ps) {
@@ -75,13 +75,16 @@ __global__ void __launch_bounds__(256) rope_pool_energy_kernel(RopePoolParams p)
         store8(xr + (size_t)t * D + D / 2 + c * 8, hi);
       }
     }
+    float ph = 0.f, pl = 0.f;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       slo[e] += lo[e];
       shi[e] += hi[e];
       const float en = fmaf(lo[e], lo[e], hi[e] * hi[e]);
-      if (c * 8 + e < p.band_pairs) eh += en; else el += en;
+      if (c * 8 + e < p.band_pairs) ph += en; else pl += en;
     }
+    eh += ph;
+    el += pl;
   }
 
   // Cross-thread reduction in float64: lanes with equal c hold the same dims.
@@ -119,9 +122,9 @@ __global__ void __launch_bounds__(256) rope_pool_energy_kernel(RopePoolParams p)
 #pragma unroll
     for (int w = 0; w < NW; ++w) s += red[w][tid];
     const double mean = s / (double)p.block;
-    float* out = (is_q ? p.qbar + ((size_t)(b * p.Hq + hh) * p.nb + j) * D
-                       : p.kbar + ((size_t)(b * p.Hkv + hh) * p.nb + j) * D);
-    out[tid] = (float)mean;
+    double* out = (is_q ? p.qbar + ((size_t)(b * p.Hq + hh) * p.nb + j) * D
+                        : p.kbar + ((size_t)(b * p.Hkv + hh) * p.nb + j) * D);
+    out[tid] = mean;
     const int m = tid % (D / 2);
     if (m < p.band_pairs) ph = mean * mean; else pl = mean * mean;
   }
@@ -137,7 +140,7 @@ __global__ void __launch_bounds__(256) rope_pool_energy_kernel(RopePoolParams p)
     double s = 0.0;
 #pragma unroll
     for (int w = 0; w < NW; ++w) s += ered[w][tid];
-    p.energy[((size_t)(b * heads + head) * p.nb + j) * 4 + tid] = (float)s;
+    p.energy[((size_t)(b * heads + head) * p.nb + j) * 4 + tid] = s;
   }
 }
 
@@ -150,16 +153,17 @@ __global__ void __launch_bounds__(256) band_temperature_kernel(TauParams p) {
   const int b = blockIdx.x / p.Hq;
   const int g = h / (p.Hq / p.Hkv);
   const int heads = p.Hq + p.Hkv;
-  const float* eq = p.energy + (size_t)(b * heads + h) * p.nb * 4;
-  const float* ek = p.energy + (size_t)(b * heads + p.Hq + g) * p.nb * 4;
+  const double* eq = p.energy + (size_t)(b * heads + h) * p.nb * 4;
+  const double* ek = p.energy + (size_t)(b * heads + p.Hq + g) * p.nb * 4;
   double acc[8];
 #pragma unroll
   for (int q = 0; q < 8; ++q) acc[q] = 0.0;
   for (int j = threadIdx.x; j < p.nb; j += blockDim.x) {
-    const float4 a = *reinterpret_cast<const float4*>(eq + (size_t)j * 4);
-    const float4 k = *reinterpret_cast<const float4*>(ek + (size_t)j * 4);
-    acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
-    acc[4] += k.x; acc[5] += k.y; acc[6] += k.z; acc[7] += k.w;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      acc[q] += eq[(size_t)j * 4 + q];
+      acc[4 + q] += ek[(size_t)j * 4 + q];
+    }
   }
   __shared__ double red[8][8];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -192,20 +196,24 @@ __global__ void __launch_bounds__(256) band_temperature_kernel(TauParams p) {
 // ---------------------------------------------------------------------------
 // block_score_softmax
 // CTA = RT query-block rows of one (b, h).  The calibrated logits of the rows
-// are kept as a float64 strip [RT][nb] in shared memory; column steps of CS
-// keys, head dim in chunks of DC.  Thread tile 4 rows x 4 columns: float32
-// products summed over 16 dims, then added into float64 accumulators.
+// are kept as a float64 strip [RT][nb] in shared memory.  Column steps of CS
+// keys; head dim in chunks of DC staged transposed in shared memory (float64).
+// Thread tile: 8 rows x 4 columns of float64 FMAs (the query operands are
+// warp-uniform broadcasts, so shared-memory traffic is 1 byte per FMA).
+// Everything is float64 because the calibration 1/tau amplifies the pooled
+// logits: float32 sums of logits of magnitude ~20 already err by ~1e-6.
 // ---------------------------------------------------------------------------
 template <int RT, int D>
 __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p) {
-  constexpr int RG = RT / 4;      // row groups
+  constexpr int TR = 8, TC = 4;
+  constexpr int RG = RT / TR;     // row groups
   constexpr int CG = 256 / RG;    // column groups
-  constexpr int CS = CG * 4;      // columns per step
-  constexpr int DC = 32;          // head-dim chunk
+  constexpr int CS = CG * TC;     // columns per step
+  constexpr int DC = RT == 16 ? 16 : 8;  // head-dim chunk
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  double* strip = reinterpret_cast<double*>(smem_raw);              // [RT][nb]
-  float* qT = reinterpret_cast<float*>(strip + (size_t)RT * p.nb);    // [D][RT]
-  float* kT = qT + D * RT;                                            // [DC][CS]
+  double* strip = reinterpret_cast<double*>(smem_raw);                 // [RT][nb]
+  double* qT = strip + (size_t)RT * p.nb;                               // [D][RT]
+  double* kT = qT + D * RT;                                             // [DC][CS]
 
   const int ntiles = (p.nb + RT - 1) / RT;
   const int tile = ntiles - 1 - (int)blockIdx.x;  // heaviest rows first
@@ -219,73 +227,61 @@ __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p)
 
   // Calibrated, pre-scaled query block means: q~ = qbar / (tau^band * sqrt(d)).
   const double* tau = p.tau + (size_t)(b * p.Hq + h) * 2;
-  const float inv_h = (float)(1.0 / (tau[0] * sqrt((double)D)));
-  const float inv_l = (float)(1.0 / (tau[1] * sqrt((double)D)));
-  const float* qsrc = p.qbar + ((size_t)(b * p.Hq + h) * p.nb + i0) * D;
+  const double inv_h = 1.0 / (tau[0] * sqrt((double)D));
+  const double inv_l = 1.0 / (tau[1] * sqrt((double)D));
+  const double* qsrc = p.qbar + ((size_t)(b * p.Hq + h) * p.nb + i0) * D;
   for (int e = tid; e < D * RT; e += 256) {
     const int r = e / D, d = e % D;
-    const float s = ((d % (D / 2)) < p.band_pairs) ? inv_h : inv_l;
-    qT[d * RT + r] = (r < rows) ? qsrc[(size_t)r * D + d] * s : 0.f;
+    const double s = ((d % (D / 2)) < p.band_pairs) ? inv_h : inv_l;
+    qT[d * RT + r] = (r < rows) ? qsrc[(size_t)r * D + d] * s : 0.0;
   }
-  const float* ksrc = p.kbar + (size_t)(b * p.Hkv + g) * p.nb * D;
+  const double* ksrc = p.kbar + (size_t)(b * p.Hkv + g) * p.nb * D;
 
   for (int col0 = 0; col0 < jend; col0 += CS) {
-    double acc[4][4];
+    double acc[TR][TC];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int r = 0; r < TR; ++r)
 #pragma unroll
-      for (int q = 0; q < 4; ++q) acc[r][q] = 0.0;
+      for (int q = 0; q < TC; ++q) acc[r][q] = 0.0;
     for (int dc = 0; dc < D; dc += DC) {
       __syncthreads();
       // kT[dd][c] = kbar[col0 + c][dc + dd]
       for (int c = tid; c < CS; c += 256) {
         const int col = col0 + c;
-        if (col < jend) {
-          const float4* src = reinterpret_cast<const float4*>(ksrc + (size_t)col * D + dc);
+        const double2* src = reinterpret_cast<const double2*>(ksrc + (size_t)col * D + dc);
 #pragma unroll
-          for (int v = 0; v < DC / 4; ++v) {
-            const float4 f = __ldg(src + v);
-            kT[(v * 4 + 0) * CS + c] = f.x;
-            kT[(v * 4 + 1) * CS + c] = f.y;
-            kT[(v * 4 + 2) * CS + c] = f.z;
-            kT[(v * 4 + 3) * CS + c] = f.w;
-          }
-        } else {
-#pragma unroll
-          for (int dd = 0; dd < DC; ++dd) kT[dd * CS + c] = 0.f;
+        for (int v = 0; v < DC / 2; ++v) {
+          const double2 f = col < jend ? __ldg(src + v) : make_double2(0.0, 0.0);
+          kT[(v * 2 + 0) * CS + c] = f.x;
+          kT[(v * 2 + 1) * CS + c] = f.y;
         }
       }
       __syncthreads();
 #pragma unroll
-      for (int half = 0; half < DC; half += 16) {
-        float a32[4][4];
+      for (int dd = 0; dd < DC; ++dd) {
+        double qv[TR], kv[TC];
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) a32[r][q] = 0.f;
-#pragma unroll
-        for (int dd = 0; dd < 16; ++dd) {
-          const float4 qa = *reinterpret_cast<const float4*>(qT + (dc + half + dd) * RT + rg * 4);
-          const float4 kb = *reinterpret_cast<const float4*>(kT + (half + dd) * CS + cg * 4);
-          const float qv[4] = {qa.x, qa.y, qa.z, qa.w};
-          const float kv[4] = {kb.x, kb.y, kb.z, kb.w};
-#pragma unroll
-          for (int r = 0; r < 4; ++r)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) a32[r][q] = fmaf(qv[r], kv[q], a32[r][q]);
+        for (int r = 0; r < TR; r += 2) {
+          const double2 t = *reinterpret_cast<const double2*>(qT + (dc + dd) * RT + rg * TR + r);
+          qv[r] = t.x; qv[r + 1] = t.y;
         }
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+        for (int q = 0; q < TC; q += 2) {
+          const double2 t = *reinterpret_cast<const double2*>(kT + dd * CS + cg * TC + q);
+          kv[q] = t.x; kv[q + 1] = t.y;
+        }
 #pragma unroll
-          for (int q = 0; q < 4; ++q) acc[r][q] += (double)a32[r][q];
+        for (int r = 0; r < TR; ++r)
+#pragma unroll
+          for (int q = 0; q < TC; ++q) acc[r][q] = fma(qv[r], kv[q], acc[r][q]);
       }
     }
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      const int rr = rg * 4 + r;
+    for (int r = 0; r < TR; ++r) {
+      const int rr = rg * TR + r;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int col = col0 + cg * 4 + q;
+      for (int q = 0; q < TC; ++q) {
+        const int col = col0 + cg * TC + q;
         if (col < jend) strip[(size_t)rr * p.nb + col] = acc[r][q];
       }
     }
@@ -340,9 +336,9 @@ int score_rows_per_cta(int nb) { return nb <= 1024 ? 16 : 8; }
 
 size_t score_smem_bytes(int nb, int D) {
   const int RT = score_rows_per_cta(nb);
-  const int CS = (256 / (RT / 4)) * 4;
-  return (size_t)RT * nb * sizeof(double) + (size_t)D * RT * sizeof(float) +
-         (size_t)32 * CS * sizeof(float);
+  const int CS = (256 / (RT / 8)) * 4;
+  const int DC = RT == 16 ? 16 : 8;
+  return ((size_t)RT * nb + (size_t)D * RT + (size_t)DC * CS) * sizeof(double);
 }
 
 template <int RT, int D>

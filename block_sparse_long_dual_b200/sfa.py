@@ -145,9 +145,9 @@ def workspace_views(ws: torch.Tensor, shape: Shape, block: int):
         nbytes = n * torch.tensor([], dtype=dt).element_size()
         return ws[off[i]:off[i] + nbytes].view(dt).view(*shp)
 
-    return (view(0, B * Hq * nb * d, torch.float32, (B, Hq, nb, d)),
-            view(1, B * Hkv * nb * d, torch.float32, (B, Hkv, nb, d)),
-            view(2, B * (Hq + Hkv) * nb * 4, torch.float32, (B, Hq + Hkv, nb, 4)),
+    return (view(0, B * Hq * nb * d, torch.float64, (B, Hq, nb, d)),
+            view(1, B * Hkv * nb * d, torch.float64, (B, Hkv, nb, d)),
+            view(2, B * (Hq + Hkv) * nb * 4, torch.float64, (B, Hq + Hkv, nb, 4)),
             view(3, B * Hq * 2, torch.float64, (B, Hq, 2)))
 
 

@@ -93,9 +93,9 @@ sfa_status sfa_rope_table(double base, int seq_len, int head_dim, float* cos, fl
  * Bytes of workspace sfa_block_scores needs for this shape and block size
  * (0 if the shape is invalid).  The workspace holds, each at a 256-byte
  * aligned offset given by sfa_workspace_layout:
- *   [0] Qbar   [B, heads_q,  nb, d] float32  block means of rotated Q
- *   [1] Kbar   [B, heads_kv, nb, d] float32  block means of rotated K
- *   [2] energy [B, heads_q + heads_kv, nb, 4] float32 per block:
+ *   [0] Qbar   [B, heads_q,  nb, d] float64  block means of rotated Q
+ *   [1] Kbar   [B, heads_kv, nb, d] float64  block means of rotated K
+ *   [2] energy [B, heads_q + heads_kv, nb, 4] float64 per block:
  *              sum_t ||x_t^H||^2, sum_t ||x_t^L||^2, ||xbar^H||^2, ||xbar^L||^2
  *              (Q heads first, then KV heads)
  *   [3] tau    [B, heads_q, 2] float64  (band H, band L)
@@ -115,14 +115,15 @@ sfa_status sfa_workspace_layout(const sfa_shape* shape, int block, size_t offset
  *
  * Per (batch, Q head, band b in {H, L}), with band H = rotary pairs
  * m < band_split (dims m and m + d/2), band L = the other dims:
- *   xbar_j  = mean of the rotated vectors of block j (float32)
+ *   xbar_j  = mean of the rotated vectors of block j
  *   rho^b   = sqrt(mean_j ||xbar_j^b||^2 / mean_t ||x_t^b||^2)   (1 if the band is empty)
  *   tau^b   = max(rho^b(Q_h) * rho^b(K_g), 1e-6)   (1 with SFA_NO_CALIB)
  *   s_ij    = sum_b (qbar_i^b . kbar_j^b) / (tau^b * sqrt(d)),  j <= i
  *   probs_ij = exp(s_ij) / sum_{j' <= i} exp(s_ij'), and 0 for j > i.
  * probs [B, heads_q, nb, nb] float32.  SFA_SINGLE_BAND puts all dims in band H.
- * The logits are accumulated with float64 partial sums and the softmax is
- * evaluated in float64, then rounded once to float32.
+ * RoPE is applied in float32; block means, energies, temperatures, logits and
+ * the softmax are float64 (the 1/tau calibration amplifies pooled logits, so
+ * float32 sums would move probabilities by ~1e-6), rounded once to float32.
  *
  * workspace: device buffer of at least sfa_block_scores_workspace() bytes,
  * 256-byte aligned; its contents are documented above and may be read back.

@@ -80,9 +80,9 @@ def test_workspace_layout_matches_documented_sizes(lib):
     nb = 16
     off = sfa.workspace_layout(shape, 128)
     assert off[0] == 0
-    assert off[1] >= 2 * 4 * nb * 128 * 4 and off[1] % 256 == 0
-    assert off[2] >= off[1] + 2 * 2 * nb * 128 * 4 and off[2] % 256 == 0
-    assert off[3] >= off[2] + 2 * 6 * nb * 4 * 4 and off[3] % 256 == 0
+    assert off[1] >= 2 * 4 * nb * 128 * 8 and off[1] % 256 == 0
+    assert off[2] >= off[1] + 2 * 2 * nb * 128 * 8 and off[2] % 256 == 0
+    assert off[3] >= off[2] + 2 * 6 * nb * 4 * 8 and off[3] % 256 == 0
     total = lib.sfa_block_scores_workspace(ctypes.byref(shape), 128)
     assert total >= off[3] + 2 * 4 * 2 * 8
 

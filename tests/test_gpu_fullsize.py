@@ -60,7 +60,8 @@ def test_full_size_sampled(w):
         sc = po.prism_scores(Qh, Kh, w.block, w.band_split, w.flags, (cos, sin))
         P = model.probs[b, h].cpu().numpy()
         err = rel_err(np.tril(P).reshape(-1), np.tril(sc.probs[0, 0]).reshape(-1), floor=1e-35)
-        assert err < 2e-6, f"block probabilities: max relative error {err:.3e}"
+        print(f"{w.name} b={b} h={h}: max relative error of block probabilities {err:.3e}")
+        assert err < 1e-6, f"block probabilities: max relative error {err:.3e}"
         sel = po.select_blocks(sc.probs, w.flags, k=w.k, mass=mass)
         stats, exact = compare_masks(sel, sc.probs, model.counts[b:b + 1, h:h + 1], model.idx[b:b + 1, h:h + 1],
                                      mass)

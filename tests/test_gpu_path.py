@@ -70,27 +70,29 @@ def test_path_matches_oracle(w):
     for got, want in ((model.Q_rot, ref.q_attn), (model.K_rot, ref.k_attn)):
         g = to_np(got).astype(np.float64)
         if w.dtype == "bf16":
-            ulp = np.abs(want) * 2.0 ** -7 + 1e-30
+            # one bf16 ulp of the value, plus the float32 rounding of x*c - y*s when it cancels
+            ulp = np.abs(want) * 2.0 ** -7 * 1.01 + 2e-6
             diff = np.abs(g - want)
-            assert np.all(diff <= ulp * 1.01), "rotated values differ by more than one bf16 ulp"
+            assert np.all(diff <= ulp), "rotated values differ by more than one bf16 ulp"
             assert np.mean(diff > 0) < 1e-3
         else:
             np.testing.assert_allclose(g, want, rtol=0, atol=2e-6)
 
     # a2/a3: block means, energies, temperatures (diagnostic tolerances at float32 rounding)
     qbar, kbar, energy, tau = sfa.workspace_views(model.workspace, model.shape, w.block)
-    np.testing.assert_allclose(to_np(qbar), sc.qbar, rtol=0, atol=3e-7)
-    np.testing.assert_allclose(to_np(kbar), sc.kbar, rtol=0, atol=3e-7)
+    np.testing.assert_allclose(to_np(qbar), sc.qbar, rtol=0, atol=1e-7)
+    np.testing.assert_allclose(to_np(kbar), sc.kbar, rtol=0, atol=1e-7)
     e = to_np(energy)
-    np.testing.assert_allclose(e[:, :w.heads_q, :, :2], sc.tok_energy_q, rtol=2e-6, atol=1e-6)
-    np.testing.assert_allclose(e[:, w.heads_q:, :, :2], sc.tok_energy_k, rtol=2e-6, atol=1e-6)
-    np.testing.assert_allclose(to_np(tau), sc.tau, rtol=2e-6, atol=0)
+    np.testing.assert_allclose(e[:, :w.heads_q, :, :2], sc.tok_energy_q, rtol=1e-6, atol=1e-9)
+    np.testing.assert_allclose(e[:, w.heads_q:, :, :2], sc.tok_energy_k, rtol=1e-6, atol=1e-9)
+    np.testing.assert_allclose(to_np(tau), sc.tau, rtol=1e-7, atol=0)
 
     # a4: probabilities (relative error of the float32 output vs float64)
     P = to_np(model.probs)
     assert np.all(np.triu(P, 1) == 0)
     err = rel_err(np.tril(P).reshape(-1), np.tril(sc.probs).reshape(-1), floor=1e-35)
-    assert err < 2e-6, f"max relative error of block probabilities {err:.3e}"
+    print(f"{w.name}: max relative error of block probabilities {err:.3e}")
+    assert err < 1e-6, f"max relative error of block probabilities {err:.3e}"
 
     # a5: masks identical except near-ties at the row threshold
     stats, exact = compare_masks(ref.selection, sc.probs, model.counts, model.idx, mass)
