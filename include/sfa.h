@@ -137,6 +137,42 @@ sfa_status sfa_block_scores(const sfa_shape* shape, const void* Q, const void* K
                             size_t workspace_bytes, void* stream);
 
 /*
+ * sfa_block_scores_noalloc - the same computation and outputs as
+ * sfa_block_scores, for callers that cannot allocate device memory.
+ * (The paper has no counterpart: this is a deployment convenience.)
+ *
+ * Some callers cannot call cudaMalloc or hand out scratch buffers at call
+ * time: plugin or callback code run by a host runtime that owns all device
+ * memory and passes in only the input and output buffers, processes whose
+ * device memory is already reserved by another framework's allocator, and
+ * latency-bound loops that must not risk the implicit device synchronisation
+ * an allocation can cause.  This entry point takes the same arguments minus
+ * the workspace; it uses a fixed scratch array of SFA_NOALLOC_SCRATCH_BYTES
+ * (16 MiB) that the library declares in device memory, so every GPU that
+ * loads the library holds those 16 MiB until the process exits.  It calls no
+ * cudaMalloc, cudaFree or allocating library routine.
+ *
+ * Limit: shapes whose sfa_block_scores_workspace() exceeds
+ * SFA_NOALLOC_SCRATCH_BYTES are rejected with SFA_ERR_WORKSPACE (e.g. the
+ * 32 query / 8 KV head, d = 128, block = 128 layer fits up to L = 32768 per
+ * batch element).  The caller still passes Q, K, Q_rot, K_rot and probs.
+ *
+ * The first call on a device looks up the scratch array's device address
+ * (cudaGetSymbolAddress, with that device current) and caches it; make that
+ * first call before any stream capture.  All calls on a device share the one
+ * scratch array and it keeps the last call's contents: calls whose kernels
+ * overlap on the GPU (different streams, no ordering between them) race on it
+ * and give wrong results.  Serialise such calls, e.g. issue them on one stream.
+ * Every scratch region is fully rewritten by each call, so nothing needs
+ * clearing between calls.  Errors: as sfa_block_scores, plus SFA_ERR_WORKSPACE
+ * for shapes over the limit and SFA_ERR_UNSUPPORTED for device ordinals >= 64.
+ */
+#define SFA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+sfa_status sfa_block_scores_noalloc(const sfa_shape* shape, const void* Q, const void* K,
+                                    const sfa_rope* rope, int band_split, int block, unsigned flags,
+                                    void* Q_rot, void* K_rot, float* probs, void* stream);
+
+/*
  * Block selection (Prism §1: attention runs over a chosen subset of key blocks).
  * For every row (b, h, i) of probs [B, heads_q, nb, nb]:
  *   forced F_i = {i}, plus {0} with SFA_KEEP_SINK;
