@@ -2,19 +2,30 @@
 // Block-Sparse Attention" §1) on the sm_100a tensor cores.
 //
 // bf16 Q/K/V, query block = key block = 128 tokens, head dim 128.
-// One CTA per (b, h, query block i); 6 warps:
-//   warps 0-3  softmax: thread r owns query row r (TMEM lane r); reads S from
-//              TMEM, online softmax in registers (lazy rescale of O), writes P
-//              (bf16) into shared memory in the 128-byte-swizzled K-major
-//              layout, final O / l epilogue.
-//   warp 4     producer: TMA loads of the Q tile and of the K_j / V_j tiles of
-//              every kept block j, fetched through the index list (two stages).
-//   warp 5     MMA issuer: S = Q K_j^T (tcgen05.mma kind::f16, M=N=128,
-//              K=16 steps) into a double-buffered TMEM S, then O += P V_j into
-//              TMEM O; completion tracked with tcgen05.commit -> mbarriers.
+// One CTA holds TWO query tiles (t = 0, 1): two consecutive entries of the tile
+// order (b, kv head, query block descending, q head in the group), i.e. two Q
+// heads of one GQA group at the same query block.  Each tile walks its own
+// index list; the two tiles ping-pong on the tensor core: while one softmax
+// warpgroup turns S_t into P_t, the tensor core runs the other tile's P.V and
+// next Q.K^T.
+//
+//   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread r owns query row r
+//                    (TMEM lane r); reads S_t from TMEM, online softmax with a
+//                    lazily rescaled O_t, writes P_t (bf16) back into the S_t
+//                    columns of TMEM, final O_t / l epilogue.
+//   warp 8           producer: TMA loads of Q_t and of K_t(j), V_t(j) for every
+//                    kept block j of each tile (one K and one V slot per tile).
+//   warp 9           MMA issuer: S_t = Q_t K_t^T (A, B from shared memory) and
+//                    O_t += P_t V_t (A = P_t from TMEM, B = V_t from shared
+//                    memory), M = N = 128, K = 16 steps; completion tracked with
+//                    tcgen05.commit -> mbarriers.  A commit covers every MMA the
+//                    thread issued before it, so the commit that signals S_t(j)
+//                    also means O_t has absorbed P_t(j-1).
+// TMEM (512 columns): S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512);
+// P_t aliases the first 64 columns of S_t (two bf16 per column).
 // Every mbarrier wait is bounded (about 2 s); a wait that runs out writes
-// SFA_ERR_TIMEOUT to the status word, raises a CTA-wide abort flag, drains
-// the copies / MMAs this CTA issued and frees its tensor memory.
+// SFA_ERR_TIMEOUT to the status word, raises a CTA-wide abort flag, drains the
+// copies / MMAs this CTA issued and frees its tensor memory.
 #include <math.h>
 
 #include "common.cuh"
@@ -28,20 +39,25 @@ namespace {
 constexpr int kHD = 128;
 constexpr uint32_t kSub = 16384;       // 128 rows x 64 bf16 (one 128B-swizzle box)
 constexpr uint32_t kTile = 2 * kSub;   // 128 x 128 bf16
-constexpr int kStages = 2;
-constexpr uint32_t OFF_Q = 0;
-constexpr uint32_t OFF_K = OFF_Q + kTile;
-constexpr uint32_t OFF_V = OFF_K + kStages * kTile;
-constexpr uint32_t OFF_P = OFF_V + kStages * kTile;
-constexpr uint32_t OFF_BAR = OFF_P + kTile;
-enum { B_Q = 0, B_KF = 1, B_VF = 3, B_KVE = 5, B_SF = 7, B_SFREE = 9, B_PF = 11, B_OD = 12, B_DRAIN = 13, NBAR = 14 };
+// Shared memory: per tile t a Q, a K and a V tile (6 x 32 KB).
+__host__ __device__ constexpr uint32_t off_q(int t) { return t * kTile; }
+__host__ __device__ constexpr uint32_t off_k(int t) { return 2 * kTile + t * kTile; }
+__host__ __device__ constexpr uint32_t off_v(int t) { return 4 * kTile + t * kTile; }
+constexpr uint32_t OFF_BAR = 6 * kTile;
+// Barriers, two of each (one per tile) except DRAIN.
+enum { B_Q = 0, B_KF = 2, B_VF = 4, B_KE = 6, B_VE = 8, B_SF = 10, B_PF = 12, B_OD = 14, B_DRAIN = 16, NBAR = 17 };
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr uint32_t SMEM_BYTES = OFF_MISC + 16 + 1024;
-constexpr int kThreads = 192;
+constexpr int kMaxList = 2048;                       // nb <= 2048, so a valid list has <= 2048 entries
+constexpr uint32_t OFF_LIST = OFF_MISC + 32;         // per tile: the validated index list
+constexpr uint32_t SMEM_BYTES = OFF_LIST + 2 * kMaxList * 4 + 1024;
+constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8, kMmaWarp = 9;
 constexpr uint32_t TMEM_COLS = 512;
-constexpr uint32_t COL_O = 256;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
+
+__host__ __device__ constexpr uint32_t col_s(int t) { return t * 128; }
+__host__ __device__ constexpr uint32_t col_o(int t) { return 256 + t * 128; }
 
 struct Ctx {
   uint32_t sbase;
@@ -75,6 +91,30 @@ __device__ void drain_wait(uint32_t bar, uint32_t parity) {
   }
 }
 
+struct Tile {
+  int b, h, g, i, n;
+  const int* list;
+  bool valid;
+};
+
+__device__ Tile decode_tile(const AttnParams& p, int t) {
+  Tile x;
+  const int group = p.Hq / p.Hkv;
+  const int total = p.B * p.Hq * p.nb;
+  x.valid = t < total;
+  if (!x.valid) t = total - 1;
+  const int hh = t % group;
+  t /= group;
+  x.i = p.nb - 1 - (t % p.nb);
+  t /= p.nb;
+  x.g = t % p.Hkv;
+  x.b = t / p.Hkv;
+  x.h = x.g * group + hh;
+  x.list = p.idx + ((size_t)(x.b * p.Hq + x.h) * p.nb + x.i) * p.kmax;
+  x.n = 0;
+  return x;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -88,55 +128,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   cx.sbase = raw + pad;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
   cx.abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
-  int* bad_flag = reinterpret_cast<int*>(sm + OFF_MISC + 8);
+  int* nsh = reinterpret_cast<int*>(sm + OFF_MISC + 8);  // validated count per tile
+  int* slist = reinterpret_cast<int*>(sm + OFF_LIST);    // [2][kMaxList] validated index lists
   cx.status = p.status;
-
-  const int group = p.Hq / p.Hkv;
-  int t = blockIdx.x;
-  const int hh = t % group;
-  t /= group;
-  const int i = p.nb - 1 - (t % p.nb);
-  t /= p.nb;
-  const int g = t % p.Hkv;
-  const int b = t / p.Hkv;
-  const int h = g * group + hh;
-  const size_t rowid = (size_t)(b * p.Hq + h) * p.nb + i;
-  const int* list = p.idx + rowid * p.kmax;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  if (warp == 0) {
-    // Validate the index list: count in [0, kmax], entries ascending in [0, nb), <= i if causal.
-    const int n = p.counts[rowid];
-    bool ok = n >= 0 && n <= p.kmax;
-    if (ok) {
-      for (int u = lane; u < n; u += 32) {
-        const int j = list[u];
-        if (j < 0 || j >= p.nb || (p.causal && j > i) || (u > 0 && list[u - 1] >= j)) ok = false;
+  Tile tl[2] = {decode_tile(p, 2 * blockIdx.x), decode_tile(p, 2 * blockIdx.x + 1)};
+
+  if (warp == 0 || warp == 4) {
+    // Validate one tile's index list: count in [0, kmax], entries ascending in [0, nb), <= i if causal.
+    const int t = warp >> 2;
+    const Tile x = t == 0 ? tl[0] : tl[1];
+    int n = 0;
+    if (x.valid) {
+      const size_t rowid = (size_t)(x.b * p.Hq + x.h) * p.nb + x.i;
+      n = p.counts[rowid];
+      bool ok = n >= 0 && n <= p.kmax;
+      if (ok) {
+        for (int u = lane; u < n; u += 32) {
+          const int j = x.list[u];
+          if (j < 0 || j >= p.nb || (p.causal && j > x.i) || (u > 0 && x.list[u - 1] >= j)) ok = false;
+          if (u < kMaxList) slist[t * kMaxList + u] = j;
+        }
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      if (!ok) {
+        if (lane == 0) report(p.status, SFA_ERR_INDEX);
+        n = 0;
       }
     }
-    ok = __all_sync(0xffffffffu, ok);
-    if (lane == 0) {
-      *bad_flag = ok ? 0 : 1;
-      if (!ok) report(p.status, SFA_ERR_INDEX);
+    if (lane == 0) nsh[t] = n;
+    if (warp == 0 && lane == 0) {
       *cx.abort_flag = 0;
-      tc::mbar_init(cx.bar(B_Q), 1);
-      for (int s = 0; s < kStages; ++s) {
-        tc::mbar_init(cx.bar(B_KF + s), 1);
-        tc::mbar_init(cx.bar(B_VF + s), 1);
-        tc::mbar_init(cx.bar(B_KVE + s), 1);
-        tc::mbar_init(cx.bar(B_SF + s), 1);
-        tc::mbar_init(cx.bar(B_SFREE + s), 128);
-      }
-      tc::mbar_init(cx.bar(B_PF), 128);
-      tc::mbar_init(cx.bar(B_OD), 1);
-      tc::mbar_init(cx.bar(B_DRAIN), 1);
+      for (int k = 0; k < NBAR; ++k) tc::mbar_init(cx.bar(k), (k == B_PF || k == B_PF + 1) ? 128 : 1);
       tc::fence_mbar_init();
     }
-  } else if (warp == 4 && lane == 0) {
+  } else if (warp == kProducerWarp && lane == 0) {
     tc::prefetch_tmap(&tmQ);
     tc::prefetch_tmap(&tmK);
     tc::prefetch_tmap(&tmV);
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
     tc::tmem_relinquish();
   }
@@ -144,79 +175,115 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const int n = *bad_flag ? 0 : p.counts[rowid];
-  const uint32_t sQ = cx.sbase + OFF_Q, sP = cx.sbase + OFF_P;
+  tl[0].n = nsh[0];
+  tl[1].n = nsh[1];
+  const int nmax = max(tl[0].n, tl[1].n);
 
-  if (n > 0 && warp == 4) {
+  if (warp == kProducerWarp) {
     // ------------------------------ producer ------------------------------
-    if (lane == 0) {
-      const int qrow = (b * p.Hq + h) * p.L + i * 128;
-      const int kvrow0 = (b * p.Hkv + g) * p.L;
-      tc::mbar_arrive_expect_tx(cx.bar(B_Q), kTile);
-      tc::tma_load_2d(sQ, &tmQ, cx.bar(B_Q), 0, qrow);
-      tc::tma_load_2d(sQ + kSub, &tmQ, cx.bar(B_Q), 64, qrow);
-      int issued[kStages] = {0, 0};
-      for (int it = 0; it < n; ++it) {
-        const int st = it & 1, use = it >> 1;
-        if (!wait_bar(cx, cx.bar(B_KVE + st), (use & 1) ^ 1)) break;
-        const int row = kvrow0 + list[it] * 128;
-        const uint32_t sK = cx.sbase + OFF_K + st * kTile, sV = cx.sbase + OFF_V + st * kTile;
-        tc::mbar_arrive_expect_tx(cx.bar(B_KF + st), kTile);
-        tc::tma_load_2d(sK, &tmK, cx.bar(B_KF + st), 0, row);
-        tc::tma_load_2d(sK + kSub, &tmK, cx.bar(B_KF + st), 64, row);
-        tc::mbar_arrive_expect_tx(cx.bar(B_VF + st), kTile);
-        tc::tma_load_2d(sV, &tmV, cx.bar(B_VF + st), 0, row);
-        tc::tma_load_2d(sV + kSub, &tmV, cx.bar(B_VF + st), 64, row);
-        issued[st] = use + 1;
+    if (lane == 0 && nmax > 0) {
+      int kissued[2] = {0, 0}, vissued[2] = {0, 0};
+      bool qissued[2] = {false, false};
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (tl[t].n == 0) continue;
+        const int qrow = (tl[t].b * p.Hq + tl[t].h) * p.L + tl[t].i * 128;
+        const uint32_t sQ = cx.sbase + off_q(t);
+        tc::mbar_arrive_expect_tx(cx.bar(B_Q + t), kTile);
+        tc::tma_load_2d(sQ, &tmQ, cx.bar(B_Q + t), 0, qrow);
+        tc::tma_load_2d(sQ + kSub, &tmQ, cx.bar(B_Q + t), 64, qrow);
+        qissued[t] = true;
+      }
+      bool ok = true;
+      for (int it = 0; ok && it < nmax; ++it) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || it >= tl[t].n) continue;
+          if (it > 0 && !wait_bar(cx, cx.bar(B_KE + t), (it - 1) & 1)) { ok = false; break; }
+          const int row = (tl[t].b * p.Hkv + tl[t].g) * p.L + slist[t * kMaxList + it] * 128;
+          const uint32_t sK = cx.sbase + off_k(t);
+          tc::mbar_arrive_expect_tx(cx.bar(B_KF + t), kTile);
+          tc::tma_load_2d(sK, &tmK, cx.bar(B_KF + t), 0, row);
+          tc::tma_load_2d(sK + kSub, &tmK, cx.bar(B_KF + t), 64, row);
+          kissued[t] = it + 1;
+        }
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || it >= tl[t].n) continue;
+          if (it > 0 && !wait_bar(cx, cx.bar(B_VE + t), (it - 1) & 1)) { ok = false; break; }
+          const int row = (tl[t].b * p.Hkv + tl[t].g) * p.L + slist[t * kMaxList + it] * 128;
+          const uint32_t sV = cx.sbase + off_v(t);
+          tc::mbar_arrive_expect_tx(cx.bar(B_VF + t), kTile);
+          tc::tma_load_2d(sV, &tmV, cx.bar(B_VF + t), 0, row);
+          tc::tma_load_2d(sV + kSub, &tmV, cx.bar(B_VF + t), 64, row);
+          vissued[t] = it + 1;
+        }
       }
       if (*cx.abort_flag) {
         // Let every copy this CTA started land before the CTA exits.
-        drain_wait(cx.bar(B_Q), 0);
-        for (int s = 0; s < kStages; ++s) {
-          if (issued[s] > 0) {
-            drain_wait(cx.bar(B_KF + s), (issued[s] - 1) & 1);
-            drain_wait(cx.bar(B_VF + s), (issued[s] - 1) & 1);
-          }
+        for (int t = 0; t < 2; ++t) {
+          if (qissued[t]) drain_wait(cx.bar(B_Q + t), 0);
+          if (kissued[t] > 0) drain_wait(cx.bar(B_KF + t), (kissued[t] - 1) & 1);
+          if (vissued[t] > 0) drain_wait(cx.bar(B_VF + t), (vissued[t] - 1) & 1);
         }
       }
     }
-  } else if (n > 0 && warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ------------------------------ MMA issuer ----------------------------
-    if (lane == 0) {
+    if (lane == 0 && nmax > 0) {
       const uint32_t id_qk = tc::idesc_bf16_f32(128, 128, false);
       const uint32_t id_pv = tc::idesc_bf16_f32(128, 128, true);
-      if (wait_bar(cx, cx.bar(B_Q), 0)) {
+      bool ok = true;
+      // S_t(0) for both tiles.
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        if (!ok || tl[t].n == 0) continue;
+        if (!wait_bar(cx, cx.bar(B_Q + t), 0) || !wait_bar(cx, cx.bar(B_KF + t), 0)) { ok = false; break; }
         tc::tc_fence_after();
-        for (int it = 0; it <= n; ++it) {
-          if (it < n) {
-            const int st = it & 1, use = it >> 1;
-            if (!wait_bar(cx, cx.bar(B_KF + st), use & 1)) break;
-            if (!wait_bar(cx, cx.bar(B_SFREE + st), (use & 1) ^ 1)) break;
+        const uint32_t sQ = cx.sbase + off_q(t), sK = cx.sbase + off_k(t);
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) {
+          const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
+          tc::mma_bf16_ss(tmem + col_s(t), tc::sw128_desc(sQ + off, 16, 1024), tc::sw128_desc(sK + off, 16, 1024),
+                          id_qk, kk > 0 ? 1u : 0u);
+        }
+        tc::mma_commit(cx.bar(B_KE + t));
+        tc::mma_commit(cx.bar(B_SF + t));
+      }
+      for (int it = 0; ok && it < nmax; ++it) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if (!ok || it >= tl[t].n) continue;
+          // O_t += P_t(it) V_t(it)
+          if (!wait_bar(cx, cx.bar(B_PF + t), it & 1) || !wait_bar(cx, cx.bar(B_VF + t), it & 1)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          const uint32_t sV = cx.sbase + off_v(t);
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            tc::mma_bf16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, tc::sw128_desc(sV + kk * 2048, kSub, 1024),
+                            id_pv, (it > 0 || kk > 0) ? 1u : 0u);
+          tc::mma_commit(cx.bar(B_VE + t));
+          if (it + 1 < tl[t].n) {
+            // S_t(it + 1) = Q_t K_t(it + 1)^T overwrites the TMEM columns holding P_t(it): issue it
+            // only once the P.V above has completed (MMAs into different accumulators are not
+            // ordered against each other).
+            if (!wait_bar(cx, cx.bar(B_VE + t), it & 1)) { ok = false; break; }
+            if (!wait_bar(cx, cx.bar(B_KF + t), (it + 1) & 1)) { ok = false; break; }
             tc::tc_fence_after();
-            const uint32_t sK = cx.sbase + OFF_K + st * kTile;
+            const uint32_t sQ = cx.sbase + off_q(t), sK = cx.sbase + off_k(t);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-              tc::mma_bf16_ss(tmem + st * 128, tc::sw128_desc(sQ + off, 16, 1024),
+              tc::mma_bf16_ss(tmem + col_s(t), tc::sw128_desc(sQ + off, 16, 1024),
                               tc::sw128_desc(sK + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
             }
-            tc::mma_commit(cx.bar(B_SF + st));
-          }
-          if (it >= 1) {
-            const int jt = it - 1, st = jt & 1, use = jt >> 1;
-            if (!wait_bar(cx, cx.bar(B_PF), jt & 1)) break;
-            if (!wait_bar(cx, cx.bar(B_VF + st), use & 1)) break;
-            tc::tc_fence_after();
-            const uint32_t sV = cx.sbase + OFF_V + st * kTile;
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint32_t offp = (kk >> 2) * kSub + (kk & 3) * 32;
-              tc::mma_bf16_ss(tmem + COL_O, tc::sw128_desc(sP + offp, 16, 1024),
-                              tc::sw128_desc(sV + kk * 2048, kSub, 1024), id_pv,
-                              (jt > 0 || kk > 0) ? 1u : 0u);
-            }
-            tc::mma_commit(cx.bar(B_KVE + st));
-            tc::mma_commit(cx.bar(B_OD));
+            tc::mma_commit(cx.bar(B_KE + t));
+            tc::mma_commit(cx.bar(B_SF + t));
+          } else {
+            tc::mma_commit(cx.bar(B_OD + t));
           }
         }
       }
@@ -224,128 +291,140 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mma_commit(cx.bar(B_DRAIN));
       drain_wait(cx.bar(B_DRAIN), 0);
     }
-  } else if (n > 0 && warp < 4) {
+  } else {
     // ------------------------------ softmax -------------------------------
-    const int r = threadIdx.x;
-    const int qt = i * 128 + r;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const int t = warp >> 2;                 // tile of this warpgroup
+    const int r = threadIdx.x & 127;         // query row = TMEM lane
+    const Tile x = t == 0 ? tl[0] : tl[1];
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + col_s(t), tO = tmem + lane_base + col_o(t);
+    const int qt = x.i * 128 + r;
     const float sl2 = p.scale * 1.4426950408889634f;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    unsigned char* prow = sm + OFF_P + r * 128;
-    for (int it = 0; it < n; ++it) {
-      const int sb = it & 1, use = it >> 1;
-      ok = __all_sync(0xffffffffu, wait_bar(cx, cx.bar(B_SF + sb), use & 1));
+    for (int it = 0; it < x.n; ++it) {
+      ok = __all_sync(0xffffffffu, wait_bar(cx, cx.bar(B_SF + t), it & 1));
       if (!ok) break;
       tc::tc_fence_after();
-      float x[128];
-      {
-        uint32_t v[32];
+      const int j = slist[t * kMaxList + it];
+      const int lim = (p.causal && j * 128 + 127 > qt) ? qt - j * 128 : 127;  // keys c <= lim visible
+      // Pass 1: row max, two 64-column halves of S per TMEM round trip.
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
+      for (int h2 = 0; h2 < 2; ++h2) {
+        uint32_t sv[2][32];
+        tc::tmem_ld32(tS + h2 * 64, sv[0]);
+        tc::tmem_ld32(tS + h2 * 64 + 32, sv[1]);
+        tc::tmem_wait_ld();
+        if (lim < 127) {  // causal diagonal: keys beyond the query row are masked
+#pragma unroll
+          for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (h2 * 64 + c * 32 + e > lim) sv[c][e] = __float_as_uint(-INFINITY);
+        }
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+          for (int e = 0; e < 32; e += 8)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              mq[q] = tc::max3(mq[q], __uint_as_float(sv[c][e + 2 * q]), __uint_as_float(sv[c][e + 2 * q + 1]));
+      }
+      const float mx = tc::max3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+      const float mnew = fmaxf(m, mx * sl2);
+      const bool need = mnew > m + kRescaleThreshold || (m == -INFINITY && mnew != -INFINITY);
+      // O_t is stable here: PV_t(it-1) completed before S_t(it) was signalled.
+      if (__any_sync(0xffffffffu, need) && it > 0) {
+        const float f = need ? exp2f(m - mnew) : 1.f;
+#pragma unroll 1
         for (int c = 0; c < 4; ++c) {
-          tc::tmem_ld32(tmem + lane_base + sb * 128 + c * 32, v);
+          uint32_t v[32];
+          tc::tmem_ld32(tO + c * 32, v);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) x[c * 32 + e] = __uint_as_float(v[e]);
+          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+          tc::tmem_st32(tO + c * 32, v);
         }
       }
-      tc::tc_fence_before();
-      tc::mbar_arrive(cx.bar(B_SFREE + sb));
-      const int j = list[it];
-      const int lim = (p.causal && j * 128 + 127 > qt) ? qt - j * 128 : 127;  // keys c <= lim visible
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        const float v = (c <= lim) ? x[c] * sl2 : -INFINITY;
-        x[c] = v;
-        mx = fmaxf(mx, v);
+      if (need) {
+        l *= exp2f(m - mnew);
+        m = mnew;
       }
-      const float mnew = fmaxf(m, mx);
-      if (it > 0) {
-        ok = __all_sync(0xffffffffu, wait_bar(cx, cx.bar(B_OD), (it - 1) & 1));
-        if (!ok) break;
-      }
-      const bool need = mnew > m + kRescaleThreshold || (m == -INFINITY && mnew != -INFINITY);
-      if (__any_sync(0xffffffffu, need)) {
-        const float f = need ? exp2f(m - mnew) : 1.f;
-        if (it > 0) {
-          tc::tc_fence_after();
-          uint32_t v[32];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const uint32_t ta = tmem + lane_base + COL_O + c * 32;
-            tc::tmem_ld32(ta, v);
-            tc::tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-            tc::tmem_st32(ta, v);
-          }
-          tc::tmem_wait_st();
-        }
-        if (need) {
-          l *= f;
-          m = mnew;
-        }
-      }
-      const float mu = (m == -INFINITY) ? 0.f : m;
-      float rs = 0.f;
-#pragma unroll
-      for (int cc = 0; cc < 16; ++cc) {
-        float pv[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pv[e] = exp2f(x[cc * 8 + e] - mu);
-          rs += pv[e];
-        }
-        uint4 u;
-        u.x = pack_bf16x2(pv[0], pv[1]);
-        u.y = pack_bf16x2(pv[2], pv[3]);
-        u.z = pack_bf16x2(pv[4], pv[5]);
-        u.w = pack_bf16x2(pv[6], pv[7]);
-        const int sub = cc >> 3, ch = cc & 7;
-        *reinterpret_cast<uint4*>(prow + sub * kSub + ((ch ^ (r & 7)) << 4)) = u;
-      }
-      l += rs;
-      tc::fence_proxy_async_smem();
-      tc::tc_fence_before();
-      tc::mbar_arrive(cx.bar(B_PF));
-    }
-    if (ok) ok = __all_sync(0xffffffffu, wait_bar(cx, cx.bar(B_OD), (n - 1) & 1));
-    if (ok) {
-      tc::tc_fence_after();
-      const float inv = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.O) + ((size_t)(b * p.Hq + h) * p.L + qt) * kHD;
-      uint32_t v[32];
+      const float nmu = (m == -INFINITY) ? 0.f : -m;
+      // Pass 2: P = 2^(s * scale * log2e - m) as bf16 pairs over the first 64 columns of S_t,
+      // reading S again 32 columns at a time (double-buffered: the next chunk's load is in
+      // flight while this chunk is exponentiated).  P chunk c lands in columns [16c, 16c+16),
+      // which this pass has already read.
+      const uint64_t sl2x2 = tc::f2_pack(sl2, sl2), nmux2 = tc::f2_pack(nmu, nmu);
+      uint64_t acc[4] = {0, 0, 0, 0};  // packed (even, odd) column partial row sums
+      uint32_t buf[2][32];
+      tc::tmem_ld32(tS, buf[0]);
+      tc::tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        tc::tmem_ld32(tmem + lane_base + COL_O + c * 32, v);
-        tc::tmem_wait_ld();
+        uint32_t (&cur)[32] = buf[c & 1];
+        if (c < 3) tc::tmem_ld32(tS + (c + 1) * 32, buf[(c + 1) & 1]);
+        if (lim < 127) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint4 u;
-          u.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]) * inv, __uint_as_float(v[q * 8 + 1]) * inv);
-          u.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]) * inv, __uint_as_float(v[q * 8 + 3]) * inv);
-          u.z = pack_bf16x2(__uint_as_float(v[q * 8 + 4]) * inv, __uint_as_float(v[q * 8 + 5]) * inv);
-          u.w = pack_bf16x2(__uint_as_float(v[q * 8 + 6]) * inv, __uint_as_float(v[q * 8 + 7]) * inv);
-          *reinterpret_cast<uint4*>(orow + c * 32 + q * 8) = u;
+          for (int e = 0; e < 32; ++e)
+            if (c * 32 + e > lim) cur[e] = __float_as_uint(-INFINITY);
         }
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float a0, a1;
+          tc::f2_unpack(tc::f2_fma(tc::f2_pack(__uint_as_float(cur[e]), __uint_as_float(cur[e + 1])), sl2x2,
+                                   nmux2), a0, a1);
+          const float p0 = tc::ex2_approx(a0), p1 = tc::ex2_approx(a1);
+          acc[(e >> 1) & 3] = tc::f2_add(acc[(e >> 1) & 3], tc::f2_pack(p0, p1));
+          pk[e >> 1] = pack_bf16x2(p0, p1);
+        }
+        tc::tmem_st16(tS + c * 16, pk);
+        if (c < 3) tc::tmem_wait_ld();
+      }
+      float rs0, rs1, rs2, rs3;
+      tc::f2_unpack(tc::f2_add(acc[0], acc[1]), rs0, rs1);
+      tc::f2_unpack(tc::f2_add(acc[2], acc[3]), rs2, rs3);
+      l += (rs0 + rs1) + (rs2 + rs3);
+      tc::tmem_wait_st();
+      tc::tc_fence_before();
+      tc::mbar_arrive(cx.bar(B_PF + t));
+    }
+    if (x.n > 0 && ok) ok = __all_sync(0xffffffffu, wait_bar(cx, cx.bar(B_OD + t), 0));
+    if (x.valid && (x.n == 0 || ok)) {
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.O) + ((size_t)(x.b * p.Hq + x.h) * p.L + qt) * kHD;
+      if (x.n > 0) {
+        tc::tc_fence_after();
+        const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t v[32];
+          tc::tmem_ld32(tO + c * 32, v);
+          tc::tmem_wait_ld();
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint4 u;
+            u.x = pack_bf16x2(__uint_as_float(v[q * 8 + 0]) * inv, __uint_as_float(v[q * 8 + 1]) * inv);
+            u.y = pack_bf16x2(__uint_as_float(v[q * 8 + 2]) * inv, __uint_as_float(v[q * 8 + 3]) * inv);
+            u.z = pack_bf16x2(__uint_as_float(v[q * 8 + 4]) * inv, __uint_as_float(v[q * 8 + 5]) * inv);
+            u.w = pack_bf16x2(__uint_as_float(v[q * 8 + 6]) * inv, __uint_as_float(v[q * 8 + 7]) * inv);
+            *reinterpret_cast<uint4*>(orow + c * 32 + q * 8) = u;
+          }
+        }
+      } else {
+#pragma unroll
+        for (int q = 0; q < 16; ++q) reinterpret_cast<uint4*>(orow)[q] = make_uint4(0, 0, 0, 0);
       }
       if (p.lse != nullptr)
-        p.lse[(size_t)(b * p.Hq + h) * p.L + qt] = l > 0.f ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+        p.lse[(size_t)(x.b * p.Hq + x.h) * p.L + qt] =
+            (x.n > 0 && l > 0.f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
-  }
-  if (n == 0 && warp < 4) {
-    const int qt = i * 128 + threadIdx.x;
-    uint4* orow = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.O) +
-                                           ((size_t)(b * p.Hq + h) * p.L + qt) * kHD);
-#pragma unroll
-    for (int q = 0; q < 16; ++q) orow[q] = make_uint4(0, 0, 0, 0);
-    if (p.lse != nullptr) p.lse[(size_t)(b * p.Hq + h) * p.L + qt] = -INFINITY;
   }
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, TMEM_COLS);
   }
@@ -356,7 +435,8 @@ cudaError_t launch_attn_tcgen05(const AttnParams& p, const CUtensorMap& tmQ, con
   cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  const unsigned grid = (unsigned)((size_t)p.B * p.Hq * p.nb);
+  const size_t tiles = (size_t)p.B * p.Hq * p.nb;
+  const unsigned grid = (unsigned)((tiles + 1) / 2);
   attn_tc_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(tmQ, tmK, tmV, p);
   return cudaGetLastError();
 }

@@ -79,6 +79,8 @@ ATT_CASES = [
     ("f32", 1, 2, 1, 7, 64, 64, True),
     ("f32", 1, 2, 2, 5, 128, 128, True),
     ("bf16", 1, 2, 1, 6, 64, 128, True),
+    ("bf16", 1, 1, 1, 7, 128, 128, True),     # odd number of query tiles, no GQA
+    ("bf16", 1, 3, 1, 3, 128, 128, False),    # group of 3: tile pairs straddle query blocks
 ]
 
 
