@@ -196,20 +196,24 @@ __global__ void __launch_bounds__(256) band_temperature_kernel(TauParams p) {
 // ---------------------------------------------------------------------------
 // block_score_softmax
 // CTA = RT query-block rows of one (b, h).  The calibrated logits of the rows
-// are kept as a float64 strip [RT][nb] in shared memory.  Column steps of CS
-// keys; head dim in chunks of DC staged transposed in shared memory (float64).
-// Thread tile: 8 rows x 4 columns of float64 FMAs (the query operands are
-// warp-uniform broadcasts, so shared-memory traffic is 1 byte per FMA).
+// are kept as a float64 strip [RT][nb] in shared memory.  Column steps of
+// CS = 256 keys; the head dim in chunks of DC staged transposed in shared
+// memory (float64), the next chunk prefetched into registers while the current
+// one is used.  Thread tile: TR rows x 2 columns of float64 FMAs (the query
+// operands are warp-uniform broadcasts).
 // Everything is float64 because the calibration 1/tau amplifies the pooled
 // logits: float32 sums of logits of magnitude ~20 already err by ~1e-6.
 // ---------------------------------------------------------------------------
 template <int RT, int D>
 __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p) {
-  constexpr int TR = 8, TC = 4;
-  constexpr int RG = RT / TR;     // row groups
-  constexpr int CG = 256 / RG;    // column groups
-  constexpr int CS = CG * TC;     // columns per step
-  constexpr int DC = RT == 16 ? 16 : 8;  // head-dim chunk
+  constexpr int TC = 2;
+  constexpr int CS = 256;                 // columns per step: one per thread when staging
+  constexpr int CG = CS / TC;             // column groups
+  constexpr int RG = 256 / CG;            // row groups
+  constexpr int TR = RT / RG;             // rows per thread
+  constexpr int DC = 16;                  // head-dim chunk
+  constexpr int NCH = D / DC;
+  static_assert(TR * RG == RT && TR % 2 == 0, "tile");
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* strip = reinterpret_cast<double*>(smem_raw);                 // [RT][nb]
   double* qT = strip + (size_t)RT * p.nb;                               // [D][RT]
@@ -237,43 +241,48 @@ __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p)
   }
   const double* ksrc = p.kbar + (size_t)(b * p.Hkv + g) * p.nb * D;
 
+  // Register stage of one K-bar chunk: column col0 + tid, dims [dc, dc + DC).
+  double2 stage[DC / 2];
+  auto fetch = [&](int col0, int dc) {
+    const int col = col0 + tid;
+    const double2* src = reinterpret_cast<const double2*>(ksrc + (size_t)col * D + dc);
+#pragma unroll
+    for (int v = 0; v < DC / 2; ++v) stage[v] = col < jend ? __ldg(src + v) : make_double2(0.0, 0.0);
+  };
+
+  fetch(0, 0);
   for (int col0 = 0; col0 < jend; col0 += CS) {
     double acc[TR][TC];
 #pragma unroll
     for (int r = 0; r < TR; ++r)
 #pragma unroll
       for (int q = 0; q < TC; ++q) acc[r][q] = 0.0;
-    for (int dc = 0; dc < D; dc += DC) {
-      __syncthreads();
-      // kT[dd][c] = kbar[col0 + c][dc + dd]
-      for (int c = tid; c < CS; c += 256) {
-        const int col = col0 + c;
-        const double2* src = reinterpret_cast<const double2*>(ksrc + (size_t)col * D + dc);
+    for (int ch = 0; ch < NCH; ++ch) {
+      __syncthreads();  // previous chunk consumed
 #pragma unroll
-        for (int v = 0; v < DC / 2; ++v) {
-          const double2 f = col < jend ? __ldg(src + v) : make_double2(0.0, 0.0);
-          kT[(v * 2 + 0) * CS + c] = f.x;
-          kT[(v * 2 + 1) * CS + c] = f.y;
-        }
+      for (int v = 0; v < DC / 2; ++v) {
+        kT[(v * 2 + 0) * CS + tid] = stage[v].x;
+        kT[(v * 2 + 1) * CS + tid] = stage[v].y;
       }
       __syncthreads();
+      // prefetch the next chunk (next column step after the last chunk)
+      if (ch + 1 < NCH) fetch(col0, (ch + 1) * DC);
+      else if (col0 + CS < jend) fetch(col0 + CS, 0);
+      const int dc = ch * DC;
 #pragma unroll
       for (int dd = 0; dd < DC; ++dd) {
-        double qv[TR], kv[TC];
+        double qv[TR];
 #pragma unroll
         for (int r = 0; r < TR; r += 2) {
           const double2 t = *reinterpret_cast<const double2*>(qT + (dc + dd) * RT + rg * TR + r);
           qv[r] = t.x; qv[r + 1] = t.y;
         }
+        const double2 kv = *reinterpret_cast<const double2*>(kT + dd * CS + cg * TC);
 #pragma unroll
-        for (int q = 0; q < TC; q += 2) {
-          const double2 t = *reinterpret_cast<const double2*>(kT + dd * CS + cg * TC + q);
-          kv[q] = t.x; kv[q + 1] = t.y;
+        for (int r = 0; r < TR; ++r) {
+          acc[r][0] = fma(qv[r], kv.x, acc[r][0]);
+          acc[r][1] = fma(qv[r], kv.y, acc[r][1]);
         }
-#pragma unroll
-        for (int r = 0; r < TR; ++r)
-#pragma unroll
-          for (int q = 0; q < TC; ++q) acc[r][q] = fma(qv[r], kv[q], acc[r][q]);
       }
     }
 #pragma unroll
@@ -336,9 +345,7 @@ int score_rows_per_cta(int nb) { return nb <= 1024 ? 16 : 8; }
 
 size_t score_smem_bytes(int nb, int D) {
   const int RT = score_rows_per_cta(nb);
-  const int CS = (256 / (RT / 8)) * 4;
-  const int DC = RT == 16 ? 16 : 8;
-  return ((size_t)RT * nb + (size_t)D * RT + (size_t)DC * CS) * sizeof(double);
+  return ((size_t)RT * nb + (size_t)D * RT + (size_t)16 * 256) * sizeof(double);
 }
 
 template <int RT, int D>

@@ -1,11 +1,19 @@
 // Per-query-block selection of key blocks ("Prism: Spectral-Aware
 // Block-Sparse Attention" §1: attention runs over a chosen subset of blocks).
 //
-// One CTA per row (b, h, i).  The candidates {0..i} minus the forced blocks
-// are sorted in shared memory by a bitonic network on (probability desc,
-// index asc); top-k takes a prefix of fixed length, cumulative mass takes the
-// shortest prefix whose float64 running sum (forced blocks included) reaches
-// `mass`.  The kept set is written ascending, padded with -1.
+// One warp per row (b, h, i); the row's probabilities sit in registers (lane l
+// holds blocks l, l + 32, l + 64, ...).  Probabilities are >= 0, so their
+// float32 bit patterns order like the values; candidates carry their bit
+// pattern as a signed key and non-candidates (forced blocks, j > i) key -1.
+//
+// The kept candidates are a prefix of the order (probability desc, index asc).
+// Such a prefix is {key > T} plus the lowest-index entries of {key == T} for
+// one threshold key T, found by bisection over the 31-bit key range:
+//   top-k:  T = the largest key with #{key >= T} >= k; take k - #{key > T} ties.
+//   mass:   T = the smallest key with forced + sum_{key > T} p < mass (float64
+//           sums), i.e. the value of the last candidate added; ties are added
+//           in index order while the running sum stays below mass.
+// The kept set (forced blocks included) is written ascending, padded with -1.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -13,132 +21,143 @@ namespace sfa {
 
 namespace {
 
-__device__ __forceinline__ bool before(float ka, int ia, float kb, int ib) {
-  return ka > kb || (ka == kb && ia < ib);
+constexpr int kWarps = 8;
+
+__device__ __forceinline__ double warp_sum(double v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
 }
 
-// Exclusive block scan of one value per thread (256 threads).
-template <typename V>
-__device__ V block_exclusive_scan(V v, V* warp_tot, V* total) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  V inc = v;
+template <int NPL>
+__global__ void __launch_bounds__(kWarps * 32) select_kernel(SelectParams p) {
+  const int lane = threadIdx.x & 31;
+  const size_t row = (size_t)blockIdx.x * kWarps + (threadIdx.x >> 5);
+  const size_t nrows = (size_t)p.B * p.Hq * p.nb;
+  if (row >= nrows) return;
+  const int i = (int)(row % p.nb);
+  const float* prow = p.probs + row * p.nb;
+  const int f1 = ((p.flags & SFA_KEEP_SINK) && i > 0) ? 0 : -1;
+  const int nforced = f1 >= 0 ? 2 : 1;
+  const int nc = i + 1 - nforced;
+  const int tmax = i / 32 + 1;  // register slots that hold blocks <= i
+
+  int key[NPL];  // candidate: bit pattern of its probability (the value is __uint_as_float(key))
 #pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const V n = __shfl_up_sync(0xffffffffu, inc, off);
-    if (lane >= off) inc += n;
+  for (int t = 0; t < NPL; ++t) {
+    const int j = t * 32 + lane;
+    int kk = -1;
+    if (t < tmax && j <= i && j != i && j != f1) kk = (int)__float_as_uint(__ldg(prow + j));
+    key[t] = kk;
   }
-  if (lane == 31) warp_tot[warp] = inc;
-  __syncthreads();
-  V base = 0, all = 0;
-  for (int w = 0; w < 8; ++w) {
-    if (w < warp) base += warp_tot[w];
-    all += warp_tot[w];
+
+  int T = -1;       // threshold key; candidates with key > T are kept
+  int take_ties = 0;  // number of key == T candidates kept, lowest index first
+  if (p.k >= 0) {
+    if (p.k >= nc) {
+      T = -1;  // every candidate
+    } else if (p.k > 0) {
+      int lo = 0, hi = 0x7F800001;  // #{key >= lo} >= k, #{key >= hi} < k
+      while (hi - lo > 1) {
+        const int mid = lo + ((hi - lo) >> 1);
+        int c = 0;
+#pragma unroll
+        for (int t = 0; t < NPL; ++t) c += (t < tmax && key[t] >= mid) ? 1 : 0;
+        c = __reduce_add_sync(0xffffffffu, c);
+        if (c >= p.k) lo = mid; else hi = mid;
+      }
+      int g = 0;
+#pragma unroll
+      for (int t = 0; t < NPL; ++t) g += (t < tmax && key[t] > lo) ? 1 : 0;
+      g = __reduce_add_sync(0xffffffffu, g);
+      T = lo;
+      take_ties = p.k - g;
+    } else {
+      T = 0x7F800001;  // k = 0: no candidate
+    }
+  } else {
+    // Running sum starts with the forced blocks.
+    const double cum_forced = (double)prow[i] + (f1 >= 0 ? (double)prow[f1] : 0.0);
+    double all = 0.0;
+#pragma unroll
+    for (int t = 0; t < NPL; ++t) all += (t < tmax && key[t] >= 0) ? (double)__uint_as_float((unsigned)key[t]) : 0.0;
+    all = warp_sum(all);
+    if (cum_forced >= p.mass) {
+      T = 0x7F800001;  // nothing added
+    } else if (cum_forced + all < p.mass) {
+      T = -1;  // every candidate added
+    } else {
+      int lo = -1, hi = 0x7F800000;  // F(lo) >= mass, F(hi) < mass, F(U) = forced + sum_{key > U} p
+      while (hi - lo > 1) {
+        const int mid = lo + ((hi - lo) >> 1);
+        double s = 0.0;
+#pragma unroll
+        for (int t = 0; t < NPL; ++t) s += (t < tmax && key[t] > mid) ? (double)__uint_as_float((unsigned)key[t]) : 0.0;
+        s = warp_sum(s);
+        if (cum_forced + s < p.mass) hi = mid; else lo = mid;
+      }
+      // hi is the key of the last candidate added; add its ties in index order while below mass.
+      double sg = 0.0;
+      int e = 0;
+#pragma unroll
+      for (int t = 0; t < NPL; ++t) {
+        if (t < tmax && key[t] > hi) sg += (double)__uint_as_float((unsigned)key[t]);
+        if (t < tmax && key[t] == hi) ++e;
+      }
+      sg = cum_forced + warp_sum(sg);
+      e = __reduce_add_sync(0xffffffffu, e);
+      const double tv = (double)__uint_as_float((unsigned)hi);
+      int r = 0;
+      double run = sg;
+      while (r < e && run < p.mass) {
+        run += tv;
+        ++r;
+      }
+      T = hi;
+      take_ties = r;
+    }
   }
-  if (total) *total = all;
-  __syncthreads();
-  return base + inc - v;
+
+  // Ascending compaction of forced + kept candidates.
+  int* out = p.idx + row * p.kmax;
+  int pos = 0, ties = 0;
+  const unsigned lt = (1u << lane) - 1u;
+#pragma unroll
+  for (int t = 0; t < NPL; ++t) {
+    if (t < tmax) {
+      const int j = t * 32 + lane;
+      const bool tie = key[t] >= 0 && key[t] == T;
+      const unsigned tb = __ballot_sync(0xffffffffu, tie);
+      const bool keep_tie = tie && (ties + __popc(tb & lt)) < take_ties;
+      const bool keep = (j <= i) && (j == i || j == f1 || key[t] > T || keep_tie);
+      const unsigned kb = __ballot_sync(0xffffffffu, keep);
+      if (keep) out[pos + __popc(kb & lt)] = j;
+      pos += __popc(kb);
+      ties += __popc(tb);
+    }
+  }
+  for (int q = pos + lane; q < p.kmax; q += 32) out[q] = -1;
+  if (lane == 0) p.counts[row] = pos;
+}
+
+template <int NPL>
+cudaError_t launch_t(const SelectParams& p, cudaStream_t st) {
+  const size_t rows = (size_t)p.B * p.Hq * p.nb;
+  const unsigned grid = (unsigned)((rows + kWarps - 1) / kWarps);
+  select_kernel<NPL><<<grid, kWarps * 32, 0, st>>>(p);
+  return cudaGetLastError();
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(256) select_kernel(SelectParams p, int nb2) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* key = reinterpret_cast<float*>(smem_raw);
-  int* id = reinterpret_cast<int*>(key + nb2);
-  unsigned char* flag = reinterpret_cast<unsigned char*>(id + nb2);
-  __shared__ double dtot[8];
-  __shared__ int itot[8];
-
-  const int row = blockIdx.x;
-  const int i = row % p.nb;
-  const float* prow = p.probs + (size_t)row * p.nb;
-  const int tid = threadIdx.x;
-  int S = 1;
-  while (S < i + 1) S <<= 1;
-  const int f0 = i;
-  const int f1 = ((p.flags & SFA_KEEP_SINK) && i > 0) ? 0 : -1;
-  const int nforced = f1 >= 0 ? 2 : 1;
-  const int nc = i + 1 - nforced;
-
-  for (int t = tid; t < S; t += 256) {
-    if (t <= i) {
-      const bool forced = (t == f0) || (t == f1);
-      key[t] = forced ? -1.f : prow[t];
-    } else {
-      key[t] = -2.f;
-    }
-    id[t] = t;
-  }
-  for (int t = tid; t < p.nb; t += 256) flag[t] = 0;
-  __syncthreads();
-
-  for (int k2 = 2; k2 <= S; k2 <<= 1) {
-    for (int j2 = k2 >> 1; j2 > 0; j2 >>= 1) {
-      for (int t = tid; t < (S >> 1); t += 256) {
-        const int a = 2 * j2 * (t / j2) + (t % j2);
-        const int c = a + j2;
-        const bool up = (a & k2) == 0;
-        const float ka = key[a], kc = key[c];
-        const int ia = id[a], ic = id[c];
-        const bool sw = up ? before(kc, ic, ka, ia) : before(ka, ia, kc, ic);
-        if (sw) {
-          key[a] = kc; key[c] = ka;
-          id[a] = ic; id[c] = ia;
-        }
-      }
-      __syncthreads();
-    }
-  }
-
-  int ntake;
-  if (p.k >= 0) {
-    ntake = min(p.k, nc);
-  } else {
-    double cum_forced = (double)prow[f0] + (f1 >= 0 ? (double)prow[f1] : 0.0);
-    const int ept = (S + 255) / 256;
-    const int t0 = tid * ept;
-    double local = 0.0;
-    for (int t = t0; t < min(t0 + ept, nc); ++t) local += (double)key[t];
-    double excl = block_exclusive_scan<double>(local, dtot, nullptr);
-    double run = cum_forced + excl;
-    int cnt = 0;
-    for (int t = t0; t < min(t0 + ept, nc); ++t) {
-      if (run < p.mass) ++cnt;
-      run += (double)key[t];
-    }
-    int total = 0;
-    block_exclusive_scan<int>(cnt, itot, &total);
-    ntake = total;
-  }
-  for (int t = tid; t < ntake; t += 256) flag[id[t]] = 1;
-  if (tid == 0) {
-    flag[f0] = 1;
-    if (f1 >= 0) flag[f1] = 1;
-  }
-  __syncthreads();
-
-  // Ascending compaction of the kept flags over [0, i].
-  const int n = i + 1;
-  const int ept = (n + 255) / 256;
-  const int t0 = tid * ept;
-  int cnt = 0;
-  for (int t = t0; t < min(t0 + ept, n); ++t) cnt += flag[t];
-  int total = 0;
-  int pos = block_exclusive_scan<int>(cnt, itot, &total);
-  int* out = p.idx + (size_t)row * p.kmax;
-  for (int t = t0; t < min(t0 + ept, n); ++t)
-    if (flag[t]) out[pos++] = t;
-  for (int t = total + tid; t < p.kmax; t += 256) out[t] = -1;
-  if (tid == 0) p.counts[row] = total;
-}
-
 cudaError_t launch_select(const SelectParams& p, cudaStream_t st) {
-  int nb2 = 1;
-  while (nb2 < p.nb) nb2 <<= 1;
-  const size_t smem = (size_t)nb2 * (sizeof(float) + sizeof(int)) + (size_t)p.nb;
-  const unsigned grid = (unsigned)((size_t)p.B * p.Hq * p.nb);
-  select_kernel<<<grid, 256, smem, st>>>(p, nb2);
-  return cudaGetLastError();
+  if (p.nb <= 32) return launch_t<1>(p, st);
+  if (p.nb <= 64) return launch_t<2>(p, st);
+  if (p.nb <= 128) return launch_t<4>(p, st);
+  if (p.nb <= 256) return launch_t<8>(p, st);
+  if (p.nb <= 512) return launch_t<16>(p, st);
+  if (p.nb <= 1024) return launch_t<32>(p, st);
+  return launch_t<64>(p, st);
 }
 
 }  // namespace sfa
