@@ -5,10 +5,10 @@
 // Three kernels, launched in order on one stream:
 //   rope_pool_energy  HBM stream over Q and K: RoPE, rotated copy, per-block
 //                     mean vectors and per-band energies (one CTA per block
-//                     and head).
+//                     and head, the block staged by bulk asynchronous copies).
 //   band_temperature  per (batch, Q head): reduce the energies to tau^H, tau^L.
-//   block_score_softmax  calibrated block logits and the causal row softmax,
-//                     both in float64.
+//   block_score_softmax  calibrated block logits (float64 tensor-core MMAs)
+//                     and the causal row softmax, both in float64.
 #include <math.h>
 
 #include "common.cuh"
@@ -18,129 +18,203 @@ namespace sfa {
 
 // ---------------------------------------------------------------------------
 // rope_pool_energy
-// Thread map: CH = D/16 threads cover one token (each owns 8 dims of the low
-// half and the matching 8 dims of the high half, i.e. 8 rotary pairs);
-// 256 / CH tokens per pass; block / (256 / CH) passes.
+// One CTA per (batch, block, group of heads).  The cos/sin slice of the block
+// (shared by every head) is read once into registers; the block's rows of Q or
+// K of each head (contiguous, 32 KB for bf16 d = 128) stream through an
+// NS-stage shared-memory ring filled by bulk asynchronous copies (mbarrier per
+// stage), so HBM reads stay in flight without holding registers.  Per head:
+// CH = D/16 threads cover one token (each owns 8 rotary pairs), 256 / CH
+// tokens per pass; RoPE in float32, the rotated row written back (input dtype,
+// round to nearest even), per-thread partial sums reduced across threads in
+// float64 to the block mean and the per-band energies.
 // ---------------------------------------------------------------------------
-template <typename T, int D>
-__global__ void __launch_bounds__(256) rope_pool_energy_kernel(RopePoolParams p) {
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               ::"r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void arm_and_load(uint32_t bar, uint32_t dst, const void* src, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}"
+               ::"r"(bar), "r"(bytes) : "memory");
+  bulk_load(dst, src, bytes, bar);
+}
+
+__device__ __forceinline__ bool wait_parity_bounded(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  for (;;) {
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}" : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    if (ok) return true;
+    if (globaltimer_ns() - t0 > 2000000000ull) return false;
+  }
+}
+
+template <typename T, int D, int PASSES, int NS>
+__global__ void __launch_bounds__(256, 1) rope_pool_energy_kernel(RopePoolParams p, int heads_per_cta) {
   constexpr int CH = D / 16;
   constexpr int TPP = 256 / CH;  // tokens per pass
   constexpr int NW = 8;
+  constexpr int BLK = TPP * PASSES;
+  constexpr uint32_t XBYTES = BLK * D * sizeof(T);
   __shared__ double red[NW][D];
   __shared__ double ered[NW][4];
+  __shared__ __align__(8) uint64_t bars[NS];
+  extern __shared__ __align__(128) unsigned char smem_dyn[];  // [NS][BLK][D] elements
 
   const int heads = p.Hq + p.Hkv;
+  const int ngroups = (heads + heads_per_cta - 1) / heads_per_cta;
   int bid = blockIdx.x;
-  const int head = bid % heads;
-  bid /= heads;
+  const int hg = bid % ngroups;
+  bid /= ngroups;
   const int j = bid % p.nb;
   const int b = bid / p.nb;
-  const bool is_q = head < p.Hq;
-  const int hh = is_q ? head : head - p.Hq;
-  const int H = is_q ? p.Hq : p.Hkv;
-  const size_t row0 = ((size_t)(b * H + hh) * p.L) + (size_t)j * p.block;
-  const T* x = static_cast<const T*>(is_q ? p.Q : p.K) + row0 * D;
-  T* xr = p.write_rot ? static_cast<T*>(is_q ? p.Qr : p.Kr) + row0 * D : nullptr;
+  const int h0 = hg * heads_per_cta;
+  const int h1 = min(heads, h0 + heads_per_cta);
+  const int nh = h1 - h0;
 
   const int tid = threadIdx.x;
   const int c = tid % CH;
   const int tk = tid / CH;
   const int lane = tid & 31, warp = tid >> 5;
 
-  float slo[8], shi[8];
-#pragma unroll
-  for (int e = 0; e < 8; ++e) slo[e] = shi[e] = 0.f;
-  double eh = 0.0, el = 0.0;
+  auto src_of = [&](int head) -> const T* {
+    const bool is_q = head < p.Hq;
+    const int hh = is_q ? head : head - p.Hq;
+    const int H = is_q ? p.Hq : p.Hkv;
+    const size_t row0 = ((size_t)(b * H + hh) * p.L) + (size_t)j * BLK;
+    return static_cast<const T*>(is_q ? p.Q : p.K) + row0 * D;
+  };
+  auto stage_ptr = [&](int st) { return reinterpret_cast<T*>(smem_dyn + (size_t)st * XBYTES); };
 
-  const int passes = p.block / TPP;
-  for (int ps = 0; ps < passes; ++ps) {
-    const int t = ps * TPP + tk;          // token within the block
-    const size_t pos = (size_t)j * p.block + t;  // absolute position
-    float lo[8], hi[8];
-    load8(x + (size_t)t * D + c * 8, lo);
-    load8(x + (size_t)t * D + D / 2 + c * 8, hi);
+  if (tid == 0) {
+    for (int st = 0; st < NS; ++st)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"((uint32_t)__cvta_generic_to_shared(&bars[st]))
+                   : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int st = 0; st < NS && st < nh; ++st)
+      arm_and_load((uint32_t)__cvta_generic_to_shared(&bars[st]),
+                   (uint32_t)__cvta_generic_to_shared(stage_ptr(st)), src_of(h0 + st), XBYTES);
+  }
+
+  // The block's cos/sin slice, once per CTA: pairs [8c, 8c+8) of tokens ps*TPP + tk.
+  float csv[PASSES][8], snv[PASSES][8];
+#pragma unroll
+  for (int ps = 0; ps < PASSES; ++ps) {
+    const size_t pos = (size_t)j * BLK + ps * TPP + tk;
     if (p.apply) {
-      float cs[8], sn[8];
-      load8(p.cos + pos * (D / 2) + c * 8, cs);
-      load8(p.sin + pos * (D / 2) + c * 8, sn);
+      load8(p.cos + pos * (D / 2) + c * 8, csv[ps]);
+      load8(p.sin + pos * (D / 2) + c * 8, snv[ps]);
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) { csv[ps][e] = 1.f; snv[ps][e] = 0.f; }
+    }
+  }
+  __syncthreads();  // barriers initialised
+
+  for (int q = 0; q < nh; ++q) {
+    const int head = h0 + q;
+    const int st = q % NS;
+    const bool landed = wait_parity_bounded((uint32_t)__cvta_generic_to_shared(&bars[st]), (q / NS) & 1);
+    const bool is_q = head < p.Hq;
+    const int hh = is_q ? head : head - p.Hq;
+    const int H = is_q ? p.Hq : p.Hkv;
+    const size_t row0 = ((size_t)(b * H + hh) * p.L) + (size_t)j * BLK;
+    T* xr = p.write_rot ? static_cast<T*>(is_q ? p.Qr : p.Kr) + row0 * D : nullptr;
+    const T* xs = stage_ptr(st);
+
+    float slo[8], shi[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) slo[e] = shi[e] = 0.f;
+    double eh = 0.0, el = 0.0;
+#pragma unroll
+    for (int ps = 0; ps < PASSES; ++ps) {
+      const int t = ps * TPP + tk;
+      float lo[8], hi[8];
+      load8_smem(xs + (size_t)t * D + c * 8, lo);
+      load8_smem(xs + (size_t)t * D + D / 2 + c * 8, hi);
+      if (p.apply) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float a = lo[e], bb = hi[e];
+          lo[e] = fmaf(a, csv[ps][e], -bb * snv[ps][e]);
+          hi[e] = fmaf(bb, csv[ps][e], a * snv[ps][e]);
+        }
+        if (xr != nullptr) {
+          store8(xr + (size_t)t * D + c * 8, lo);
+          store8(xr + (size_t)t * D + D / 2 + c * 8, hi);
+        }
+      }
+      float ph = 0.f, pl = 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
-        const float a = lo[e], bb = hi[e];
-        lo[e] = fmaf(a, cs[e], -bb * sn[e]);
-        hi[e] = fmaf(bb, cs[e], a * sn[e]);
+        slo[e] += lo[e];
+        shi[e] += hi[e];
+        const float en = fmaf(lo[e], lo[e], hi[e] * hi[e]);
+        if (c * 8 + e < p.band_pairs) ph += en; else pl += en;
       }
-      if (xr != nullptr) {
-        store8(xr + (size_t)t * D + c * 8, lo);
-        store8(xr + (size_t)t * D + D / 2 + c * 8, hi);
+      eh += ph;
+      el += pl;
+    }
+
+    // Cross-thread reduction in float64: lanes with equal c hold the same dims.
+    double dlo[8], dhi[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) { dlo[e] = slo[e]; dhi[e] = shi[e]; }
+#pragma unroll
+    for (int off = CH; off < 32; off <<= 1) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        dlo[e] += __shfl_xor_sync(0xffffffffu, dlo[e], off);
+        dhi[e] += __shfl_xor_sync(0xffffffffu, dhi[e], off);
       }
     }
-    float ph = 0.f, pl = 0.f;
+    if (lane < CH) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      slo[e] += lo[e];
-      shi[e] += hi[e];
-      const float en = fmaf(lo[e], lo[e], hi[e] * hi[e]);
-      if (c * 8 + e < p.band_pairs) ph += en; else pl += en;
+      for (int e = 0; e < 8; ++e) {
+        red[warp][lane * 8 + e] = dlo[e];
+        red[warp][D / 2 + lane * 8 + e] = dhi[e];
+      }
     }
-    eh += ph;
-    el += pl;
-  }
+    double deh = eh, del = el;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      deh += __shfl_xor_sync(0xffffffffu, deh, off);
+      del += __shfl_xor_sync(0xffffffffu, del, off);
+    }
+    if (lane == 0) { ered[warp][0] = deh; ered[warp][1] = del; }
+    __syncthreads();  // stage st fully read; partial sums visible
+    if (tid == 0 && q + NS < nh)
+      arm_and_load((uint32_t)__cvta_generic_to_shared(&bars[st]), (uint32_t)__cvta_generic_to_shared(stage_ptr(st)),
+                   src_of(h0 + q + NS), XBYTES);
 
-  // Cross-thread reduction in float64: lanes with equal c hold the same dims.
-  double dlo[8], dhi[8];
+    // One thread per dim: block mean, pooled energy per band.
+    double ph = 0.0, pl = 0.0;
+    if (tid < D) {
+      double sacc = 0.0;
 #pragma unroll
-  for (int e = 0; e < 8; ++e) { dlo[e] = slo[e]; dhi[e] = shi[e]; }
-#pragma unroll
-  for (int off = CH; off < 32; off <<= 1) {
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      dlo[e] += __shfl_xor_sync(0xffffffffu, dlo[e], off);
-      dhi[e] += __shfl_xor_sync(0xffffffffu, dhi[e], off);
+      for (int w = 0; w < NW; ++w) sacc += red[w][tid];
+      const double mean = landed ? sacc / (double)BLK : (double)NAN;  // a copy that never landed poisons tau
+      double* out = (is_q ? p.qbar + ((size_t)(b * p.Hq + hh) * p.nb + j) * D
+                          : p.kbar + ((size_t)(b * p.Hkv + hh) * p.nb + j) * D);
+      out[tid] = mean;
+      const int m = tid % (D / 2);
+      if (m < p.band_pairs) ph = mean * mean; else pl = mean * mean;
     }
-  }
-  if (lane < CH) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      red[warp][lane * 8 + e] = dlo[e];
-      red[warp][D / 2 + lane * 8 + e] = dhi[e];
+    for (int off = 16; off > 0; off >>= 1) {
+      ph += __shfl_xor_sync(0xffffffffu, ph, off);
+      pl += __shfl_xor_sync(0xffffffffu, pl, off);
     }
-  }
-  double deh = eh, del = el;
+    if (lane == 0) { ered[warp][2] = ph; ered[warp][3] = pl; }
+    __syncthreads();
+    if (tid < 4) {
+      double sacc = 0.0;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    deh += __shfl_xor_sync(0xffffffffu, deh, off);
-    del += __shfl_xor_sync(0xffffffffu, del, off);
-  }
-  if (lane == 0) { ered[warp][0] = deh; ered[warp][1] = del; }
-  __syncthreads();
-
-  // One thread per dim: block mean, pooled energy per band.
-  double ph = 0.0, pl = 0.0;
-  if (tid < D) {
-    double s = 0.0;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) s += red[w][tid];
-    const double mean = s / (double)p.block;
-    double* out = (is_q ? p.qbar + ((size_t)(b * p.Hq + hh) * p.nb + j) * D
-                        : p.kbar + ((size_t)(b * p.Hkv + hh) * p.nb + j) * D);
-    out[tid] = mean;
-    const int m = tid % (D / 2);
-    if (m < p.band_pairs) ph = mean * mean; else pl = mean * mean;
-  }
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) {
-    ph += __shfl_xor_sync(0xffffffffu, ph, off);
-    pl += __shfl_xor_sync(0xffffffffu, pl, off);
-  }
-  __syncthreads();  // everyone has read red / ered partials of the token energy
-  if (lane == 0) { ered[warp][2] = ph; ered[warp][3] = pl; }
-  __syncthreads();
-  if (tid < 4) {
-    double s = 0.0;
-#pragma unroll
-    for (int w = 0; w < NW; ++w) s += ered[w][tid];
-    p.energy[((size_t)(b * heads + head) * p.nb + j) * 4 + tid] = s;
+      for (int w = 0; w < NW; ++w) sacc += ered[w][tid];
+      p.energy[((size_t)(b * heads + head) * p.nb + j) * 4 + tid] = landed ? sacc : (double)NAN;
+    }
+    __syncthreads();  // red / ered free for the next head
   }
 }
 
@@ -196,28 +270,32 @@ __global__ void __launch_bounds__(256) band_temperature_kernel(TauParams p) {
 // ---------------------------------------------------------------------------
 // block_score_softmax
 // CTA = RT query-block rows of one (b, h).  The calibrated logits of the rows
-// are kept as a float64 strip [RT][nb] in shared memory.  Column steps of
-// CS = 256 keys; the head dim in chunks of DC staged transposed in shared
-// memory (float64), the next chunk prefetched into registers while the current
-// one is used.  Thread tile: TR rows x 2 columns of float64 FMAs (the query
-// operands are warp-uniform broadcasts).
+// are kept as a float64 strip [RT][nb] in shared memory, computed on the
+// float64 tensor cores (mma.sync m8n8k4 .f64: tcgen05 has no float64 kind):
+// column steps of 256 key blocks, each warp owns 4 column tiles of 8 and all
+// RT/8 row tiles, the head dim in k-steps of 4.  A fragments (calibrated query
+// means) come from shared memory, B fragments (key means) straight from L2,
+// prefetched one k-step ahead.  Column tiles past the causal diagonal are
+// skipped.  Then the causal row softmax in float64, one warp per row.
 // Everything is float64 because the calibration 1/tau amplifies the pooled
 // logits: float32 sums of logits of magnitude ~20 already err by ~1e-6.
 // ---------------------------------------------------------------------------
+__device__ __forceinline__ void dmma_8x8x4(double (&c)[2], double a, double b) {
+  asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
+               : "+d"(c[0]), "+d"(c[1])
+               : "d"(a), "d"(b));
+}
+
 template <int RT, int D>
 __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p) {
-  constexpr int TC = 2;
-  constexpr int CS = 256;                 // columns per step: one per thread when staging
-  constexpr int CG = CS / TC;             // column groups
-  constexpr int RG = 256 / CG;            // row groups
-  constexpr int TR = RT / RG;             // rows per thread
-  constexpr int DC = 16;                  // head-dim chunk
-  constexpr int NCH = D / DC;
-  static_assert(TR * RG == RT && TR % 2 == 0, "tile");
+  constexpr int RTL = RT / 8;             // row tiles
+  constexpr int CS = 256;                 // columns per step
+  constexpr int CTW = 4;                  // column tiles per warp (8 warps x 4 x 8 = 256)
+  constexpr int QLD = D + 4;              // padded row of the query tile (doubles)
+  constexpr int KS = D / 4;               // k-steps
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* strip = reinterpret_cast<double*>(smem_raw);                 // [RT][nb]
-  double* qT = strip + (size_t)RT * p.nb;                               // [D][RT]
-  double* kT = qT + D * RT;                                             // [DC][CS]
+  double* qs = strip + (size_t)RT * p.nb;                               // [RT][QLD]
 
   const int ntiles = (p.nb + RT - 1) / RT;
   const int tile = ntiles - 1 - (int)blockIdx.x;  // heaviest rows first
@@ -226,8 +304,8 @@ __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p)
   const int i0 = tile * RT;
   const int rows = min(RT, p.nb - i0);
   const int jend = i0 + rows;  // columns [0, jend)
-  const int tid = threadIdx.x;
-  const int rg = tid / CG, cg = tid % CG;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int gq = lane >> 2, tq = lane & 3;  // mma fragment coordinates
 
   // Calibrated, pre-scaled query block means: q~ = qbar / (tau^band * sqrt(d)).
   const double* tau = p.tau + (size_t)(b * p.Hq + h) * 2;
@@ -237,68 +315,69 @@ __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p)
   for (int e = tid; e < D * RT; e += 256) {
     const int r = e / D, d = e % D;
     const double s = ((d % (D / 2)) < p.band_pairs) ? inv_h : inv_l;
-    qT[d * RT + r] = (r < rows) ? qsrc[(size_t)r * D + d] * s : 0.0;
+    qs[r * QLD + d] = (r < rows) ? qsrc[(size_t)r * D + d] * s : 0.0;
   }
+  __syncthreads();
   const double* ksrc = p.kbar + (size_t)(b * p.Hkv + g) * p.nb * D;
 
-  // Register stage of one K-bar chunk: column col0 + tid, dims [dc, dc + DC).
-  double2 stage[DC / 2];
-  auto fetch = [&](int col0, int dc) {
-    const int col = col0 + tid;
-    const double2* src = reinterpret_cast<const double2*>(ksrc + (size_t)col * D + dc);
-#pragma unroll
-    for (int v = 0; v < DC / 2; ++v) stage[v] = col < jend ? __ldg(src + v) : make_double2(0.0, 0.0);
-  };
-
-  fetch(0, 0);
   for (int col0 = 0; col0 < jend; col0 += CS) {
-    double acc[TR][TC];
+    // this warp's column tiles: col0 + (warp * CTW + ct) * 8 .. + 8
+    int ntl = 0;
 #pragma unroll
-    for (int r = 0; r < TR; ++r)
+    for (int ct = 0; ct < CTW; ++ct) ntl += (col0 + (warp * CTW + ct) * 8 < jend) ? 1 : 0;
+    if (ntl > 0) {
+      double acc[RTL][CTW][2];
 #pragma unroll
-      for (int q = 0; q < TC; ++q) acc[r][q] = 0.0;
-    for (int ch = 0; ch < NCH; ++ch) {
-      __syncthreads();  // previous chunk consumed
+      for (int rt = 0; rt < RTL; ++rt)
 #pragma unroll
-      for (int v = 0; v < DC / 2; ++v) {
-        kT[(v * 2 + 0) * CS + tid] = stage[v].x;
-        kT[(v * 2 + 1) * CS + tid] = stage[v].y;
+        for (int ct = 0; ct < CTW; ++ct) acc[rt][ct][0] = acc[rt][ct][1] = 0.0;
+      // B fragment of column tile ct at k-step ks: kbar[col][4 ks + tq], col = tile start + gq.
+      const double* kb[CTW];
+#pragma unroll
+      for (int ct = 0; ct < CTW; ++ct) {
+        const int col = min(col0 + (warp * CTW + ct) * 8 + gq, p.nb - 1);
+        kb[ct] = ksrc + (size_t)col * D + tq;
       }
-      __syncthreads();
-      // prefetch the next chunk (next column step after the last chunk)
-      if (ch + 1 < NCH) fetch(col0, (ch + 1) * DC);
-      else if (col0 + CS < jend) fetch(col0 + CS, 0);
-      const int dc = ch * DC;
+      double bcur[CTW], bnxt[CTW];
 #pragma unroll
-      for (int dd = 0; dd < DC; ++dd) {
-        double qv[TR];
+      for (int ct = 0; ct < CTW; ++ct) bcur[ct] = __ldg(kb[ct]);
+#pragma unroll 4
+      for (int ks = 0; ks < KS; ++ks) {
+        if (ks + 1 < KS) {
 #pragma unroll
-        for (int r = 0; r < TR; r += 2) {
-          const double2 t = *reinterpret_cast<const double2*>(qT + (dc + dd) * RT + rg * TR + r);
-          qv[r] = t.x; qv[r + 1] = t.y;
+          for (int ct = 0; ct < CTW; ++ct) bnxt[ct] = __ldg(kb[ct] + 4 * (ks + 1));
         }
-        const double2 kv = *reinterpret_cast<const double2*>(kT + dd * CS + cg * TC);
+        double a[RTL];
 #pragma unroll
-        for (int r = 0; r < TR; ++r) {
-          acc[r][0] = fma(qv[r], kv.x, acc[r][0]);
-          acc[r][1] = fma(qv[r], kv.y, acc[r][1]);
+        for (int rt = 0; rt < RTL; ++rt) a[rt] = qs[(rt * 8 + gq) * QLD + 4 * ks + tq];
+#pragma unroll
+        for (int ct = 0; ct < CTW; ++ct) {
+          if (ct < ntl) {
+#pragma unroll
+            for (int rt = 0; rt < RTL; ++rt) dmma_8x8x4(acc[rt][ct], a[rt], bcur[ct]);
+          }
         }
+#pragma unroll
+        for (int ct = 0; ct < CTW; ++ct) bcur[ct] = bnxt[ct];
       }
-    }
+      // C fragment: (row gq, cols 2 tq, 2 tq + 1) of each tile
 #pragma unroll
-    for (int r = 0; r < TR; ++r) {
-      const int rr = rg * TR + r;
+      for (int rt = 0; rt < RTL; ++rt) {
+        const int rr = rt * 8 + gq;
 #pragma unroll
-      for (int q = 0; q < TC; ++q) {
-        const int col = col0 + cg * TC + q;
-        if (col < jend) strip[(size_t)rr * p.nb + col] = acc[r][q];
+        for (int ct = 0; ct < CTW; ++ct) {
+          const int col = col0 + (warp * CTW + ct) * 8 + 2 * tq;
+          if (ct < ntl) {  // scalar stores: nb may be odd, so a row need not start 16-byte aligned
+            if (col < jend) strip[(size_t)rr * p.nb + col] = acc[rt][ct][0];
+            if (col + 1 < jend) strip[(size_t)rr * p.nb + col + 1] = acc[rt][ct][1];
+          }
+        }
       }
     }
   }
   __syncthreads();
 
   // Causal row softmax in float64, one warp per row.
-  const int lane = tid & 31, warp = tid >> 5;
   for (int r = warp; r < rows; r += 8) {
     const int i = i0 + r;
     double* srow = strip + (size_t)r * p.nb;
@@ -323,12 +402,30 @@ __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p)
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
+template <typename T, int D, int PASSES>
+static cudaError_t launch_rope_pool_tdp(const RopePoolParams& p, cudaStream_t st) {
+  constexpr int NS = sizeof(T) == 2 ? 3 : 2;  // ring stages of one head's block rows
+  const size_t smem = (size_t)NS * (256 / (D / 16)) * PASSES * D * sizeof(T);
+  auto kern = rope_pool_energy_kernel<T, D, PASSES, NS>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  // Enough CTAs for about four waves of 148 SMs; each CTA reads the table slice once for its heads.
+  const int heads = p.Hq + p.Hkv;
+  const long long blocks = (long long)p.B * p.nb;
+  int groups = (int)((4LL * 148 + blocks - 1) / blocks);
+  groups = groups < 1 ? 1 : (groups > heads ? heads : groups);
+  const int per = (heads + groups - 1) / groups;
+  groups = (heads + per - 1) / per;
+  const unsigned grid = (unsigned)(blocks * groups);
+  kern<<<grid, 256, smem, st>>>(p, per);
+  return cudaGetLastError();
+}
+
 template <typename T>
 static cudaError_t launch_rope_pool_t(const RopePoolParams& p, int D, cudaStream_t st) {
-  const unsigned grid = (unsigned)((size_t)p.B * p.nb * (p.Hq + p.Hkv));
-  if (D == 128) rope_pool_energy_kernel<T, 128><<<grid, 256, 0, st>>>(p);
-  else rope_pool_energy_kernel<T, 64><<<grid, 256, 0, st>>>(p);
-  return cudaGetLastError();
+  // tokens per pass: 256 / (D / 16) = 32 (D = 128) or 64 (D = 64)
+  if (D == 128) return p.block == 128 ? launch_rope_pool_tdp<T, 128, 4>(p, st) : launch_rope_pool_tdp<T, 128, 2>(p, st);
+  return p.block == 128 ? launch_rope_pool_tdp<T, 64, 2>(p, st) : launch_rope_pool_tdp<T, 64, 1>(p, st);
 }
 
 cudaError_t launch_rope_pool_energy(const RopePoolParams& p, int dtype, int D, cudaStream_t st) {
@@ -345,7 +442,7 @@ int score_rows_per_cta(int nb) { return nb <= 1024 ? 16 : 8; }
 
 size_t score_smem_bytes(int nb, int D) {
   const int RT = score_rows_per_cta(nb);
-  return ((size_t)RT * nb + (size_t)D * RT + (size_t)16 * 256) * sizeof(double);
+  return ((size_t)RT * nb + (size_t)RT * (D + 4)) * sizeof(double);
 }
 
 template <int RT, int D>
