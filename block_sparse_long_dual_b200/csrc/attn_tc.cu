@@ -9,20 +9,25 @@
 // warpgroup turns S_t into P_t, the tensor core runs the other tile's P.V and
 // next Q.K^T.
 //
-//   warps 0-3 / 4-7  softmax of tile 0 / tile 1: thread r owns query row r
-//                    (TMEM lane r); reads S_t from TMEM, online softmax with a
-//                    lazily rescaled O_t, writes P_t (bf16) back into the S_t
-//                    columns of TMEM, final O_t / l epilogue.
-//   warp 8           producer: TMA loads of Q_t and of K_t(j), V_t(j) for every
+//   warps 0-7 / 8-15 softmax of tile 0 / tile 1: two threads per query row r
+//                    (TMEM lane r; warps w and w+4 share lanes), each owning 64
+//                    of the 128 key columns, row maxima exchanged through shared
+//                    memory; reads S_t from TMEM, online softmax with a lazily
+//                    rescaled O_t, writes P_t (bf16) back into the S_t columns of
+//                    TMEM, final O_t / l epilogue.  Two softmax warps per SM
+//                    sub-partition work on a tile at once, hiding each other's
+//                    latency.
+//   warp 16          producer: TMA loads of Q_t and of K_t(j), V_t(j) for every
 //                    kept block j of each tile (one K and one V slot per tile).
-//   warp 9           MMA issuer: S_t = Q_t K_t^T (A, B from shared memory) and
+//   warp 17          MMA issuer: S_t = Q_t K_t^T (A, B from shared memory) and
 //                    O_t += P_t V_t (A = P_t from TMEM, B = V_t from shared
 //                    memory), M = N = 128, K = 16 steps; completion tracked with
 //                    tcgen05.commit -> mbarriers.  A commit covers every MMA the
 //                    thread issued before it, so the commit that signals S_t(j)
 //                    also means O_t has absorbed P_t(j-1).
 // TMEM (512 columns): S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512);
-// P_t aliases the first 64 columns of S_t (two bf16 per column).
+// P_t aliases S_t (two bf16 per column): keys [0,64) in S columns [0,32), keys
+// [64,128) in S columns [64,96), each half written by the threads that read it.
 // Every mbarrier wait is bounded (about 2 s); a wait that runs out writes
 // SFA_ERR_TIMEOUT to the status word, raises a CTA-wide abort flag, drains the
 // copies / MMAs this CTA issued and frees its tensor memory.
@@ -45,13 +50,17 @@ __host__ __device__ constexpr uint32_t off_k(int t) { return 2 * kTile + t * kTi
 __host__ __device__ constexpr uint32_t off_v(int t) { return 4 * kTile + t * kTile; }
 constexpr uint32_t OFF_BAR = 6 * kTile;
 // Barriers, two of each (one per tile) except DRAIN.
-enum { B_Q = 0, B_KF = 2, B_VF = 4, B_KE = 6, B_VE = 8, B_SF = 10, B_PF = 12, B_OD = 14, B_DRAIN = 16, NBAR = 17 };
+enum { B_Q = 0, B_KF = 2, B_VF = 4, B_KE = 6, B_VE = 8, B_SF = 10, B_PF = 12, B_OD = 14, B_X = 16, B_DRAIN = 20,
+       NBAR = 21 };  // B_X: [tile][parity] row-max / row-sum exchange of the two column halves
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+constexpr uint32_t OFF_XCHG = OFF_MISC + 32;         // [2 tiles][2 parities][2 halves][128 rows] float
 constexpr int kMaxList = 2048;                       // nb <= 2048, so a valid list has <= 2048 entries
-constexpr uint32_t OFF_LIST = OFF_MISC + 32;         // per tile: the validated index list
+constexpr uint32_t OFF_LIST = OFF_XCHG + 2 * 2 * 2 * 128 * 4;  // per tile: the validated index list
 constexpr uint32_t SMEM_BYTES = OFF_LIST + 2 * kMaxList * 4 + 1024;
-constexpr int kThreads = 320;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
+// Warps 0-7 softmax of tile 0, 8-15 of tile 1 (two threads per query row: warps w and w+4
+// share TMEM lanes and split the 128 key columns), 16 producer, 17 MMA issuer.
+constexpr int kThreads = 576;
+constexpr int kProducerWarp = 16, kMmaWarp = 17;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
@@ -135,9 +144,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   Tile tl[2] = {decode_tile(p, 2 * blockIdx.x), decode_tile(p, 2 * blockIdx.x + 1)};
 
-  if (warp == 0 || warp == 4) {
+  if (warp == 0 || warp == 8) {
     // Validate one tile's index list: count in [0, kmax], entries ascending in [0, nb), <= i if causal.
-    const int t = warp >> 2;
+    const int t = warp >> 3;
     const Tile x = t == 0 ? tl[0] : tl[1];
     int n = 0;
     if (x.valid) {
@@ -160,7 +169,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) nsh[t] = n;
     if (warp == 0 && lane == 0) {
       *cx.abort_flag = 0;
-      for (int k = 0; k < NBAR; ++k) tc::mbar_init(cx.bar(k), (k == B_PF || k == B_PF + 1) ? 128 : 1);
+      for (int k = 0; k < NBAR; ++k)
+        tc::mbar_init(cx.bar(k), (k == B_PF || k == B_PF + 1 || (k >= B_X && k < B_X + 4)) ? 256 : 1);
       tc::fence_mbar_init();
     }
   } else if (warp == kProducerWarp && lane == 0) {
@@ -263,8 +273,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t sV = cx.sbase + off_v(t);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            tc::mma_bf16_ts(tmem + col_o(t), tmem + col_s(t) + kk * 8, tc::sw128_desc(sV + kk * 2048, kSub, 1024),
-                            id_pv, (it > 0 || kk > 0) ? 1u : 0u);
+            // P keys [16 kk, 16 kk + 16): half kk / 4 wrote them into its own S columns
+            tc::mma_bf16_ts(tmem + col_o(t), tmem + col_s(t) + (kk >> 2) * 64 + (kk & 3) * 8,
+                            tc::sw128_desc(sV + kk * 2048, kSub, 1024), id_pv, (it > 0 || kk > 0) ? 1u : 0u);
           tc::mma_commit(cx.bar(B_VE + t));
           if (it + 1 < tl[t].n) {
             // S_t(it + 1) = Q_t K_t(it + 1)^T overwrites the TMEM columns holding P_t(it): issue it
@@ -293,35 +304,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------ softmax -------------------------------
-    const int t = warp >> 2;                 // tile of this warpgroup
-    const int r = threadIdx.x & 127;         // query row = TMEM lane
+    const int t = warp >> 3;                 // tile of this warp
+    const int hf = (warp >> 2) & 1;          // key-column half: [64 hf, 64 hf + 64)
+    const int r = ((warp & 3) << 5) | lane;  // query row = TMEM lane
     const Tile x = t == 0 ? tl[0] : tl[1];
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + col_s(t), tO = tmem + lane_base + col_o(t);
+    const uint32_t tS = tmem + lane_base + col_s(t) + 64 * hf;     // this half's S columns
+    const uint32_t tP = tmem + lane_base + col_s(t) + 64 * hf;     // this half's P columns (2 bf16 each)
+    const uint32_t tO = tmem + lane_base + col_o(t) + 64 * hf;     // this half's O columns
+    float* xchg = reinterpret_cast<float*>(sm + OFF_XCHG) + t * 512;  // [parity][half][row]
+    // Exchange with the other half of the row: write, arrive on the tile's parity barrier (256
+    // arrivals), bounded wait, read.  Use u of parity q waits for phase parity (u / 2) & 1.
+    auto exchange = [&](int use, float v) -> float {
+      float* xc = xchg + (use & 1) * 256;
+      xc[hf * 128 + r] = v;
+      const uint32_t xb = cx.bar(B_X + t * 2 + (use & 1));
+      tc::mbar_arrive(xb);
+      if (!wait_bar(cx, xb, (use >> 1) & 1)) return NAN;
+      return xc[(1 - hf) * 128 + r];
+    };
     const int qt = x.i * 128 + r;
     const float sl2 = p.scale * 1.4426950408889634f;
-    float m = -INFINITY, l = 0.f;
+    float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
     bool ok = true;
     for (int it = 0; it < x.n; ++it) {
       ok = __all_sync(0xffffffffu, wait_bar(cx, cx.bar(B_SF + t), it & 1));
       if (!ok) break;
       tc::tc_fence_after();
       const int j = slist[t * kMaxList + it];
-      const int lim = (p.causal && j * 128 + 127 > qt) ? qt - j * 128 : 127;  // keys c <= lim visible
-      // Pass 1: row max, two 64-column halves of S per TMEM round trip.
+      // keys c (0..127 of the block) with c <= lim are visible; this half holds c = 64 hf + cc
+      const int lim = ((p.causal && j * 128 + 127 > qt) ? qt - j * 128 : 127) - 64 * hf;
+      // Pass 1: max over this half, then the row max through shared memory.
       float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
+      {
         uint32_t sv[2][32];
-        tc::tmem_ld32(tS + h2 * 64, sv[0]);
-        tc::tmem_ld32(tS + h2 * 64 + 32, sv[1]);
+        tc::tmem_ld32(tS, sv[0]);
+        tc::tmem_ld32(tS + 32, sv[1]);
         tc::tmem_wait_ld();
-        if (lim < 127) {  // causal diagonal: keys beyond the query row are masked
+        if (lim < 63) {  // causal diagonal: keys beyond the query row are masked
 #pragma unroll
           for (int c = 0; c < 2; ++c)
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (h2 * 64 + c * 32 + e > lim) sv[c][e] = __float_as_uint(-INFINITY);
+              if (c * 32 + e > lim) sv[c][e] = __float_as_uint(-INFINITY);
         }
 #pragma unroll
         for (int c = 0; c < 2; ++c)
@@ -331,14 +356,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int q = 0; q < 4; ++q)
               mq[q] = tc::max3(mq[q], __uint_as_float(sv[c][e + 2 * q]), __uint_as_float(sv[c][e + 2 * q + 1]));
       }
-      const float mx = tc::max3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+      const float mhalf = tc::max3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
+      const float mx = fmaxf(mhalf, exchange(it, mhalf));
       const float mnew = fmaxf(m, mx * sl2);
       const bool need = mnew > m + kRescaleThreshold || (m == -INFINITY && mnew != -INFINITY);
       // O_t is stable here: PV_t(it-1) completed before S_t(it) was signalled.
       if (__any_sync(0xffffffffu, need) && it > 0) {
         const float f = need ? exp2f(m - mnew) : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
           tc::tmem_ld32(tO + c * 32, v);
           tc::tmem_wait_ld();
@@ -352,27 +378,26 @@ __global__ void __launch_bounds__(kThreads, 1)
         m = mnew;
       }
       const float nmu = (m == -INFINITY) ? 0.f : -m;
-      // Pass 2: P = 2^(s * scale * log2e - m) as bf16 pairs over the first 64 columns of S_t,
-      // reading S again 32 columns at a time (double-buffered: the next chunk's load is in
-      // flight while this chunk is exponentiated).  P chunk c lands in columns [16c, 16c+16),
-      // which this pass has already read.
+      // Pass 2: P = 2^(s * scale * log2e - m) as bf16 pairs, 16 columns at a time
+      // (double-buffered TMEM loads).  P chunk c of this half lands in S columns
+      // [64 hf + 8 c, +8), which this thread has already read.
       const uint64_t sl2x2 = tc::f2_pack(sl2, sl2), nmux2 = tc::f2_pack(nmu, nmu);
       uint64_t acc[4] = {0, 0, 0, 0};  // packed (even, odd) column partial row sums
-      uint32_t buf[2][32];
-      tc::tmem_ld32(tS, buf[0]);
+      uint32_t buf[2][16];
+      tc::tmem_ld16(tS, buf[0]);
       tc::tmem_wait_ld();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
-        uint32_t (&cur)[32] = buf[c & 1];
-        if (c < 3) tc::tmem_ld32(tS + (c + 1) * 32, buf[(c + 1) & 1]);
-        if (lim < 127) {
+        uint32_t (&cur)[16] = buf[c & 1];
+        if (c < 3) tc::tmem_ld16(tS + (c + 1) * 16, buf[(c + 1) & 1]);
+        if (lim < 63) {
 #pragma unroll
-          for (int e = 0; e < 32; ++e)
-            if (c * 32 + e > lim) cur[e] = __float_as_uint(-INFINITY);
+          for (int e = 0; e < 16; ++e)
+            if (c * 16 + e > lim) cur[e] = __float_as_uint(-INFINITY);
         }
-        uint32_t pk[16];
+        uint32_t pk[8];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
+        for (int e = 0; e < 16; e += 2) {
           float a0, a1;
           tc::f2_unpack(tc::f2_fma(tc::f2_pack(__uint_as_float(cur[e]), __uint_as_float(cur[e + 1])), sl2x2,
                                    nmux2), a0, a1);
@@ -380,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc[(e >> 1) & 3] = tc::f2_add(acc[(e >> 1) & 3], tc::f2_pack(p0, p1));
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        tc::tmem_st16(tS + c * 16, pk);
+        tc::tmem_st8(tP + c * 8, pk);
         if (c < 3) tc::tmem_wait_ld();
       }
       float rs0, rs1, rs2, rs3;
@@ -392,13 +417,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc::mbar_arrive(cx.bar(B_PF + t));
     }
     if (x.n > 0 && ok) ok = __all_sync(0xffffffffu, wait_bar(cx, cx.bar(B_OD + t), 0));
+    // Both halves of a row take the same branch: ok and x.n are uniform over the tile.
     if (x.valid && (x.n == 0 || ok)) {
-      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.O) + ((size_t)(x.b * p.Hq + x.h) * p.L + qt) * kHD;
+      __nv_bfloat16* orow =
+          static_cast<__nv_bfloat16*>(p.O) + ((size_t)(x.b * p.Hq + x.h) * p.L + qt) * kHD + 64 * hf;
+      float ltot = 0.f;
       if (x.n > 0) {
+        ltot = l + exchange(x.n, l);  // use n: the parity the last iteration did not touch
         tc::tc_fence_after();
-        const float inv = l > 0.f ? 1.f / l : 0.f;
+        const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+        for (int c = 0; c < 2; ++c) {
           uint32_t v[32];
           tc::tmem_ld32(tO + c * 32, v);
           tc::tmem_wait_ld();
@@ -414,11 +443,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
 #pragma unroll
-        for (int q = 0; q < 16; ++q) reinterpret_cast<uint4*>(orow)[q] = make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < 8; ++q) reinterpret_cast<uint4*>(orow)[q] = make_uint4(0, 0, 0, 0);
       }
-      if (p.lse != nullptr)
+      if (p.lse != nullptr && hf == 0)
         p.lse[(size_t)(x.b * p.Hq + x.h) * p.L + qt] =
-            (x.n > 0 && l > 0.f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
+            (x.n > 0 && ltot > 0.f) ? (m + log2f(ltot)) * 0.6931471805599453f : -INFINITY;
     }
   }
 
