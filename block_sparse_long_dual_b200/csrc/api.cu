@@ -19,7 +19,7 @@ namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
 constexpr int kMaxBlocks = 2048;
-constexpr unsigned kKnownFlags = SFA_KEEP_SINK | SFA_NO_CALIB | SFA_SINGLE_BAND;
+constexpr unsigned kKnownFlags = SFA_KEEP_SINK | SFA_NO_CALIB | SFA_SINGLE_BAND | SFA_RELATIVE_CALIB;
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 

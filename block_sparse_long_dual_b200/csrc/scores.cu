@@ -220,7 +220,8 @@ __global__ void __launch_bounds__(256, 1) rope_pool_energy_kernel(RopePoolParams
 
 // ---------------------------------------------------------------------------
 // band_temperature: tau^b = max(rho^b(Q_h) * rho^b(K_g), 1e-6),
-// rho = sqrt(mean_j ||xbar_j^b||^2 / mean_t ||x_t^b||^2), 1 for an empty band.
+// rho = sqrt(mean_j ||xbar_j^b||^2 / mean_t ||x_t^b||^2), 1 for an empty band;
+// with SFA_RELATIVE_CALIB tau^H / tau^L and 1.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) band_temperature_kernel(TauParams p) {
   const int h = blockIdx.x % p.Hq;
@@ -248,22 +249,29 @@ __global__ void __launch_bounds__(256) band_temperature_kernel(TauParams p) {
     if (lane == 0) red[warp][q] = acc[q];
   }
   __syncthreads();
-  if (threadIdx.x < 2) {
-    const int band = threadIdx.x;  // 0 = H, 1 = L
-    double tq = 0, pq = 0, tk = 0, pk = 0;
-    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
-      tq += red[w][band]; pq += red[w][2 + band];
-      tk += red[w][4 + band]; pk += red[w][6 + band];
-    }
-    double tau = 1.0;
+  if (threadIdx.x == 0) {
+    double tau[2] = {1.0, 1.0};  // band H, band L
     if (!(p.flags & SFA_NO_CALIB)) {
-      const double etq = tq / (double)p.L, epq = pq / (double)p.nb;
-      const double etk = tk / (double)p.L, epk = pk / (double)p.nb;
-      const double rq = etq > 0.0 ? sqrt(epq / etq) : 1.0;
-      const double rk = etk > 0.0 ? sqrt(epk / etk) : 1.0;
-      tau = fmax(rq * rk, 1e-6);
+      for (int band = 0; band < 2; ++band) {
+        double tq = 0, pq = 0, tk = 0, pk = 0;
+        for (int w = 0; w < (int)(blockDim.x >> 5); ++w) {
+          tq += red[w][band]; pq += red[w][2 + band];
+          tk += red[w][4 + band]; pk += red[w][6 + band];
+        }
+        const double etq = tq / (double)p.L, epq = pq / (double)p.nb;
+        const double etk = tk / (double)p.L, epk = pk / (double)p.nb;
+        const double rq = etq > 0.0 ? sqrt(epq / etq) : 1.0;
+        const double rk = etk > 0.0 ? sqrt(epk / etk) : 1.0;
+        tau[band] = fmax(rq * rk, 1e-6);
+      }
+      if (p.flags & SFA_RELATIVE_CALIB) {
+        // Alternative reading: only the high band's amplitude relative to the low band is restored.
+        tau[0] = (p.flags & SFA_SINGLE_BAND) ? 1.0 : tau[0] / tau[1];
+        tau[1] = 1.0;
+      }
     }
-    p.tau[(size_t)(b * p.Hq + h) * 2 + band] = tau;
+    p.tau[(size_t)(b * p.Hq + h) * 2 + 0] = tau[0];
+    p.tau[(size_t)(b * p.Hq + h) * 2 + 1] = tau[1];
   }
 }
 

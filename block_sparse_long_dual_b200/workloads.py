@@ -15,6 +15,7 @@ from dataclasses import dataclass, replace
 KEEP_SINK = 1
 NO_CALIB = 2
 SINGLE_BAND = 4
+RELATIVE_CALIB = 8
 
 
 @dataclass(frozen=True)

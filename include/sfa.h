@@ -68,7 +68,8 @@ typedef struct {
 enum {
   SFA_KEEP_SINK = 1,   /* select: also force key block 0 into every row */
   SFA_NO_CALIB = 2,    /* scores: temperature tau = 1 (plain mean pooling) */
-  SFA_SINGLE_BAND = 4  /* scores: all d dims form one band (one tau) */
+  SFA_SINGLE_BAND = 4, /* scores: all d dims form one band (one tau) */
+  SFA_RELATIVE_CALIB = 8 /* scores: restore band H relative to band L only: tau^H <- tau^H / tau^L, tau^L <- 1 */
 };
 
 /* Library version: major * 10000 + minor * 100 + patch. */
@@ -121,6 +122,8 @@ sfa_status sfa_workspace_layout(const sfa_shape* shape, int block, size_t offset
  *   s_ij    = sum_b (qbar_i^b . kbar_j^b) / (tau^b * sqrt(d)),  j <= i
  *   probs_ij = exp(s_ij) / sum_{j' <= i} exp(s_ij'), and 0 for j > i.
  * probs [B, heads_q, nb, nb] float32.  SFA_SINGLE_BAND puts all dims in band H.
+ * SFA_RELATIVE_CALIB (an alternative reading of the temperature) divides
+ * tau^H by tau^L and sets tau^L = 1 (1 for both with a single band).
  * RoPE is applied in float32; block means, energies, temperatures, logits and
  * the softmax are float64 (the 1/tau calibration amplifies pooled logits, so
  * float32 sums would move probabilities by ~1e-6), rounded once to float32.

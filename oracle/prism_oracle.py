@@ -38,6 +38,9 @@ R4  Energy and tau, per (batch, Q head, band):
         rho    = sqrt(E_pool / E_tok)            (rho = 1 if E_tok == 0)
         tau    = max(rho(Q_h) * rho(K_g), 1e-6)
     NO_CALIB sets tau = 1; SINGLE_BAND treats all d dims as one band.
+R4b (alternative reading, flag RELATIVE_CALIB): restore the high band's
+    amplitude relative to the low band only: tau^H <- tau^H / tau^L,
+    tau^L <- 1 (the low band keeps its plain mean-pooling scale).
 R5  Logits: s_ij = (1/sqrt(d)) * sum_b (qbar_i^b . kbar_j^b) / tau^b, j <= i.
 R6  Probabilities: causal row softmax over j <= i; p_ij = 0 for j > i.
 R7  Selection: forced F_i = {i} (and {0} with KEEP_SINK); candidates ordered
@@ -69,6 +72,7 @@ import numpy as np
 FLAG_KEEP_SINK = 1
 FLAG_NO_CALIB = 2
 FLAG_SINGLE_BAND = 4
+FLAG_RELATIVE_CALIB = 8
 
 TAU_FLOOR = 1e-6
 
@@ -167,6 +171,12 @@ def temperatures(qr, kr, qbar, kbar, band_split, flags, group):
         rk = retained_amplitude(kr, kbar, band)            # [B, Hkv]
         rk_per_q = np.repeat(rk, group, axis=1)            # Q head h -> KV head h // group
         tau[:, :, bi] = np.maximum(rq * rk_per_q, TAU_FLOOR)
+    if flags & FLAG_RELATIVE_CALIB:
+        if single:
+            tau[:] = 1.0
+        else:
+            tau[:, :, 0] = tau[:, :, 0] / tau[:, :, 1]
+            tau[:, :, 1] = 1.0
     return tau
 
 

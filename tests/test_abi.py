@@ -98,7 +98,7 @@ def test_argument_validation_before_launch(lib):
     assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 0, d, d, None, d, ws, None) == 1
     assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 65, 128, 0, d, d, d, d, ws, None) == 1
     assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), -1, 128, 0, d, d, d, d, ws, None) == 1
-    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 8, d, d, d, d, ws, None) == 1
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 16, d, d, d, d, ws, None) == 1
     assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 0, None, d, d, d, ws, None) == 1
     # misaligned pointers
     assert bs(ctypes.byref(shape), ctypes.c_void_p((1 << 20) + 2), d, ctypes.byref(rope), 16, 128, 0, d, d, d, d,
@@ -116,7 +116,7 @@ def test_argument_validation_before_launch(lib):
     assert sel(ctypes.byref(shape), 128, d, 3, 0.0, 0, d, d, 3, None) == 1       # kmax < k + 1
     assert sel(ctypes.byref(shape), 128, d, 3, 0.0, 1, d, d, 4, None) == 1       # kmax < k + 2 with sink
     assert sel(ctypes.byref(shape), 128, None, 3, 0.0, 0, d, d, 4, None) == 1
-    assert sel(ctypes.byref(shape), 128, d, 3, 0.0, 16, d, d, 4, None) == 1      # unknown flag
+    assert sel(ctypes.byref(shape), 128, d, 3, 0.0, 32, d, d, 4, None) == 1      # unknown flag
     at = lib.sfa_block_sparse_attn
     assert at(ctypes.byref(shape), 128, d, d, d, d, d, 0, 1, 0.0, d, None, None, None) == 1  # kmax 0
     assert at(ctypes.byref(shape), 128, d, None, d, d, d, 4, 1, 0.0, d, None, None, None) == 1

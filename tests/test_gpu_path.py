@@ -13,7 +13,7 @@ import torch
 
 from block_sparse_long_dual_b200 import sfa
 from block_sparse_long_dual_b200.synthetic import make_inputs
-from block_sparse_long_dual_b200.workloads import KEEP_SINK, NO_CALIB, SINGLE_BAND, TINY, Workload
+from block_sparse_long_dual_b200.workloads import KEEP_SINK, NO_CALIB, RELATIVE_CALIB, SINGLE_BAND, TINY, Workload
 from oracle import prism_oracle as po
 from tests.parity import compare_masks, rel_err, to_np
 
@@ -41,6 +41,8 @@ CASES = [
     W("bf16-d64-b64", head_dim=64, block=64, band_split=16, seq_len=33 * 64, k=4, flags=KEEP_SINK),
     W("f32-d128-b64-mass", dtype="f32", block=64, seq_len=24 * 64, k=None, mass=0.5, slash=True),
     W("bf16-one-block", seq_len=128, k=1),
+    W("bf16-relative-calib-mass", seq_len=12 * 128, k=None, mass=0.9, slash=True, flags=RELATIVE_CALIB),
+    W("bf16-relative-calib-single", seq_len=6 * 128, k=2, flags=RELATIVE_CALIB | SINGLE_BAND | KEEP_SINK),
 ]
 
 

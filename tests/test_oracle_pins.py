@@ -373,3 +373,40 @@ def test_tiny_path_structure():
         assert i in kept and (i == 0 or 0 in kept)
         assert len(kept) == min(i + 1, w.k + (2 if i else 1))
     assert np.all(np.isfinite(r.out))
+
+
+# ---------------------------------------------------------------------------
+# Alternative reading R4b (RELATIVE_CALIB): band H restored relative to band L.
+# ---------------------------------------------------------------------------
+def test_relative_calibration_closed_form_and_low_band_untouched():
+    base, d, beta, L, bs = 1e4, 16, 8, 64, 3
+    cos, sin = po.rope_tables(base, L, d)
+    rng = np.random.default_rng(21)
+    qv, kv = rng.normal(size=d), rng.normal(size=d)
+    Q = np.broadcast_to(qv, (1, 1, L, d)).copy()
+    K = np.broadcast_to(kv, (1, 1, L, d)).copy()
+    rel = po.prism_scores(Q, K, beta, bs, po.FLAG_RELATIVE_CALIB, (cos, sin))
+    theta = po.rope_frequencies(base, d)
+    Dm = np.abs(np.sin(beta * theta / 2)) / (beta * np.abs(np.sin(theta / 2)))
+
+    def rho(v, pairs):
+        e = v[pairs] ** 2 + v[pairs + d // 2] ** 2
+        return math.sqrt((e * Dm[pairs] ** 2).sum() / e.sum())
+
+    hi, lo = np.arange(bs), np.arange(bs, d // 2)
+    want = (rho(qv, hi) * rho(kv, hi)) / (rho(qv, lo) * rho(kv, lo))
+    assert rel.tau[0, 0, 0] == pytest.approx(want, rel=1e-5)
+    assert rel.tau[0, 0, 1] == 1.0
+    # Q, K with no high-band energy: identical to plain mean pooling
+    rng = np.random.default_rng(22)
+    Qr_, Kr_ = rng.normal(size=(1, 2, 96, d)), rng.normal(size=(1, 1, 96, d))
+    hm = po.high_band_mask(d, bs)
+    Qr_[..., hm] = 0.0
+    Kr_[..., hm] = 0.0
+    cos2, sin2 = po.rope_tables(base, 96, d)
+    a = po.prism_scores(Qr_, Kr_, beta, bs, po.FLAG_RELATIVE_CALIB, (cos2, sin2))
+    b = po.prism_scores(Qr_, Kr_, beta, bs, po.FLAG_NO_CALIB, (cos2, sin2))
+    np.testing.assert_allclose(a.probs, b.probs, rtol=0, atol=1e-13)
+    # one band relative to itself: no calibration
+    c = po.prism_scores(Qr_, Kr_, beta, bs, po.FLAG_RELATIVE_CALIB | po.FLAG_SINGLE_BAND, (cos2, sin2))
+    np.testing.assert_allclose(c.tau, 1.0)
