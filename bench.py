@@ -344,8 +344,10 @@ def main():
             "roofline": {"kernel": "attn_tc_kernel (sfa_block_sparse_attn)", "bound": "tensor",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": f"{pk_src} bf16 burst",
-                         "traffic": (tr["bytes_per_launch"] * (flops_step / tr["flops_per_launch"])
+                         "traffic": (tr["bytes_per_launch"] * (w.batch * w.heads_q * w.nb) / tr["tiles_per_launch"]
                                      if tr else None),
+                         "traffic_note": (f"ncu DRAM bytes of one launch at {tr['workload']}, scaled by query tiles"
+                                          if tr else "no capture for the current kernel source"),
                          "flops_per_launch": flops_step},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
