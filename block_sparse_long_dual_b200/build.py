@@ -21,7 +21,7 @@ BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsfa.so")
 
 SOURCES = ["api.cu", "scores.cu", "scores_noalloc.cu", "select.cu", "attn_simt.cu", "attn_tc.cu"]
-HEADERS = ["common.cuh", "kernels.h", "tc_ptx.cuh"]
+HEADERS = ["common.cuh", "kernels.h", "tc_ptx.cuh", "select_row.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -161,16 +161,49 @@ sfa_status sfa_workspace_layout(const sfa_shape* shape, int block, size_t offset
   return SFA_OK;
 }
 
-sfa_status sfa_block_scores(const sfa_shape* shape, const void* Q, const void* K, const sfa_rope* rope,
-                            int band_split, int block, unsigned flags, void* Q_rot, void* K_rot, float* probs,
-                            void* workspace, size_t workspace_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+struct FusedSelect {
+  int k;
+  float mass;
+  int* counts;
+  int* idx;
+  int kmax;
+};
+
+// Selection-rule checks shared by sfa_select and sfa_block_scores_select.
+sfa_status check_select(int nb, int k, float mass, unsigned flags, const int* counts, const int* idx, int kmax) {
+  if (counts == nullptr || idx == nullptr) return SFA_ERR_INVALID_ARG;
+  if (flags & ~kKnownFlags) return SFA_ERR_INVALID_ARG;
+  const int nforced = (flags & SFA_KEEP_SINK) && nb > 1 ? 2 : 1;
+  int need;
+  if (k >= 0) {
+    need = k + nforced < nb ? k + nforced : nb;
+  } else {
+    if (!(mass > 0.f && mass <= 1.f)) return SFA_ERR_INVALID_ARG;
+    need = nb;
+  }
+  if (kmax < need || kmax < 1) return SFA_ERR_INVALID_ARG;
+  return SFA_OK;
+}
+
+sfa_status run_block_scores(const sfa_shape* shape, const void* Q, const void* K, const sfa_rope* rope, int band_split,
+                            int block, unsigned flags, void* Q_rot, void* K_rot, float* probs, void* workspace,
+                            size_t workspace_bytes, void* stream, const FusedSelect* fused) {
   int nb = 0;
   sfa_status st = check_shape(shape, block, &nb);
   if (st != SFA_OK) return st;
   const int D = shape->head_dim;
-  if (Q == nullptr || K == nullptr || rope == nullptr || probs == nullptr) return SFA_ERR_INVALID_ARG;
+  if (Q == nullptr || K == nullptr || rope == nullptr || (probs == nullptr && fused == nullptr))
+    return SFA_ERR_INVALID_ARG;
   if (flags & ~kKnownFlags) return SFA_ERR_INVALID_ARG;
   if (band_split < 0 || band_split > D / 2) return SFA_ERR_INVALID_ARG;
+  if (fused != nullptr) {
+    st = check_select(nb, fused->k, fused->mass, flags, fused->counts, fused->idx, fused->kmax);
+    if (st != SFA_OK) return st;
+  }
   if (rope->apply && (rope->cos == nullptr || rope->sin == nullptr || Q_rot == nullptr || K_rot == nullptr))
     return SFA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || (rope->apply && (!aligned16(Q_rot) || !aligned16(K_rot) ||
@@ -206,7 +239,33 @@ sfa_status sfa_block_scores(const sfa_shape* shape, const void* Q, const void* K
   ScoreParams sp;
   sp.qbar = rp.qbar; sp.kbar = rp.kbar; sp.tau = tp.tau; sp.probs = probs;
   sp.B = rp.B; sp.Hq = rp.Hq; sp.Hkv = rp.Hkv; sp.nb = nb; sp.band_pairs = band_pairs;
+  sp.counts = fused ? fused->counts : nullptr;
+  sp.idx = fused ? fused->idx : nullptr;
+  sp.kmax = fused ? fused->kmax : 0;
+  sp.k = fused ? fused->k : 0;
+  sp.mass = fused ? (double)fused->mass : 0.0;
+  sp.flags = flags;
   return cuda_status(launch_block_score_softmax(sp, D, cs));
+}
+
+}  // namespace
+
+extern "C" {
+
+sfa_status sfa_block_scores(const sfa_shape* shape, const void* Q, const void* K, const sfa_rope* rope,
+                            int band_split, int block, unsigned flags, void* Q_rot, void* K_rot, float* probs,
+                            void* workspace, size_t workspace_bytes, void* stream) {
+  return run_block_scores(shape, Q, K, rope, band_split, block, flags, Q_rot, K_rot, probs, workspace,
+                          workspace_bytes, stream, nullptr);
+}
+
+sfa_status sfa_block_scores_select(const sfa_shape* shape, const void* Q, const void* K, const sfa_rope* rope,
+                                   int band_split, int block, unsigned flags, int k, float mass, void* Q_rot,
+                                   void* K_rot, float* probs, int* counts, int* idx, int kmax, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  const FusedSelect f{k, mass, counts, idx, kmax};
+  return run_block_scores(shape, Q, K, rope, band_split, block, flags, Q_rot, K_rot, probs, workspace,
+                          workspace_bytes, stream, &f);
 }
 
 sfa_status sfa_select(const sfa_shape* shape, int block, const float* probs, int k, float mass, unsigned flags,
@@ -214,17 +273,9 @@ sfa_status sfa_select(const sfa_shape* shape, int block, const float* probs, int
   int nb = 0;
   sfa_status st = check_shape(shape, block, &nb);
   if (st != SFA_OK) return st;
-  if (probs == nullptr || counts == nullptr || idx == nullptr) return SFA_ERR_INVALID_ARG;
-  if (flags & ~kKnownFlags) return SFA_ERR_INVALID_ARG;
-  const int nforced = (flags & SFA_KEEP_SINK) && nb > 1 ? 2 : 1;
-  int need;
-  if (k >= 0) {
-    need = k + nforced < nb ? k + nforced : nb;
-  } else {
-    if (!(mass > 0.f && mass <= 1.f)) return SFA_ERR_INVALID_ARG;
-    need = nb;
-  }
-  if (kmax < need || kmax < 1) return SFA_ERR_INVALID_ARG;
+  if (probs == nullptr) return SFA_ERR_INVALID_ARG;
+  st = check_select(nb, k, mass, flags, counts, idx, kmax);
+  if (st != SFA_OK) return st;
   SelectParams p;
   p.probs = probs; p.counts = counts; p.idx = idx;
   p.B = shape->batch; p.Hq = shape->heads_q; p.nb = nb; p.kmax = kmax;

@@ -35,9 +35,16 @@ struct ScoreParams {
   const double* qbar;
   const double* kbar;
   const double* tau;
-  float* probs;
+  float* probs;  // may be null when the selection is fused
   int B, Hq, Hkv, nb;
   int band_pairs;
+  // fused selection (counts != null): the rule of SelectParams
+  int* counts;
+  int* idx;
+  int kmax;
+  int k;
+  double mass;
+  unsigned flags;
 };
 
 struct SelectParams {

@@ -13,6 +13,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "select_row.cuh"
 
 namespace sfa {
 
@@ -294,7 +295,7 @@ __device__ __forceinline__ void dmma_8x8x4(double (&c)[2], double a, double b) {
                : "d"(a), "d"(b));
 }
 
-template <int RT, int D>
+template <int RT, int D, int NPL, bool FUSED>
 __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p) {
   constexpr int RTL = RT / 8;             // row tiles
   constexpr int CS = 256;                 // columns per step
@@ -402,8 +403,18 @@ __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p)
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
     const double inv = 1.0 / sum;
-    float* prow = p.probs + ((size_t)(b * p.Hq + h) * p.nb + i) * p.nb;
-    for (int jj = lane; jj < p.nb; jj += 32) prow[jj] = (jj <= i) ? (float)(srow[jj] * inv) : 0.f;
+    const size_t rowid = (size_t)(b * p.Hq + h) * p.nb + i;
+    if (p.probs != nullptr) {
+      float* prow = p.probs + rowid * p.nb;
+      for (int jj = lane; jj < p.nb; jj += 32) prow[jj] = (jj <= i) ? (float)(srow[jj] * inv) : 0.f;
+    }
+    if constexpr (FUSED) {
+      // Select on exactly the float32 probabilities the unfused path would write.
+      __syncwarp();
+      const int n = select_row_warp<NPL>([&](int j) { return (float)(srow[j] * inv); }, i, p.k, p.mass, p.flags,
+                                         p.idx + rowid * p.kmax, p.kmax);
+      if (lane == 0) p.counts[rowid] = n;
+    }
   }
 }
 
@@ -453,10 +464,10 @@ size_t score_smem_bytes(int nb, int D) {
   return ((size_t)RT * nb + (size_t)RT * (D + 4)) * sizeof(double);
 }
 
-template <int RT, int D>
+template <int RT, int D, int NPL, bool FUSED>
 static cudaError_t launch_score_t(const ScoreParams& p, cudaStream_t st) {
   const size_t smem = score_smem_bytes(p.nb, D);
-  auto kern = block_score_softmax_kernel<RT, D>;
+  auto kern = block_score_softmax_kernel<RT, D, NPL, FUSED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   dim3 grid((p.nb + RT - 1) / RT, p.Hq, p.B);
@@ -464,10 +475,23 @@ static cudaError_t launch_score_t(const ScoreParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+template <int D>
+static cudaError_t launch_score_d(const ScoreParams& p, cudaStream_t st) {
+  if (p.counts == nullptr) {
+    return score_rows_per_cta(p.nb) == 16 ? launch_score_t<16, D, 1, false>(p, st)
+                                          : launch_score_t<8, D, 1, false>(p, st);
+  }
+  if (p.nb <= 32) return launch_score_t<16, D, 1, true>(p, st);
+  if (p.nb <= 64) return launch_score_t<16, D, 2, true>(p, st);
+  if (p.nb <= 128) return launch_score_t<16, D, 4, true>(p, st);
+  if (p.nb <= 256) return launch_score_t<16, D, 8, true>(p, st);
+  if (p.nb <= 512) return launch_score_t<16, D, 16, true>(p, st);
+  if (p.nb <= 1024) return launch_score_t<16, D, 32, true>(p, st);
+  return launch_score_t<8, D, 64, true>(p, st);
+}
+
 cudaError_t launch_block_score_softmax(const ScoreParams& p, int D, cudaStream_t st) {
-  const int RT = score_rows_per_cta(p.nb);
-  if (RT == 16) return D == 128 ? launch_score_t<16, 128>(p, st) : launch_score_t<16, 64>(p, st);
-  return D == 128 ? launch_score_t<8, 128>(p, st) : launch_score_t<8, 64>(p, st);
+  return D == 128 ? launch_score_d<128>(p, st) : launch_score_d<64>(p, st);
 }
 
 }  // namespace sfa

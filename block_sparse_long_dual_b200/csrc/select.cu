@@ -1,33 +1,15 @@
 // Per-query-block selection of key blocks ("Prism: Spectral-Aware
-// Block-Sparse Attention" §1: attention runs over a chosen subset of blocks).
-//
-// One warp per row (b, h, i); the row's probabilities sit in registers (lane l
-// holds blocks l, l + 32, l + 64, ...).  Probabilities are >= 0, so their
-// float32 bit patterns order like the values; candidates carry their bit
-// pattern as a signed key and non-candidates (forced blocks, j > i) key -1.
-//
-// The kept candidates are a prefix of the order (probability desc, index asc).
-// Such a prefix is {key > T} plus the lowest-index entries of {key == T} for
-// one threshold key T, found by bisection over the 31-bit key range:
-//   top-k:  T = the largest key with #{key >= T} >= k; take k - #{key > T} ties.
-//   mass:   T = the smallest key with forced + sum_{key > T} p < mass (float64
-//           sums), i.e. the value of the last candidate added; ties are added
-//           in index order while the running sum stays below mass.
-// The kept set (forced blocks included) is written ascending, padded with -1.
+// Block-Sparse Attention" §1): one warp per row (b, h, i) running the shared
+// warp routine of select_row.cuh on the row's float32 probabilities.
 #include "common.cuh"
 #include "kernels.h"
+#include "select_row.cuh"
 
 namespace sfa {
 
 namespace {
 
 constexpr int kWarps = 8;
-
-__device__ __forceinline__ double warp_sum(double v) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  return v;
-}
 
 template <int NPL>
 __global__ void __launch_bounds__(kWarps * 32) select_kernel(SelectParams p) {
@@ -37,107 +19,9 @@ __global__ void __launch_bounds__(kWarps * 32) select_kernel(SelectParams p) {
   if (row >= nrows) return;
   const int i = (int)(row % p.nb);
   const float* prow = p.probs + row * p.nb;
-  const int f1 = ((p.flags & SFA_KEEP_SINK) && i > 0) ? 0 : -1;
-  const int nforced = f1 >= 0 ? 2 : 1;
-  const int nc = i + 1 - nforced;
-  const int tmax = i / 32 + 1;  // register slots that hold blocks <= i
-
-  int key[NPL];  // candidate: bit pattern of its probability (the value is __uint_as_float(key))
-#pragma unroll
-  for (int t = 0; t < NPL; ++t) {
-    const int j = t * 32 + lane;
-    int kk = -1;
-    if (t < tmax && j <= i && j != i && j != f1) kk = (int)__float_as_uint(__ldg(prow + j));
-    key[t] = kk;
-  }
-
-  int T = -1;       // threshold key; candidates with key > T are kept
-  int take_ties = 0;  // number of key == T candidates kept, lowest index first
-  if (p.k >= 0) {
-    if (p.k >= nc) {
-      T = -1;  // every candidate
-    } else if (p.k > 0) {
-      int lo = 0, hi = 0x7F800001;  // #{key >= lo} >= k, #{key >= hi} < k
-      while (hi - lo > 1) {
-        const int mid = lo + ((hi - lo) >> 1);
-        int c = 0;
-#pragma unroll
-        for (int t = 0; t < NPL; ++t) c += (t < tmax && key[t] >= mid) ? 1 : 0;
-        c = __reduce_add_sync(0xffffffffu, c);
-        if (c >= p.k) lo = mid; else hi = mid;
-      }
-      int g = 0;
-#pragma unroll
-      for (int t = 0; t < NPL; ++t) g += (t < tmax && key[t] > lo) ? 1 : 0;
-      g = __reduce_add_sync(0xffffffffu, g);
-      T = lo;
-      take_ties = p.k - g;
-    } else {
-      T = 0x7F800001;  // k = 0: no candidate
-    }
-  } else {
-    // Running sum starts with the forced blocks.
-    const double cum_forced = (double)prow[i] + (f1 >= 0 ? (double)prow[f1] : 0.0);
-    double all = 0.0;
-#pragma unroll
-    for (int t = 0; t < NPL; ++t) all += (t < tmax && key[t] >= 0) ? (double)__uint_as_float((unsigned)key[t]) : 0.0;
-    all = warp_sum(all);
-    if (cum_forced >= p.mass) {
-      T = 0x7F800001;  // nothing added
-    } else if (cum_forced + all < p.mass) {
-      T = -1;  // every candidate added
-    } else {
-      int lo = -1, hi = 0x7F800000;  // F(lo) >= mass, F(hi) < mass, F(U) = forced + sum_{key > U} p
-      while (hi - lo > 1) {
-        const int mid = lo + ((hi - lo) >> 1);
-        double s = 0.0;
-#pragma unroll
-        for (int t = 0; t < NPL; ++t) s += (t < tmax && key[t] > mid) ? (double)__uint_as_float((unsigned)key[t]) : 0.0;
-        s = warp_sum(s);
-        if (cum_forced + s < p.mass) hi = mid; else lo = mid;
-      }
-      // hi is the key of the last candidate added; add its ties in index order while below mass.
-      double sg = 0.0;
-      int e = 0;
-#pragma unroll
-      for (int t = 0; t < NPL; ++t) {
-        if (t < tmax && key[t] > hi) sg += (double)__uint_as_float((unsigned)key[t]);
-        if (t < tmax && key[t] == hi) ++e;
-      }
-      sg = cum_forced + warp_sum(sg);
-      e = __reduce_add_sync(0xffffffffu, e);
-      const double tv = (double)__uint_as_float((unsigned)hi);
-      int r = 0;
-      double run = sg;
-      while (r < e && run < p.mass) {
-        run += tv;
-        ++r;
-      }
-      T = hi;
-      take_ties = r;
-    }
-  }
-
-  // Ascending compaction of forced + kept candidates.
-  int* out = p.idx + row * p.kmax;
-  int pos = 0, ties = 0;
-  const unsigned lt = (1u << lane) - 1u;
-#pragma unroll
-  for (int t = 0; t < NPL; ++t) {
-    if (t < tmax) {
-      const int j = t * 32 + lane;
-      const bool tie = key[t] >= 0 && key[t] == T;
-      const unsigned tb = __ballot_sync(0xffffffffu, tie);
-      const bool keep_tie = tie && (ties + __popc(tb & lt)) < take_ties;
-      const bool keep = (j <= i) && (j == i || j == f1 || key[t] > T || keep_tie);
-      const unsigned kb = __ballot_sync(0xffffffffu, keep);
-      if (keep) out[pos + __popc(kb & lt)] = j;
-      pos += __popc(kb);
-      ties += __popc(tb);
-    }
-  }
-  for (int q = pos + lane; q < p.kmax; q += 32) out[q] = -1;
-  if (lane == 0) p.counts[row] = pos;
+  const int n = select_row_warp<NPL>([&](int j) { return __ldg(prow + j); }, i, p.k, p.mass, p.flags,
+                                     p.idx + row * p.kmax, p.kmax);
+  if (lane == 0) p.counts[row] = n;
 }
 
 template <int NPL>

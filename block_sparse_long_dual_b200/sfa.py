@@ -66,6 +66,10 @@ def load() -> ctypes.CDLL:
     lib.sfa_block_scores.restype = c_int
     lib.sfa_block_scores.argtypes = [POINTER(Shape), c_void_p, c_void_p, POINTER(Rope), c_int, c_int, c_uint,
                                      c_void_p, c_void_p, c_void_p, c_void_p, c_size_t, c_void_p]
+    lib.sfa_block_scores_select.restype = c_int
+    lib.sfa_block_scores_select.argtypes = [POINTER(Shape), c_void_p, c_void_p, POINTER(Rope), c_int, c_int, c_uint,
+                                            c_int, c_float, c_void_p, c_void_p, c_void_p, c_void_p, c_void_p,
+                                            c_int, c_void_p, c_size_t, c_void_p]
     lib.sfa_select.restype = c_int
     lib.sfa_select.argtypes = [POINTER(Shape), c_int, c_void_p, c_int, c_float, c_uint, c_void_p, c_void_p,
                                c_int, c_void_p]
@@ -175,6 +179,41 @@ def block_scores(Q, K, cos, sin, *, band_split: int, block: int, flags: int = 0,
     return (Q_rot if apply_rope else Q), (K_rot if apply_rope else K), probs, workspace
 
 
+def block_scores_select(Q, K, cos, sin, *, band_split: int, block: int, k: int | None = None,
+                        mass: float | None = None, flags: int = 0, apply_rope: bool = True, Q_rot=None, K_rot=None,
+                        probs=None, want_probs: bool = False, kmax: int | None = None, counts=None, idx=None,
+                        workspace=None, stream=None):
+    """sfa_block_scores_select: returns (Q_rot, K_rot, probs or None, counts, idx, workspace)."""
+    lib = load()
+    _cuda(Q, "Q"); _cuda(K, "K")
+    if (k is None) == (mass is None):
+        raise ValueError("give exactly one of k / mass")
+    shape = make_shape(Q, K)
+    nb = shape.seq_len // block if block > 0 else 0
+    if apply_rope:
+        Q_rot = torch.empty_like(Q) if Q_rot is None else Q_rot
+        K_rot = torch.empty_like(K) if K_rot is None else K_rot
+        _cuda(cos, "cos"); _cuda(sin, "sin")
+    if probs is None and want_probs:
+        probs = torch.empty((shape.batch, shape.heads_q, nb, nb), dtype=torch.float32, device=Q.device)
+    kmax = kmax_for(nb, k, flags) if kmax is None else kmax
+    if counts is None:
+        counts = torch.empty((shape.batch, shape.heads_q, nb), dtype=torch.int32, device=Q.device)
+    if idx is None:
+        idx = torch.empty((shape.batch, shape.heads_q, nb, max(kmax, 1)), dtype=torch.int32, device=Q.device)
+    if workspace is None:
+        workspace = torch.empty(max(workspace_bytes(shape, block), 256), dtype=torch.uint8, device=Q.device)
+    rope = Rope(cos.data_ptr() if apply_rope else None, sin.data_ptr() if apply_rope else None,
+                1 if apply_rope else 0)
+    _check(lib.sfa_block_scores_select(ctypes.byref(shape), _ptr(Q), _ptr(K), ctypes.byref(rope), band_split,
+                                       block, flags, -1 if k is None else int(k),
+                                       0.0 if mass is None else float(mass),
+                                       _ptr(Q_rot) if apply_rope else None, _ptr(K_rot) if apply_rope else None,
+                                       _ptr(probs), _ptr(counts), _ptr(idx), kmax, _ptr(workspace),
+                                       workspace.numel(), _stream(stream)), "sfa_block_scores_select")
+    return (Q_rot if apply_rope else Q), (K_rot if apply_rope else K), probs, counts, idx, workspace
+
+
 def kmax_for(nb: int, k: int | None, flags: int) -> int:
     if k is None:
         return nb
@@ -221,13 +260,16 @@ class PrismAttention:
     """The whole path for one layer shape: estimate -> select -> exact sparse attention.
 
     Buffers (rotated Q/K, probabilities, workspace, index lists, output) are
-    allocated once here; ``__call__`` only launches the library's kernels."""
+    allocated once here; ``__call__`` only launches the library's kernels.
+    With ``fused=True`` the estimate and the selection run as one call
+    (sfa_block_scores_select) and the block probabilities are not stored."""
 
     def __init__(self, *, batch, heads_q, heads_kv, seq_len, head_dim, dtype, block, rope_base, band_split,
-                 k=None, mass=None, flags=0, causal=True, device="cuda", with_lse=False):
+                 k=None, mass=None, flags=0, causal=True, device="cuda", with_lse=False, fused=False):
         tdt = torch.bfloat16 if dtype in ("bf16", torch.bfloat16) else torch.float32
         self.block, self.band_split, self.k, self.mass, self.flags, self.causal = (
             block, band_split, k, mass, flags, causal)
+        self.fused = fused
         self.shape = Shape(batch, heads_q, heads_kv, seq_len, head_dim, BF16 if tdt == torch.bfloat16 else F32)
         nb = seq_len // block
         self.nb = nb
@@ -236,7 +278,7 @@ class PrismAttention:
         self.cos, self.sin = rope_table(rope_base, seq_len, head_dim, device=dev)
         self.Q_rot = torch.empty((batch, heads_q, seq_len, head_dim), dtype=tdt, device=dev)
         self.K_rot = torch.empty((batch, heads_kv, seq_len, head_dim), dtype=tdt, device=dev)
-        self.probs = torch.empty((batch, heads_q, nb, nb), dtype=torch.float32, device=dev)
+        self.probs = None if fused else torch.empty((batch, heads_q, nb, nb), dtype=torch.float32, device=dev)
         self.workspace = torch.empty(workspace_bytes(self.shape, block), dtype=torch.uint8, device=dev)
         self.counts = torch.empty((batch, heads_q, nb), dtype=torch.int32, device=dev)
         self.idx = torch.empty((batch, heads_q, nb, self.kmax), dtype=torch.int32, device=dev)
@@ -249,6 +291,12 @@ class PrismAttention:
                      Q_rot=self.Q_rot, K_rot=self.K_rot, probs=self.probs, workspace=self.workspace,
                      stream=stream)
 
+    def scores_select(self, Q, K, stream=None):
+        block_scores_select(Q, K, self.cos, self.sin, band_split=self.band_split, block=self.block, k=self.k,
+                            mass=self.mass, flags=self.flags, Q_rot=self.Q_rot, K_rot=self.K_rot,
+                            probs=self.probs, kmax=self.kmax, counts=self.counts, idx=self.idx,
+                            workspace=self.workspace, stream=stream)
+
     def select(self, stream=None):
         select(self.probs, self.shape, block=self.block, k=self.k, mass=self.mass, flags=self.flags,
                kmax=self.kmax, counts=self.counts, idx=self.idx, stream=stream)
@@ -258,8 +306,11 @@ class PrismAttention:
                           causal=self.causal, O=self.O, lse=self.lse, status=self.status, stream=stream)
 
     def __call__(self, Q, K, V, stream=None):
-        self.scores(Q, K, stream)
-        self.select(stream)
+        if self.fused:
+            self.scores_select(Q, K, stream)
+        else:
+            self.scores(Q, K, stream)
+            self.select(stream)
         self.attend(V, stream)
         return self.O
 

@@ -140,6 +140,21 @@ sfa_status sfa_block_scores(const sfa_shape* shape, const void* Q, const void* K
                             size_t workspace_bytes, void* stream);
 
 /*
+ * sfa_block_scores_select: sfa_block_scores followed by sfa_select in one
+ * pass, the selection running on each row of block probabilities while it is
+ * still in shared memory (the same float32 values, so the same index lists as
+ * the two calls), so the probabilities need not be written to device memory:
+ * `probs` may be NULL.  Arguments as in sfa_block_scores and sfa_select (k >= 0
+ * top-k, else cumulative mass; counts [B, heads_q, nb], idx [B, heads_q, nb,
+ * kmax]).  Errors: the union of both calls' errors.
+ */
+sfa_status sfa_block_scores_select(const sfa_shape* shape, const void* Q, const void* K,
+                                   const sfa_rope* rope, int band_split, int block, unsigned flags,
+                                   int k, float mass, void* Q_rot, void* K_rot, float* probs,
+                                   int* counts, int* idx, int kmax, void* workspace,
+                                   size_t workspace_bytes, void* stream);
+
+/*
  * sfa_block_scores_noalloc - the same computation and outputs as
  * sfa_block_scores, for callers that cannot allocate device memory.
  * (The paper has no counterpart: this is a deployment convenience.)

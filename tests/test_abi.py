@@ -32,7 +32,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = declared_functions()
-    for required in ("sfa_block_scores", "sfa_select", "sfa_block_sparse_attn", "sfa_rope_table",
+    for required in ("sfa_block_scores", "sfa_select", "sfa_block_sparse_attn", "sfa_block_scores_select",
+                     "sfa_rope_table",
                      "sfa_block_scores_workspace", "sfa_workspace_layout", "sfa_status_string", "sfa_version"):
         assert required in names
 
@@ -71,6 +72,8 @@ def test_shape_validation(lib, shape, block, code):
     assert lib.sfa_block_scores(ctypes.byref(shape), dummy, dummy, ctypes.byref(rope), 16, block, 0, None, None,
                                 dummy, dummy, 1 << 30, None) == code
     assert lib.sfa_select(ctypes.byref(shape), block, dummy, 4, 0.0, 0, dummy, dummy, 64, None) == code
+    assert lib.sfa_block_scores_select(ctypes.byref(shape), dummy, dummy, ctypes.byref(rope), 16, block, 0, 4, 0.0,
+                                       None, None, None, dummy, dummy, 64, dummy, 1 << 30, None) == code
     assert lib.sfa_block_sparse_attn(ctypes.byref(shape), block, dummy, dummy, dummy, dummy, dummy, 8, 1, 0.0,
                                      dummy, None, None, None) == code
 
@@ -124,6 +127,32 @@ def test_argument_validation_before_launch(lib):
     assert lib.sfa_rope_table(0.0, 16, 64, d, d, None) == 1
     assert lib.sfa_rope_table(1e4, 16, 63, d, d, None) == 2
     assert lib.sfa_rope_table(1e4, 0, 64, d, d, None) == 2
+
+
+def test_fused_scores_select_validation(lib):
+    shape = S()  # nb = 8
+    d = ctypes.c_void_p(1 << 20)
+    rope = sfa.Rope(d, d, 1)
+    ws = lib.sfa_block_scores_workspace(ctypes.byref(shape), 128)
+    f = lib.sfa_block_scores_select
+    R = ctypes.byref(rope)
+    sh = ctypes.byref(shape)
+    # score-side errors: null Q, band_split, unknown flag, rope outputs, workspace
+    assert f(sh, None, d, R, 16, 128, 0, 4, 0.0, d, d, None, d, d, 5, d, ws, None) == 1
+    assert f(sh, d, d, R, 65, 128, 0, 4, 0.0, d, d, None, d, d, 5, d, ws, None) == 1
+    assert f(sh, d, d, R, 16, 128, 16, 4, 0.0, d, d, None, d, d, 6, d, ws, None) == 1
+    assert f(sh, d, d, R, 16, 128, 0, 4, 0.0, None, d, None, d, d, 5, d, ws, None) == 1
+    assert f(sh, d, d, R, 16, 128, 0, 4, 0.0, d, d, None, d, d, 5, d, ws - 1, None) == 5
+    # selection-side errors: null counts / idx, kmax too small, mass out of range
+    assert f(sh, d, d, R, 16, 128, 0, 4, 0.0, d, d, None, None, d, 5, d, ws, None) == 1
+    assert f(sh, d, d, R, 16, 128, 0, 4, 0.0, d, d, None, d, None, 5, d, ws, None) == 1
+    assert f(sh, d, d, R, 16, 128, 0, 4, 0.0, d, d, None, d, d, 4, d, ws, None) == 1
+    assert f(sh, d, d, R, 16, 128, 1, 4, 0.0, d, d, None, d, d, 5, d, ws, None) == 1
+    assert f(sh, d, d, R, 16, 128, 0, -1, 0.0, d, d, None, d, d, 8, d, ws, None) == 1
+    assert f(sh, d, d, R, 16, 128, 0, -1, 1.5, d, d, None, d, d, 8, d, ws, None) == 1
+    assert f(sh, d, d, R, 16, 128, 0, -1, 0.9, d, d, None, d, d, 7, d, ws, None) == 1
+    # probs may be NULL here, unlike sfa_block_scores
+    assert lib.sfa_block_scores(sh, d, d, R, 16, 128, 0, d, d, None, d, ws, None) == 1
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

@@ -108,3 +108,42 @@ def test_path_matches_oracle(w):
     assert rows.mean() > 0.9
     np.testing.assert_allclose(O[rows], ref.out[rows], rtol=0, atol=TOL_O[w.dtype])
     np.testing.assert_allclose(lse[rows], ref.lse[rows], rtol=0, atol=TOL_O[w.dtype])
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_fused_scores_select_matches(w):
+    """sfa_block_scores_select: the same index lists as sfa_block_scores + sfa_select
+    (bit for bit), with and without the probabilities stored, and the oracle's masks."""
+    Q, K, V = make_inputs(w, seed=1)
+    dev = torch.device("cuda")
+    kw = dict(batch=w.batch, heads_q=w.heads_q, heads_kv=w.heads_kv, seq_len=w.seq_len, head_dim=w.head_dim,
+              dtype=w.dtype, block=w.block, rope_base=w.rope_base, band_split=w.band_split, k=w.k, mass=w.mass,
+              flags=w.flags, device=dev)
+    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    sep = sfa.PrismAttention(**kw)
+    fused = sfa.PrismAttention(**kw, fused=True)
+    assert fused.probs is None
+    sep(Qd, Kd, Vd)
+    fused.idx.fill_(-7)
+    fused(Qd, Kd, Vd)
+    torch.cuda.synchronize()
+    assert torch.equal(sep.counts, fused.counts)
+    assert torch.equal(sep.idx, fused.idx)
+    assert torch.equal(sep.Q_rot, fused.Q_rot) and torch.equal(sep.K_rot, fused.K_rot)
+    assert torch.equal(sep.O, fused.O)
+    assert int(fused.status.item()) == 0
+
+    # probabilities requested from the fused call: identical to sfa_block_scores'
+    mass = None if w.mass is None else float(np.float32(w.mass))
+    _, _, P, counts, idx, _ = sfa.block_scores_select(Qd, Kd, sep.cos, sep.sin, band_split=w.band_split,
+                                                      block=w.block, k=w.k, mass=w.mass, flags=w.flags,
+                                                      want_probs=True)
+    torch.cuda.synchronize()
+    assert torch.equal(P, sep.probs)
+    assert torch.equal(counts, sep.counts) and torch.equal(idx, sep.idx)
+
+    cos, sin = po.rope_tables(w.rope_base, w.seq_len, w.head_dim)
+    sc = po.prism_scores(to_np(Q), to_np(K), w.block, w.band_split, w.flags, (cos, sin))
+    sel = po.select_blocks(sc.probs, w.flags, k=w.k, mass=mass)
+    stats, _ = compare_masks(sel, sc.probs, fused.counts, fused.idx, mass)
+    assert stats["mismatches"] == 0, stats["bad_rows"][:5]
