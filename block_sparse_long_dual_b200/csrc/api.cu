@@ -204,7 +204,8 @@ sfa_status run_block_scores(const sfa_shape* shape, const void* Q, const void* K
     st = check_select(nb, fused->k, fused->mass, flags, fused->counts, fused->idx, fused->kmax);
     if (st != SFA_OK) return st;
   }
-  if (rope->apply && (rope->cos == nullptr || rope->sin == nullptr || Q_rot == nullptr || K_rot == nullptr))
+  // Q_rot may be NULL: the rotated Q is then not stored (sfa_block_sparse_attn_rope rotates it on load).
+  if (rope->apply && (rope->cos == nullptr || rope->sin == nullptr || K_rot == nullptr))
     return SFA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || (rope->apply && (!aligned16(Q_rot) || !aligned16(K_rot) ||
                                                          !aligned16(rope->cos) || !aligned16(rope->sin))))
@@ -283,9 +284,13 @@ sfa_status sfa_select(const sfa_shape* shape, int block, const float* probs, int
   return cuda_status(launch_select(p, as_stream(stream)));
 }
 
-sfa_status sfa_block_sparse_attn(const sfa_shape* shape, int block, const void* Q, const void* K, const void* V,
-                                 const int* counts, const int* idx, int kmax, int causal, float scale, void* O,
-                                 float* lse, int* status_word, void* stream) {
+}  // extern "C"
+
+namespace {
+
+sfa_status run_attn(const sfa_shape* shape, int block, const void* Q, const void* K, const void* V,
+                    const sfa_rope* rope, const int* counts, const int* idx, int kmax, int causal, float scale,
+                    void* O, float* lse, int* status_word, void* stream) {
   int nb = 0;
   sfa_status st = check_shape(shape, block, &nb);
   if (st != SFA_OK) return st;
@@ -293,9 +298,14 @@ sfa_status sfa_block_sparse_attn(const sfa_shape* shape, int block, const void* 
     return SFA_ERR_INVALID_ARG;
   if (kmax < 1 || !(isfinite(scale))) return SFA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || !aligned16(O)) return SFA_ERR_INVALID_ARG;
+  const bool rot = rope != nullptr && rope->apply;
+  if (rot && (rope->cos == nullptr || rope->sin == nullptr || !aligned16(rope->cos) || !aligned16(rope->sin)))
+    return SFA_ERR_INVALID_ARG;
   const int D = shape->head_dim;
   AttnParams p;
   p.Q = Q; p.K = K; p.V = V; p.counts = counts; p.idx = idx; p.O = O; p.lse = lse; p.status = status_word;
+  p.rope_cos = rot ? rope->cos : nullptr;
+  p.rope_sin = rot ? rope->sin : nullptr;
   p.B = shape->batch; p.Hq = shape->heads_q; p.Hkv = shape->heads_kv; p.L = shape->seq_len;
   p.block = block; p.nb = nb; p.kmax = kmax; p.causal = causal ? 1 : 0;
   p.scale = scale > 0.f ? scale : (float)(1.0 / sqrt((double)D));
@@ -308,6 +318,24 @@ sfa_status sfa_block_sparse_attn(const sfa_shape* shape, int block, const void* 
     return cuda_status(launch_attn_tcgen05(p, tq, tk, tv, cs));
   }
   return cuda_status(launch_attn_simt(p, shape->dtype, D, cs));
+}
+
+}  // namespace
+
+extern "C" {
+
+sfa_status sfa_block_sparse_attn(const sfa_shape* shape, int block, const void* Q, const void* K, const void* V,
+                                 const int* counts, const int* idx, int kmax, int causal, float scale, void* O,
+                                 float* lse, int* status_word, void* stream) {
+  return run_attn(shape, block, Q, K, V, nullptr, counts, idx, kmax, causal, scale, O, lse, status_word, stream);
+}
+
+sfa_status sfa_block_sparse_attn_rope(const sfa_shape* shape, int block, const void* Q, const sfa_rope* rope,
+                                      const void* K_rot, const void* V, const int* counts, const int* idx, int kmax,
+                                      int causal, float scale, void* O, float* lse, int* status_word,
+                                      void* stream) {
+  if (rope == nullptr || !rope->apply) return SFA_ERR_INVALID_ARG;
+  return run_attn(shape, block, Q, K_rot, V, rope, counts, idx, kmax, causal, scale, O, lse, status_word, stream);
 }
 
 }  // extern "C"

@@ -54,10 +54,28 @@ __global__ void __launch_bounds__(BLK * 4) attn_simt_kernel(AttnParams p) {
   float q[DP], o[DP];
   {
     const T* qp = static_cast<const T*>(p.Q) + qrow * D + part * DP;
+    // RoPE on load: dims [part DP, +DP) pair with the other half's dims (+-d/2).
+    const bool rot = p.rope_cos != nullptr;
+    const bool upper = part >= 2;
+    const T* pp = static_cast<const T*>(p.Q) + qrow * D + (part ^ 2) * DP;
+    const size_t tpos = (size_t)i * BLK + r;
+    const int m0 = (part & 1) * DP;  // first rotary pair index of this thread's dims
 #pragma unroll
     for (int d = 0; d < DP; d += 8) {
       float v[8];
       load8(qp + d, v);
+      if (rot) {
+        float w[8], c[8], sn[8];
+        load8(pp + d, w);
+        load8(p.rope_cos + tpos * (D / 2) + m0 + d, c);
+        load8(p.rope_sin + tpos * (D / 2) + m0 + d, sn);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          float lo, hi;
+          if (upper) rope_pair(w[e], v[e], c[e], sn[e], lo, hi); else rope_pair(v[e], w[e], c[e], sn[e], lo, hi);
+          v[e] = round_as(upper ? hi : lo, T());
+        }
+      }
 #pragma unroll
       for (int e = 0; e < 8; ++e) { q[d + e] = v[e] * p.scale; o[d + e] = 0.f; }
     }

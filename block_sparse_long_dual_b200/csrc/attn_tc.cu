@@ -51,7 +51,8 @@ __host__ __device__ constexpr uint32_t off_v(int t) { return 4 * kTile + t * kTi
 constexpr uint32_t OFF_BAR = 6 * kTile;
 // Barriers, two of each (one per tile) except DRAIN.
 enum { B_Q = 0, B_KF = 2, B_VF = 4, B_KE = 6, B_VE = 8, B_SF = 10, B_PF = 12, B_OD = 14, B_X = 16, B_DRAIN = 20,
-       NBAR = 21 };  // B_X: [tile][parity] row-max / row-sum exchange of the two column halves
+       B_QR = 21, NBAR = 22 };  // B_X: [tile][parity] row-max / row-sum exchange of the two column halves;
+                                // B_QR: both Q tiles rotated in shared memory (RoPE on load)
 constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
 constexpr uint32_t OFF_XCHG = OFF_MISC + 32;         // [2 tiles][2 parities][2 halves][128 rows] float
 constexpr int kMaxList = 2048;                       // nb <= 2048, so a valid list has <= 2048 entries
@@ -124,6 +125,75 @@ __device__ Tile decode_tile(const AttnParams& p, int t) {
   return x;
 }
 
+// RoPE on load: the 512 softmax threads rotate the CTA's Q tiles in shared
+// memory once their TMA copies have landed (bounded waits on the tiles' B_Q
+// barriers); returns false if a wait gave up.  Work unit = (row, 16-byte
+// chunk c) of a tile: chunk c of box 0 holds dims [8c, 8c + 8) and the same
+// offset of box 1 holds their rotary partners [64 + 8c, 64 + 8c + 8) (chunk c of
+// row r is stored at chunk c ^ (r & 7) of the 128-byte row).  Thread st takes
+// chunk st & 7 of rows st / 8 and st / 8 + 64, so a warp touches four whole
+// rows: conflict-free in shared memory, and each row's table entries are one
+// contiguous 256-byte run.  The two tiles usually share the query block (two
+// heads of a GQA group), so the table entries are fetched once, before the
+// waits, and their latency hides behind the copies.  Kept out of line: it runs
+// once per CTA and must not add to the register pressure of the softmax loop.
+__device__ __noinline__ bool rope_q_on_load(volatile int* abort_flag, int* status, uint32_t bar_q0,
+                                            unsigned char* sm, const float* cos_t, const float* sin_t, int i0,
+                                            int i1, int n0, int n1, int st) {
+  Ctx cx;
+  cx.sbase = 0;
+  cx.abort_flag = abort_flag;
+  cx.status = status;
+  const int c = st & 7;
+  const bool two = n0 > 0 && n1 > 0 && i1 != i0;  // tiles at different query blocks need two table slices
+  const int ia = n0 > 0 ? i0 : i1;
+  float ca[2][8], sa[2][8], cb[2][8], sb[2][8];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int row = (st >> 3) + 64 * k;
+    load8(cos_t + ((size_t)ia * 128 + row) * 64 + c * 8, ca[k]);
+    load8(sin_t + ((size_t)ia * 128 + row) * 64 + c * 8, sa[k]);
+    if (two) {
+      load8(cos_t + ((size_t)i1 * 128 + row) * 64 + c * 8, cb[k]);
+      load8(sin_t + ((size_t)i1 * 128 + row) * 64 + c * 8, sb[k]);
+    }
+  }
+  bool ok = true;
+  if (n0 > 0) ok = wait_bar(cx, bar_q0, 0);
+  if (ok && n1 > 0) ok = wait_bar(cx, bar_q0 + 8, 0);  // B_Q + 1
+  if (!__all_sync(0xffffffffu, ok)) return false;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    if ((t == 0 ? n0 : n1) == 0) continue;
+    const bool use_b = t == 1 && two;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int row = (st >> 3) + 64 * k;
+      unsigned char* rp = sm + off_q(t) + row * 128 + ((c ^ (row & 7)) << 4);
+      uint4* plo = reinterpret_cast<uint4*>(rp);
+      uint4* phi = reinterpret_cast<uint4*>(rp + kSub);
+      const uint4 ulo = *plo, uhi = *phi;
+      const uint32_t wl[4] = {ulo.x, ulo.y, ulo.z, ulo.w}, wh[4] = {uhi.x, uhi.y, uhi.z, uhi.w};
+      uint32_t ol[4], oh[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float c0 = use_b ? cb[k][2 * e] : ca[k][2 * e], s0 = use_b ? sb[k][2 * e] : sa[k][2 * e];
+        const float c1 = use_b ? cb[k][2 * e + 1] : ca[k][2 * e + 1];
+        const float s1 = use_b ? sb[k][2 * e + 1] : sa[k][2 * e + 1];
+        float l0, l1, h0, h1;
+        rope_pair(__uint_as_float(wl[e] << 16), __uint_as_float(wh[e] << 16), c0, s0, l0, h0);
+        rope_pair(__uint_as_float(wl[e] & 0xFFFF0000u), __uint_as_float(wh[e] & 0xFFFF0000u), c1, s1, l1, h1);
+        ol[e] = pack_bf16x2(l0, l1);
+        oh[e] = pack_bf16x2(h0, h1);
+      }
+      *plo = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+      *phi = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+    }
+  }
+  tc::fence_proxy_async_smem();  // the generic-proxy writes become visible to the MMAs
+  return true;
+}
+
 }  // namespace
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -170,7 +240,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
       *cx.abort_flag = 0;
       for (int k = 0; k < NBAR; ++k)
-        tc::mbar_init(cx.bar(k), (k == B_PF || k == B_PF + 1 || (k >= B_X && k < B_X + 4)) ? 256 : 1);
+        tc::mbar_init(cx.bar(k), k == B_QR ? 512
+                                 : (k == B_PF || k == B_PF + 1 || (k >= B_X && k < B_X + 4)) ? 256 : 1);
       tc::fence_mbar_init();
     }
   } else if (warp == kProducerWarp && lane == 0) {
@@ -243,12 +314,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0 && nmax > 0) {
       const uint32_t id_qk = tc::idesc_bf16_f32(128, 128, false);
       const uint32_t id_pv = tc::idesc_bf16_f32(128, 128, true);
+      const bool rot = p.rope_cos != nullptr;  // Q_t ready: landed (B_Q + t), or both landed and rotated (B_QR)
       bool ok = true;
       // S_t(0) for both tiles.
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
         if (!ok || tl[t].n == 0) continue;
-        if (!wait_bar(cx, cx.bar(B_Q + t), 0) || !wait_bar(cx, cx.bar(B_KF + t), 0)) { ok = false; break; }
+        if (!wait_bar(cx, cx.bar(rot ? B_QR : B_Q + t), 0) || !wait_bar(cx, cx.bar(B_KF + t), 0)) {
+          ok = false;
+          break;
+        }
         tc::tc_fence_after();
         const uint32_t sQ = cx.sbase + off_q(t), sK = cx.sbase + off_k(t);
 #pragma unroll
@@ -327,7 +402,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float sl2 = p.scale * 1.4426950408889634f;
     float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
     bool ok = true;
-    for (int it = 0; it < x.n; ++it) {
+    if (p.rope_cos != nullptr && nmax > 0) {
+      // RoPE on load: all 512 softmax threads rotate both Q tiles, then one arrival each on B_QR.
+      ok = rope_q_on_load(cx.abort_flag, cx.status, cx.bar(B_Q), sm, p.rope_cos, p.rope_sin, tl[0].i, tl[1].i,
+                          tl[0].n, tl[1].n, warp * 32 + lane);
+      tc::mbar_arrive(cx.bar(B_QR));
+    }
+    for (int it = 0; ok && it < x.n; ++it) {
       ok = __all_sync(0xffffffffu, wait_bar(cx, cx.bar(B_SF + t), it & 1));
       if (!ok) break;
       tc::tc_fence_after();

@@ -71,6 +71,21 @@ __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
   *reinterpret_cast<uint4*>(p) = u;
 }
 
+// Rotate-half RoPE of one pair (x_m, x_{m + d/2}) by the float32 table entry
+// (c, s) of its position and frequency.  Every kernel that rotates Q or K uses
+// this one routine, so a value rotated on load equals the stored rotated copy
+// bit for bit.
+__device__ __forceinline__ void rope_pair(float a, float b, float c, float s, float& lo, float& hi) {
+  lo = fmaf(a, c, -(b * s));
+  hi = fmaf(b, c, a * s);
+}
+
+// Round to the storage type and back (the value a rotated copy would hold).
+__device__ __forceinline__ float round_as(float x, float) { return x; }
+__device__ __forceinline__ float round_as(float x, __nv_bfloat16) {
+  return __bfloat162float(__float2bfloat16_rn(x));
+}
+
 // First error wins; 0 means ok.
 __device__ __forceinline__ void report(int* status_word, int code) {
   if (status_word != nullptr) atomicCAS(status_word, 0, code);

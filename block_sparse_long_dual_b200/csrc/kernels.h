@@ -66,6 +66,8 @@ struct AttnParams {
   void* O;
   float* lse;
   int* status;
+  const float* rope_cos;  // non-null: Q is pre-RoPE and is rotated on load with these [L, d/2] tables
+  const float* rope_sin;
   int B, Hq, Hkv, L, block, nb, kmax;
   int causal;
   float scale;  // softmax scale (natural-log units)

@@ -121,7 +121,8 @@ __global__ void __launch_bounds__(256, 1) rope_pool_energy_kernel(RopePoolParams
     const int hh = is_q ? head : head - p.Hq;
     const int H = is_q ? p.Hq : p.Hkv;
     const size_t row0 = ((size_t)(b * H + hh) * p.L) + (size_t)j * BLK;
-    T* xr = p.write_rot ? static_cast<T*>(is_q ? p.Qr : p.Kr) + row0 * D : nullptr;
+    void* xdst = p.write_rot ? (is_q ? p.Qr : p.Kr) : nullptr;  // Qr may be NULL: Q rotated on load later
+    T* xr = xdst != nullptr ? static_cast<T*>(xdst) + row0 * D : nullptr;
     const T* xs = stage_ptr(st);
 
     float slo[8], shi[8];
@@ -136,11 +137,7 @@ __global__ void __launch_bounds__(256, 1) rope_pool_energy_kernel(RopePoolParams
       load8_smem(xs + (size_t)t * D + D / 2 + c * 8, hi);
       if (p.apply) {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float a = lo[e], bb = hi[e];
-          lo[e] = fmaf(a, csv[ps][e], -bb * snv[ps][e]);
-          hi[e] = fmaf(bb, csv[ps][e], a * snv[ps][e]);
-        }
+        for (int e = 0; e < 8; ++e) rope_pair(lo[e], hi[e], csv[ps][e], snv[ps][e], lo[e], hi[e]);
         if (xr != nullptr) {
           store8(xr + (size_t)t * D + c * 8, lo);
           store8(xr + (size_t)t * D + D / 2 + c * 8, hi);

@@ -77,6 +77,10 @@ def load() -> ctypes.CDLL:
     lib.sfa_block_sparse_attn.argtypes = [POINTER(Shape), c_int, c_void_p, c_void_p, c_void_p, c_void_p,
                                           c_void_p, c_int, c_int, c_float, c_void_p, c_void_p, c_void_p,
                                           c_void_p]
+    lib.sfa_block_sparse_attn_rope.restype = c_int
+    lib.sfa_block_sparse_attn_rope.argtypes = [POINTER(Shape), c_int, c_void_p, POINTER(Rope), c_void_p, c_void_p,
+                                               c_void_p, c_void_p, c_int, c_int, c_float, c_void_p, c_void_p,
+                                               c_void_p, c_void_p]
     _lib = lib
     return lib
 
@@ -156,13 +160,17 @@ def workspace_views(ws: torch.Tensor, shape: Shape, block: int):
 
 
 def block_scores(Q, K, cos, sin, *, band_split: int, block: int, flags: int = 0, apply_rope: bool = True,
-                 Q_rot=None, K_rot=None, probs=None, workspace=None, stream=None):
-    """sfa_block_scores: returns (Q_rot, K_rot, probs, workspace)."""
+                 Q_rot=None, K_rot=None, probs=None, workspace=None, store_q_rot: bool = True, stream=None):
+    """sfa_block_scores: returns (Q_rot, K_rot, probs, workspace).
+
+    ``store_q_rot=False`` passes a NULL Q_rot (the rotated Q is not written; Q_rot is returned as None)."""
     lib = load()
     _cuda(Q, "Q"); _cuda(K, "K")
     shape = make_shape(Q, K)
     nb = shape.seq_len // block if block > 0 else 0
-    if apply_rope:
+    if apply_rope and not store_q_rot:
+        Q_rot = None
+    elif apply_rope:
         Q_rot = torch.empty_like(Q) if Q_rot is None else Q_rot
         K_rot = torch.empty_like(K) if K_rot is None else K_rot
         _cuda(cos, "cos"); _cuda(sin, "sin")
@@ -182,7 +190,7 @@ def block_scores(Q, K, cos, sin, *, band_split: int, block: int, flags: int = 0,
 def block_scores_select(Q, K, cos, sin, *, band_split: int, block: int, k: int | None = None,
                         mass: float | None = None, flags: int = 0, apply_rope: bool = True, Q_rot=None, K_rot=None,
                         probs=None, want_probs: bool = False, kmax: int | None = None, counts=None, idx=None,
-                        workspace=None, stream=None):
+                        workspace=None, store_q_rot: bool = True, stream=None):
     """sfa_block_scores_select: returns (Q_rot, K_rot, probs or None, counts, idx, workspace)."""
     lib = load()
     _cuda(Q, "Q"); _cuda(K, "K")
@@ -190,7 +198,9 @@ def block_scores_select(Q, K, cos, sin, *, band_split: int, block: int, k: int |
         raise ValueError("give exactly one of k / mass")
     shape = make_shape(Q, K)
     nb = shape.seq_len // block if block > 0 else 0
-    if apply_rope:
+    if apply_rope and not store_q_rot:
+        Q_rot = None
+    elif apply_rope:
         Q_rot = torch.empty_like(Q) if Q_rot is None else Q_rot
         K_rot = torch.empty_like(K) if K_rot is None else K_rot
         _cuda(cos, "cos"); _cuda(sin, "sin")
@@ -256,27 +266,51 @@ def block_sparse_attn(Q, K, V, counts, idx, *, block: int, causal: bool = True, 
     return O
 
 
+def block_sparse_attn_rope(Q, cos, sin, K_rot, V, counts, idx, *, block: int, causal: bool = True,
+                           scale: float = 0.0, O=None, lse=None, status=None, stream=None):
+    """sfa_block_sparse_attn_rope: Q pre-RoPE (rotated on load with the cos/sin tables); returns O."""
+    lib = load()
+    for t, n in ((Q, "Q"), (cos, "cos"), (sin, "sin"), (K_rot, "K_rot"), (V, "V"), (counts, "counts"),
+                 (idx, "idx")):
+        _cuda(t, n)
+    shape = make_shape(Q, K_rot)
+    if V.shape != K_rot.shape or V.dtype != K_rot.dtype:
+        raise ValueError("V must match K_rot")
+    O = torch.empty_like(Q) if O is None else O
+    rope = Rope(cos.data_ptr(), sin.data_ptr(), 1)
+    _check(lib.sfa_block_sparse_attn_rope(ctypes.byref(shape), block, _ptr(Q), ctypes.byref(rope), _ptr(K_rot),
+                                          _ptr(V), _ptr(counts), _ptr(idx), idx.shape[-1], 1 if causal else 0,
+                                          float(scale), _ptr(O), _ptr(lse), _ptr(status), _stream(stream)),
+           "sfa_block_sparse_attn_rope")
+    return O
+
+
 class PrismAttention:
     """The whole path for one layer shape: estimate -> select -> exact sparse attention.
 
     Buffers (rotated Q/K, probabilities, workspace, index lists, output) are
     allocated once here; ``__call__`` only launches the library's kernels.
     With ``fused=True`` the estimate and the selection run as one call
-    (sfa_block_scores_select) and the block probabilities are not stored."""
+    (sfa_block_scores_select) and the block probabilities are not stored.
+    With ``rope_on_load=True`` the rotated Q is not stored: the attention
+    (sfa_block_sparse_attn_rope) rotates Q tiles as it loads them."""
 
     def __init__(self, *, batch, heads_q, heads_kv, seq_len, head_dim, dtype, block, rope_base, band_split,
-                 k=None, mass=None, flags=0, causal=True, device="cuda", with_lse=False, fused=False):
+                 k=None, mass=None, flags=0, causal=True, device="cuda", with_lse=False, fused=False,
+                 rope_on_load=False):
         tdt = torch.bfloat16 if dtype in ("bf16", torch.bfloat16) else torch.float32
         self.block, self.band_split, self.k, self.mass, self.flags, self.causal = (
             block, band_split, k, mass, flags, causal)
         self.fused = fused
+        self.rope_on_load = rope_on_load
         self.shape = Shape(batch, heads_q, heads_kv, seq_len, head_dim, BF16 if tdt == torch.bfloat16 else F32)
         nb = seq_len // block
         self.nb = nb
         self.kmax = kmax_for(nb, k, flags)
         dev = torch.device(device)
         self.cos, self.sin = rope_table(rope_base, seq_len, head_dim, device=dev)
-        self.Q_rot = torch.empty((batch, heads_q, seq_len, head_dim), dtype=tdt, device=dev)
+        self.Q_rot = None if rope_on_load else torch.empty((batch, heads_q, seq_len, head_dim), dtype=tdt,
+                                                           device=dev)
         self.K_rot = torch.empty((batch, heads_kv, seq_len, head_dim), dtype=tdt, device=dev)
         self.probs = None if fused else torch.empty((batch, heads_q, nb, nb), dtype=torch.float32, device=dev)
         self.workspace = torch.empty(workspace_bytes(self.shape, block), dtype=torch.uint8, device=dev)
@@ -289,21 +323,28 @@ class PrismAttention:
     def scores(self, Q, K, stream=None):
         block_scores(Q, K, self.cos, self.sin, band_split=self.band_split, block=self.block, flags=self.flags,
                      Q_rot=self.Q_rot, K_rot=self.K_rot, probs=self.probs, workspace=self.workspace,
-                     stream=stream)
+                     store_q_rot=not self.rope_on_load, stream=stream)
 
     def scores_select(self, Q, K, stream=None):
         block_scores_select(Q, K, self.cos, self.sin, band_split=self.band_split, block=self.block, k=self.k,
                             mass=self.mass, flags=self.flags, Q_rot=self.Q_rot, K_rot=self.K_rot,
                             probs=self.probs, kmax=self.kmax, counts=self.counts, idx=self.idx,
-                            workspace=self.workspace, stream=stream)
+                            workspace=self.workspace, store_q_rot=not self.rope_on_load, stream=stream)
 
     def select(self, stream=None):
         select(self.probs, self.shape, block=self.block, k=self.k, mass=self.mass, flags=self.flags,
                kmax=self.kmax, counts=self.counts, idx=self.idx, stream=stream)
 
-    def attend(self, V, stream=None):
-        block_sparse_attn(self.Q_rot, self.K_rot, V, self.counts, self.idx, block=self.block,
-                          causal=self.causal, O=self.O, lse=self.lse, status=self.status, stream=stream)
+    def attend(self, V, Q=None, stream=None):
+        """Attention over the selection; ``Q`` (pre-RoPE) is needed only with rope_on_load."""
+        if self.rope_on_load:
+            if Q is None:
+                raise ValueError("rope_on_load: attend() needs the pre-RoPE Q")
+            block_sparse_attn_rope(Q, self.cos, self.sin, self.K_rot, V, self.counts, self.idx, block=self.block,
+                                   causal=self.causal, O=self.O, lse=self.lse, status=self.status, stream=stream)
+        else:
+            block_sparse_attn(self.Q_rot, self.K_rot, V, self.counts, self.idx, block=self.block,
+                              causal=self.causal, O=self.O, lse=self.lse, status=self.status, stream=stream)
 
     def __call__(self, Q, K, V, stream=None):
         if self.fused:
@@ -311,7 +352,7 @@ class PrismAttention:
         else:
             self.scores(Q, K, stream)
             self.select(stream)
-        self.attend(V, stream)
+        self.attend(V, Q, stream)
         return self.O
 
     def run_host(self, Q_host, K_host, V_host, O_host, dev_in=None, stream=None):

@@ -113,6 +113,8 @@ sfa_status sfa_workspace_layout(const sfa_shape* shape, int block, size_t offset
  * when rope->apply, else already rotated.  With rope->apply the rotated
  * tensors are written to Q_rot / K_rot (same shape and dtype, rounded to
  * nearest even); they are the Q and K the attention call should read.
+ * Q_rot may be NULL: the rotated Q is then not stored, and the attention runs
+ * through sfa_block_sparse_attn_rope, which rotates Q tiles as it loads them.
  *
  * Per (batch, Q head, band b in {H, L}), with band H = rotary pairs
  * m < band_split (dims m and m + d/2), band L = the other dims:
@@ -228,6 +230,24 @@ sfa_status sfa_block_sparse_attn(const sfa_shape* shape, int block, const void* 
                                  const void* V, const int* counts, const int* idx, int kmax,
                                  int causal, float scale, void* O, float* lse, int* status_word,
                                  void* stream);
+
+/*
+ * sfa_block_sparse_attn with RoPE applied to Q on load (Prism §5: the rotated
+ * Q is used only by this call, so it need not make a round trip through
+ * device memory).  Q is the pre-RoPE query tensor; rope->cos / rope->sin the
+ * [L, d/2] float32 tables of sfa_rope_table (rope->apply must be nonzero);
+ * K_rot the rotated keys written by sfa_block_scores.  Each Q tile is rotated
+ * with the same float32 arithmetic and rounding to the storage dtype as
+ * sfa_block_scores' Q_rot, so O and lse equal those of
+ * sfa_block_sparse_attn(Q_rot, K_rot, V) bit for bit.  Other arguments,
+ * layouts and errors as sfa_block_sparse_attn; SFA_ERR_INVALID_ARG also for a
+ * missing or misaligned table.
+ */
+sfa_status sfa_block_sparse_attn_rope(const sfa_shape* shape, int block, const void* Q,
+                                      const sfa_rope* rope, const void* K_rot, const void* V,
+                                      const int* counts, const int* idx, int kmax, int causal,
+                                      float scale, void* O, float* lse, int* status_word,
+                                      void* stream);
 
 #ifdef __cplusplus
 }

@@ -33,6 +33,7 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("sfa_block_scores", "sfa_select", "sfa_block_sparse_attn", "sfa_block_scores_select",
+                     "sfa_block_sparse_attn_rope",
                      "sfa_rope_table",
                      "sfa_block_scores_workspace", "sfa_workspace_layout", "sfa_status_string", "sfa_version"):
         assert required in names
@@ -102,7 +103,7 @@ def test_argument_validation_before_launch(lib):
     assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 65, 128, 0, d, d, d, d, ws, None) == 1
     assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), -1, 128, 0, d, d, d, d, ws, None) == 1
     assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 16, d, d, d, d, ws, None) == 1
-    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 0, None, d, d, d, ws, None) == 1
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 0, d, None, d, d, ws, None) == 1  # no K_rot
     # misaligned pointers
     assert bs(ctypes.byref(shape), ctypes.c_void_p((1 << 20) + 2), d, ctypes.byref(rope), 16, 128, 0, d, d, d, d,
               ws, None) == 1
@@ -141,7 +142,7 @@ def test_fused_scores_select_validation(lib):
     assert f(sh, None, d, R, 16, 128, 0, 4, 0.0, d, d, None, d, d, 5, d, ws, None) == 1
     assert f(sh, d, d, R, 65, 128, 0, 4, 0.0, d, d, None, d, d, 5, d, ws, None) == 1
     assert f(sh, d, d, R, 16, 128, 16, 4, 0.0, d, d, None, d, d, 6, d, ws, None) == 1
-    assert f(sh, d, d, R, 16, 128, 0, 4, 0.0, None, d, None, d, d, 5, d, ws, None) == 1
+    assert f(sh, d, d, R, 16, 128, 0, 4, 0.0, d, None, None, d, d, 5, d, ws, None) == 1  # no K_rot
     assert f(sh, d, d, R, 16, 128, 0, 4, 0.0, d, d, None, d, d, 5, d, ws - 1, None) == 5
     # selection-side errors: null counts / idx, kmax too small, mass out of range
     assert f(sh, d, d, R, 16, 128, 0, 4, 0.0, d, d, None, None, d, 5, d, ws, None) == 1
@@ -153,6 +154,23 @@ def test_fused_scores_select_validation(lib):
     assert f(sh, d, d, R, 16, 128, 0, -1, 0.9, d, d, None, d, d, 7, d, ws, None) == 1
     # probs may be NULL here, unlike sfa_block_scores
     assert lib.sfa_block_scores(sh, d, d, R, 16, 128, 0, d, d, None, d, ws, None) == 1
+
+
+def test_attn_rope_validation(lib):
+    shape = S()
+    d = ctypes.c_void_p(1 << 20)
+    f = lib.sfa_block_sparse_attn_rope
+    sh = ctypes.byref(shape)
+    good = sfa.Rope(d, d, 1)
+    assert f(sh, 128, d, None, d, d, d, d, 8, 1, 0.0, d, None, None, None) == 1            # no tables
+    assert f(sh, 128, d, ctypes.byref(sfa.Rope(d, d, 0)), d, d, d, d, 8, 1, 0.0, d, None, None, None) == 1
+    assert f(sh, 128, d, ctypes.byref(sfa.Rope(None, d, 1)), d, d, d, d, 8, 1, 0.0, d, None, None, None) == 1
+    assert f(sh, 128, d, ctypes.byref(sfa.Rope(ctypes.c_void_p((1 << 20) + 4), d, 1)), d, d, d, d, 8, 1, 0.0, d,
+             None, None, None) == 1                                                       # misaligned table
+    assert f(sh, 128, d, ctypes.byref(good), None, d, d, d, 8, 1, 0.0, d, None, None, None) == 1  # no K_rot
+    assert f(sh, 128, d, ctypes.byref(good), d, d, d, d, 0, 1, 0.0, d, None, None, None) == 1     # kmax 0
+    bad = S(L=1000)
+    assert f(ctypes.byref(bad), 128, d, ctypes.byref(good), d, d, d, d, 8, 1, 0.0, d, None, None, None) == 2
 
 
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):

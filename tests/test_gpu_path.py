@@ -147,3 +147,28 @@ def test_fused_scores_select_matches(w):
     sel = po.select_blocks(sc.probs, w.flags, k=w.k, mass=mass)
     stats, _ = compare_masks(sel, sc.probs, fused.counts, fused.idx, mass)
     assert stats["mismatches"] == 0, stats["bad_rows"][:5]
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_rope_on_load_matches(w):
+    """sfa_block_sparse_attn_rope on pre-RoPE Q (Q_rot never stored) gives the same O and lse,
+    bit for bit, as sfa_block_sparse_attn on the stored Q_rot; alone and with the fused selection."""
+    Q, K, V = make_inputs(w, seed=2)
+    dev = torch.device("cuda")
+    kw = dict(batch=w.batch, heads_q=w.heads_q, heads_kv=w.heads_kv, seq_len=w.seq_len, head_dim=w.head_dim,
+              dtype=w.dtype, block=w.block, rope_base=w.rope_base, band_split=w.band_split, k=w.k, mass=w.mass,
+              flags=w.flags, device=dev, with_lse=True)
+    Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
+    ref = sfa.PrismAttention(**kw)
+    ref(Qd, Kd, Vd)
+    for fused in (False, True):
+        rol = sfa.PrismAttention(**kw, rope_on_load=True, fused=fused)
+        assert rol.Q_rot is None
+        rol.O.fill_(7)
+        rol(Qd, Kd, Vd)
+        torch.cuda.synchronize()
+        assert int(rol.status.item()) == 0
+        assert torch.equal(ref.K_rot, rol.K_rot)
+        assert torch.equal(ref.counts, rol.counts) and torch.equal(ref.idx, rol.idx)
+        assert torch.equal(ref.O, rol.O), f"fused={fused}: O differs"
+        assert torch.equal(ref.lse, rol.lse), f"fused={fused}: lse differs"
