@@ -41,8 +41,19 @@ R4  Energy and tau, per (batch, Q head, band):
 R4b (alternative reading, flag RELATIVE_CALIB): restore the high band's
     amplitude relative to the low band only: tau^H <- tau^H / tau^L,
     tau^L <- 1 (the low band keeps its plain mean-pooling scale).
+R4c (alternative reading, flag BLOCK_TAU): the temperature is per block pair,
+    tau^b_ij = rho^b_i(Q_h) * rho^b_j(K_g), with each block's own retained
+    amplitude rho^b_i(X) = sqrt(||xbar_i^b||^2 / ((1/block) sum_{t in i}
+    ||x_t^b||^2)), floored at 1e-3 (so tau >= 1e-6 as in R4) and 1 when the
+    block's band energy is 0.  Exclusive with NO_CALIB and RELATIVE_CALIB.
 R5  Logits: s_ij = (1/sqrt(d)) * sum_b (qbar_i^b . kbar_j^b) / tau^b, j <= i.
 R6  Probabilities: causal row softmax over j <= i; p_ij = 0 for j > i.
+R5b (alternative reading, flag BAND_MAX; §3 "two parallel branches"): each
+    band's calibrated logits s^b_ij = (qbar_i^b . kbar_j^b) / (tau^b sqrt(d))
+    get their own causal softmax p^b; the branches combine by the elementwise
+    maximum, renormalised over j <= i:
+        p_ij = max_b p^b_ij / sum_{j' <= i} max_b p^b_ij'.
+    A band with no dims has no branch (then p is the R5/R6 result).
 R7  Selection: forced F_i = {i} (and {0} with KEEP_SINK); candidates ordered
     by (p desc, index asc); top-k keeps F_i plus the first min(k, |C_i|);
     mass keeps F_i and adds candidates in order while the running sum
@@ -58,7 +69,11 @@ Pins (tests/test_oracle_pins.py): the Dirichlet amplitude-collapse closed form
 to token-level causal softmax, mean pooling cross-checked with torch's
 avg_pool1d, RoPE against the transformers Llama rotary routine, brute-force
 selection, and all-blocks-kept attention against brute-force dense causal
-attention.  Parity of the *selection rule itself* with the pages' own
+attention.  R4c: per-block rho equal to the golden Dirichlet factor for a
+constant pair, the 1e-3 floor on a full turn per block, restoration of each
+block's token RMS, block size 1 giving token softmax.  R5b: mirrored bands
+giving the half-logit softmax, a one-hot branch against a uniform branch in
+closed form, and a single band reducing to R5/R6.  Parity of the *selection rule itself* with the pages' own
 selections is unpinned: the pages print no worked example.
 """
 
@@ -73,8 +88,11 @@ FLAG_KEEP_SINK = 1
 FLAG_NO_CALIB = 2
 FLAG_SINGLE_BAND = 4
 FLAG_RELATIVE_CALIB = 8
+FLAG_BAND_MAX = 16
+FLAG_BLOCK_TAU = 32
 
 TAU_FLOOR = 1e-6
+BLOCK_RHO_FLOOR = 1e-3
 
 
 # ---------------------------------------------------------------------------
@@ -155,6 +173,19 @@ def retained_amplitude(xr: np.ndarray, xbar: np.ndarray, band: np.ndarray) -> np
     return rho
 
 
+def block_retained_amplitude(xr: np.ndarray, xbar: np.ndarray, band: np.ndarray) -> np.ndarray:
+    """R4c: rho of every block [..., nb] for one band: sqrt(||xbar_j||^2 / mean_{t in j} ||x_t||^2),
+    floored at BLOCK_RHO_FLOOR; 1 where the block's band energy is 0."""
+    nb = xbar.shape[-2]
+    block = xr.shape[-2] // nb
+    e_tok = (xr[..., band] ** 2).sum(axis=-1).reshape(*xr.shape[:-2], nb, block).mean(axis=-1)
+    e_pool = (xbar[..., band] ** 2).sum(axis=-1)
+    rho = np.ones_like(e_tok)
+    nz = e_tok > 0
+    rho[nz] = np.maximum(np.sqrt(e_pool[nz] / e_tok[nz]), BLOCK_RHO_FLOOR)
+    return rho
+
+
 def temperatures(qr, kr, qbar, kbar, band_split, flags, group):
     """tau [B, Hq, 2] (index 0 = band H, 1 = band L); band L is all ones with SINGLE_BAND."""
     B, Hq = qr.shape[0], qr.shape[1]
@@ -183,20 +214,45 @@ def temperatures(qr, kr, qbar, kbar, band_split, flags, group):
 # ---------------------------------------------------------------------------
 # R5/R6: calibrated block logits and causal block softmax (Prism §3.2, §5).
 # ---------------------------------------------------------------------------
-def block_logits(qbar, kbar, tau, band_split, flags, group):
-    """s [B, Hq, nb, nb] (all entries; the caller masks j > i)."""
+def band_logits(qbar, kbar, tau, band_split, flags, group, qr=None, kr=None):
+    """Per-band calibrated logits [(band index, s^b [B, Hq, nb, nb])] for the bands that have dims.
+
+    R5 divides band b by tau^b [B, Hq, 2]; with BLOCK_TAU (R4c) by rho^b_i(Q) rho^b_j(K)
+    from the rotated tokens ``qr``, ``kr``."""
     d = qbar.shape[-1]
     single = bool(flags & FLAG_SINGLE_BAND)
     kq = np.repeat(kbar, group, axis=1)
-    s = np.zeros(qbar.shape[:-1] + (kbar.shape[-2],), dtype=np.float64)
+    out = []
     for bi, band in enumerate(band_masks(d, band_split, single)):
         if single and bi == 1:
             break
         if not band.any():
             continue
         part = qbar[..., band] @ np.swapaxes(kq[..., band], -1, -2)
-        s += part / tau[:, :, bi][:, :, None, None]
-    return s / math.sqrt(d)
+        if flags & FLAG_BLOCK_TAU:
+            rq = block_retained_amplitude(qr, qbar, band)                                 # [B, Hq, nb]
+            rk = np.repeat(block_retained_amplitude(kr, kbar, band), group, axis=1)      # [B, Hq, nb]
+            part = part / (rq[..., :, None] * rk[..., None, :])
+        else:
+            part = part / tau[:, :, bi][:, :, None, None]
+        out.append((bi, part / math.sqrt(d)))
+    return out
+
+
+def block_logits(qbar, kbar, tau, band_split, flags, group, qr=None, kr=None):
+    """s [B, Hq, nb, nb] = sum of the band logits (all entries; the caller masks j > i)."""
+    s = np.zeros(qbar.shape[:-1] + (kbar.shape[-2],), dtype=np.float64)
+    for _, part in band_logits(qbar, kbar, tau, band_split, flags, group, qr, kr):
+        s = s + part
+    return s
+
+
+def band_max_probs(band_probs):
+    """R5b: elementwise maximum of the per-band causal softmaxes, renormalised per row."""
+    c = band_probs[0]
+    for q in band_probs[1:]:
+        c = np.maximum(c, q)
+    return c / c.sum(axis=-1, keepdims=True)
 
 
 def causal_block_softmax(s: np.ndarray) -> np.ndarray:
@@ -239,6 +295,8 @@ def prism_scores(Q, K, block, band_split, flags=0, rope=None) -> ScoreResult:
     """Steps R1-R6 for Q [B, Hq, L, d] and K [B, Hkv, L, d] (pre-RoPE values).
 
     ``rope`` is (cos32, sin32) tables or None when Q, K are already rotated."""
+    if (flags & FLAG_BLOCK_TAU) and (flags & (FLAG_NO_CALIB | FLAG_RELATIVE_CALIB)):
+        raise ValueError("BLOCK_TAU excludes NO_CALIB and RELATIVE_CALIB")
     Q = np.asarray(Q, dtype=np.float64)
     K = np.asarray(K, dtype=np.float64)
     group = Q.shape[1] // K.shape[1]
@@ -250,8 +308,14 @@ def prism_scores(Q, K, block, band_split, flags=0, rope=None) -> ScoreResult:
     qbar = pool_blocks(qr, block)
     kbar = pool_blocks(kr, block)
     tau = temperatures(qr, kr, qbar, kbar, band_split, flags, group)
-    s = block_logits(qbar, kbar, tau, band_split, flags, group)
-    p = causal_block_softmax(s)
+    parts = band_logits(qbar, kbar, tau, band_split, flags, group, qr, kr)
+    s = np.zeros(qbar.shape[:-1] + (kbar.shape[-2],), dtype=np.float64)
+    for _, part in parts:
+        s = s + part
+    if (flags & FLAG_BAND_MAX) and len(parts) == 2:
+        p = band_max_probs([causal_block_softmax(part) for _, part in parts])
+    else:
+        p = causal_block_softmax(s)
     return ScoreResult(qr, kr, qbar, kbar,
                        block_token_energy(qr, block, band_split, flags),
                        block_token_energy(kr, block, band_split, flags),

@@ -410,3 +410,122 @@ def test_relative_calibration_closed_form_and_low_band_untouched():
     # one band relative to itself: no calibration
     c = po.prism_scores(Qr_, Kr_, beta, bs, po.FLAG_RELATIVE_CALIB | po.FLAG_SINGLE_BAND, (cos2, sin2))
     np.testing.assert_allclose(c.tau, 1.0)
+
+
+# ---------------------------------------------------------------------------
+# Alternative readings of §3: per-block temperature (BLOCK_TAU) and the two
+# spectral branches combined by their maximum (BAND_MAX).
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("row", _golden_rows()[:2])
+def test_block_tau_rho_is_dirichlet_factor_per_block(row):
+    """A constant vector in one rotary pair: every block's own retained amplitude is the
+    Dirichlet factor of that pair (golden), and a band without energy gets rho = 1."""
+    base, d, m, beta, theta, D = row
+    L = 5 * beta
+    cos, sin = po.rope_tables(base, L, d)
+    x = np.zeros((1, 1, L, d))
+    x[..., m] = 1.0
+    xr = po.apply_rope(x, cos, sin)
+    xbar = po.pool_blocks(xr, beta)
+    h, l = po.band_masks(d, m + 1)
+    np.testing.assert_allclose(po.block_retained_amplitude(xr, xbar, h), D, rtol=0, atol=3e-6)
+    np.testing.assert_allclose(po.block_retained_amplitude(xr, xbar, l), 1.0)
+    # a block with no energy: rho = 1
+    assert po.block_retained_amplitude(xr * 0.0, xbar * 0.0, h).min() == 1.0
+
+
+def test_block_tau_rho_floor_on_full_turn():
+    """theta = 2 pi / beta: each block holds one full turn of the pair, its mean cancels (to the
+    float32 table's rounding) and rho is floored at 1e-3."""
+    beta, d, L = 8, 4, 32
+    base = (beta / (2 * math.pi)) ** 2          # theta_1 = base**(-2/4) = 2 pi / beta
+    cos, sin = po.rope_tables(base, L, d)
+    x = np.zeros((1, 1, L, d))
+    x[..., 1] = 1.0
+    xr = po.apply_rope(x, cos, sin)
+    xbar = po.pool_blocks(xr, beta)
+    assert np.abs(xbar).max() < 1e-6
+    h, _ = po.band_masks(d, 2)
+    np.testing.assert_array_equal(po.block_retained_amplitude(xr, xbar, h), po.BLOCK_RHO_FLOOR)
+
+
+def test_block_tau_restores_each_block_to_its_token_rms():
+    """Dividing a block mean by its own rho gives a vector whose squared norm is the block's
+    mean token energy in that band (checked against the rotated tokens with torch)."""
+    base, d, beta, L, bs = 1e4, 16, 8, 64, 3
+    cos, sin = po.rope_tables(base, L, d)
+    rng = np.random.default_rng(31)
+    X = rng.normal(size=(1, 2, L, d))
+    xr = po.apply_rope(X, cos, sin)
+    xbar = po.pool_blocks(xr, beta)
+    for band in po.band_masks(d, bs):
+        rho = po.block_retained_amplitude(xr, xbar, band)
+        lhs = ((xbar[..., band] / rho[..., None]) ** 2).sum(-1)
+        t = _torch_rotate(X, cos, sin)[..., torch.from_numpy(band)]
+        rms2 = (t ** 2).sum(-1).reshape(1, 2, L // beta, beta).mean(-1).numpy()
+        np.testing.assert_allclose(lhs, rms2, rtol=1e-12)
+
+
+def test_block_tau_block_one_equals_token_causal_softmax():
+    B, Hq, Hkv, L, d = 1, 4, 2, 10, 8
+    cos, sin = po.rope_tables(1e4, L, d)
+    rng = np.random.default_rng(32)
+    Q = rng.normal(size=(B, Hq, L, d))
+    K = rng.normal(size=(B, Hkv, L, d))
+    sc = po.prism_scores(Q, K, 1, 2, po.FLAG_BLOCK_TAU, (cos, sin))
+    qt = _torch_rotate(Q, cos, sin)
+    kt = torch.repeat_interleave(_torch_rotate(K, cos, sin), Hq // Hkv, dim=1)
+    logits = qt @ kt.transpose(-1, -2) / math.sqrt(d)
+    mask = torch.ones(L, L, dtype=torch.bool).tril()
+    ref = torch.softmax(logits.masked_fill(~mask, float("-inf")), dim=-1)
+    np.testing.assert_allclose(sc.probs, ref.numpy(), rtol=0, atol=1e-12)
+    with pytest.raises(ValueError):
+        po.prism_scores(Q, K, 1, 2, po.FLAG_BLOCK_TAU | po.FLAG_NO_CALIB, (cos, sin))
+
+
+def test_band_max_mirrored_bands_is_half_logit_softmax():
+    """Identical bands: both branches give softmax(s^H), while the sum reading gives softmax(2 s^H)."""
+    L, d = 9, 4
+    rng = np.random.default_rng(33)
+    q = rng.normal(size=(1, 1, L, 2))
+    k = rng.normal(size=(1, 1, L, 2))
+    Q = np.stack([q[..., 0], q[..., 0], q[..., 1], q[..., 1]], -1)   # dims (0, 2) = band H, (1, 3) = band L
+    K = np.stack([k[..., 0], k[..., 0], k[..., 1], k[..., 1]], -1)
+    mx = po.prism_scores(Q, K, 1, 1, po.FLAG_BAND_MAX, None)
+    sm = po.prism_scores(Q, K, 1, 1, 0, None)
+    sH = torch.from_numpy(q[0, 0] @ k[0, 0].T / math.sqrt(d))
+    mask = torch.ones(L, L, dtype=torch.bool).tril()
+    np.testing.assert_allclose(mx.probs[0, 0], torch.softmax(sH.masked_fill(~mask, -math.inf), -1).numpy(),
+                               rtol=0, atol=1e-13)
+    np.testing.assert_allclose(sm.probs[0, 0], torch.softmax((2 * sH).masked_fill(~mask, -math.inf), -1).numpy(),
+                               rtol=0, atol=1e-13)
+
+
+def test_band_max_one_hot_branch_against_uniform_branch():
+    """Band H one-hot at block j* (huge logit), band L uniform (zero logits): row i >= j* keeps
+    (i+1)/(2i+1) on j* and 1/(2i+1) elsewhere; rows i < j* stay uniform."""
+    L, d, js, A = 8, 4, 3, 12.0
+    Q = np.zeros((1, 1, L, d))
+    K = np.zeros((1, 1, L, d))
+    Q[..., 0] = A
+    K[0, 0, js, 0] = A
+    p = po.prism_scores(Q, K, 1, 1, po.FLAG_BAND_MAX, None).probs[0, 0]
+    for i in range(L):
+        want = np.zeros(L)
+        if i < js:
+            want[:i + 1] = 1.0 / (i + 1)
+        else:
+            want[:i + 1] = 1.0 / (2 * i + 1)
+            want[js] = (i + 1) / (2 * i + 1)
+        np.testing.assert_allclose(p[i], want, rtol=0, atol=1e-12)
+
+
+def test_band_max_single_band_is_default():
+    base, d, beta, L = 1e4, 16, 8, 64
+    cos, sin = po.rope_tables(base, L, d)
+    rng = np.random.default_rng(34)
+    Q, K = rng.normal(size=(1, 2, L, d)), rng.normal(size=(1, 1, L, d))
+    for flags, bs in ((po.FLAG_SINGLE_BAND, 3), (0, 0), (0, d // 2)):
+        a = po.prism_scores(Q, K, beta, bs, flags | po.FLAG_BAND_MAX, (cos, sin))
+        b = po.prism_scores(Q, K, beta, bs, flags, (cos, sin))
+        np.testing.assert_array_equal(a.probs, b.probs)
