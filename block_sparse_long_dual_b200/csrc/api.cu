@@ -19,7 +19,8 @@ namespace {
 
 constexpr int kVersion = 100;  // 0.1.0
 constexpr int kMaxBlocks = 2048;
-constexpr unsigned kKnownFlags = SFA_KEEP_SINK | SFA_NO_CALIB | SFA_SINGLE_BAND | SFA_RELATIVE_CALIB;
+constexpr unsigned kKnownFlags =
+    SFA_KEEP_SINK | SFA_NO_CALIB | SFA_SINGLE_BAND | SFA_RELATIVE_CALIB | SFA_BAND_MAX | SFA_BLOCK_TAU;
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
 
@@ -200,6 +201,7 @@ sfa_status run_block_scores(const sfa_shape* shape, const void* Q, const void* K
     return SFA_ERR_INVALID_ARG;
   if (flags & ~kKnownFlags) return SFA_ERR_INVALID_ARG;
   if (band_split < 0 || band_split > D / 2) return SFA_ERR_INVALID_ARG;
+  if ((flags & SFA_BLOCK_TAU) && (flags & (SFA_NO_CALIB | SFA_RELATIVE_CALIB))) return SFA_ERR_INVALID_ARG;
   if (fused != nullptr) {
     st = check_select(nb, fused->k, fused->mass, flags, fused->counts, fused->idx, fused->kmax);
     if (st != SFA_OK) return st;
@@ -238,8 +240,8 @@ sfa_status run_block_scores(const sfa_shape* shape, const void* Q, const void* K
   if (st != SFA_OK) return st;
 
   ScoreParams sp;
-  sp.qbar = rp.qbar; sp.kbar = rp.kbar; sp.tau = tp.tau; sp.probs = probs;
-  sp.B = rp.B; sp.Hq = rp.Hq; sp.Hkv = rp.Hkv; sp.nb = nb; sp.band_pairs = band_pairs;
+  sp.qbar = rp.qbar; sp.kbar = rp.kbar; sp.tau = tp.tau; sp.energy = rp.energy; sp.probs = probs;
+  sp.B = rp.B; sp.Hq = rp.Hq; sp.Hkv = rp.Hkv; sp.nb = nb; sp.block = block; sp.band_pairs = band_pairs;
   sp.counts = fused ? fused->counts : nullptr;
   sp.idx = fused ? fused->idx : nullptr;
   sp.kmax = fused ? fused->kmax : 0;

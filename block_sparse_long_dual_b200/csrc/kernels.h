@@ -35,8 +35,9 @@ struct ScoreParams {
   const double* qbar;
   const double* kbar;
   const double* tau;
+  const double* energy;  // per-block energies (SFA_BLOCK_TAU)
   float* probs;  // may be null when the selection is fused
-  int B, Hq, Hkv, nb;
+  int B, Hq, Hkv, nb, block;
   int band_pairs;
   // fused selection (counts != null): the rule of SelectParams
   int* counts;
@@ -76,7 +77,7 @@ struct AttnParams {
 cudaError_t launch_rope_pool_energy(const RopePoolParams& p, int dtype, int D, cudaStream_t st);
 cudaError_t launch_band_temperature(const TauParams& p, cudaStream_t st);
 cudaError_t launch_block_score_softmax(const ScoreParams& p, int D, cudaStream_t st);
-size_t score_smem_bytes(int nb, int D);
+size_t score_smem_bytes(int nb, int D, bool band_max);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnParams& p, int dtype, int D, cudaStream_t st);
 cudaError_t launch_attn_tcgen05(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,

@@ -285,7 +285,22 @@ __global__ void __launch_bounds__(256) band_temperature_kernel(TauParams p) {
 // skipped.  Then the causal row softmax in float64, one warp per row.
 // Everything is float64 because the calibration 1/tau amplifies the pooled
 // logits: float32 sums of logits of magnitude ~20 already err by ~1e-6.
+//
+// Alternative readings (flags):
+//   SFA_BLOCK_TAU  per-block temperature: the query means of row i are scaled
+//                  by 1/rho^b_i(Q) and each key mean element by 1/rho^b_j(K)
+//                  as its fragment is loaded (rho from the block energies).
+//   SFA_BAND_MAX   one GEMM pass per band (the other band's query dims zeroed),
+//                  each with its own causal softmax; band H's probabilities
+//                  wait in a float32 strip [RT][nb] until band L's pass takes
+//                  the elementwise maximum and renormalises.
 // ---------------------------------------------------------------------------
+// Retained amplitude of one block and band: sqrt(||xbar||^2 / mean_t ||x_t||^2),
+// floored at 1e-3, 1 when the block's band has no energy.
+__device__ __forceinline__ double block_rho(double tok, double pool, int block) {
+  return tok == 0.0 ? 1.0 : fmax(sqrt(pool * (double)block / tok), 1e-3);
+}
+
 __device__ __forceinline__ void dmma_8x8x4(double (&c)[2], double a, double b) {
   asm volatile("mma.sync.aligned.m8n8k4.row.col.f64.f64.f64.f64 {%0, %1}, {%2}, {%3}, {%0, %1};"
                : "+d"(c[0]), "+d"(c[1])
@@ -293,7 +308,7 @@ __device__ __forceinline__ void dmma_8x8x4(double (&c)[2], double a, double b) {
 }
 
 template <int RT, int D, int NPL, bool FUSED>
-__global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p) {
+__global__ void __launch_bounds__(256, 1) block_score_softmax_kernel(ScoreParams p) {
   constexpr int RTL = RT / 8;             // row tiles
   constexpr int CS = 256;                 // columns per step
   constexpr int CTW = 4;                  // column tiles per warp (8 warps x 4 x 8 = 256)
@@ -302,6 +317,7 @@ __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p)
   extern __shared__ __align__(16) unsigned char smem_raw[];
   double* strip = reinterpret_cast<double*>(smem_raw);                 // [RT][nb]
   double* qs = strip + (size_t)RT * p.nb;                               // [RT][QLD]
+  float* pstrip = reinterpret_cast<float*>(qs + RT * QLD);              // [RT][nb], band-max only
 
   const int ntiles = (p.nb + RT - 1) / RT;
   const int tile = ntiles - 1 - (int)blockIdx.x;  // heaviest rows first
@@ -313,75 +329,123 @@ __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p)
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int gq = lane >> 2, tq = lane & 3;  // mma fragment coordinates
 
-  // Calibrated, pre-scaled query block means: q~ = qbar / (tau^band * sqrt(d)).
+  const bool block_tau = (p.flags & SFA_BLOCK_TAU) != 0;
+  const bool two = (p.flags & SFA_BAND_MAX) && p.band_pairs > 0 && p.band_pairs < D / 2;
+  const int heads = p.Hq + p.Hkv;
   const double* tau = p.tau + (size_t)(b * p.Hq + h) * 2;
   const double inv_h = 1.0 / (tau[0] * sqrt((double)D));
   const double inv_l = 1.0 / (tau[1] * sqrt((double)D));
   const double* qsrc = p.qbar + ((size_t)(b * p.Hq + h) * p.nb + i0) * D;
-  for (int e = tid; e < D * RT; e += 256) {
-    const int r = e / D, d = e % D;
-    const double s = ((d % (D / 2)) < p.band_pairs) ? inv_h : inv_l;
-    qs[r * QLD + d] = (r < rows) ? qsrc[(size_t)r * D + d] * s : 0.0;
-  }
-  __syncthreads();
   const double* ksrc = p.kbar + (size_t)(b * p.Hkv + g) * p.nb * D;
+  const double* eq = p.energy + ((size_t)(b * heads + h) * p.nb) * 4;
+  const double* ek = p.energy + ((size_t)(b * heads + p.Hq + g) * p.nb) * 4;
 
-  for (int col0 = 0; col0 < jend; col0 += CS) {
-    // this warp's column tiles: col0 + (warp * CTW + ct) * 8 .. + 8
-    int ntl = 0;
-#pragma unroll
-    for (int ct = 0; ct < CTW; ++ct) ntl += (col0 + (warp * CTW + ct) * 8 < jend) ? 1 : 0;
-    if (ntl > 0) {
-      double acc[RTL][CTW][2];
-#pragma unroll
-      for (int rt = 0; rt < RTL; ++rt)
-#pragma unroll
-        for (int ct = 0; ct < CTW; ++ct) acc[rt][ct][0] = acc[rt][ct][1] = 0.0;
-      // B fragment of column tile ct at k-step ks: kbar[col][4 ks + tq], col = tile start + gq.
-      const double* kb[CTW];
-#pragma unroll
-      for (int ct = 0; ct < CTW; ++ct) {
-        const int col = min(col0 + (warp * CTW + ct) * 8 + gq, p.nb - 1);
-        kb[ct] = ksrc + (size_t)col * D + tq;
+  for (int pass = 0; pass < (two ? 2 : 1); ++pass) {
+    // Calibrated, pre-scaled query block means: q~ = qbar / (tau^band * sqrt(d)) (per-block
+    // rho^band_i(Q) instead of tau with SFA_BLOCK_TAU); with SFA_BAND_MAX pass 0 keeps band H's
+    // dims only and pass 1 band L's.
+    for (int e = tid; e < D * RT; e += 256) {
+      const int r = e / D, d = e % D;
+      const bool hb = (d % (D / 2)) < p.band_pairs;
+      double sc;
+      if (block_tau) {
+        const double* er = eq + (size_t)min(i0 + r, p.nb - 1) * 4;
+        sc = 1.0 / (block_rho(er[hb ? 0 : 1], er[hb ? 2 : 3], p.block) * sqrt((double)D));
+      } else {
+        sc = hb ? inv_h : inv_l;
       }
-      double bcur[CTW], bnxt[CTW];
+      if (two && hb != (pass == 0)) sc = 0.0;
+      qs[r * QLD + d] = (r < rows) ? qsrc[(size_t)r * D + d] * sc : 0.0;
+    }
+    __syncthreads();
+
+    for (int col0 = 0; col0 < jend; col0 += CS) {
+      // this warp's column tiles: col0 + (warp * CTW + ct) * 8 .. + 8
+      int ntl = 0;
 #pragma unroll
-      for (int ct = 0; ct < CTW; ++ct) bcur[ct] = __ldg(kb[ct]);
-#pragma unroll 4
-      for (int ks = 0; ks < KS; ++ks) {
-        if (ks + 1 < KS) {
+      for (int ct = 0; ct < CTW; ++ct) ntl += (col0 + (warp * CTW + ct) * 8 < jend) ? 1 : 0;
+      if (ntl > 0) {
+        double acc[RTL][CTW][2];
 #pragma unroll
-          for (int ct = 0; ct < CTW; ++ct) bnxt[ct] = __ldg(kb[ct] + 4 * (ks + 1));
-        }
-        double a[RTL];
+        for (int rt = 0; rt < RTL; ++rt)
 #pragma unroll
-        for (int rt = 0; rt < RTL; ++rt) a[rt] = qs[(rt * 8 + gq) * QLD + 4 * ks + tq];
+          for (int ct = 0; ct < CTW; ++ct) acc[rt][ct][0] = acc[rt][ct][1] = 0.0;
+        // B fragment of column tile ct at k-step ks: kbar[col][4 ks + tq], col = tile start + gq.
+        const double* kb[CTW];
+        double kih[CTW], kil[CTW];  // 1 / rho^band_col(K) with SFA_BLOCK_TAU, else 1
 #pragma unroll
         for (int ct = 0; ct < CTW; ++ct) {
-          if (ct < ntl) {
-#pragma unroll
-            for (int rt = 0; rt < RTL; ++rt) dmma_8x8x4(acc[rt][ct], a[rt], bcur[ct]);
+          const int col = min(col0 + (warp * CTW + ct) * 8 + gq, p.nb - 1);
+          kb[ct] = ksrc + (size_t)col * D + tq;
+          kih[ct] = kil[ct] = 1.0;
+          if (block_tau) {
+            const double* er = ek + (size_t)col * 4;
+            kih[ct] = 1.0 / block_rho(er[0], er[2], p.block);
+            kil[ct] = 1.0 / block_rho(er[1], er[3], p.block);
           }
         }
+        double bcur[CTW], bnxt[CTW];
+        {
+          const bool hb = (tq % (D / 2)) < p.band_pairs;
 #pragma unroll
-        for (int ct = 0; ct < CTW; ++ct) bcur[ct] = bnxt[ct];
-      }
-      // C fragment: (row gq, cols 2 tq, 2 tq + 1) of each tile
+          for (int ct = 0; ct < CTW; ++ct) bcur[ct] = __ldg(kb[ct]) * (hb ? kih[ct] : kil[ct]);
+        }
+#pragma unroll 4
+        for (int ks = 0; ks < KS; ++ks) {
+          if (ks + 1 < KS) {
+            const bool hb = ((4 * (ks + 1) + tq) % (D / 2)) < p.band_pairs;
 #pragma unroll
-      for (int rt = 0; rt < RTL; ++rt) {
-        const int rr = rt * 8 + gq;
+            for (int ct = 0; ct < CTW; ++ct) bnxt[ct] = __ldg(kb[ct] + 4 * (ks + 1)) * (hb ? kih[ct] : kil[ct]);
+          }
+          double a[RTL];
 #pragma unroll
-        for (int ct = 0; ct < CTW; ++ct) {
-          const int col = col0 + (warp * CTW + ct) * 8 + 2 * tq;
-          if (ct < ntl) {  // scalar stores: nb may be odd, so a row need not start 16-byte aligned
-            if (col < jend) strip[(size_t)rr * p.nb + col] = acc[rt][ct][0];
-            if (col + 1 < jend) strip[(size_t)rr * p.nb + col + 1] = acc[rt][ct][1];
+          for (int rt = 0; rt < RTL; ++rt) a[rt] = qs[(rt * 8 + gq) * QLD + 4 * ks + tq];
+#pragma unroll
+          for (int ct = 0; ct < CTW; ++ct) {
+            if (ct < ntl) {
+#pragma unroll
+              for (int rt = 0; rt < RTL; ++rt) dmma_8x8x4(acc[rt][ct], a[rt], bcur[ct]);
+            }
+          }
+#pragma unroll
+          for (int ct = 0; ct < CTW; ++ct) bcur[ct] = bnxt[ct];
+        }
+        // C fragment: (row gq, cols 2 tq, 2 tq + 1) of each tile
+#pragma unroll
+        for (int rt = 0; rt < RTL; ++rt) {
+          const int rr = rt * 8 + gq;
+#pragma unroll
+          for (int ct = 0; ct < CTW; ++ct) {
+            const int col = col0 + (warp * CTW + ct) * 8 + 2 * tq;
+            if (ct < ntl) {  // scalar stores: nb may be odd, so a row need not start 16-byte aligned
+              if (col < jend) strip[(size_t)rr * p.nb + col] = acc[rt][ct][0];
+              if (col + 1 < jend) strip[(size_t)rr * p.nb + col + 1] = acc[rt][ct][1];
+            }
           }
         }
       }
     }
+    __syncthreads();
+    if (two && pass == 0) {
+      // Band H's causal softmax, kept as float32 probabilities for pass 1.
+      for (int r = warp; r < rows; r += 8) {
+        const int i = i0 + r;
+        const double* srow = strip + (size_t)r * p.nb;
+        double m = -INFINITY;
+        for (int jj = lane; jj <= i; jj += 32) m = fmax(m, srow[jj]);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) m = fmax(m, __shfl_xor_sync(0xffffffffu, m, off));
+        double sum = 0.0;
+        for (int jj = lane; jj <= i; jj += 32) sum += exp(srow[jj] - m);
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+        const double inv = 1.0 / sum;
+        float* prow = pstrip + (size_t)r * p.nb;
+        for (int jj = lane; jj <= i; jj += 32) prow[jj] = (float)(exp(srow[jj] - m) * inv);
+      }
+      __syncthreads();  // strip free for band L; pstrip complete
+    }
   }
-  __syncthreads();
 
   // Causal row softmax in float64, one warp per row.
   for (int r = warp; r < rows; r += 8) {
@@ -399,7 +463,20 @@ __global__ void __launch_bounds__(256) block_score_softmax_kernel(ScoreParams p)
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-    const double inv = 1.0 / sum;
+    double inv = 1.0 / sum;
+    if (two) {
+      // Band max: c_j = max(p^H_j, p^L_j), renormalised over j <= i.
+      const float* prow = pstrip + (size_t)r * p.nb;
+      double z = 0.0;
+      for (int jj = lane; jj <= i; jj += 32) {
+        const double c = fmax((double)prow[jj], srow[jj] * inv);
+        srow[jj] = c;
+        z += c;
+      }
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+      inv = 1.0 / z;
+    }
     const size_t rowid = (size_t)(b * p.Hq + h) * p.nb + i;
     if (p.probs != nullptr) {
       float* prow = p.probs + rowid * p.nb;
@@ -456,14 +533,15 @@ cudaError_t launch_band_temperature(const TauParams& p, cudaStream_t st) {
 
 int score_rows_per_cta(int nb) { return nb <= 1024 ? 16 : 8; }
 
-size_t score_smem_bytes(int nb, int D) {
+size_t score_smem_bytes(int nb, int D, bool band_max) {
   const int RT = score_rows_per_cta(nb);
-  return ((size_t)RT * nb + (size_t)RT * (D + 4)) * sizeof(double);
+  return ((size_t)RT * nb + (size_t)RT * (D + 4)) * sizeof(double) + (band_max ? (size_t)RT * nb * sizeof(float) : 0);
 }
 
 template <int RT, int D, int NPL, bool FUSED>
 static cudaError_t launch_score_t(const ScoreParams& p, cudaStream_t st) {
-  const size_t smem = score_smem_bytes(p.nb, D);
+  const size_t smem =
+      score_smem_bytes(p.nb, D, (p.flags & SFA_BAND_MAX) && p.band_pairs > 0 && p.band_pairs < D / 2);
   auto kern = block_score_softmax_kernel<RT, D, NPL, FUSED>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;

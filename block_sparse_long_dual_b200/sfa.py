@@ -22,7 +22,7 @@ import torch
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsfa.so")
 
 F32, BF16 = 0, 1
-KEEP_SINK, NO_CALIB, SINGLE_BAND, RELATIVE_CALIB = 1, 2, 4, 8
+KEEP_SINK, NO_CALIB, SINGLE_BAND, RELATIVE_CALIB, BAND_MAX, BLOCK_TAU = 1, 2, 4, 8, 16, 32
 STATUS = {0: "SFA_OK", 1: "SFA_ERR_INVALID_ARG", 2: "SFA_ERR_SHAPE", 3: "SFA_ERR_DTYPE",
           4: "SFA_ERR_UNSUPPORTED", 5: "SFA_ERR_WORKSPACE", 6: "SFA_ERR_CUDA", 7: "SFA_ERR_TIMEOUT",
           8: "SFA_ERR_INDEX"}

@@ -16,6 +16,8 @@ KEEP_SINK = 1
 NO_CALIB = 2
 SINGLE_BAND = 4
 RELATIVE_CALIB = 8
+BAND_MAX = 16
+BLOCK_TAU = 32
 
 
 @dataclass(frozen=True)

@@ -69,7 +69,9 @@ enum {
   SFA_KEEP_SINK = 1,   /* select: also force key block 0 into every row */
   SFA_NO_CALIB = 2,    /* scores: temperature tau = 1 (plain mean pooling) */
   SFA_SINGLE_BAND = 4, /* scores: all d dims form one band (one tau) */
-  SFA_RELATIVE_CALIB = 8 /* scores: restore band H relative to band L only: tau^H <- tau^H / tau^L, tau^L <- 1 */
+  SFA_RELATIVE_CALIB = 8, /* scores: restore band H relative to band L only: tau^H <- tau^H / tau^L, tau^L <- 1 */
+  SFA_BAND_MAX = 16,      /* scores: one causal softmax per band, combined by the renormalised elementwise max */
+  SFA_BLOCK_TAU = 32      /* scores: per-block temperature rho^b_i(Q) rho^b_j(K) (excludes NO_CALIB, RELATIVE_CALIB) */
 };
 
 /* Library version: major * 10000 + minor * 100 + patch. */
@@ -126,6 +128,16 @@ sfa_status sfa_workspace_layout(const sfa_shape* shape, int block, size_t offset
  * probs [B, heads_q, nb, nb] float32.  SFA_SINGLE_BAND puts all dims in band H.
  * SFA_RELATIVE_CALIB (an alternative reading of the temperature) divides
  * tau^H by tau^L and sets tau^L = 1 (1 for both with a single band).
+ * SFA_BLOCK_TAU (alternative reading, Prism §3.2): band b of s_ij is divided by
+ * rho^b_i(Q_h) rho^b_j(K_g) instead of tau^b, where a block's own retained
+ * amplitude is rho^b_j = sqrt(||xbar_j^b||^2 * block / sum_{t in j} ||x_t^b||^2),
+ * floored at 1e-3, 1 if the block's band energy is 0 (the workspace tau still
+ * holds the global values).  Combined with SFA_NO_CALIB or
+ * SFA_RELATIVE_CALIB it is SFA_ERR_INVALID_ARG.
+ * SFA_BAND_MAX (alternative reading, Prism §3 "two parallel branches"): each
+ * band's part of s_ij gets its own causal softmax p^b; then
+ * probs_ij = max_b p^b_ij / sum_{j' <= i} max_b p^b_ij'.  With one band (band
+ * H or L empty, or SFA_SINGLE_BAND) it changes nothing.
  * RoPE is applied in float32; block means, energies, temperatures, logits and
  * the softmax are float64 (the 1/tau calibration amplifies pooled logits, so
  * float32 sums would move probabilities by ~1e-6), rounded once to float32.

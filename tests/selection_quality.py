@@ -26,11 +26,13 @@ if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
 from block_sparse_long_dual_b200.synthetic import make_inputs, planted_blocks  # noqa: E402
-from block_sparse_long_dual_b200.workloads import NO_CALIB, RELATIVE_CALIB, SINGLE_BAND, Workload  # noqa: E402
+from block_sparse_long_dual_b200.workloads import (BAND_MAX, BLOCK_TAU, NO_CALIB, RELATIVE_CALIB,  # noqa: E402
+                                                   SINGLE_BAND, Workload)
 from oracle import prism_oracle as po  # noqa: E402
 
 VARIANTS = (("calibrated dual band", 0), ("plain mean pooling", NO_CALIB), ("single band", SINGLE_BAND),
-            ("relative calibration", RELATIVE_CALIB))
+            ("relative calibration", RELATIVE_CALIB), ("band max", BAND_MAX),
+            ("band max + relative calibration", BAND_MAX | RELATIVE_CALIB), ("per-block temperature", BLOCK_TAU))
 
 
 def token_mass_recall(qa, ka, kept, block, b, h, g, i, causal=True, scale=None):

@@ -102,7 +102,9 @@ def test_argument_validation_before_launch(lib):
     assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 0, d, d, None, d, ws, None) == 1
     assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 65, 128, 0, d, d, d, d, ws, None) == 1
     assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), -1, 128, 0, d, d, d, d, ws, None) == 1
-    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 16, d, d, d, d, ws, None) == 1
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 64, d, d, d, d, ws, None) == 1
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 32 | 2, d, d, d, d, ws, None) == 1  # block tau + no calib
+    assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 32 | 8, d, d, d, d, ws, None) == 1
     assert bs(ctypes.byref(shape), d, d, ctypes.byref(rope), 16, 128, 0, d, None, d, d, ws, None) == 1  # no K_rot
     # misaligned pointers
     assert bs(ctypes.byref(shape), ctypes.c_void_p((1 << 20) + 2), d, ctypes.byref(rope), 16, 128, 0, d, d, d, d,
@@ -120,7 +122,7 @@ def test_argument_validation_before_launch(lib):
     assert sel(ctypes.byref(shape), 128, d, 3, 0.0, 0, d, d, 3, None) == 1       # kmax < k + 1
     assert sel(ctypes.byref(shape), 128, d, 3, 0.0, 1, d, d, 4, None) == 1       # kmax < k + 2 with sink
     assert sel(ctypes.byref(shape), 128, None, 3, 0.0, 0, d, d, 4, None) == 1
-    assert sel(ctypes.byref(shape), 128, d, 3, 0.0, 32, d, d, 4, None) == 1      # unknown flag
+    assert sel(ctypes.byref(shape), 128, d, 3, 0.0, 64, d, d, 4, None) == 1      # unknown flag
     at = lib.sfa_block_sparse_attn
     assert at(ctypes.byref(shape), 128, d, d, d, d, d, 0, 1, 0.0, d, None, None, None) == 1  # kmax 0
     assert at(ctypes.byref(shape), 128, d, None, d, d, d, 4, 1, 0.0, d, None, None, None) == 1
@@ -141,7 +143,7 @@ def test_fused_scores_select_validation(lib):
     # score-side errors: null Q, band_split, unknown flag, rope outputs, workspace
     assert f(sh, None, d, R, 16, 128, 0, 4, 0.0, d, d, None, d, d, 5, d, ws, None) == 1
     assert f(sh, d, d, R, 65, 128, 0, 4, 0.0, d, d, None, d, d, 5, d, ws, None) == 1
-    assert f(sh, d, d, R, 16, 128, 16, 4, 0.0, d, d, None, d, d, 6, d, ws, None) == 1
+    assert f(sh, d, d, R, 16, 128, 64, 4, 0.0, d, d, None, d, d, 6, d, ws, None) == 1
     assert f(sh, d, d, R, 16, 128, 0, 4, 0.0, d, None, None, d, d, 5, d, ws, None) == 1  # no K_rot
     assert f(sh, d, d, R, 16, 128, 0, 4, 0.0, d, d, None, d, d, 5, d, ws - 1, None) == 5
     # selection-side errors: null counts / idx, kmax too small, mass out of range

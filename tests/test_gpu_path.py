@@ -13,7 +13,8 @@ import torch
 
 from block_sparse_long_dual_b200 import sfa
 from block_sparse_long_dual_b200.synthetic import make_inputs
-from block_sparse_long_dual_b200.workloads import KEEP_SINK, NO_CALIB, RELATIVE_CALIB, SINGLE_BAND, TINY, Workload
+from block_sparse_long_dual_b200.workloads import (BAND_MAX, BLOCK_TAU, KEEP_SINK, NO_CALIB, RELATIVE_CALIB,
+                                                   SINGLE_BAND, TINY, Workload)
 from oracle import prism_oracle as po
 from tests.parity import compare_masks, rel_err, to_np
 
@@ -43,6 +44,13 @@ CASES = [
     W("bf16-one-block", seq_len=128, k=1),
     W("bf16-relative-calib-mass", seq_len=12 * 128, k=None, mass=0.9, slash=True, flags=RELATIVE_CALIB),
     W("bf16-relative-calib-single", seq_len=6 * 128, k=2, flags=RELATIVE_CALIB | SINGLE_BAND | KEEP_SINK),
+    W("bf16-band-max-mass", seq_len=14 * 128, k=None, mass=0.9, slash=True, flags=BAND_MAX),
+    W("bf16-band-max-topk-sink", seq_len=11 * 128, k=3, flags=BAND_MAX | KEEP_SINK),
+    W("bf16-block-tau-topk", seq_len=12 * 128, k=3, flags=BLOCK_TAU),
+    W("bf16-block-tau-band-max-mass", seq_len=10 * 128, k=None, mass=0.8, slash=True, flags=BLOCK_TAU | BAND_MAX),
+    W("f32-d64-b64-band-max-block-tau", dtype="f32", head_dim=64, block=64, band_split=16, seq_len=20 * 64, k=2,
+      flags=BAND_MAX | BLOCK_TAU),
+    W("bf16-band-max-single-band", seq_len=5 * 128, k=1, flags=BAND_MAX | SINGLE_BAND),
 ]
 
 
