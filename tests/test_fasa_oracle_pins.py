@@ -1,0 +1,165 @@
+"""Pins of the decode-side oracle ("FASA: Frequency-aware Sparse Attention", §2)
+against closed forms, torch routines, brute force and RoPE invariants."""
+
+import itertools
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import fasa_oracle as fo
+
+
+def _rope_torch(x, pos, base, d):
+    """Rotate-half RoPE at integer positions ``pos`` through transformers' rotate_half (float64)."""
+    from transformers.models.llama.modeling_llama import rotate_half
+    theta = base ** (-2.0 * torch.arange(d // 2, dtype=torch.float64) / d)
+    ang = torch.as_tensor(pos, dtype=torch.float64)[..., None] * theta
+    c = torch.cat([ang.cos(), ang.cos()], -1)
+    s = torch.cat([ang.sin(), ang.sin()], -1)
+    x = torch.as_tensor(x, dtype=torch.float64)
+    return x * c + rotate_half(x) * s
+
+
+def _inputs(B=2, Hq=4, Hkv=2, L=40, d=16, seed=0):
+    rng = np.random.default_rng(seed)
+    return (rng.normal(size=(B, Hq, d)), rng.normal(size=(B, Hkv, L, d)), rng.normal(size=(B, Hkv, L, d)))
+
+
+def test_all_pairs_dominant_is_full_dot_product():
+    q, K, _ = _inputs()
+    d = q.shape[-1]
+    fc = np.tile(np.arange(d // 2), (K.shape[1], 1))
+    s = fo.tip_scores(q, K, fc)
+    Kq = torch.repeat_interleave(torch.from_numpy(K), q.shape[1] // K.shape[1], dim=1)
+    ref = torch.einsum("bhd,bhtd->bht", torch.from_numpy(q), Kq).numpy()
+    np.testing.assert_allclose(s, ref, rtol=0, atol=1e-12)
+
+
+def test_subset_score_is_sum_over_chosen_pairs_only():
+    """Zeroing every dim outside the chosen pairs leaves the full dot product equal to the TIP score."""
+    q, K, _ = _inputs(seed=1)
+    d = q.shape[-1]
+    fc = np.array([[1, 5, 6], [0, 2, 7]])
+    s = fo.tip_scores(q, K, fc)
+    group = q.shape[1] // K.shape[1]
+    for h in range(q.shape[1]):
+        g = h // group
+        keep = np.zeros(d, dtype=bool)
+        keep[fc[g]] = True
+        keep[fc[g] + d // 2] = True
+        qm = torch.from_numpy(np.where(keep, q[:, h], 0.0))
+        ref = torch.einsum("bd,btd->bt", qm, torch.from_numpy(K[:, g])).numpy()
+        np.testing.assert_allclose(s[:, h], ref, rtol=0, atol=1e-12)
+
+
+def test_tip_scores_invariant_under_common_position_shift():
+    """Each rotary pair's dot product depends on the position difference only, so any subset of
+    pairs gives scores invariant under shifting the query and all keys by the same offset."""
+    B, Hq, Hkv, L, d, base = 1, 2, 1, 24, 16, 1e4
+    rng = np.random.default_rng(2)
+    q0, K0 = rng.normal(size=(B, Hq, d)), rng.normal(size=(B, Hkv, L, d))
+    fc = np.array([[0, 3, 6]])
+    out = []
+    for shift in (0, 37, 1000):
+        pos_k = np.arange(L) + shift
+        pos_q = np.full((B, Hq), L - 1 + shift)
+        q = _rope_torch(q0, pos_q, base, d).numpy()
+        K = _rope_torch(K0, pos_k, base, d).numpy()
+        out.append(fo.tip_scores(q, K, fc))
+    np.testing.assert_allclose(out[1], out[0], rtol=0, atol=1e-10)
+    np.testing.assert_allclose(out[2], out[0], rtol=0, atol=1e-10)
+    # the invariance is a property of the true pairs: mixing dims across pairs breaks it
+    bad = []
+    for shift in (0, 37):
+        pos_k = np.arange(L) + shift
+        q = _rope_torch(q0, np.full((B, Hq), L - 1 + shift), base, d).numpy()
+        K = _rope_torch(K0, pos_k, base, d).numpy()
+        dims = np.array([0, 1])  # halves of two different pairs
+        bad.append(np.einsum("bhd,btd->bht", q[..., dims], K[:, 0][..., dims]))
+    assert np.abs(bad[1] - bad[0]).max() > 1e-3
+
+
+def test_gather_fc_layout_gives_the_same_scores():
+    q, K, _ = _inputs(seed=3)
+    d = q.shape[-1]
+    fc = np.array([[2, 4, 0, 7], [1, 3, 5, 6]])
+    Kfc = fo.gather_fc(K, fc)
+    assert Kfc.shape == K.shape[:3] + (8,)
+    np.testing.assert_array_equal(Kfc[:, 1, :, 0], K[:, 1, :, 1])
+    np.testing.assert_array_equal(Kfc[:, 1, :, 4], K[:, 1, :, 1 + d // 2])
+    group = q.shape[1] // K.shape[1]
+    for h in range(q.shape[1]):
+        g = h // group
+        qd = q[:, h][:, fo.fc_dims(fc[g], d)]
+        np.testing.assert_allclose(np.einsum("bc,btc->bt", qd, Kfc[:, g]), fo.tip_scores(q, K, fc)[:, h],
+                                   rtol=0, atol=1e-12)
+
+
+def _dominates(a, ia, b, ib):
+    return a > b or (a == b and ia < ib)
+
+
+@pytest.mark.parametrize("seed", range(5))
+def test_selection_matches_bruteforce(seed):
+    rng = np.random.default_rng(seed)
+    L = 9
+    keys = (rng.integers(0, 5, size=L).astype(np.float32) - 2.0) / 4.0   # many exact ties, negatives
+    for k in range(0, L + 2):
+        got = fo.select_row(keys, k)
+        n = min(k, L)
+        found = [set(S) for S in itertools.combinations(range(L), n)
+                 if all(_dominates(keys[a], a, keys[b], b) for a in S for b in set(range(L)) - set(S))]
+        assert len(found) == 1
+        assert set(got.tolist()) == found[0]
+        assert list(got) == sorted(got)
+        best = max(sum(float(keys[t]) for t in S) for S in itertools.combinations(range(L), n)) if n else 0.0
+        assert sum(float(keys[t]) for t in got) == best
+    idx = fo.select_tokens(keys[None, None], L + 3)
+    assert list(idx[0, 0, :L]) == list(range(L)) and np.all(idx[0, 0, L:] == -1)
+
+
+def test_all_tokens_kept_is_dense_single_query_attention():
+    q, K, V = _inputs(seed=4)
+    B, Hq, d = q.shape
+    L = K.shape[2]
+    idx = np.tile(np.arange(L), (B, Hq, 1))
+    o, lse = fo.focused_attention(q, K, V, idx)
+    group = Hq // K.shape[1]
+    Kq = torch.repeat_interleave(torch.from_numpy(K), group, dim=1)
+    Vq = torch.repeat_interleave(torch.from_numpy(V), group, dim=1)
+    qt = torch.from_numpy(q)[:, :, None, :]
+    ref = torch.nn.functional.scaled_dot_product_attention(qt, Kq, Vq)[:, :, 0]
+    np.testing.assert_allclose(o, ref.numpy(), rtol=0, atol=1e-12)
+    lse_ref = torch.logsumexp(torch.einsum("bhd,bhtd->bht", torch.from_numpy(q), Kq) / math.sqrt(d), -1)
+    np.testing.assert_allclose(lse, lse_ref.numpy(), rtol=0, atol=1e-12)
+
+
+def test_single_kept_token_returns_its_value():
+    q, K, V = _inputs(seed=5)
+    B, Hq, d = q.shape
+    idx = -np.ones((B, Hq, 3), dtype=np.int64)
+    idx[..., 0] = 7
+    o, lse = fo.focused_attention(q, K, V, idx, scale=0.3)
+    group = Hq // K.shape[1]
+    for h in range(Hq):
+        np.testing.assert_array_equal(o[:, h], V[:, h // group, 7])
+        np.testing.assert_allclose(lse[:, h], 0.3 * np.einsum("bd,bd->b", q[:, h], K[:, h // group, 7]),
+                                   rtol=0, atol=1e-12)
+    # no kept token: zero output, lse = -inf
+    o0, lse0 = fo.focused_attention(q, K, V, -np.ones((B, Hq, 2), dtype=np.int64))
+    assert np.all(o0 == 0) and np.all(np.isneginf(lse0))
+
+
+def test_decode_step_top1_picks_planted_key():
+    """A key equal to a large multiple of the query in the dominant pairs wins the TIP, and FAC over
+    that single token returns its value."""
+    q, K, V = _inputs(B=1, Hq=2, Hkv=1, L=30, d=16, seed=6)
+    fc = np.array([[1, 4]])
+    d = 16
+    dims = fo.fc_dims(fc[0], d)
+    K[0, 0, 11, dims] = 50.0 * q[0, 0, dims]
+    _, _, idx, o, _ = fo.decode_step(q, K, V, fc, 1)
+    assert idx[0, 0, 0] == 11
+    np.testing.assert_array_equal(o[0, 0], V[0, 0, 11])
