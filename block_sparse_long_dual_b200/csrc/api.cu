@@ -341,3 +341,116 @@ sfa_status sfa_block_sparse_attn_rope(const sfa_shape* shape, int block, const v
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Decode step
+// ---------------------------------------------------------------------------
+namespace {
+
+sfa_status check_decode_shape(const sfa_shape* s) {
+  if (s == nullptr) return SFA_ERR_INVALID_ARG;
+  if (s->dtype != SFA_BF16) return SFA_ERR_DTYPE;
+  if (s->batch < 1 || s->heads_q < 1 || s->heads_kv < 1 || s->seq_len < 1) return SFA_ERR_SHAPE;
+  if (s->head_dim != 64 && s->head_dim != 128) return SFA_ERR_SHAPE;
+  if (s->heads_q % s->heads_kv != 0) return SFA_ERR_SHAPE;
+  const int group = s->heads_q / s->heads_kv;
+  if (group != 1 && group != 2 && group != 4 && group != 8) return SFA_ERR_UNSUPPORTED;
+  if ((long long)s->batch * s->heads_kv * s->seq_len >= (1LL << 31)) return SFA_ERR_UNSUPPORTED;
+  return SFA_OK;
+}
+
+// Fills the shape fields and the dominant-pair table of p; validates fc.
+sfa_status decode_params(const sfa_shape* s, const int* fc, int nfc, DecodeParams* p) {
+  sfa_status st = check_decode_shape(s);
+  if (st != SFA_OK) return st;
+  memset(p, 0, sizeof(*p));
+  p->B = s->batch; p->Hq = s->heads_q; p->Hkv = s->heads_kv; p->L = s->seq_len; p->D = s->head_dim;
+  const int half = s->head_dim / 2;
+  // Without a pair list (sizing, attention) the geometry of the widest list bounds the workspace.
+  const DecodeGeometry geo = decode_geometry(s->heads_q / s->heads_kv, fc == nullptr ? half : nfc);
+  p->chunk = geo.chunk;
+  p->tps = geo.tps;
+  p->nstages = geo.nstages;
+  p->nchunks = (s->seq_len + p->chunk - 1) / p->chunk;
+  if (p->nchunks > decode_max_chunks()) return SFA_ERR_UNSUPPORTED;
+  if (fc == nullptr) return nfc == 0 ? SFA_OK : SFA_ERR_INVALID_ARG;
+  if (nfc < 4 || nfc > half || nfc % 4 != 0 || s->heads_kv * nfc > (int)sizeof(p->fc)) return SFA_ERR_INVALID_ARG;
+  for (int g = 0; g < s->heads_kv; ++g) {
+    unsigned long long seen = 0;
+    for (int c = 0; c < nfc; ++c) {
+      const int m = fc[g * nfc + c];
+      if (m < 0 || m >= half || (seen >> m) & 1ull) return SFA_ERR_INVALID_ARG;
+      seen |= 1ull << m;
+      p->fc[g * nfc + c] = (uint8_t)m;
+    }
+  }
+  p->nfc = nfc;
+  return SFA_OK;
+}
+
+// Candidate slots: every chunk of every row may keep up to all its tokens.  Sized for the
+// largest chunk geometry (4096 tokens) and the most chunks (1024 tokens each), so one
+// workspace serves every pair list.
+size_t decode_ws_bytes(const DecodeParams& p, int /*k*/) {
+  const size_t rows = (size_t)p.B * p.Hq;
+  const size_t slots = rows * (((size_t)p.L + 4095) / 4096) * 4096;
+  const size_t counts = rows * (((size_t)p.L + 1023) / 1024) * 8;
+  return 2 * align256(slots * sizeof(uint32_t)) + align256(counts * sizeof(int));
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sfa_decode_workspace(const sfa_shape* shape, int k) {
+  DecodeParams p;
+  if (k < 1 || decode_params(shape, nullptr, 0, &p) != SFA_OK) return 0;
+  return decode_ws_bytes(p, k);
+}
+
+sfa_status sfa_decode_fc_gather(const sfa_shape* shape, const void* K_cache, const int* fc, int nfc, int pos0,
+                                int npos, void* K_fc, void* stream) {
+  DecodeParams p;
+  sfa_status st = decode_params(shape, fc, nfc, &p);
+  if (st != SFA_OK) return st;
+  if (fc == nullptr || K_cache == nullptr || K_fc == nullptr) return SFA_ERR_INVALID_ARG;
+  if (pos0 < 0 || npos < 0 || (long long)pos0 + npos > shape->seq_len) return SFA_ERR_INVALID_ARG;
+  if (!aligned16(K_cache) || !aligned16(K_fc)) return SFA_ERR_INVALID_ARG;
+  return cuda_status(launch_fc_gather(p, K_cache, K_fc, pos0, npos, as_stream(stream)));
+}
+
+sfa_status sfa_decode_select(const sfa_shape* shape, const void* q, const void* K_fc, const int* fc, int nfc, int k,
+                             int* idx, void* workspace, size_t workspace_bytes, int* status_word, void* stream) {
+  DecodeParams p;
+  sfa_status st = decode_params(shape, fc, nfc, &p);
+  if (st != SFA_OK) return st;
+  if (fc == nullptr || q == nullptr || K_fc == nullptr || idx == nullptr || k < 1) return SFA_ERR_INVALID_ARG;
+  if (!aligned16(K_fc)) return SFA_ERR_INVALID_ARG;
+  const size_t need = decode_ws_bytes(p, k);
+  if (workspace == nullptr || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255))
+    return SFA_ERR_WORKSPACE;
+  const size_t n = (size_t)p.B * p.Hq * p.nchunks * p.chunk;
+  unsigned char* ws = static_cast<unsigned char*>(workspace);
+  p.q = q; p.Kfc = K_fc; p.idx = idx; p.k = k; p.status = status_word;
+  p.cand_key = reinterpret_cast<uint32_t*>(ws);
+  p.cand_idx = reinterpret_cast<int*>(ws + align256(n * sizeof(uint32_t)));
+  p.cand_count = reinterpret_cast<int*>(ws + 2 * align256(n * sizeof(uint32_t)));
+  return cuda_status(launch_decode_select(p, as_stream(stream)));
+}
+
+sfa_status sfa_decode_attn(const sfa_shape* shape, const void* q, const void* K_cache, const void* V_cache,
+                           const int* idx, int k, float scale, void* o, float* lse, int* status_word, void* stream) {
+  DecodeParams p;
+  sfa_status st = decode_params(shape, nullptr, 0, &p);
+  if (st != SFA_OK) return st;
+  if (q == nullptr || K_cache == nullptr || V_cache == nullptr || idx == nullptr || o == nullptr || k < 1)
+    return SFA_ERR_INVALID_ARG;
+  if (!isfinite(scale)) return SFA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(K_cache) || !aligned16(V_cache)) return SFA_ERR_INVALID_ARG;
+  p.q = q; p.Kc = K_cache; p.Vc = V_cache; p.idx = const_cast<int*>(idx); p.k = k;
+  p.o = o; p.lse = lse; p.status = status_word;
+  p.scale = scale > 0.f ? scale : (float)(1.0 / sqrt((double)shape->head_dim));
+  return cuda_status(launch_decode_attn(p, as_stream(stream)));
+}
+
+}  // extern "C"

@@ -1,0 +1,846 @@
+// Decode-side estimate -> exact attention ("FASA: Frequency-aware Sparse
+// Attention" §2B): one query token per (batch, Q head) against a KV cache.
+//
+//   fc_gather      compact copy K_fc [B, Hkv, L, 2 nfc] of the dominant rotary
+//                  pairs of the rotated key cache (low dims, then partners);
+//                  run once over the cache, then per appended token range.
+//   tip_chunk      Token Importance Predictor: CTA = (chunk of C tokens, KV
+//                  head); streams the chunk's K_fc rows once for all Q heads of
+//                  the group; each score is a float32 FMA chain over the
+//                  compact columns in order (a bf16 x bf16 product is exact in
+//                  float32, so every step rounds once and the value is
+//                  reproducible); then each head's local top-k of the
+//                  chunk by a block-wide radix select, written in token order.
+//   tip_merge      CTA per (b, h): radix select over the chunks' candidates
+//                  (already in token order), ascending index list, -1 padded.
+//   fac            Focused Attention Computation: CTA per (b, h), 16 warps,
+//                  each warp gathers the K / V rows of its share of the kept
+//                  tokens (eight tokens' loads in flight per lane), float32
+//                  online softmax, warps merged through shared memory.
+//
+// Ranking: key = order-preserving uint32 of the float32 score (+0 for both
+// zeros); the first k by (key desc, index asc).
+#include <math.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace sfa {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = kThreads / 32;
+
+__device__ __forceinline__ uint32_t order_key(float f) {
+  uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+// The k-th largest of n keys (1 <= k <= n) by MSB-first 8-bit radix select over a
+// block of kThreads threads: returns T and sets *gt = #{key > T}.
+template <typename KeyAt>
+__device__ uint32_t block_kth_largest(KeyAt key_at, int n, int k, uint32_t* hist, int* sh, int* gt) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  uint32_t prefix = 0, pmask = 0;
+  int krem = k;
+  for (int shift = 24; shift >= 0; shift -= 8) {
+    for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
+    __syncthreads();
+    // Warp-aggregated increments: keys cluster in a few digits (float exponents), so lanes with
+    // the same digit add once through their lowest lane instead of serialising on one bin.
+    for (int i0 = 0; i0 < n; i0 += kThreads) {
+      const int i = i0 + tid;
+      int bin = -1;
+      if (i < n) {
+        const uint32_t u = key_at(i);
+        if ((u & pmask) == prefix) bin = (int)((u >> shift) & 255u);
+      }
+      const unsigned same = __match_any_sync(0xffffffffu, bin);
+      if (bin >= 0 && lane == __ffs(same) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(same));
+    }
+    __syncthreads();
+    if (warp == 0) {
+      // lane l owns digits 255 - 8l - j, j = 0..7 (descending)
+      uint32_t c[8];
+      int s = 0;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        c[j] = hist[255 - 8 * lane - j];
+        s += (int)c[j];
+      }
+      int incl = s;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, incl, off);
+        if (lane >= off) incl += y;
+      }
+      const int excl = incl - s;  // keys in higher digits than this lane's
+      if (excl < krem && krem <= incl) {
+        int above = excl;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          if (above < krem && krem <= above + (int)c[j]) {
+            sh[0] = 255 - 8 * lane - j;
+            sh[1] = above;
+          }
+          above += (int)c[j];
+        }
+      }
+    }
+    __syncthreads();
+    const uint32_t digit = (uint32_t)sh[0];
+    krem -= sh[1];
+    prefix |= digit << shift;
+    pmask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  *gt = k - krem;
+  return prefix;
+}
+
+// Sum of a warp-uniform value over the warps before this one (and the block total).
+__device__ int warp_exclusive_sum(int v, int* sh, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) sh[warp] = v;
+  __syncthreads();
+  int before = 0, all = 0;
+#pragma unroll
+  for (int w = 0; w < kWarps; ++w) {
+    const int x = sh[w];
+    before += w < warp ? x : 0;
+    all += x;
+  }
+  __syncthreads();
+  *total = all;
+  return before;
+}
+
+// Stable compaction of the first k keys by (key desc, index asc) out of n (k >= n keeps all):
+// emit(rank, i) for the kept i in ascending i, rank = 0, 1, ...  Returns the kept count.
+// Warp w owns a contiguous range of 32-key groups; lane j takes key 32 g + j of each group, so
+// shared-memory reads are conflict-free and global reads coalesced; ranks come from ballots.
+template <typename KeyAt, typename Emit>
+__device__ int block_select_ordered(KeyAt key_at, int n, int k, Emit emit, uint32_t* hist, int* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  uint32_t T = 0;
+  int take = n;  // ties at T to keep (all when every key is kept)
+  const bool all = k >= n;
+  if (!all) {
+    int gt = 0;
+    T = block_kth_largest(key_at, n, k, hist, sh, &gt);
+    take = k - gt;
+  }
+  const int S = ((n + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  const int w0 = min(n, warp * S), w1 = min(n, w0 + S);
+  int nt = 0;
+  if (!all)
+    for (int b = w0; b < w1; b += 32) {
+      const int i = b + lane;
+      nt += __popc(__ballot_sync(0xffffffffu, i < w1 && key_at(i) == T));
+    }
+  int tot = 0;
+  const int tie_base = warp_exclusive_sum(nt, sh + 4, &tot);
+  int nk = 0, tr = tie_base;
+  for (int b = w0; b < w1; b += 32) {
+    const int i = b + lane;
+    const uint32_t u = (i < w1 && !all) ? key_at(i) : 0u;
+    const bool tie = i < w1 && !all && u == T;
+    const unsigned tb = __ballot_sync(0xffffffffu, tie);
+    const bool keep = i < w1 && (all || u > T || (tie && tr + __popc(tb & lt) < take));
+    nk += __popc(__ballot_sync(0xffffffffu, keep));
+    tr += __popc(tb);
+  }
+  int kept = 0;
+  int pos = warp_exclusive_sum(nk, sh + 4, &kept);
+  tr = tie_base;
+  for (int b = w0; b < w1; b += 32) {
+    const int i = b + lane;
+    const uint32_t u = (i < w1 && !all) ? key_at(i) : 0u;
+    const bool tie = i < w1 && !all && u == T;
+    const unsigned tb = __ballot_sync(0xffffffffu, tie);
+    const bool keep = i < w1 && (all || u > T || (tie && tr + __popc(tb & lt) < take));
+    const unsigned kb = __ballot_sync(0xffffffffu, keep);
+    if (keep) emit(pos + __popc(kb & lt), i);
+    pos += __popc(kb);
+    tr += __popc(tb);
+  }
+  return kept;
+}
+
+// Block-wide: emit(rank, i) for every i in [0, n) with key_at(i) >= LB, in ascending i; returns
+// the count.  Warp-contiguous ranges of 32-key groups, ranks from ballots.
+template <typename KeyAt, typename Emit>
+__device__ int block_filter_ordered(KeyAt key_at, int n, uint32_t LB, Emit emit, int* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  const int S = ((n + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+  const int w0 = min(n, warp * S), w1 = min(n, w0 + S);
+  int nk = 0;
+  for (int b = w0; b < w1; b += 32) {
+    const int i = b + lane;
+    nk += __popc(__ballot_sync(0xffffffffu, i < w1 && key_at(i) >= LB));
+  }
+  int total = 0;
+  int pos = warp_exclusive_sum(nk, sh, &total);
+  for (int b = w0; b < w1; b += 32) {
+    const int i = b + lane;
+    const bool keep = i < w1 && key_at(i) >= LB;
+    const unsigned kb = __ballot_sync(0xffffffffu, keep);
+    if (keep) emit(pos + __popc(kb & lt), i);
+    pos += __popc(kb);
+  }
+  return total;
+}
+
+// Block-wide lower bound, NH independent problems at once: for each h, a value LB with at
+// least k of the block's values v[h][.] >= LB (every thread holds NV of them; k <= 256 NV).
+// Bisection from the bracket [min, max + 1) keeps that invariant at every step, so stopping
+// after ITERS steps gives a valid (if looser) bound.  One barrier per step: the per-warp counts
+// alternate between two halves of sh (2 * 8 * NH ints).
+template <int NH, int NV, int ITERS>
+__device__ void block_lower_bound(const uint32_t (&v)[NH][NV], int k, uint32_t (&LB)[NH], int* sh) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint64_t lo[NH], hi[NH];
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+    for (int j = 0; j < NV; ++j) { mn = min(mn, v[h][j]); mx = max(mx, v[h][j]); }
+    mn = __reduce_min_sync(0xffffffffu, mn);
+    mx = __reduce_max_sync(0xffffffffu, mx);
+    if (lane == 0) { sh[warp * NH + h] = (int)mn; sh[(kWarps + warp) * NH + h] = (int)mx; }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < NH; ++h) {
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      mn = min(mn, (uint32_t)sh[w * NH + h]);
+      mx = max(mx, (uint32_t)sh[(kWarps + w) * NH + h]);
+    }
+    lo[h] = mn;  // every value >= min: #{>= lo} = 256 NV >= k
+    hi[h] = (uint64_t)mx + 1;
+  }
+  __syncthreads();
+  for (int it = 0; it < ITERS; ++it) {
+    int* cs = sh + (it & 1) * kWarps * NH;
+    uint32_t mid[NH];
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      mid[h] = (uint32_t)(lo[h] + ((hi[h] - lo[h]) >> 1));
+      int c = 0;
+#pragma unroll
+      for (int j = 0; j < NV; ++j) c += v[h][j] >= mid[h] ? 1 : 0;
+      c = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+      if (lane == 0) cs[warp * NH + h] = c;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int h = 0; h < NH; ++h) {
+      int c = 0;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) c += cs[w * NH + h];
+      if (hi[h] - lo[h] > 1) {
+        if (c >= k) lo[h] = mid[h]; else hi[h] = mid[h];
+      }
+    }
+  }
+  __syncthreads();
+#pragma unroll
+  for (int h = 0; h < NH; ++h) LB[h] = (uint32_t)lo[h];
+}
+
+// Block-wide bisection over n values in shared memory (1 <= k <= n): the k-th largest T and
+// *gt = #{> T}.  Bracketed by the values' minimum and maximum.
+__device__ uint32_t block_kth_largest_smem(const uint32_t* vals, int n, int k, int* sh, int* gt) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+  for (int i = threadIdx.x; i < n; i += kThreads) {
+    mn = min(mn, vals[i]);
+    mx = max(mx, vals[i]);
+  }
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  if (lane == 0) { sh[warp] = (int)mn; sh[kWarps + warp] = (int)mx; }
+  __syncthreads();
+  for (int w = 0; w < kWarps; ++w) {
+    mn = min(mn, (uint32_t)sh[w]);
+    mx = max(mx, (uint32_t)sh[kWarps + w]);
+  }
+  __syncthreads();
+  uint64_t lo = mn, hi = (uint64_t)mx + 1;
+  while (hi - lo > 1) {  // uniform across the block
+    const uint32_t mid = (uint32_t)(lo + ((hi - lo) >> 1));
+    int c = 0;
+    for (int i = threadIdx.x; i < n; i += kThreads) c += vals[i] >= mid ? 1 : 0;
+    c = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
+    if (lane == 0) sh[warp] = c;
+    __syncthreads();
+    int t = 0;
+    for (int w = 0; w < kWarps; ++w) t += sh[w];
+    __syncthreads();
+    if (t >= k) lo = mid; else hi = mid;
+  }
+  const uint32_t T = (uint32_t)lo;
+  int g = 0;
+  for (int i = threadIdx.x; i < n; i += kThreads) g += vals[i] > T ? 1 : 0;
+  g = (int)__reduce_add_sync(0xffffffffu, (unsigned)g);
+  if (lane == 0) sh[warp] = g;
+  __syncthreads();
+  int t = 0;
+  for (int w = 0; w < kWarps; ++w) t += sh[w];
+  __syncthreads();
+  *gt = t;
+  return T;
+}
+
+// ---------------------------------------------------------------------------
+// fc_gather
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kThreads) fc_gather_kernel(DecodeParams p, const void* Kc, void* Kfc, int pos0,
+                                                             int npos) {
+  const int W = 2 * p.nfc;          // columns of a compact row
+  const int G8 = W / 8;             // 16-byte groups per compact row
+  const size_t items = (size_t)p.B * p.Hkv * npos * G8;
+  for (size_t it = (size_t)blockIdx.x * kThreads + threadIdx.x; it < items; it += (size_t)gridDim.x * kThreads) {
+    const int grp = (int)(it % G8);
+    size_t r = it / G8;
+    const int t = pos0 + (int)(r % npos);
+    const int bg = (int)(r / npos);  // b * Hkv + g
+    const int g = bg % p.Hkv;
+    const __nv_bfloat16* krow = static_cast<const __nv_bfloat16*>(Kc) + ((size_t)bg * p.L + t) * p.D;
+    uint16_t v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int c = grp * 8 + e;
+      const int dim = c < p.nfc ? p.fc[g * p.nfc + c] : p.fc[g * p.nfc + c - p.nfc] + p.D / 2;
+      v[e] = reinterpret_cast<const uint16_t*>(krow)[dim];
+    }
+    uint4 o;
+    o.x = v[0] | ((uint32_t)v[1] << 16);
+    o.y = v[2] | ((uint32_t)v[3] << 16);
+    o.z = v[4] | ((uint32_t)v[5] << 16);
+    o.w = v[6] | ((uint32_t)v[7] << 16);
+    reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(Kfc) + ((size_t)bg * p.L + t) * W)[grp] = o;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// tip_chunk: persistent, one CTA per SM, looping over tiles (chunk, b, KV head);
+// G = Q heads per KV head, TPS = tokens per thread per slab, NGR = groups of 4
+// keys per thread per chunk.  The chunk's compact key rows stream through an
+// NS-stage ring of slabs (ST = 256 TPS tokens) filled by bulk copies; the ring
+// runs across tiles, so the next tile's first slabs are in flight while this
+// tile's candidates are selected.
+// ---------------------------------------------------------------------------
+template <int G, int TPS, int NGR>
+__global__ void __launch_bounds__(kThreads, 1) tip_chunk_kernel(DecodeParams p) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  constexpr int ST = kThreads * TPS;
+  const int W = 2 * p.nfc;
+  const int C = p.chunk;
+  const int NS = p.nstages;
+  const uint32_t SB = (uint32_t)ST * W * 2;                                                // slab bytes
+  unsigned char* ring = smem_raw;                                                           // [NS][SB]
+  uint32_t* keys = reinterpret_cast<uint32_t*>(ring + (size_t)NS * SB);                   // [G][C]
+  float* qd = reinterpret_cast<float*>(keys + (size_t)G * C);                              // [W][G]
+  __shared__ __align__(8) uint64_t bars[4];
+  __shared__ int scratch[128];
+  __shared__ int lost;
+
+  const int tid = threadIdx.x;
+  const int ntiles = p.nchunks * p.B * p.Hkv;
+  const __nv_bfloat16* kfc_all = static_cast<const __nv_bfloat16*>(p.Kfc);
+  auto slabs_of = [&](int tile) {
+    const int n = min(C, p.L - (tile % p.nchunks) * C);
+    return (n + ST - 1) / ST;
+  };
+  // Producer state (thread 0): next (tile, slab) to copy and the stage it goes to.
+  int ptile = blockIdx.x, pslab = 0, issued = 0;
+  auto issue_next = [&]() {
+    if (ptile >= ntiles) return;
+    const int chunk = ptile % p.nchunks, bg = ptile / p.nchunks;
+    const int n = min(C, p.L - chunk * C);
+    const int rows = min(ST, n - pslab * ST);
+    const __nv_bfloat16* src = kfc_all + ((size_t)bg * p.L + (size_t)chunk * C + (size_t)pslab * ST) * W;
+    const int stg = issued % NS;
+    arm_and_load((uint32_t)__cvta_generic_to_shared(&bars[stg]), (uint32_t)__cvta_generic_to_shared(ring + (size_t)stg * SB),
+                 src, (uint32_t)rows * W * 2);
+    ++issued;
+    if (++pslab == slabs_of(ptile)) {
+      pslab = 0;
+      ptile += gridDim.x;
+    }
+  };
+  if (tid == 0) {
+    lost = 0;
+    for (int st = 0; st < NS; ++st)
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"((uint32_t)__cvta_generic_to_shared(&bars[st]))
+                   : "memory");
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    for (int st = 0; st < NS; ++st) issue_next();
+  }
+  __syncthreads();
+
+  int consumed = 0;
+  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+    const int chunk = tile % p.nchunks, bg = tile / p.nchunks;
+    const int b = bg / p.Hkv, g = bg % p.Hkv;
+    const int t0 = chunk * C;
+    const int n = min(C, p.L - t0);
+    const int nsl = (n + ST - 1) / ST;
+
+    // The group's query values on the dominant dims, column-major: qd[c * G + head].
+    for (int e = tid; e < G * W; e += kThreads) {
+      const int hh = e % G, c = e / G;
+      const int dim = c < p.nfc ? p.fc[g * p.nfc + c] : p.fc[g * p.nfc + c - p.nfc] + p.D / 2;
+      const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + g * G + hh) * p.D;
+      qd[c * G + hh] = __bfloat162float(qrow[dim]);
+    }
+    __syncthreads();
+
+    // Scores: a float32 FMA chain per (token, head) over the columns in order.  Thread tid takes
+    // tokens tid + 256 u of each slab; its j-th key of the chunk (j = slab TPS + u) joins group j / 4.
+    uint32_t gmax[G][NGR];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh)
+#pragma unroll
+      for (int r = 0; r < NGR; ++r) gmax[hh][r] = 0u;
+    for (int sl = 0; sl < nsl; ++sl, ++consumed) {
+      const int stg = consumed % NS;
+      if (!wait_parity_bounded((uint32_t)__cvta_generic_to_shared(&bars[stg]), (consumed / NS) & 1)) lost = 1;
+      const __nv_bfloat16* slab = reinterpret_cast<const __nv_bfloat16*>(ring + (size_t)stg * SB);
+      float acc[TPS][G];
+#pragma unroll
+      for (int u = 0; u < TPS; ++u)
+#pragma unroll
+        for (int hh = 0; hh < G; ++hh) acc[u][hh] = 0.f;
+      for (int q8 = 0; q8 < W / 8; ++q8) {
+        uint32_t w4[TPS][4];
+#pragma unroll
+        for (int u = 0; u < TPS; ++u) {
+          const uint4 v = reinterpret_cast<const uint4*>(slab + (size_t)(u * kThreads + tid) * W)[q8];
+          w4[u][0] = v.x; w4[u][1] = v.y; w4[u][2] = v.z; w4[u][3] = v.w;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const int c = q8 * 8 + e;
+          float qv[G];
+          if constexpr (G % 4 == 0) {
+#pragma unroll
+            for (int h4 = 0; h4 < G; h4 += 4) {
+              const float4 f = *reinterpret_cast<const float4*>(qd + c * G + h4);
+              qv[h4] = f.x; qv[h4 + 1] = f.y; qv[h4 + 2] = f.z; qv[h4 + 3] = f.w;
+            }
+          } else {
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) qv[hh] = qd[c * G + hh];
+          }
+#pragma unroll
+          for (int u = 0; u < TPS; ++u) {
+            const uint32_t w = w4[u][e >> 1];
+            const float kv = __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
+#pragma unroll
+            for (int hh = 0; hh < G; ++hh) acc[u][hh] = fmaf(qv[hh], kv, acc[u][hh]);
+          }
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < TPS; ++u) {
+        const int t = sl * ST + u * kThreads + tid;
+        const int grp = (sl * TPS + u) >> 2;
+        if (t < n) {
+#pragma unroll
+          for (int hh = 0; hh < G; ++hh) {
+            const uint32_t key = order_key(acc[u][hh]);
+            keys[(size_t)hh * C + t] = key;
+#pragma unroll
+            for (int r = 0; r < NGR; ++r)
+              if (r == grp) gmax[hh][r] = max(gmax[hh][r], key);
+          }
+        }
+      }
+      __syncthreads();  // stage consumed
+      if (tid == 0) issue_next();
+    }
+
+    // Per head, a lower bound LB of the chunk's k-th largest key: a value with at least k of the
+    // 256 NGR group maxima (each a distinct key, or 0) at or above it, when k <= 256 NGR.  Every
+    // token of the row's top k has a key >= the row's k-th largest >= the chunk's k-th largest
+    // >= LB, so keys below LB are dropped.
+    uint32_t LB[G];
+    if (p.k <= kThreads * NGR) {
+      block_lower_bound<G, NGR, 16>(gmax, p.k, LB, scratch);
+    } else {
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) LB[hh] = 0u;
+    }
+    // Candidates in token order: warp w scans its contiguous range [w S, w S + S) of the chunk
+    // and writes its own segment of the slot; counts per (slot, warp).
+    const int bad = lost;
+    {
+      const int lane = tid & 31, warp = tid >> 5;
+      const unsigned lt = (1u << lane) - 1u;
+      const int S = C / kWarps;
+      const int w0 = min(n, warp * S), w1 = min(n, w0 + S);
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) {
+        const size_t slot = ((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk;
+        uint32_t* ck = p.cand_key + slot * C + (size_t)warp * S;
+        int* ci = p.cand_idx + slot * C + (size_t)warp * S;
+        const uint32_t* hk = keys + (size_t)hh * C;
+        int cnt = 0;
+        for (int b0 = w0; b0 < w1; b0 += 32) {
+          const int i = b0 + lane;
+          const uint32_t u = i < w1 ? hk[i] : 0u;
+          const bool keep = i < w1 && u >= LB[hh];
+          const unsigned kb = __ballot_sync(0xffffffffu, keep);
+          if (keep) {
+            ck[cnt + __popc(kb & lt)] = u;
+            ci[cnt + __popc(kb & lt)] = t0 + i;
+          }
+          cnt += __popc(kb);
+        }
+        if (lane == 0) p.cand_count[slot * kWarps + warp] = bad ? 0 : cnt;
+      }
+    }
+    if (bad && tid == 0) report(p.status, SFA_ERR_TIMEOUT);
+    __syncthreads();  // keys / qd free for the next tile
+  }
+  // After a wait that gave up, let this CTA's copies land (bounded) before it exits.
+  if (tid == 0 && lost) {
+    for (int st = 0; st < NS && st < issued; ++st) {
+      const int uses = (issued - st + NS - 1) / NS;
+      wait_parity_bounded((uint32_t)__cvta_generic_to_shared(&bars[st]), (uses - 1) & 1);
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------
+// tip_merge: CTA per (b, h).  The chunks' candidates (token order, counts per
+// chunk) are staged in shared memory when they fit (kMergeSmem); bounded again
+// (with k <= 256, the least of the 256 threads' maxima is at most the k-th
+// largest), compacted, and the exact k-th largest found by block bisection;
+// the first k by (key desc, index asc) are written ascending.  More
+// candidates than fit use the block radix select over global memory.
+// ---------------------------------------------------------------------------
+constexpr int kMergeSmem = 12288;
+constexpr int kMaxChunks = 512;
+
+__global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
+  extern __shared__ __align__(16) uint32_t msm[];
+  __shared__ uint32_t hist[256];
+  __shared__ int sh[64];
+  const size_t row = blockIdx.x;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nseg = p.nchunks * kWarps;
+  const int S = p.chunk / kWarps;
+  const uint32_t* ck = p.cand_key + row * p.nchunks * p.chunk;
+  const int* ci = p.cand_idx + row * p.nchunks * p.chunk;
+  const int* cc = p.cand_count + row * nseg;
+  int* out = p.idx + row * p.k;
+  int* off = reinterpret_cast<int*>(msm);  // [nseg + 1] prefix of the segment counts
+  {
+    // block scan of the segment counts, kThreads segments at a time
+    int carry = 0;
+    for (int base = 0; base < nseg; base += kThreads) {
+      const int sidx = base + tid;
+      const int v = sidx < nseg ? cc[sidx] : 0;
+      int tot = 0;
+      int x = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (lane == 31) sh[warp] = x;
+      __syncthreads();
+      int before = 0;
+      for (int w = 0; w < kWarps; ++w) {
+        before += w < warp ? sh[w] : 0;
+        tot += sh[w];
+      }
+      if (sidx < nseg) off[sidx] = carry + before + x - v;
+      carry += tot;
+      __syncthreads();
+    }
+    if (tid == 0) off[nseg] = carry;
+    __syncthreads();
+  }
+  const int n = off[nseg];
+  // flat candidate position -> offset in the slot array (segment by binary search)
+  auto locate = [&](int i) -> size_t {
+    int lo = 0, hi = nseg;  // off[lo] <= i < off[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (off[mid] <= i) lo = mid; else hi = mid;
+    }
+    return (size_t)lo * S + (i - off[lo]);
+  };
+  int kept;
+  const int ob = (nseg + 1 + 3) & ~3;  // keys start after the offsets (16-byte aligned)
+  if (n <= kMergeSmem) {
+    uint32_t* sk = msm + ob;                              // [n] keys
+    int* st = reinterpret_cast<int*>(sk + n);             // [n] token indices
+    int* sv = st + n;                                     // [n] survivor positions
+    uint32_t* gk = reinterpret_cast<uint32_t*>(sv + n);   // [n] survivor keys
+    for (int i = tid; i < n; i += kThreads) {
+      const size_t o = locate(i);
+      sk[i] = __ldg(ck + o);
+      st[i] = __ldg(ci + o);
+    }
+    __syncthreads();
+    if (p.k >= n) {
+      for (int i = tid; i < n; i += kThreads) out[i] = st[i];
+      kept = n;
+    } else {
+      uint32_t LB = 0u;
+      if (p.k <= kThreads) {
+        // the least of the 256 threads' maxima is at most the k-th largest when k <= 256
+        uint32_t m = 0u;
+        for (int i = tid; i < n; i += kThreads) m = max(m, sk[i]);
+        m = __reduce_min_sync(0xffffffffu, m);
+        if (lane == 0) sh[warp] = (int)m;
+        __syncthreads();
+        LB = 0xFFFFFFFFu;
+        for (int w = 0; w < kWarps; ++w) LB = min(LB, (uint32_t)sh[w]);
+        __syncthreads();
+      }
+      const int ns = block_filter_ordered([&](int i) { return sk[i]; }, n, LB, [&](int r, int i) { sv[r] = i; },
+                                          sh + 16);
+      __syncthreads();
+      for (int j = tid; j < ns; j += kThreads) gk[j] = sk[sv[j]];
+      __syncthreads();
+      int gt = 0;
+      const uint32_t T = block_kth_largest_smem(gk, ns, p.k, sh, &gt);
+      const int take = p.k - gt;
+      // ordered emission over the survivors with ties by index
+      const unsigned lt = (1u << lane) - 1u;
+      const int SW = ((ns + kWarps * 32 - 1) / (kWarps * 32)) * 32;
+      const int w0 = min(ns, warp * SW), w1 = min(ns, w0 + SW);
+      int nt = 0;
+      for (int b = w0; b < w1; b += 32) {
+        const int j = b + lane;
+        nt += __popc(__ballot_sync(0xffffffffu, j < w1 && gk[j] == T));
+      }
+      int tot = 0;
+      const int tie_base = warp_exclusive_sum(nt, sh + 16, &tot);
+      int nk = 0, tr = tie_base;
+      for (int b = w0; b < w1; b += 32) {
+        const int j = b + lane;
+        const uint32_t u = j < w1 ? gk[j] : 0u;
+        const bool tie = j < w1 && u == T;
+        const unsigned tb = __ballot_sync(0xffffffffu, tie);
+        const bool keep = j < w1 && (u > T || (tie && tr + __popc(tb & lt) < take));
+        nk += __popc(__ballot_sync(0xffffffffu, keep));
+        tr += __popc(tb);
+      }
+      int pos = warp_exclusive_sum(nk, sh + 16, &kept);
+      tr = tie_base;
+      for (int b = w0; b < w1; b += 32) {
+        const int j = b + lane;
+        const uint32_t u = j < w1 ? gk[j] : 0u;
+        const bool tie = j < w1 && u == T;
+        const unsigned tb = __ballot_sync(0xffffffffu, tie);
+        const bool keep = j < w1 && (u > T || (tie && tr + __popc(tb & lt) < take));
+        const unsigned kb = __ballot_sync(0xffffffffu, keep);
+        if (keep) out[pos + __popc(kb & lt)] = st[sv[j]];
+        pos += __popc(kb);
+        tr += __popc(tb);
+      }
+    }
+  } else {
+    kept = block_select_ordered([&](int i) { return __ldg(ck + locate(i)); }, n, p.k,
+                                [&](int r, int i) { out[r] = __ldg(ci + locate(i)); }, hist, sh);
+  }
+  for (int r = kept + tid; r < p.k; r += kThreads) out[r] = -1;
+}
+
+// ---------------------------------------------------------------------------
+// fac: CTA per (b, h), 16 warps
+// ---------------------------------------------------------------------------
+constexpr int kFacWarps = 16;
+constexpr int kFacBatch = 8;  // tokens per warp with loads in flight
+
+template <int D>
+__global__ void __launch_bounds__(kFacWarps * 32) fac_kernel(DecodeParams p) {
+  constexpr int DPL = D / 32;  // dims per lane (4 for d = 128, 2 for d = 64)
+  __shared__ float wm[kFacWarps], wl[kFacWarps];
+  __shared__ float wacc[kFacWarps][D];
+  __shared__ int bad;
+  const size_t row = blockIdx.x;
+  const int b = (int)(row / p.Hq), h = (int)(row % p.Hq);
+  const int g = h / (p.Hq / p.Hkv);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int* list = p.idx + row * p.k;
+  if (threadIdx.x == 0) bad = 0;
+  __syncthreads();
+
+  float q[DPL];
+  {
+    const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + row * D + lane * DPL;
+#pragma unroll
+    for (int e = 0; e < DPL; ++e) q[e] = __bfloat162float(qrow[e]) * p.scale;
+  }
+  const __nv_bfloat16* kbase = static_cast<const __nv_bfloat16*>(p.Kc) + (size_t)(b * p.Hkv + g) * p.L * D;
+  const __nv_bfloat16* vbase = static_cast<const __nv_bfloat16*>(p.Vc) + (size_t)(b * p.Hkv + g) * p.L * D;
+  float m = -INFINITY, l = 0.f, acc[DPL];
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
+
+  for (int base = warp * kFacBatch; base < p.k; base += kFacWarps * kFacBatch) {
+    int tok[kFacBatch];
+    float kv[kFacBatch][DPL], vv[kFacBatch][DPL];
+#pragma unroll
+    for (int u = 0; u < kFacBatch; ++u) {
+      const int r = base + u;
+      int t = r < p.k ? __ldg(list + r) : -1;
+      if (t >= p.L || t < -1) {  // out of range (-1 is padding): record, skip the row
+        if (lane == 0) bad = 1;
+        t = -1;
+      }
+      tok[u] = t;
+      const int ts = t < 0 ? 0 : t;
+      const __nv_bfloat16* kr = kbase + (size_t)ts * D + lane * DPL;
+      const __nv_bfloat16* vr = vbase + (size_t)ts * D + lane * DPL;
+      if constexpr (DPL == 4) {
+        const uint2 ku = __ldg(reinterpret_cast<const uint2*>(kr));
+        const uint2 vu = __ldg(reinterpret_cast<const uint2*>(vr));
+        kv[u][0] = __uint_as_float(ku.x << 16); kv[u][1] = __uint_as_float(ku.x & 0xFFFF0000u);
+        kv[u][2] = __uint_as_float(ku.y << 16); kv[u][3] = __uint_as_float(ku.y & 0xFFFF0000u);
+        vv[u][0] = __uint_as_float(vu.x << 16); vv[u][1] = __uint_as_float(vu.x & 0xFFFF0000u);
+        vv[u][2] = __uint_as_float(vu.y << 16); vv[u][3] = __uint_as_float(vu.y & 0xFFFF0000u);
+      } else {
+        const uint32_t ku = __ldg(reinterpret_cast<const uint32_t*>(kr));
+        const uint32_t vu = __ldg(reinterpret_cast<const uint32_t*>(vr));
+        kv[u][0] = __uint_as_float(ku << 16); kv[u][1] = __uint_as_float(ku & 0xFFFF0000u);
+        vv[u][0] = __uint_as_float(vu << 16); vv[u][1] = __uint_as_float(vu & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < kFacBatch; ++u) {
+      float s = 0.f;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) s = fmaf(q[e], kv[u][e], s);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+      if (tok[u] < 0) continue;  // padding (warp-uniform)
+      const float mn = fmaxf(m, s);
+      const float f = expf(m - mn), pe = expf(s - mn);
+      l = l * f + pe;
+#pragma unroll
+      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(acc[e], f, pe * vv[u][e]);
+      m = mn;
+    }
+  }
+  if (lane == 0) { wm[warp] = m; wl[warp] = l; }
+#pragma unroll
+  for (int e = 0; e < DPL; ++e) wacc[warp][lane * DPL + e] = acc[e];
+  __syncthreads();
+  if (bad) {
+    if (threadIdx.x == 0) report(p.status, SFA_ERR_INDEX);
+  }
+  if (threadIdx.x < D) {
+    const int dd = threadIdx.x;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kFacWarps; ++w) M = fmaxf(M, wm[w]);
+    float L = 0.f, o = 0.f;
+    if (M != -INFINITY) {
+#pragma unroll
+      for (int w = 0; w < kFacWarps; ++w) {
+        const float f = wm[w] == -INFINITY ? 0.f : expf(wm[w] - M);
+        L += wl[w] * f;
+        o += wacc[w][dd] * f;
+      }
+    }
+    const float out = (bad || L == 0.f) ? 0.f : o / L;
+    static_cast<__nv_bfloat16*>(p.o)[row * D + dd] = __float2bfloat16_rn(out);
+    if (dd == 0 && p.lse != nullptr) p.lse[row] = (bad || L == 0.f) ? -INFINITY : M + logf(L);
+  }
+}
+
+}  // namespace
+
+// Chunk geometry for a group size and compact row width: C tokens per chunk, TPS tokens per
+// thread per slab, NS ring stages; shared memory = NS slabs + G C keys + the query table.
+DecodeGeometry decode_geometry(int group, int nfc) {
+  DecodeGeometry d;
+  const int W = 2 * nfc;
+  d.tps = W <= 32 ? 2 : 1;
+  const size_t slab = (size_t)kThreads * d.tps * W * 2;
+  // Two CTAs per SM when the keys and a two-stage ring fit in half the shared memory.
+  size_t budget = 110 * 1024;
+  if ((size_t)group * 4096 * 4 + 2 * slab > budget) budget = 200 * 1024;
+  d.chunk = 4096;
+  while (d.chunk > 1024 && (size_t)group * d.chunk * 4 + 2 * slab > budget) d.chunk /= 2;
+  d.nstages = (int)((budget - (size_t)group * d.chunk * 4) / slab);
+  d.nstages = d.nstages > 4 ? 4 : d.nstages;
+  d.ctas_per_sm = budget < 150 * 1024 ? 2 : 1;
+  d.smem = d.nstages * slab + (size_t)group * d.chunk * 4 + (size_t)group * W * 4;
+  return d;
+}
+
+int decode_max_chunks() { return kMaxChunks; }
+
+cudaError_t launch_fc_gather(const DecodeParams& p, const void* Kc, void* Kfc, int pos0, int npos, cudaStream_t st) {
+  const size_t items = (size_t)p.B * p.Hkv * npos * (2 * p.nfc / 8);
+  if (items == 0) return cudaSuccess;
+  size_t blocks = (items + kThreads - 1) / kThreads;
+  if (blocks > (size_t)148 * 16) blocks = (size_t)148 * 16;
+  const unsigned grid = (unsigned)blocks;
+  fc_gather_kernel<<<grid, kThreads, 0, st>>>(p, Kc, Kfc, pos0, npos);
+  return cudaGetLastError();
+}
+
+template <int G, int TPS, int NGR>
+static cudaError_t launch_tip_chunk_t(const DecodeParams& p, cudaStream_t st) {
+  const DecodeGeometry d = decode_geometry(G, p.nfc);
+  auto kern = tip_chunk_kernel<G, TPS, NGR>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)d.smem);
+  if (e != cudaSuccess) return e;
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int ntiles = p.nchunks * p.B * p.Hkv;
+  const int grid = sms * d.ctas_per_sm;
+  kern<<<ntiles < grid ? ntiles : grid, kThreads, d.smem, st>>>(p);
+  return cudaGetLastError();
+}
+
+template <int G>
+static cudaError_t launch_tip_chunk(const DecodeParams& p, cudaStream_t st) {
+  const bool two = p.tps == 2;
+  const bool four = p.chunk == 4096;  // groups of 4 keys per thread: C / 1024
+  if (two) return four ? launch_tip_chunk_t<G, 2, 4>(p, st) : (p.chunk == 2048 ? launch_tip_chunk_t<G, 2, 2>(p, st)
+                                                                                : launch_tip_chunk_t<G, 2, 1>(p, st));
+  return four ? launch_tip_chunk_t<G, 1, 4>(p, st)
+              : (p.chunk == 2048 ? launch_tip_chunk_t<G, 1, 2>(p, st) : launch_tip_chunk_t<G, 1, 1>(p, st));
+}
+
+cudaError_t launch_decode_select(const DecodeParams& p, cudaStream_t st) {
+  const int G = p.Hq / p.Hkv;
+  cudaError_t e = G == 1 ? launch_tip_chunk<1>(p, st)
+                  : G == 2 ? launch_tip_chunk<2>(p, st)
+                  : G == 4 ? launch_tip_chunk<4>(p, st)
+                           : launch_tip_chunk<8>(p, st);
+  if (e != cudaSuccess) return e;
+  const size_t msmem = ((size_t)p.nchunks * kWarps + 8 + (size_t)4 * kMergeSmem) * sizeof(uint32_t);
+  e = cudaFuncSetAttribute(tip_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+  if (e != cudaSuccess) return e;
+  tip_merge_kernel<<<p.B * p.Hq, kThreads, msmem, st>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_decode_attn(const DecodeParams& p, cudaStream_t st) {
+  if (p.D == 128)
+    fac_kernel<128><<<p.B * p.Hq, kFacWarps * 32, 0, st>>>(p);
+  else
+    fac_kernel<64><<<p.B * p.Hq, kFacWarps * 32, 0, st>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace sfa

@@ -74,12 +74,39 @@ struct AttnParams {
   float scale;  // softmax scale (natural-log units)
 };
 
+// Decode step (one query token per (b, h) against a KV cache of L tokens).
+struct DecodeParams {
+  const void* q;     // [B, Hq, D] bf16, rotated at the query's position
+  const void* Kfc;   // [B, Hkv, L, 2 nfc] bf16 compact dominant-pair keys
+  const void* Kc;    // [B, Hkv, L, D] bf16 rotated key cache
+  const void* Vc;    // [B, Hkv, L, D] bf16 value cache
+  uint32_t* cand_key;  // [B * Hq, nchunks, chunk] candidates of each chunk, token order
+  int* cand_idx;
+  int* cand_count;     // [B * Hq, nchunks, 8] per warp segment of each chunk
+  int* idx;          // [B, Hq, k]
+  void* o;           // [B, Hq, D] bf16
+  float* lse;        // [B, Hq] (nullable)
+  int* status;
+  int B, Hq, Hkv, L, D, nfc, k, chunk, nchunks, tps, nstages;
+  float scale;
+  uint8_t fc[1024];  // [Hkv][nfc] dominant pair indices
+};
+
 cudaError_t launch_rope_pool_energy(const RopePoolParams& p, int dtype, int D, cudaStream_t st);
 cudaError_t launch_band_temperature(const TauParams& p, cudaStream_t st);
 cudaError_t launch_block_score_softmax(const ScoreParams& p, int D, cudaStream_t st);
 size_t score_smem_bytes(int nb, int D, bool band_max);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnParams& p, int dtype, int D, cudaStream_t st);
+struct DecodeGeometry {
+  int chunk, tps, nstages, ctas_per_sm;
+  size_t smem;
+};
+DecodeGeometry decode_geometry(int group, int nfc);
+int decode_max_chunks();
+cudaError_t launch_fc_gather(const DecodeParams& p, const void* Kc, void* Kfc, int pos0, int npos, cudaStream_t st);
+cudaError_t launch_decode_select(const DecodeParams& p, cudaStream_t st);
+cudaError_t launch_decode_attn(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_attn_tcgen05(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                 const CUtensorMap& tmV, cudaStream_t st);
 

@@ -81,6 +81,16 @@ def load() -> ctypes.CDLL:
     lib.sfa_block_sparse_attn_rope.argtypes = [POINTER(Shape), c_int, c_void_p, POINTER(Rope), c_void_p, c_void_p,
                                                c_void_p, c_void_p, c_int, c_int, c_float, c_void_p, c_void_p,
                                                c_void_p, c_void_p]
+    lib.sfa_decode_workspace.restype = c_size_t
+    lib.sfa_decode_workspace.argtypes = [POINTER(Shape), c_int]
+    lib.sfa_decode_fc_gather.restype = c_int
+    lib.sfa_decode_fc_gather.argtypes = [POINTER(Shape), c_void_p, c_void_p, c_int, c_int, c_int, c_void_p, c_void_p]
+    lib.sfa_decode_select.restype = c_int
+    lib.sfa_decode_select.argtypes = [POINTER(Shape), c_void_p, c_void_p, c_void_p, c_int, c_int, c_void_p, c_void_p,
+                                      c_size_t, c_void_p, c_void_p]
+    lib.sfa_decode_attn.restype = c_int
+    lib.sfa_decode_attn.argtypes = [POINTER(Shape), c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_float,
+                                    c_void_p, c_void_p, c_void_p, c_void_p]
     _lib = lib
     return lib
 
@@ -364,3 +374,105 @@ class PrismAttention:
         self(*dev_in, stream=stream)
         O_host.copy_(self.O, non_blocking=True)
         return O_host
+
+
+# ---------------------------------------------------------------------------
+# Decode step (token importance on dominant rotary pairs -> top-k -> attention)
+# ---------------------------------------------------------------------------
+def _fc_host(fc) -> tuple:
+    """fc [Hkv, nfc] (any int array-like) -> (ctypes int32 array, nfc)."""
+    import numpy as np
+    a = np.ascontiguousarray(np.asarray(fc, dtype=np.int32))
+    if a.ndim != 2:
+        raise ValueError("fc must be [heads_kv, nfc]")
+    return (ctypes.c_int * a.size)(*a.reshape(-1).tolist()), a.shape[1]
+
+
+def decode_shape(q, K_cache) -> Shape:
+    B, Hq, d = q.shape
+    return Shape(B, Hq, K_cache.shape[1], K_cache.shape[2], d, _dtype_code(q))
+
+
+def decode_fc_gather(K_cache, fc, *, K_fc=None, pos0: int = 0, npos: int | None = None, stream=None):
+    """sfa_decode_fc_gather: returns K_fc [B, Hkv, L, 2 nfc]."""
+    lib = load()
+    _cuda(K_cache, "K_cache")
+    B, Hkv, L, d = K_cache.shape
+    fch, nfc = _fc_host(fc)
+    shape = Shape(B, Hkv, Hkv, L, d, _dtype_code(K_cache))
+    if K_fc is None:
+        K_fc = torch.empty((B, Hkv, L, 2 * nfc), dtype=K_cache.dtype, device=K_cache.device)
+    npos = L - pos0 if npos is None else npos
+    _check(lib.sfa_decode_fc_gather(ctypes.byref(shape), _ptr(K_cache), fch, nfc, pos0, npos, _ptr(K_fc),
+                                    _stream(stream)), "sfa_decode_fc_gather")
+    return K_fc
+
+
+def decode_select(q, K_fc, fc, L: int, *, k: int, idx=None, workspace=None, status=None, stream=None):
+    """sfa_decode_select: returns idx [B, Hq, k] int32 (ascending, -1 padded)."""
+    lib = load()
+    _cuda(q, "q"); _cuda(K_fc, "K_fc")
+    B, Hq, d = q.shape
+    fch, nfc = _fc_host(fc)
+    shape = Shape(B, Hq, K_fc.shape[1], L, d, _dtype_code(q))
+    if idx is None:
+        idx = torch.empty((B, Hq, k), dtype=torch.int32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(max(lib.sfa_decode_workspace(ctypes.byref(shape), k), 256), dtype=torch.uint8,
+                                device=q.device)
+    _check(lib.sfa_decode_select(ctypes.byref(shape), _ptr(q), _ptr(K_fc), fch, nfc, k, _ptr(idx),
+                                 _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
+           "sfa_decode_select")
+    return idx
+
+
+def decode_attn(q, K_cache, V_cache, idx, *, scale: float = 0.0, o=None, lse=None, status=None, stream=None):
+    """sfa_decode_attn: returns o [B, Hq, d]."""
+    lib = load()
+    for t, n in ((q, "q"), (K_cache, "K_cache"), (V_cache, "V_cache"), (idx, "idx")):
+        _cuda(t, n)
+    shape = decode_shape(q, K_cache)
+    o = torch.empty_like(q) if o is None else o
+    _check(lib.sfa_decode_attn(ctypes.byref(shape), _ptr(q), _ptr(K_cache), _ptr(V_cache), _ptr(idx),
+                               idx.shape[-1], float(scale), _ptr(o), _ptr(lse), _ptr(status), _stream(stream)),
+           "sfa_decode_attn")
+    return o
+
+
+class FasaDecode:
+    """One decode step for a fixed cache shape: TIP on the compact dominant-pair keys, top-k,
+    focused attention.  ``fc`` [Hkv, nfc] are the dominant pairs (an input: the offline
+    calibration that finds them is not part of this library).  Buffers are allocated once;
+    ``refresh_keys`` (re)builds the compact key copy for a position range, ``__call__`` runs
+    the step's three kernels."""
+
+    def __init__(self, *, batch, heads_q, heads_kv, seq_len, head_dim, fc, k, device="cuda", with_lse=True):
+        self.fc = fc
+        self.k = k
+        self.shape = Shape(batch, heads_q, heads_kv, seq_len, head_dim, BF16)
+        dev = torch.device(device)
+        _, nfc = _fc_host(fc)
+        self.K_fc = torch.empty((batch, heads_kv, seq_len, 2 * nfc), dtype=torch.bfloat16, device=dev)
+        ws = load().sfa_decode_workspace(ctypes.byref(self.shape), k)
+        if ws == 0:
+            raise SfaError(1, "sfa_decode_workspace")
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=dev)
+        self.idx = torch.empty((batch, heads_q, k), dtype=torch.int32, device=dev)
+        self.o = torch.empty((batch, heads_q, head_dim), dtype=torch.bfloat16, device=dev)
+        self.lse = torch.empty((batch, heads_q), dtype=torch.float32, device=dev) if with_lse else None
+        self.status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def refresh_keys(self, K_cache, pos0=0, npos=None, stream=None):
+        decode_fc_gather(K_cache, self.fc, K_fc=self.K_fc, pos0=pos0, npos=npos, stream=stream)
+
+    def select(self, q, stream=None):
+        decode_select(q, self.K_fc, self.fc, self.shape.seq_len, k=self.k, idx=self.idx, workspace=self.workspace,
+                      status=self.status, stream=stream)
+
+    def attend(self, q, K_cache, V_cache, stream=None):
+        decode_attn(q, K_cache, V_cache, self.idx, o=self.o, lse=self.lse, status=self.status, stream=stream)
+
+    def __call__(self, q, K_cache, V_cache, stream=None):
+        self.select(q, stream)
+        self.attend(q, K_cache, V_cache, stream)
+        return self.o

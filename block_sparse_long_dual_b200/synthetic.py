@@ -14,13 +14,22 @@ arithmetic.  Recipe (pre-RoPE Q, K, V, layout [B, H, L, d]):
   constant c ~ N(0, 1) from seed 3 on the high-band dims, added to every Q and
   K token.  After RoPE, q.k gains sum_m |c_m|^2 cos((p_q - p_k) theta_m): a
   recency diagonal that block mean pooling attenuates (§2).
+
+Decode inputs (``make_decode_inputs``; "FASA: Frequency-aware Sparse
+Attention" §2B): q [B, Hq, d], K, V [B, Hkv, L, d] drawn N(0, 1) from
+``seed`` and cast to bf16 (K and q stand for already-rotated values: a random
+vector's rotation is again random).  Dominant pairs ``fc`` [Hkv, nfc]: nfc
+distinct pairs per KV head drawn with seed 5 (a stand-in for the offline
+calibration the page describes).  Needles: round(needle_frac * L) tokens per
+(b, KV head), drawn with seed 6, get 2 x the group's mean query added on that
+head's dominant dims, so the estimate has real winners to find.
 """
 
 from __future__ import annotations
 
 import torch
 
-from .workloads import Workload
+from .workloads import DecodeWorkload, Workload
 
 
 def _band_dims(head_dim: int, band_split: int):
@@ -77,3 +86,33 @@ def make_inputs(w: Workload, seed: int = 0, device: str | torch.device = "cpu"):
     K = draw(w.heads_kv, k_all, k_pl)
     V = draw(w.heads_kv, None, None)
     return Q, K, V
+
+
+def decode_fc(w: DecodeWorkload):
+    """Dominant pair lists [Hkv, nfc] (int64, sorted per head)."""
+    g = torch.Generator().manual_seed(5)
+    rows = [torch.sort(torch.randperm(w.head_dim // 2, generator=g)[:w.nfc]).values for _ in range(w.heads_kv)]
+    return torch.stack(rows).numpy()
+
+
+def make_decode_inputs(w: DecodeWorkload, seed: int = 0, device: str | torch.device = "cpu"):
+    """q [B,Hq,d], K [B,Hkv,L,d], V [B,Hkv,L,d] bf16 on ``device``, and fc [Hkv, nfc]."""
+    g = torch.Generator().manual_seed(seed)
+    fc = decode_fc(w)
+    q = torch.randn((w.batch, w.heads_q, w.head_dim), generator=g)
+    K = torch.empty((w.batch, w.heads_kv, w.seq_len, w.head_dim), dtype=torch.bfloat16, device=device)
+    V = torch.empty_like(K)
+    gn = torch.Generator().manual_seed(6)
+    nneedle = int(round(w.needle_frac * w.seq_len))
+    half = w.head_dim // 2
+    for b in range(w.batch):
+        for h in range(w.heads_kv):
+            x = torch.randn((w.seq_len, w.head_dim), generator=g)
+            if nneedle:
+                dims = torch.cat([torch.as_tensor(fc[h]), torch.as_tensor(fc[h]) + half])
+                qm = q[b, h * w.group:(h + 1) * w.group].mean(0)
+                pos = torch.randperm(w.seq_len, generator=gn)[:nneedle]
+                x[pos[:, None], dims[None, :]] += 2.0 * qm[dims]
+            K[b, h].copy_(x.to(torch.bfloat16))
+            V[b, h].copy_(torch.randn((w.seq_len, w.head_dim), generator=g).to(torch.bfloat16))
+    return q.to(torch.bfloat16).to(device), K, V, fc

@@ -104,3 +104,36 @@ SWEEP_DENSITIES = (0.01, 0.02, 0.05, 0.10, 0.25, 1.0)
 
 ALL = {w.name: w for w in [TINY, LLAMA_32K, LLAMA_128K, QWEN_64K_B2]
        + [sweep(x) for x in SWEEP_DENSITIES]}
+
+
+# ---------------------------------------------------------------------------
+# Decode step ("FASA: Frequency-aware Sparse Attention" §2B): one query token
+# per (batch, Q head) against a KV cache.  nfc = 12 of 64 rotary pairs is
+# 18.75% of the key dims, the share of the cache the page's FASA-C reads
+# (18.9%, §4); k = 256 is the page's extreme token budget (§4, LongBench).
+# ---------------------------------------------------------------------------
+@dataclass(frozen=True)
+class DecodeWorkload:
+    name: str
+    batch: int
+    heads_q: int
+    heads_kv: int
+    seq_len: int      # cache length L
+    head_dim: int
+    nfc: int          # dominant rotary pairs per KV head
+    k: int            # token budget
+    needle_frac: float = 0.01   # fraction of cache tokens aligned with the query on the dominant pairs
+
+    @property
+    def group(self) -> int:
+        return self.heads_q // self.heads_kv
+
+    def scaled(self, **kw) -> "DecodeWorkload":
+        return replace(self, **kw)
+
+
+FASA_DECODE_128K_B4 = DecodeWorkload(name="fasa-decode-llama3.1-8b-128k-b4", batch=4, heads_q=32, heads_kv=8,
+                                     seq_len=131072, head_dim=128, nfc=12, k=256)
+FASA_DECODE_32K_B16 = DecodeWorkload(name="fasa-decode-llama3.1-8b-32k-b16", batch=16, heads_q=32, heads_kv=8,
+                                     seq_len=32768, head_dim=128, nfc=12, k=256)
+DECODE = {w.name: w for w in [FASA_DECODE_128K_B4, FASA_DECODE_32K_B16]}

@@ -261,6 +261,66 @@ sfa_status sfa_block_sparse_attn_rope(const sfa_shape* shape, int block, const v
                                       float scale, void* O, float* lse, int* status_word,
                                       void* stream);
 
+/*
+ * ---------------------------------------------------------------------------
+ * Decode step ("FASA: Frequency-aware Sparse Attention" §2B): one query token
+ * per (batch, Q head) against a KV cache.  shape->seq_len is the cache length
+ * L; shape->dtype must be SFA_BF16 (SFA_ERR_DTYPE otherwise); heads_q /
+ * heads_kv in {1, 2, 4, 8} and L <= 2^21 (SFA_ERR_UNSUPPORTED otherwise).  q [B, heads_q, d] is the newest token's query, already
+ * rotated at its position; K_cache, V_cache [B, heads_kv, L, d] hold the
+ * rotated keys and the values at their original positions.
+ *
+ * fc: HOST array [heads_kv][nfc] of each KV head's dominant rotary pairs
+ * (pair m = dims m and m + d/2; found by an offline calibration that this
+ * library does not perform), distinct entries in [0, d/2); 4 <= nfc <= d/2,
+ * nfc % 4 == 0, heads_kv * nfc <= 1024.  The Q heads of a group share their
+ * KV head's list.  Violations: SFA_ERR_INVALID_ARG.
+ * ---------------------------------------------------------------------------
+ */
+
+/*
+ * Compact dominant-pair key copy (§2C, FASA-C reads only this part of the
+ * keys for the estimate): K_fc [B, heads_kv, L, 2 nfc] bf16, column c < nfc =
+ * dim fc[g][c], column nfc + c = dim fc[g][c] + d/2.  Writes the rows of
+ * positions [pos0, pos0 + npos) only (the whole cache once, then each
+ * appended range).  K_cache and K_fc 16-byte aligned.
+ */
+sfa_status sfa_decode_fc_gather(const sfa_shape* shape, const void* K_cache, const int* fc, int nfc,
+                                int pos0, int npos, void* K_fc, void* stream);
+
+/* Workspace bytes sfa_decode_select needs for a budget of k tokens (0 if invalid). */
+size_t sfa_decode_workspace(const sfa_shape* shape, int k);
+
+/*
+ * Token Importance Predictor (§2B.1): for Q head h of KV group g,
+ *   s_t = sum_{m in fc[g]} q_m k_{t,m} + q_{m+d/2} k_{t,m+d/2}
+ * from K_fc, summed in float64 and rounded once to float32; then the first
+ * min(k, L) tokens by (s desc, index asc).  idx [B, heads_q, k] int32: the kept
+ * token indices ascending, padded with -1.  k >= 1.  workspace: device, at
+ * least sfa_decode_workspace() bytes, 256-byte aligned (SFA_ERR_WORKSPACE).
+ * status_word (device, nullable): SFA_ERR_TIMEOUT if a copy of the compact
+ * keys did not land within about 2 s (that chunk then contributes no tokens).
+ * Launches 2 kernels: a persistent one (per chunk of the cache: scores, a
+ * lower bound of the chunk's k-th largest, the tokens above it) and a merge
+ * (exact top k of the candidates).
+ */
+sfa_status sfa_decode_select(const sfa_shape* shape, const void* q, const void* K_fc, const int* fc,
+                             int nfc, int k, int* idx, void* workspace, size_t workspace_bytes,
+                             int* status_word, void* stream);
+
+/*
+ * Focused Attention Computation (§2B.2): full-dimension attention of q over
+ * the tokens listed in idx [B, heads_q, k] (-1 entries skipped; the cached
+ * keys keep their original positions):
+ *   o = sum_t softmax_t(scale * q . k_t) v_t,  lse = log sum_t exp(scale * q . k_t)
+ * o [B, heads_q, d] bf16; lse [B, heads_q] float32 (nullable; natural log).
+ * scale <= 0 selects 1/sqrt(d).  An entry outside [-1, L) sets status_word to
+ * SFA_ERR_INDEX and that row's o = 0, lse = -inf; an empty row likewise.
+ */
+sfa_status sfa_decode_attn(const sfa_shape* shape, const void* q, const void* K_cache,
+                           const void* V_cache, const int* idx, int k, float scale, void* o,
+                           float* lse, int* status_word, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -27,8 +27,12 @@ D1  A frequency chunk is one rotary pair (m, m + d/2) of the rotate-half
     GQA group share their KV head's list, so one compact key copy serves the group.
 D2  TIP score of Q head h for cached token t:
         s_t = sum_{m in fc[g(h)]} q_m k_{t,m} + q_{m+d/2} k_{t,m+d/2}
-    from the rotated query (at the newest position) and the rotated cache;
-    float64 sum, then rounded once to float32 (the value both sides rank).
+    from the rotated query (at the newest position) and the rotated cache.
+    The page fixes no precision, so the ranked value takes the kernel's: a
+    float32 sum taken left to right over the compact copy's columns (D5
+    order), each step one rounding of (running sum + product).  A product of
+    two bf16 values is exact in float32, so this value is reproducible
+    bit for bit; ``tip_scores`` keeps the exact float64 sum for the pins.
 D3  T_t = the first min(k, L) tokens in the order (score desc, index asc),
     output ascending, padded with -1.  No forced tokens (the page names none).
 D4  FAC: o = sum_{t in T_t} softmax_t(scale * q . k_t) v_t over all d dims,
@@ -79,9 +83,22 @@ def tip_scores(q: np.ndarray, K: np.ndarray, fc: np.ndarray) -> np.ndarray:
     return out
 
 
-def tip_keys(scores64: np.ndarray) -> np.ndarray:
-    """D2: the float32 values the selection ranks."""
-    return np.asarray(scores64, dtype=np.float64).astype(np.float32)
+def tip_keys(q: np.ndarray, K: np.ndarray, fc: np.ndarray) -> np.ndarray:
+    """D2: the float32 values the selection ranks [B, Hq, L]: running float32 sum over the
+    compact columns in order, starting from 0, each step rounding (sum + q_c * k_c) once."""
+    q = np.asarray(q, dtype=np.float32)
+    K = np.asarray(K, dtype=np.float32)
+    B, Hq, d = q.shape
+    group = Hq // K.shape[1]
+    out = np.zeros((B, Hq, K.shape[2]), dtype=np.float32)
+    for h in range(Hq):
+        g = h // group
+        acc = np.zeros((B, K.shape[2]), dtype=np.float32)
+        for dim in fc_dims(fc[g], d):
+            prod = q[:, h, dim][:, None] * K[:, g, :, dim]   # float32 product, exact for bf16 inputs
+            acc = acc + prod                                 # float32 add: one rounding per step
+        out[:, h] = acc
+    return out
 
 
 def select_row(keys: np.ndarray, k: int) -> np.ndarray:
@@ -130,7 +147,7 @@ def focused_attention(q, K, V, idx, scale=None):
 def decode_step(q, K, V, fc, k, scale=None):
     """TIP -> select -> FAC for one decode step: (scores64, keys32, idx, o, lse)."""
     s = tip_scores(q, K, fc)
-    keys = tip_keys(s)
+    keys = tip_keys(q, K, fc)
     idx = select_tokens(keys, k)
     o, lse = focused_attention(q, K, V, idx, scale)
     return s, keys, idx, o, lse

@@ -175,6 +175,38 @@ def test_attn_rope_validation(lib):
     assert f(ctypes.byref(bad), 128, d, ctypes.byref(good), d, d, d, d, 8, 1, 0.0, d, None, None, None) == 2
 
 
+def test_decode_validation(lib):
+    d = ctypes.c_void_p(1 << 20)
+    sh = S(B=2, Hq=8, Hkv=2, L=5000)
+    fc = (ctypes.c_int * 8)(0, 5, 9, 63, 1, 2, 3, 4)
+    ws = lib.sfa_decode_workspace(ctypes.byref(sh), 256)
+    assert ws >= 2 * 8 * 2 * 256 * 8
+    g = lib.sfa_decode_fc_gather
+    assert g(ctypes.byref(sh), d, fc, 4, 0, 5000, d, None) != 1                    # valid (no GPU: not 1)
+    assert g(ctypes.byref(S(B=2, Hq=8, Hkv=2, L=5000, dt=sfa.F32)), d, fc, 4, 0, 5000, d, None) == 3
+    assert g(ctypes.byref(S(B=1, Hq=18, Hkv=2, L=50)), d, fc, 4, 0, 50, d, None) == 4  # group 9
+    assert g(ctypes.byref(sh), d, fc, 3, 0, 5000, d, None) == 1                    # nfc % 4
+    assert g(ctypes.byref(sh), d, fc, 68, 0, 5000, d, None) == 1                   # nfc > d/2 (rejected before fc is read)
+    bad = (ctypes.c_int * 8)(0, 5, 9, 64, 1, 2, 3, 4)                             # pair 64 >= d/2
+    assert g(ctypes.byref(sh), d, bad, 4, 0, 5000, d, None) == 1
+    dup = (ctypes.c_int * 8)(0, 5, 5, 6, 1, 2, 3, 4)
+    assert g(ctypes.byref(sh), d, dup, 4, 0, 5000, d, None) == 1
+    assert g(ctypes.byref(sh), d, fc, 4, 4000, 1001, d, None) == 1                 # past L
+    assert g(ctypes.byref(sh), d, fc, 4, -1, 10, d, None) == 1
+    assert g(ctypes.byref(sh), d, None, 4, 0, 10, d, None) == 1
+    s = lib.sfa_decode_select
+    assert s(ctypes.byref(sh), d, d, fc, 4, 0, d, d, ws, None, None) == 1          # k = 0
+    assert s(ctypes.byref(sh), d, d, fc, 4, 256, d, d, ws - 1, None, None) == 5
+    assert s(ctypes.byref(sh), d, d, fc, 4, 256, d, None, ws, None, None) == 5
+    assert s(ctypes.byref(sh), None, d, fc, 4, 256, d, d, ws, None, None) == 1
+    a = lib.sfa_decode_attn
+    assert a(ctypes.byref(sh), d, d, d, d, 0, 0.0, d, None, None, None) == 1        # k = 0
+    assert a(ctypes.byref(sh), d, d, d, None, 8, 0.0, d, None, None, None) == 1
+    assert a(ctypes.byref(sh), d, d, d, d, 8, float("inf"), d, None, None, None) == 1
+    assert a(ctypes.byref(S(d=96)), d, d, d, d, 8, 0.0, d, None, None, None) == 2
+    assert lib.sfa_decode_workspace(ctypes.byref(sh), 0) == 0
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(sfa, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(sfa, "_lib", None)

@@ -163,3 +163,23 @@ def test_decode_step_top1_picks_planted_key():
     _, _, idx, o, _ = fo.decode_step(q, K, V, fc, 1)
     assert idx[0, 0, 0] == 11
     np.testing.assert_array_equal(o[0, 0], V[0, 0, 11])
+
+
+def test_ranked_float32_score_is_within_the_recursive_summation_bound():
+    """|fl32 running sum - exact sum| <= (n u / (1 - n u)) sum |q_c k_c| with u = 2**-24, n = 2 nfc
+    terms (products exact for bf16 inputs); and an all-dyadic case where the float32 sum is exact."""
+    q, K, _ = _inputs(seed=8)
+    qb = torch.from_numpy(q).to(torch.bfloat16).to(torch.float64).numpy()
+    Kb = torch.from_numpy(K).to(torch.bfloat16).to(torch.float64).numpy()
+    fc = np.array([[1, 5, 6, 7], [0, 2, 3, 4]])
+    keys = fo.tip_keys(qb, Kb, fc).astype(np.float64)
+    exact = fo.tip_scores(qb, Kb, fc)
+    n, u = 8, 2.0 ** -24
+    group = q.shape[1] // K.shape[1]
+    for h in range(q.shape[1]):
+        dims = fo.fc_dims(fc[h // group], q.shape[-1])
+        mag = np.einsum("bd,btd->bt", np.abs(qb[:, h][:, dims]), np.abs(Kb[:, h // group][..., dims]))
+        assert np.all(np.abs(keys[:, h] - exact[:, h]) <= n * u / (1 - n * u) * mag)
+    qi = np.round(q * 4) / 4
+    Ki = np.round(K * 4) / 4
+    np.testing.assert_array_equal(fo.tip_keys(qi, Ki, fc).astype(np.float64), fo.tip_scores(qi, Ki, fc))

@@ -1,0 +1,113 @@
+"""GPU decode step (token importance on dominant rotary pairs -> top-k -> focused attention)
+against the CPU oracle ("FASA: Frequency-aware Sparse Attention" §2B), through the C ABI.
+
+The compact key copy and the index lists are compared bit for bit (both sides rank the same
+float32 rounding of an exact float64 score); outputs within the bf16 tolerance."""
+
+import numpy as np
+import pytest
+import torch
+
+from block_sparse_long_dual_b200 import sfa
+from block_sparse_long_dual_b200.synthetic import make_decode_inputs
+from block_sparse_long_dual_b200.workloads import FASA_DECODE_128K_B4, DecodeWorkload
+from oracle import fasa_oracle as fo
+
+pytestmark = pytest.mark.gpu
+
+TOL_O = 2e-2
+
+
+def D(name, **kw):
+    base = dict(batch=1, heads_q=4, heads_kv=1, seq_len=5000, head_dim=128, nfc=12, k=256)
+    base.update(kw)
+    return DecodeWorkload(name=name, **base)
+
+
+CASES = [
+    D("ragged-two-chunks", batch=2, heads_q=8, heads_kv=2),
+    D("k-above-L-d64", seq_len=300, head_dim=64, nfc=8, k=512),
+    D("all-pairs-group8", heads_q=8, heads_kv=1, seq_len=9000, nfc=64, k=64),
+    D("k1-mha-one-chunk", batch=3, heads_q=2, heads_kv=2, seq_len=4096, nfc=4, k=1),
+    D("single-token-cache", heads_q=4, heads_kv=2, seq_len=1, head_dim=64, nfc=4, k=3),
+    D("k-above-chunk", heads_q=2, heads_kv=1, seq_len=10000, head_dim=64, nfc=8, k=5000),
+    D("no-needles-many-ties", heads_q=4, heads_kv=1, seq_len=7000, nfc=4, k=100, needle_frac=0.0),
+]
+
+
+def run(w: DecodeWorkload, seed=0):
+    q, K, V, fc = make_decode_inputs(w, seed=seed)
+    dev = torch.device("cuda")
+    m = sfa.FasaDecode(batch=w.batch, heads_q=w.heads_q, heads_kv=w.heads_kv, seq_len=w.seq_len,
+                       head_dim=w.head_dim, fc=fc, k=w.k, device=dev)
+    qd, Kd, Vd = q.to(dev), K.to(dev), V.to(dev)
+    m.refresh_keys(Kd)
+    m(qd, Kd, Vd)
+    torch.cuda.synchronize()
+    return m, q, K, V, fc
+
+
+@pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
+def test_decode_matches_oracle(w):
+    m, q, K, V, fc = run(w)
+    qn, Kn, Vn = (t.to(torch.float64).numpy() for t in (q, K, V))
+    # compact key copy: exact
+    np.testing.assert_array_equal(m.K_fc.cpu().view(torch.int16).numpy(),
+                                  fo.gather_fc(K.view(torch.int16).numpy(), fc))
+    # selection: bit-exact
+    s, keys, idx, o, lse = fo.decode_step(qn, Kn, Vn, fc, w.k)
+    got = m.idx.cpu().numpy()
+    mism = np.argwhere((got != idx).any(-1))
+    assert mism.size == 0, f"rows differ: {mism[:5].tolist()}"
+    # attention over the kept tokens
+    assert int(m.status.item()) == 0
+    np.testing.assert_allclose(m.o.cpu().to(torch.float64).numpy(), o, rtol=0, atol=TOL_O)
+    np.testing.assert_allclose(m.lse.cpu().numpy(), lse, rtol=0, atol=1e-3)
+
+
+def test_fc_gather_range_touches_only_that_range():
+    w = D("range", heads_q=4, heads_kv=2, seq_len=3000, nfc=8)
+    q, K, V, fc = make_decode_inputs(w)
+    dev = torch.device("cuda")
+    Kd = K.to(dev)
+    Kfc = torch.full((1, 2, 3000, 16), 7.0, dtype=torch.bfloat16, device=dev)
+    sfa.decode_fc_gather(Kd, fc, K_fc=Kfc, pos0=1000, npos=777)
+    torch.cuda.synchronize()
+    want = fo.gather_fc(K.view(torch.int16).numpy(), fc)
+    got = Kfc.cpu().view(torch.int16).numpy()
+    np.testing.assert_array_equal(got[:, :, 1000:1777], want[:, :, 1000:1777])
+    seven = torch.tensor(7.0, dtype=torch.bfloat16).view(torch.int16).item()
+    assert np.all(got[:, :, :1000] == seven) and np.all(got[:, :, 1777:] == seven)
+
+
+def test_decode_attn_rejects_bad_index():
+    w = D("bad", heads_q=4, heads_kv=1, seq_len=600, nfc=4, k=8)
+    m, q, K, V, fc = run(w)
+    dev = torch.device("cuda")
+    idx = m.idx.clone()
+    idx[0, 2, 3] = 600          # out of range
+    idx[0, 1, 0] = -2           # below the padding value
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    lse = torch.empty((1, 4), dtype=torch.float32, device=dev)
+    o = sfa.decode_attn(q.to(dev), K.to(dev), V.to(dev), idx, lse=lse, status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 8  # SFA_ERR_INDEX
+    assert torch.all(o[0, 2] == 0) and torch.all(o[0, 1] == 0)
+    assert torch.isneginf(lse[0, 2]) and torch.isneginf(lse[0, 1])
+    assert torch.equal(o[0, 0], m.o[0, 0]) and torch.equal(o[0, 3], m.o[0, 3])
+
+
+def test_decode_full_size_sampled_rows():
+    """The 128K-token, batch-4 cache of the decode bench: sampled rows against the oracle."""
+    w = FASA_DECODE_128K_B4
+    m, q, K, V, fc = run(w, seed=3)
+    rng = np.random.default_rng(0)
+    for _ in range(4):
+        b, h = int(rng.integers(w.batch)), int(rng.integers(w.heads_q))
+        g = h // w.group
+        qn = q[b:b + 1, h:h + 1].to(torch.float64).numpy()
+        Kn = K[b:b + 1, g:g + 1].to(torch.float64).numpy()
+        Vn = V[b:b + 1, g:g + 1].to(torch.float64).numpy()
+        s, keys, idx, o, lse = fo.decode_step(qn, Kn, Vn, fc[g:g + 1], w.k)
+        np.testing.assert_array_equal(m.idx[b, h].cpu().numpy(), idx[0, 0])
+        np.testing.assert_allclose(m.o[b, h].cpu().to(torch.float64).numpy(), o[0, 0], rtol=0, atol=TOL_O)
