@@ -16,6 +16,11 @@ e2e    = the same metric through PrismAttention.run_host from pinned host
          tensors: H2D of Q, K, V and D2H of O inside every timed step.
 --impl reference times the CPU oracle (the slow fp64 restatement) on a
 bounded sample of the same workload (see cpu_baseline.sample).
+
+--workload fasa-decode-* runs the decode step instead (one query token per
+sequence against a KV cache: compact-key append for the new position, token
+importance + top-k, focused attention): value = decode tokens/s (sequences x
+steps / time), roofline of the selection on the compact-key stream (HBM).
 """
 
 from __future__ import annotations
@@ -49,7 +54,7 @@ def parse():
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default=wl.LLAMA_128K.name, choices=sorted(wl.ALL))
+    ap.add_argument("--workload", default=wl.LLAMA_128K.name, choices=sorted(wl.ALL) + sorted(wl.DECODE))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
     return ap.parse_args()
@@ -73,11 +78,11 @@ def attention_flops(counts: np.ndarray, block: int, d: int) -> float:
 
 def scoring_bytes(w: wl.Workload) -> float:
     """Algorithmic HBM bytes of sfa_block_scores: read Q, K; write Q_r, K_r; read the cos/sin
-    table once; write the block means; write probs [B, Hq, nb, nb]."""
+    table once; write the float64 block means; write probs [B, Hq, nb, nb]."""
     e = 2 if w.dtype == "bf16" else 4
     qk = w.batch * (w.heads_q + w.heads_kv) * w.seq_len * w.head_dim * e
     table = 2 * w.seq_len * (w.head_dim // 2) * 4
-    means = w.batch * (w.heads_q + w.heads_kv) * w.nb * w.head_dim * 4
+    means = w.batch * (w.heads_q + w.heads_kv) * w.nb * w.head_dim * 8
     probs = w.batch * w.heads_q * w.nb * w.nb * 4
     return float(2 * qk + table + means + probs)
 
@@ -203,6 +208,169 @@ def blas_threads():
         return None
 
 
+DECODE_METRIC = "decode tokens/s (one query token per sequence per step, TIP + top-k + focused attention)"
+
+
+def decode_bytes(w: wl.DecodeWorkload):
+    """Algorithmic HBM bytes of one decode step: (selection) the compact keys [B, Hkv, L, 2 nfc]
+    and q; (attention) the k kept K and V rows of every (b, h), q, o; (append) one compact row per
+    (b, KV head).  Returns (selection bytes, attention bytes, total)."""
+    sel = w.batch * w.heads_kv * w.seq_len * 2 * w.nfc * 2 + w.batch * w.heads_q * w.head_dim * 2
+    att = w.batch * w.heads_q * (w.k * 2 * w.head_dim * 2 + 2 * w.head_dim * 2 + w.k * 4)
+    app = w.batch * w.heads_kv * (w.head_dim * 2 + 2 * w.nfc * 2)
+    return float(sel), float(att), float(sel + att + app)
+
+
+def oracle_decode_sample(w: wl.DecodeWorkload, q, K, V, fc, b=0, h=0):
+    """Time the oracle's decode step on one (b, h) row; returns (tokens/s, seconds, sample text)."""
+    from oracle import fasa_oracle as fo
+    g = h // w.group
+    qn = q[b:b + 1, h:h + 1].to(torch.float64).numpy()
+    Kn = K[b:b + 1, g:g + 1].to(torch.float64).numpy()
+    Vn = V[b:b + 1, g:g + 1].to(torch.float64).numpy()
+    t0 = time.perf_counter()
+    fo.decode_step(qn, Kn, Vn, fc[g:g + 1], w.k)
+    secs = time.perf_counter() - t0
+    # a step is batch x heads_q such rows for batch tokens
+    value = w.batch / (secs * w.batch * w.heads_q)
+    text = (f"one (sequence, Q head) row of {w.batch} x {w.heads_q}: float32 importance over the {w.seq_len}-token "
+            f"cache, top-{w.k}, float64 attention; scaled to the full step")
+    return value, secs, text
+
+
+def run_decode(args, w: wl.DecodeWorkload, rank, world):
+    from block_sparse_long_dual_b200 import sfa
+    from block_sparse_long_dual_b200.synthetic import make_decode_inputs
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        q, K, V, fc = make_decode_inputs(w.scaled(batch=1), seed=0)
+        per = []
+        text = ""
+        for s_ in range(args.warmup + args.steps):
+            v, secs, text = oracle_decode_sample(w.scaled(batch=1), q, K, V, fc, 0, s_ % w.heads_q)
+            if s_ >= args.warmup:
+                per.append((v, secs))
+        value = float(np.mean([v for v, _ in per]))
+        line = {"metric": DECODE_METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": float(np.mean([s for _, s in per])) * 1e3 * w.heads_q,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+                "data": "synthetic", "impl": "reference",
+                "config": {"workload": w.name},
+                "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads() or
+                                 len(os.sched_getaffinity(0)), "kind": "oracle", "sample": text},
+                "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    q, K, V, fc = make_decode_inputs(w, seed=rank)
+    m = sfa.FasaDecode(batch=w.batch, heads_q=w.heads_q, heads_kv=w.heads_kv, seq_len=w.seq_len,
+                       head_dim=w.head_dim, fc=fc, k=w.k, device=dev)
+    qd, Kd, Vd = q.to(dev), K.to(dev), V.to(dev)
+    m.refresh_keys(Kd)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        m.refresh_keys(Kd, pos0=w.seq_len - 1, npos=1)   # compact row of the newest position
+        m.select(qd)
+        m.attend(qd, Kd, Vd)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize(dev)
+    if int(m.status.item()) != 0:
+        raise RuntimeError(f"device status {int(m.status.item())}")
+    K_ = max(args.steps, 50)
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    with ClockSampler(local) as clk:
+        start.record(stream)
+        for s_ in range(K_):
+            ev[s_][0].record(stream)
+            m.refresh_keys(Kd, pos0=w.seq_len - 1, npos=1)
+            ev[s_][1].record(stream)
+            m.select(qd)
+            ev[s_][2].record(stream)
+            m.attend(qd, Kd, Vd)
+            ev[s_][3].record(stream)
+        stop.record(stream)
+        torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    total_ms = start.elapsed_time(stop)
+    t_sel = float(np.mean([ev[s_][1].elapsed_time(ev[s_][2]) for s_ in range(K_)]))
+    t_att = float(np.mean([ev[s_][2].elapsed_time(ev[s_][3]) for s_ in range(K_)]))
+    t_app = float(np.mean([ev[s_][0].elapsed_time(ev[s_][1]) for s_ in range(K_)]))
+
+    # e2e: pinned host q in, o out, through the public API
+    qh = q.pin_memory()
+    oh = torch.empty(m.o.shape, dtype=m.o.dtype).pin_memory()
+    qdev = torch.empty_like(qd)
+
+    def host_step():
+        qdev.copy_(qh, non_blocking=True)
+        m.refresh_keys(Kd, pos0=w.seq_len - 1, npos=1)
+        m(qdev, Kd, Vd)
+        oh.copy_(m.o, non_blocking=True)
+
+    host_step()
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(K_):
+        host_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1)
+    vals = torch.tensor([total_ms, e2e_ms, t_sel, t_att, t_app], dtype=torch.float64, device=dev)
+    if dist:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, e2e_ms, t_sel, t_att, t_app = vals.tolist()
+    if rank == 0:
+        pk, pk_src = peaks()
+        sel_b, att_b, all_b = decode_bytes(w)
+        achieved = sel_b / (t_sel * 1e-3) / 1e9
+        line = {
+            "metric": DECODE_METRIC, "value": w.batch * world * K_ / (total_ms * 1e-3), "unit": "tokens/s",
+            "n_gpus": world, "steps": K_, "warmup": max(args.warmup, 3), "ms_per_step": total_ms / K_,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name,
+                       "cache": f"B={w.batch} Hq={w.heads_q} Hkv={w.heads_kv} L={w.seq_len} d={w.head_dim}",
+                       "dominant_pairs": w.nfc, "k": w.k, "parallelism": f"replicas x{world}",
+                       "l2": "compact keys 201 MB, K/V cache 2.1 GB per GPU (larger than L2); no flush"},
+            "stages_us": {"append": t_app * 1e3, "select": t_sel * 1e3, "attention": t_att * 1e3},
+            "roofline": {"kernel": "tip_chunk + tip_merge (sfa_decode_select)", "bound": "hbm",
+                         "achieved": achieved, "peak": float(pk["hbm_gbs"]), "unit": "GB/s",
+                         "frac": achieved / float(pk["hbm_gbs"]), "peak_source": f"{pk_src} HBM copy",
+                         "traffic": None, "bytes_per_launch": sel_b},
+            "step_bytes": all_b,
+            "e2e": {"value": w.batch * K_ / (e2e_ms * 1e-3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": qh.numel() * qh.element_size(),
+                    "d2h_bytes_per_step": oh.numel() * oh.element_size()},
+            "gpu_launches": 4 * K_,
+            "clocks": clk.summary(),
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            v, secs, text = oracle_decode_sample(w, q, K, V, fc)
+            line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": blas_threads() or
+                                    len(os.sched_getaffinity(0)), "kind": "oracle", "sample": text,
+                                    "seconds": secs}
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
 def run_reference(args, w, rank, world):
     """The reference arm: the CPU oracle as it stands, on host cores, bounded sample per step."""
     if rank != 0:
@@ -235,6 +403,9 @@ def main():
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.workload in wl.DECODE:
+        run_decode(args, wl.DECODE[args.workload], rank, world)
+        return
     w = wl.ALL[args.workload]
     if args.impl == "reference":
         run_reference(args, w, rank, world)
