@@ -4,15 +4,19 @@
 //   fc_gather      compact copy K_fc [B, Hkv, L, 2 nfc] of the dominant rotary
 //                  pairs of the rotated key cache (low dims, then partners);
 //                  run once over the cache, then per appended token range.
-//   tip_chunk      Token Importance Predictor: CTA = (chunk of C tokens, KV
-//                  head); streams the chunk's K_fc rows once for all Q heads of
-//                  the group; each score is a float32 FMA chain over the
-//                  compact columns in order (a bf16 x bf16 product is exact in
-//                  float32, so every step rounds once and the value is
-//                  reproducible); then each head's local top-k of the
-//                  chunk by a block-wide radix select, written in token order.
-//   tip_merge      CTA per (b, h): radix select over the chunks' candidates
-//                  (already in token order), ascending index list, -1 padded.
+//   tip_chunk      Token Importance Predictor, persistent (one or two CTAs per
+//                  SM) over tiles (chunk of C tokens, b, KV head): the chunk's
+//                  K_fc rows stream through a bulk-copy ring once for all Q
+//                  heads of the group; each score is a float32 FMA chain over
+//                  the compact columns in order (a bf16 x bf16 product is exact
+//                  in float32, so every step rounds once and the value is
+//                  reproducible); then per head a lower bound of the chunk's
+//                  k-th largest score (from group maxima) and the tokens at or
+//                  above it, written per warp segment in token order.
+//   tip_merge      CTA per (b, h): the candidates staged in shared memory,
+//                  bounded again, exact k-th largest by block bisection, ties
+//                  by index; ascending index list, -1 padded (radix select over
+//                  global memory when the candidates do not fit).
 //   fac            Focused Attention Computation: CTA per (b, h), 16 warps,
 //                  each warp gathers the K / V rows of its share of the kept
 //                  tokens (eight tokens' loads in flight per lane), float32
