@@ -515,6 +515,7 @@ def main():
             "roofline": {"kernel": "attn_tc_kernel (sfa_block_sparse_attn)", "bound": "tensor",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": f"{pk_src} bf16 burst",
+                         "frac_of_sustained": achieved / float(pk.get("bf16_tflops_sustained", peak)),
                          "traffic": (tr["bytes_per_launch"] * (w.batch * w.heads_q * w.nb) / tr["tiles_per_launch"]
                                      if tr else None),
                          "traffic_note": (f"ncu DRAM bytes of one launch at {tr['workload']}, scaled by query tiles"

@@ -2,14 +2,16 @@
 // Block-Sparse Attention" §1) on the sm_100a tensor cores.
 //
 // bf16 Q/K/V, query block = key block = 128 tokens, head dim 128.
-// One CTA holds TWO query tiles (t = 0, 1): two consecutive entries of the tile
-// order (b, kv head, query block descending, q head in the group), i.e. two Q
-// heads of one GQA group at the same query block.  Each tile walks its own
-// index list; the two tiles ping-pong on the tensor core: while one softmax
-// warpgroup turns S_t into P_t, the tensor core runs the other tile's P.V and
-// next Q.K^T.
+// A CTA holds KT query tiles (Layout<KT>): consecutive entries of the tile order
+// (b, kv head, query block descending, q head in the group).  With KT = 2 (long
+// index lists) the two tiles, two Q heads of one GQA group at the same query
+// block, ping-pong on the tensor core: while one softmax warpgroup turns S_t
+// into P_t, the tensor core runs the other tile's P.V and next Q.K^T.  With
+// KT = 1 (short lists) two CTAs share each SM and play the same game, and one
+// CTA's prologue (barriers, tensor memory, Q) and epilogue (O) hide behind the
+// other's main loop.
 //
-//   warps 0-7 / 8-15 softmax of tile 0 / tile 1: two threads per query row r
+//   warps 0 .. 8 KT - 1  softmax of tile w / 8: two threads per query row r
 //                    (TMEM lane r; warps w and w+4 share lanes), each owning 64
 //                    of the 128 key columns, row maxima exchanged through shared
 //                    memory; reads S_t from TMEM, online softmax with a lazily
@@ -17,15 +19,15 @@
 //                    TMEM, final O_t / l epilogue.  Two softmax warps per SM
 //                    sub-partition work on a tile at once, hiding each other's
 //                    latency.
-//   warp 16          producer: TMA loads of Q_t and of K_t(j), V_t(j) for every
+//   warp 8 KT        producer: TMA loads of Q_t and of K_t(j), V_t(j) for every
 //                    kept block j of each tile (one K and one V slot per tile).
-//   warp 17          MMA issuer: S_t = Q_t K_t^T (A, B from shared memory) and
+//   warp 8 KT + 1    MMA issuer: S_t = Q_t K_t^T (A, B from shared memory) and
 //                    O_t += P_t V_t (A = P_t from TMEM, B = V_t from shared
 //                    memory), M = N = 128, K = 16 steps; completion tracked with
 //                    tcgen05.commit -> mbarriers.  A commit covers every MMA the
 //                    thread issued before it, so the commit that signals S_t(j)
 //                    also means O_t has absorbed P_t(j-1).
-// TMEM (512 columns): S_0 [0,128) S_1 [128,256) O_0 [256,384) O_1 [384,512);
+// TMEM (256 KT columns): S_t at [128 t, 128 t + 128), O_t at [128 (KT + t), +128);
 // P_t aliases S_t (two bf16 per column): keys [0,64) in S columns [0,32), keys
 // [64,128) in S columns [64,96), each half written by the threads that read it.
 // Every mbarrier wait is bounded (about 2 s); a wait that runs out writes
@@ -44,36 +46,44 @@ namespace {
 constexpr int kHD = 128;
 constexpr uint32_t kSub = 16384;       // 128 rows x 64 bf16 (one 128B-swizzle box)
 constexpr uint32_t kTile = 2 * kSub;   // 128 x 128 bf16
-// Shared memory: per tile t a Q, a K and a V tile (6 x 32 KB).
-__host__ __device__ constexpr uint32_t off_q(int t) { return t * kTile; }
-__host__ __device__ constexpr uint32_t off_k(int t) { return 2 * kTile + t * kTile; }
-__host__ __device__ constexpr uint32_t off_v(int t) { return 4 * kTile + t * kTile; }
-constexpr uint32_t OFF_BAR = 6 * kTile;
-// Barriers, two of each (one per tile) except DRAIN.
+// Barriers, two of each (one per tile) except DRAIN and QR.
 enum { B_Q = 0, B_KF = 2, B_VF = 4, B_KE = 6, B_VE = 8, B_SF = 10, B_PF = 12, B_OD = 14, B_X = 16, B_DRAIN = 20,
        B_QR = 21, NBAR = 22 };  // B_X: [tile][parity] row-max / row-sum exchange of the two column halves;
-                                // B_QR: both Q tiles rotated in shared memory (RoPE on load)
-constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-constexpr uint32_t OFF_XCHG = OFF_MISC + 32;         // [2 tiles][2 parities][2 halves][128 rows] float
-constexpr int kMaxList = 2048;                       // nb <= 2048, so a valid list has <= 2048 entries
-constexpr uint32_t OFF_LIST = OFF_XCHG + 2 * 2 * 2 * 128 * 4;  // per tile: the validated index list
-constexpr uint32_t SMEM_BYTES = OFF_LIST + 2 * kMaxList * 4 + 1024;
-// Warps 0-7 softmax of tile 0, 8-15 of tile 1 (two threads per query row: warps w and w+4
-// share TMEM lanes and split the 128 key columns), 16 producer, 17 MMA issuer.
-constexpr int kThreads = 576;
-constexpr int kProducerWarp = 16, kMmaWarp = 17;
-constexpr uint32_t TMEM_COLS = 512;
+                                // B_QR: the CTA's Q tiles rotated in shared memory (RoPE on load)
+constexpr int kMaxList = 2048;  // nb <= 2048, so a valid list has <= 2048 entries
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
 
-__host__ __device__ constexpr uint32_t col_s(int t) { return t * 128; }
-__host__ __device__ constexpr uint32_t col_o(int t) { return 256 + t * 128; }
+// Layout for KT query tiles per CTA.  KT = 2: one CTA ping-pongs two tiles on the tensor core;
+// KT = 1: half the shared memory and tensor memory, so two CTAs share an SM and each one's
+// prologue and epilogue overlap the other's main loop (better when the index lists are short).
+template <int KT>
+struct Layout {
+  static_assert(KT == 1 || KT == 2, "one or two query tiles per CTA");
+  // Shared memory: per tile t a Q, a K and a V tile (3 KT x 32 KB), barriers, exchange, lists.
+  static __host__ __device__ constexpr uint32_t off_q(int t) { return t * kTile; }
+  static __host__ __device__ constexpr uint32_t off_k(int t) { return KT * kTile + t * kTile; }
+  static __host__ __device__ constexpr uint32_t off_v(int t) { return 2 * KT * kTile + t * kTile; }
+  static constexpr uint32_t OFF_BAR = 3 * KT * kTile;
+  static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr uint32_t OFF_XCHG = OFF_MISC + 32;  // [KT tiles][2 parities][2 halves][128 rows] float
+  static constexpr uint32_t OFF_LIST = OFF_XCHG + KT * 2 * 2 * 128 * 4;  // per tile: the validated index list
+  static constexpr uint32_t SMEM_BYTES = OFF_LIST + KT * kMaxList * 4 + 1024;
+  // Warps 0 .. 8 KT - 1: softmax of tile w / 8 (two threads per query row: warps w and w + 4
+  // share TMEM lanes and split the 128 key columns); then the TMA producer and the MMA issuer.
+  static constexpr int kThreads = KT * 256 + 64;
+  static constexpr int kProducerWarp = KT * 8, kMmaWarp = KT * 8 + 1;
+  static constexpr uint32_t TMEM_COLS = KT * 256;
+  static __host__ __device__ constexpr uint32_t col_s(int t) { return t * 128; }
+  static __host__ __device__ constexpr uint32_t col_o(int t) { return KT * 128 + t * 128; }
+};
 
 struct Ctx {
   uint32_t sbase;
+  uint32_t bars;  // shared address of barrier 0
   volatile int* abort_flag;
   int* status;
-  __device__ uint32_t bar(int k) const { return sbase + OFF_BAR + 8u * k; }
+  __device__ uint32_t bar(int k) const { return bars + 8u * k; }
 };
 
 // Bounded wait on an mbarrier phase.  Returns false if the CTA aborted or the wait ran out.
@@ -125,32 +135,35 @@ __device__ Tile decode_tile(const AttnParams& p, int t) {
   return x;
 }
 
-// RoPE on load: the 512 softmax threads rotate the CTA's Q tiles in shared
+// RoPE on load: the 256 KT softmax threads rotate the CTA's Q tiles in shared
 // memory once their TMA copies have landed (bounded waits on the tiles' B_Q
 // barriers); returns false if a wait gave up.  Work unit = (row, 16-byte
 // chunk c) of a tile: chunk c of box 0 holds dims [8c, 8c + 8) and the same
 // offset of box 1 holds their rotary partners [64 + 8c, 64 + 8c + 8) (chunk c of
 // row r is stored at chunk c ^ (r & 7) of the 128-byte row).  Thread st takes
-// chunk st & 7 of rows st / 8 and st / 8 + 64, so a warp touches four whole
+// chunk st & 7 of rows st / 8 + 32 KT j (j < 4 / KT), so a warp touches four whole
 // rows: conflict-free in shared memory, and each row's table entries are one
 // contiguous 256-byte run.  The two tiles usually share the query block (two
 // heads of a GQA group), so the table entries are fetched once, before the
 // waits, and their latency hides behind the copies.  Kept out of line: it runs
 // once per CTA and must not add to the register pressure of the softmax loop.
+template <int KT>
 __device__ __noinline__ bool rope_q_on_load(volatile int* abort_flag, int* status, uint32_t bar_q0,
                                             unsigned char* sm, const float* cos_t, const float* sin_t, int i0,
                                             int i1, int n0, int n1, int st) {
   Ctx cx;
   cx.sbase = 0;
+  cx.bars = 0;
   cx.abort_flag = abort_flag;
   cx.status = status;
+  constexpr int RPT = 4 / KT, RS = 32 * KT;  // rows per thread, row stride between them
   const int c = st & 7;
-  const bool two = n0 > 0 && n1 > 0 && i1 != i0;  // tiles at different query blocks need two table slices
+  const bool two = KT == 2 && n0 > 0 && n1 > 0 && i1 != i0;  // tiles at different query blocks: two slices
   const int ia = n0 > 0 ? i0 : i1;
-  float ca[2][8], sa[2][8], cb[2][8], sb[2][8];
+  float ca[RPT][8], sa[RPT][8], cb[RPT][8], sb[RPT][8];
 #pragma unroll
-  for (int k = 0; k < 2; ++k) {
-    const int row = (st >> 3) + 64 * k;
+  for (int k = 0; k < RPT; ++k) {
+    const int row = (st >> 3) + RS * k;
     load8(cos_t + ((size_t)ia * 128 + row) * 64 + c * 8, ca[k]);
     load8(sin_t + ((size_t)ia * 128 + row) * 64 + c * 8, sa[k]);
     if (two) {
@@ -160,16 +173,16 @@ __device__ __noinline__ bool rope_q_on_load(volatile int* abort_flag, int* statu
   }
   bool ok = true;
   if (n0 > 0) ok = wait_bar(cx, bar_q0, 0);
-  if (ok && n1 > 0) ok = wait_bar(cx, bar_q0 + 8, 0);  // B_Q + 1
+  if (ok && KT == 2 && n1 > 0) ok = wait_bar(cx, bar_q0 + 8, 0);  // B_Q + 1
   if (!__all_sync(0xffffffffu, ok)) return false;
 #pragma unroll
-  for (int t = 0; t < 2; ++t) {
+  for (int t = 0; t < KT; ++t) {
     if ((t == 0 ? n0 : n1) == 0) continue;
     const bool use_b = t == 1 && two;
 #pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const int row = (st >> 3) + 64 * k;
-      unsigned char* rp = sm + off_q(t) + row * 128 + ((c ^ (row & 7)) << 4);
+    for (int k = 0; k < RPT; ++k) {
+      const int row = (st >> 3) + RS * k;
+      unsigned char* rp = sm + Layout<KT>::off_q(t) + row * 128 + ((c ^ (row & 7)) << 4);
       uint4* plo = reinterpret_cast<uint4*>(rp);
       uint4* phi = reinterpret_cast<uint4*>(rp + kSub);
       const uint4 ulo = *plo, uhi = *phi;
@@ -196,25 +209,31 @@ __device__ __noinline__ bool rope_q_on_load(volatile int* abort_flag, int* statu
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1)
+template <int KT>
+__global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
     attn_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                    const __grid_constant__ CUtensorMap tmV, AttnParams p) {
+  using L = Layout<KT>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t raw = tc::smem_u32(smem_raw);
   const uint32_t pad = (1024u - (raw & 1023u)) & 1023u;
   unsigned char* sm = smem_raw + pad;
   Ctx cx;
   cx.sbase = raw + pad;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + OFF_MISC);
-  cx.abort_flag = reinterpret_cast<volatile int*>(sm + OFF_MISC + 4);
-  int* nsh = reinterpret_cast<int*>(sm + OFF_MISC + 8);  // validated count per tile
-  int* slist = reinterpret_cast<int*>(sm + OFF_LIST);    // [2][kMaxList] validated index lists
+  cx.bars = cx.sbase + L::OFF_BAR;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(sm + L::OFF_MISC);
+  cx.abort_flag = reinterpret_cast<volatile int*>(sm + L::OFF_MISC + 4);
+  int* nsh = reinterpret_cast<int*>(sm + L::OFF_MISC + 8);  // validated count per tile
+  int* slist = reinterpret_cast<int*>(sm + L::OFF_LIST);    // [KT][kMaxList] validated index lists
   cx.status = p.status;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  Tile tl[2] = {decode_tile(p, 2 * blockIdx.x), decode_tile(p, 2 * blockIdx.x + 1)};
+  Tile tl[2];
+  tl[0] = decode_tile(p, KT * blockIdx.x);
+  tl[1] = decode_tile(p, KT == 2 ? 2 * blockIdx.x + 1 : KT * blockIdx.x);
+  if (KT == 1) tl[1].valid = false;
 
-  if (warp == 0 || warp == 8) {
+  if (warp == 0 || (KT == 2 && warp == 8)) {
     // Validate one tile's index list: count in [0, kmax], entries ascending in [0, nb), <= i if causal.
     const int t = warp >> 3;
     const Tile x = t == 0 ? tl[0] : tl[1];
@@ -240,16 +259,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == 0 && lane == 0) {
       *cx.abort_flag = 0;
       for (int k = 0; k < NBAR; ++k)
-        tc::mbar_init(cx.bar(k), k == B_QR ? 512
+        tc::mbar_init(cx.bar(k), k == B_QR ? KT * 256
                                  : (k == B_PF || k == B_PF + 1 || (k >= B_X && k < B_X + 4)) ? 256 : 1);
       tc::fence_mbar_init();
     }
-  } else if (warp == kProducerWarp && lane == 0) {
+  } else if (warp == L::kProducerWarp && lane == 0) {
     tc::prefetch_tmap(&tmQ);
     tc::prefetch_tmap(&tmK);
     tc::prefetch_tmap(&tmV);
-  } else if (warp == kMmaWarp) {
-    tc::tmem_alloc(tc::smem_u32(tmem_slot), TMEM_COLS);
+  } else if (warp == L::kMmaWarp) {
+    tc::tmem_alloc(tc::smem_u32(tmem_slot), L::TMEM_COLS);
     tc::tmem_relinquish();
   }
   tc::tc_fence_before();
@@ -257,19 +276,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc::tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   tl[0].n = nsh[0];
-  tl[1].n = nsh[1];
+  tl[1].n = KT == 2 ? nsh[1] : 0;
   const int nmax = max(tl[0].n, tl[1].n);
 
-  if (warp == kProducerWarp) {
+  if (warp == L::kProducerWarp) {
     // ------------------------------ producer ------------------------------
     if (lane == 0 && nmax > 0) {
       int kissued[2] = {0, 0}, vissued[2] = {0, 0};
       bool qissued[2] = {false, false};
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
+      for (int t = 0; t < KT; ++t) {
         if (tl[t].n == 0) continue;
         const int qrow = (tl[t].b * p.Hq + tl[t].h) * p.L + tl[t].i * 128;
-        const uint32_t sQ = cx.sbase + off_q(t);
+        const uint32_t sQ = cx.sbase + L::off_q(t);
         tc::mbar_arrive_expect_tx(cx.bar(B_Q + t), kTile);
         tc::tma_load_2d(sQ, &tmQ, cx.bar(B_Q + t), 0, qrow);
         tc::tma_load_2d(sQ + kSub, &tmQ, cx.bar(B_Q + t), 64, qrow);
@@ -278,22 +297,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int it = 0; ok && it < nmax; ++it) {
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < KT; ++t) {
           if (!ok || it >= tl[t].n) continue;
           if (it > 0 && !wait_bar(cx, cx.bar(B_KE + t), (it - 1) & 1)) { ok = false; break; }
           const int row = (tl[t].b * p.Hkv + tl[t].g) * p.L + slist[t * kMaxList + it] * 128;
-          const uint32_t sK = cx.sbase + off_k(t);
+          const uint32_t sK = cx.sbase + L::off_k(t);
           tc::mbar_arrive_expect_tx(cx.bar(B_KF + t), kTile);
           tc::tma_load_2d(sK, &tmK, cx.bar(B_KF + t), 0, row);
           tc::tma_load_2d(sK + kSub, &tmK, cx.bar(B_KF + t), 64, row);
           kissued[t] = it + 1;
         }
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < KT; ++t) {
           if (!ok || it >= tl[t].n) continue;
           if (it > 0 && !wait_bar(cx, cx.bar(B_VE + t), (it - 1) & 1)) { ok = false; break; }
           const int row = (tl[t].b * p.Hkv + tl[t].g) * p.L + slist[t * kMaxList + it] * 128;
-          const uint32_t sV = cx.sbase + off_v(t);
+          const uint32_t sV = cx.sbase + L::off_v(t);
           tc::mbar_arrive_expect_tx(cx.bar(B_VF + t), kTile);
           tc::tma_load_2d(sV, &tmV, cx.bar(B_VF + t), 0, row);
           tc::tma_load_2d(sV + kSub, &tmV, cx.bar(B_VF + t), 64, row);
@@ -302,14 +321,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*cx.abort_flag) {
         // Let every copy this CTA started land before the CTA exits.
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < KT; ++t) {
           if (qissued[t]) drain_wait(cx.bar(B_Q + t), 0);
           if (kissued[t] > 0) drain_wait(cx.bar(B_KF + t), (kissued[t] - 1) & 1);
           if (vissued[t] > 0) drain_wait(cx.bar(B_VF + t), (vissued[t] - 1) & 1);
         }
       }
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == L::kMmaWarp) {
     // ------------------------------ MMA issuer ----------------------------
     if (lane == 0 && nmax > 0) {
       const uint32_t id_qk = tc::idesc_bf16_f32(128, 128, false);
@@ -318,18 +337,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       // S_t(0) for both tiles.
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
+      for (int t = 0; t < KT; ++t) {
         if (!ok || tl[t].n == 0) continue;
         if (!wait_bar(cx, cx.bar(rot ? B_QR : B_Q + t), 0) || !wait_bar(cx, cx.bar(B_KF + t), 0)) {
           ok = false;
           break;
         }
         tc::tc_fence_after();
-        const uint32_t sQ = cx.sbase + off_q(t), sK = cx.sbase + off_k(t);
+        const uint32_t sQ = cx.sbase + L::off_q(t), sK = cx.sbase + L::off_k(t);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk) {
           const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-          tc::mma_bf16_ss(tmem + col_s(t), tc::sw128_desc(sQ + off, 16, 1024), tc::sw128_desc(sK + off, 16, 1024),
+          tc::mma_bf16_ss(tmem + L::col_s(t), tc::sw128_desc(sQ + off, 16, 1024), tc::sw128_desc(sK + off, 16, 1024),
                           id_qk, kk > 0 ? 1u : 0u);
         }
         tc::mma_commit(cx.bar(B_KE + t));
@@ -337,7 +356,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       for (int it = 0; ok && it < nmax; ++it) {
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < KT; ++t) {
           if (!ok || it >= tl[t].n) continue;
           // O_t += P_t(it) V_t(it)
           if (!wait_bar(cx, cx.bar(B_PF + t), it & 1) || !wait_bar(cx, cx.bar(B_VF + t), it & 1)) {
@@ -345,11 +364,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           tc::tc_fence_after();
-          const uint32_t sV = cx.sbase + off_v(t);
+          const uint32_t sV = cx.sbase + L::off_v(t);
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
             // P keys [16 kk, 16 kk + 16): half kk / 4 wrote them into its own S columns
-            tc::mma_bf16_ts(tmem + col_o(t), tmem + col_s(t) + (kk >> 2) * 64 + (kk & 3) * 8,
+            tc::mma_bf16_ts(tmem + L::col_o(t), tmem + L::col_s(t) + (kk >> 2) * 64 + (kk & 3) * 8,
                             tc::sw128_desc(sV + kk * 2048, kSub, 1024), id_pv, (it > 0 || kk > 0) ? 1u : 0u);
           tc::mma_commit(cx.bar(B_VE + t));
           if (it + 1 < tl[t].n) {
@@ -359,11 +378,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait_bar(cx, cx.bar(B_VE + t), it & 1)) { ok = false; break; }
             if (!wait_bar(cx, cx.bar(B_KF + t), (it + 1) & 1)) { ok = false; break; }
             tc::tc_fence_after();
-            const uint32_t sQ = cx.sbase + off_q(t), sK = cx.sbase + off_k(t);
+            const uint32_t sQ = cx.sbase + L::off_q(t), sK = cx.sbase + L::off_k(t);
 #pragma unroll
             for (int kk = 0; kk < 8; ++kk) {
               const uint32_t off = (kk >> 2) * kSub + (kk & 3) * 32;
-              tc::mma_bf16_ss(tmem + col_s(t), tc::sw128_desc(sQ + off, 16, 1024),
+              tc::mma_bf16_ss(tmem + L::col_s(t), tc::sw128_desc(sQ + off, 16, 1024),
                               tc::sw128_desc(sK + off, 16, 1024), id_qk, kk > 0 ? 1u : 0u);
             }
             tc::mma_commit(cx.bar(B_KE + t));
@@ -384,10 +403,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = ((warp & 3) << 5) | lane;  // query row = TMEM lane
     const Tile x = t == 0 ? tl[0] : tl[1];
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + col_s(t) + 64 * hf;     // this half's S columns
-    const uint32_t tP = tmem + lane_base + col_s(t) + 64 * hf;     // this half's P columns (2 bf16 each)
-    const uint32_t tO = tmem + lane_base + col_o(t) + 64 * hf;     // this half's O columns
-    float* xchg = reinterpret_cast<float*>(sm + OFF_XCHG) + t * 512;  // [parity][half][row]
+    const uint32_t tS = tmem + lane_base + L::col_s(t) + 64 * hf;     // this half's S columns
+    const uint32_t tP = tmem + lane_base + L::col_s(t) + 64 * hf;     // this half's P columns (2 bf16 each)
+    const uint32_t tO = tmem + lane_base + L::col_o(t) + 64 * hf;     // this half's O columns
+    float* xchg = reinterpret_cast<float*>(sm + L::OFF_XCHG) + t * 512;  // [parity][half][row]
     // Exchange with the other half of the row: write, arrive on the tile's parity barrier (256
     // arrivals), bounded wait, read.  Use u of parity q waits for phase parity (u / 2) & 1.
     auto exchange = [&](int use, float v) -> float {
@@ -403,8 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
     bool ok = true;
     if (p.rope_cos != nullptr && nmax > 0) {
-      // RoPE on load: all 512 softmax threads rotate both Q tiles, then one arrival each on B_QR.
-      ok = rope_q_on_load(cx.abort_flag, cx.status, cx.bar(B_Q), sm, p.rope_cos, p.rope_sin, tl[0].i, tl[1].i,
+      // RoPE on load: all softmax threads rotate the CTA's Q tiles, then one arrival each on B_QR.
+      ok = rope_q_on_load<KT>(cx.abort_flag, cx.status, cx.bar(B_Q), sm, p.rope_cos, p.rope_sin, tl[0].i, tl[1].i,
                           tl[0].n, tl[1].n, warp * 32 + lane);
       tc::mbar_arrive(cx.bar(B_QR));
     }
@@ -534,21 +553,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc::tc_fence_before();
   __syncthreads();
-  if (warp == kMmaWarp) {
+  if (warp == L::kMmaWarp) {
     tc::tc_fence_after();
-    tc::tmem_dealloc(tmem, TMEM_COLS);
+    tc::tmem_dealloc(tmem, L::TMEM_COLS);
   }
 }
 
+template <int KT>
+static cudaError_t launch_attn_t(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
+                                 const CUtensorMap& tmV, cudaStream_t st) {
+  using L = Layout<KT>;
+  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel<KT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)L::SMEM_BYTES);
+  if (e != cudaSuccess) return e;
+  if (KT == 1) {  // room for two CTAs per SM
+    e = cudaFuncSetAttribute(attn_tc_kernel<KT>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+  }
+  const size_t tiles = (size_t)p.B * p.Hq * p.nb;
+  const unsigned grid = (unsigned)((tiles + KT - 1) / KT);
+  attn_tc_kernel<KT><<<grid, L::kThreads, L::SMEM_BYTES, st>>>(tmQ, tmK, tmV, p);
+  return cudaGetLastError();
+}
+
+// Short index lists (few key blocks per query tile) leave each CTA's prologue and epilogue
+// exposed: one tile per CTA lets two CTAs per SM hide them behind each other.  Long lists
+// favour the two-tile ping-pong inside one CTA.  (Measured on this B200, one vs two tiles per
+// CTA: 64K layer at 1% density (lists of 3) 0.78 vs 0.85 ms; at 25% (69) 9.2 vs 9.0 ms; the
+// 32K layer (14) 1.077 vs 1.066 ms; the 128K layer (26) within run-to-run noise.)
+constexpr int kShortList = 12;
+
 cudaError_t launch_attn_tcgen05(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                 const CUtensorMap& tmV, cudaStream_t st) {
-  cudaError_t e = cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)SMEM_BYTES);
-  if (e != cudaSuccess) return e;
-  const size_t tiles = (size_t)p.B * p.Hq * p.nb;
-  const unsigned grid = (unsigned)((tiles + 1) / 2);
-  attn_tc_kernel<<<grid, kThreads, SMEM_BYTES, st>>>(tmQ, tmK, tmV, p);
-  return cudaGetLastError();
+  return p.kmax <= kShortList ? launch_attn_t<1>(p, tmQ, tmK, tmV, st) : launch_attn_t<2>(p, tmQ, tmK, tmV, st);
 }
 
 }  // namespace sfa

@@ -8,6 +8,11 @@ importance).  So the units (b, g) are independent and can be given to
 different ranks with no exchange on the data path; only the timing is
 reduced across ranks (max), and outputs are gathered only if a caller wants
 them in one place.
+
+The decode step splits the same way ("FASA: Frequency-aware Sparse
+Attention" §2B): the compact keys, token scores, selection and focused
+attention of a Q head read only its sequence's cache of its KV head, so the
+(b, g) units of a decode batch are independent too.
 """
 
 from __future__ import annotations

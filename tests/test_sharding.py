@@ -92,3 +92,61 @@ def test_two_rank_gloo_split_equals_single_process():
     full = run_units(sharding.units(W.batch, W.heads_kv), Q, K, V)
     for u in keys:
         np.testing.assert_array_equal(merged[u], full[u])
+
+
+# ---------------------------------------------------------------------------
+# Decode step: the same (batch, KV group) split
+# ---------------------------------------------------------------------------
+from block_sparse_long_dual_b200.synthetic import make_decode_inputs  # noqa: E402
+from block_sparse_long_dual_b200.workloads import DecodeWorkload  # noqa: E402
+from oracle import fasa_oracle as fo  # noqa: E402
+
+DW = DecodeWorkload(name="shard-decode", batch=2, heads_q=4, heads_kv=2, seq_len=300, head_dim=16, nfc=4, k=20)
+
+
+def run_decode_units(us, q, K, V, fc):
+    out = {}
+    for b, g in us:
+        hs = list(sharding.q_heads(g, DW.heads_q, DW.heads_kv))
+        _, _, idx, o, _ = fo.decode_step(q[b:b + 1, hs].double().numpy(), K[b:b + 1, g:g + 1].double().numpy(),
+                                         V[b:b + 1, g:g + 1].double().numpy(), fc[g:g + 1], DW.k)
+        out[(b, g)] = (idx[0], o[0])
+    return out
+
+
+def _decode_worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        qq, K, V, fc = make_decode_inputs(DW, seed=0)
+        mine = sharding.shard(sharding.units(DW.batch, DW.heads_kv), world, rank)
+        gathered = [None] * world
+        dist.all_gather_object(gathered, run_decode_units(mine, qq, K, V, fc))
+        if rank == 0:
+            merged = {}
+            for part in gathered:
+                assert not (set(part) & set(merged))
+                merged.update(part)
+            q.put(merged)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_rank_gloo_decode_split_equals_single_process():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_decode_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    merged = q.get(timeout=180)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    qq, K, V, fc = make_decode_inputs(DW, seed=0)
+    _, _, idx, o, _ = fo.decode_step(qq.double().numpy(), K.double().numpy(), V.double().numpy(), fc, DW.k)
+    assert sorted(merged) == sharding.units(DW.batch, DW.heads_kv)
+    for (b, g), (ii, oo) in merged.items():
+        hs = list(sharding.q_heads(g, DW.heads_q, DW.heads_kv))
+        np.testing.assert_array_equal(ii, idx[b, hs])
+        np.testing.assert_array_equal(oo, o[b, hs])
