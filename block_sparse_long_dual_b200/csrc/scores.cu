@@ -349,12 +349,12 @@ __global__ void __launch_bounds__(256, 1) block_score_softmax_kernel(ScoreParams
 #pragma unroll
           for (int ct = 0; ct < CTW; ++ct) acc[rt][ct][0] = acc[rt][ct][1] = 0.0;
         // B fragment of column tile ct at k-step ks: kbar[col][4 ks + tq], col = tile start + gq.
-        const double* kb[CTW];
+        const double* kptr[CTW];
         double kih[CTW], kil[CTW];  // 1 / rho^band_col(K) with SFA_BLOCK_TAU, else 1
 #pragma unroll
         for (int ct = 0; ct < CTW; ++ct) {
           const int col = min(col0 + (warp * CTW + ct) * 8 + gq, p.nb - 1);
-          kb[ct] = ksrc + (size_t)col * D + tq;
+          kptr[ct] = ksrc + (size_t)col * D + tq;
           kih[ct] = kil[ct] = 1.0;
           if (block_tau) {
             const double* er = ek + (size_t)col * 4;
@@ -362,31 +362,38 @@ __global__ void __launch_bounds__(256, 1) block_score_softmax_kernel(ScoreParams
             kil[ct] = 1.0 / block_rho(er[1], er[3], p.block);
           }
         }
-        double bcur[CTW], bnxt[CTW];
-        {
-          const bool hb = (tq % (D / 2)) < p.band_pairs;
+        // B fragments in batches of KB k-steps, double-buffered in registers: the next batch's L2
+        // loads are in flight while this batch's MMAs run.
+        constexpr int KB = 4;
+        constexpr int NKB = KS / KB;
+        double bb[2][KB][CTW];
+        auto load_batch = [&](int kb, double (&dst)[KB][CTW]) {
 #pragma unroll
-          for (int ct = 0; ct < CTW; ++ct) bcur[ct] = __ldg(kb[ct]) * (hb ? kih[ct] : kil[ct]);
-        }
-#pragma unroll 4
-        for (int ks = 0; ks < KS; ++ks) {
-          if (ks + 1 < KS) {
-            const bool hb = ((4 * (ks + 1) + tq) % (D / 2)) < p.band_pairs;
+          for (int u = 0; u < KB; ++u) {
+            const int ks = kb * KB + u;
+            const bool hb = ((4 * ks + tq) % (D / 2)) < p.band_pairs;
 #pragma unroll
-            for (int ct = 0; ct < CTW; ++ct) bnxt[ct] = __ldg(kb[ct] + 4 * (ks + 1)) * (hb ? kih[ct] : kil[ct]);
+            for (int ct = 0; ct < CTW; ++ct) dst[u][ct] = __ldg(kptr[ct] + 4 * ks) * (hb ? kih[ct] : kil[ct]);
           }
-          double a[RTL];
+        };
+        load_batch(0, bb[0]);
 #pragma unroll
-          for (int rt = 0; rt < RTL; ++rt) a[rt] = qs[(rt * 8 + gq) * QLD + 4 * ks + tq];
+        for (int kb = 0; kb < NKB; ++kb) {
+          if (kb + 1 < NKB) load_batch(kb + 1, bb[(kb + 1) & 1]);
 #pragma unroll
-          for (int ct = 0; ct < CTW; ++ct) {
-            if (ct < ntl) {
+          for (int u = 0; u < KB; ++u) {
+            const int ks = kb * KB + u;
+            double a[RTL];
 #pragma unroll
-              for (int rt = 0; rt < RTL; ++rt) dmma_8x8x4(acc[rt][ct], a[rt], bcur[ct]);
+            for (int rt = 0; rt < RTL; ++rt) a[rt] = qs[(rt * 8 + gq) * QLD + 4 * ks + tq];
+#pragma unroll
+            for (int ct = 0; ct < CTW; ++ct) {
+              if (ct < ntl) {
+#pragma unroll
+                for (int rt = 0; rt < RTL; ++rt) dmma_8x8x4(acc[rt][ct], a[rt], bb[kb & 1][u][ct]);
+              }
             }
           }
-#pragma unroll
-          for (int ct = 0; ct < CTW; ++ct) bcur[ct] = bnxt[ct];
         }
         // C fragment: (row gq, cols 2 tq, 2 tq + 1) of each tile
 #pragma unroll
