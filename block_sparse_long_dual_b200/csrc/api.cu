@@ -454,3 +454,13 @@ sfa_status sfa_decode_attn(const sfa_shape* shape, const void* q, const void* K_
 }
 
 }  // extern "C"
+
+extern "C" {
+
+sfa_status sfa_selftest_bounded_wait(int* status_word, unsigned limit_ms, int complete, void* stream) {
+  if (status_word == nullptr || limit_ms == 0 || limit_ms > 10000) return SFA_ERR_INVALID_ARG;
+  return cuda_status(launch_bounded_wait_selftest(status_word, (uint64_t)limit_ms * 1000000ull, complete ? 1 : 0,
+                                                  as_stream(stream)));
+}
+
+}  // extern "C"

@@ -91,6 +91,8 @@ def load() -> ctypes.CDLL:
     lib.sfa_decode_attn.restype = c_int
     lib.sfa_decode_attn.argtypes = [POINTER(Shape), c_void_p, c_void_p, c_void_p, c_void_p, c_int, c_float,
                                     c_void_p, c_void_p, c_void_p, c_void_p]
+    lib.sfa_selftest_bounded_wait.restype = c_int
+    lib.sfa_selftest_bounded_wait.argtypes = [c_void_p, ctypes.c_uint, c_int, c_void_p]
     _lib = lib
     return lib
 
@@ -476,3 +478,12 @@ class FasaDecode:
         self.select(q, stream)
         self.attend(q, K_cache, V_cache, stream)
         return self.o
+
+
+def selftest_bounded_wait(limit_ms: int, complete: bool, device="cuda", stream=None) -> int:
+    """sfa_selftest_bounded_wait: returns the device status word (0 or SFA_ERR_TIMEOUT)."""
+    lib = load()
+    status = torch.full((1,), -1, dtype=torch.int32, device=device)
+    _check(lib.sfa_selftest_bounded_wait(_ptr(status), int(limit_ms), 1 if complete else 0, _stream(stream)),
+           "sfa_selftest_bounded_wait")
+    return int(status.item())

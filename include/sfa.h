@@ -321,6 +321,16 @@ sfa_status sfa_decode_attn(const sfa_shape* shape, const void* q, const void* K_
                            const void* V_cache, const int* idx, int k, float scale, void* o,
                            float* lse, int* status_word, void* stream);
 
+/*
+ * Diagnostics (no counterpart in the pages): exercises the bounded wait that
+ * every kernel of this library uses on its mbarriers.  One CTA waits on a
+ * barrier phase that nothing completes (complete == 0) or that it completes
+ * itself (complete != 0), giving up after limit_ms (1 .. 10000) milliseconds;
+ * writes SFA_ERR_TIMEOUT or SFA_OK to *status_word (device).  Returns
+ * SFA_ERR_INVALID_ARG for a NULL status word or a limit out of range.
+ */
+sfa_status sfa_selftest_bounded_wait(int* status_word, unsigned limit_ms, int complete, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

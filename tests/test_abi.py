@@ -207,6 +207,13 @@ def test_decode_validation(lib):
     assert lib.sfa_decode_workspace(ctypes.byref(sh), 0) == 0
 
 
+def test_selftest_validation(lib):
+    d = ctypes.c_void_p(1 << 20)
+    assert lib.sfa_selftest_bounded_wait(None, 100, 0, None) == 1
+    assert lib.sfa_selftest_bounded_wait(d, 0, 0, None) == 1
+    assert lib.sfa_selftest_bounded_wait(d, 20000, 0, None) == 1
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(sfa, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(sfa, "_lib", None)
