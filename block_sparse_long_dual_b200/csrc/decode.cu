@@ -198,65 +198,6 @@ __device__ int block_filter_ordered(KeyAt key_at, int n, uint32_t LB, Emit emit,
   return total;
 }
 
-// Block-wide lower bound, NH independent problems at once: for each h, a value LB with at
-// least k of the block's values v[h][.] >= LB (every thread holds NV of them; k <= 256 NV).
-// Bisection from the bracket [min, max + 1) keeps that invariant at every step, so stopping
-// after ITERS steps gives a valid (if looser) bound.  One barrier per step: the per-warp counts
-// alternate between two halves of sh (2 * 8 * NH ints).
-template <int NH, int NV, int ITERS>
-__device__ void block_lower_bound(const uint32_t (&v)[NH][NV], int k, uint32_t (&LB)[NH], int* sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint64_t lo[NH], hi[NH];
-#pragma unroll
-  for (int h = 0; h < NH; ++h) {
-    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-#pragma unroll
-    for (int j = 0; j < NV; ++j) { mn = min(mn, v[h][j]); mx = max(mx, v[h][j]); }
-    mn = __reduce_min_sync(0xffffffffu, mn);
-    mx = __reduce_max_sync(0xffffffffu, mx);
-    if (lane == 0) { sh[warp * NH + h] = (int)mn; sh[(kWarps + warp) * NH + h] = (int)mx; }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int h = 0; h < NH; ++h) {
-    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) {
-      mn = min(mn, (uint32_t)sh[w * NH + h]);
-      mx = max(mx, (uint32_t)sh[(kWarps + w) * NH + h]);
-    }
-    lo[h] = mn;  // every value >= min: #{>= lo} = 256 NV >= k
-    hi[h] = (uint64_t)mx + 1;
-  }
-  __syncthreads();
-  for (int it = 0; it < ITERS; ++it) {
-    int* cs = sh + (it & 1) * kWarps * NH;
-    uint32_t mid[NH];
-#pragma unroll
-    for (int h = 0; h < NH; ++h) {
-      mid[h] = (uint32_t)(lo[h] + ((hi[h] - lo[h]) >> 1));
-      int c = 0;
-#pragma unroll
-      for (int j = 0; j < NV; ++j) c += v[h][j] >= mid[h] ? 1 : 0;
-      c = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
-      if (lane == 0) cs[warp * NH + h] = c;
-    }
-    __syncthreads();
-#pragma unroll
-    for (int h = 0; h < NH; ++h) {
-      int c = 0;
-#pragma unroll
-      for (int w = 0; w < kWarps; ++w) c += cs[w * NH + h];
-      if (hi[h] - lo[h] > 1) {
-        if (c >= k) lo[h] = mid[h]; else hi[h] = mid[h];
-      }
-    }
-  }
-  __syncthreads();
-#pragma unroll
-  for (int h = 0; h < NH; ++h) LB[h] = (uint32_t)lo[h];
-}
-
 // Block-wide bisection over n values in shared memory (1 <= k <= n): the k-th largest T and
 // *gt = #{> T}.  Bracketed by the values' minimum and maximum.
 __device__ uint32_t block_kth_largest_smem(const uint32_t* vals, int n, int k, int* sh, int* gt) {
@@ -341,7 +282,7 @@ __global__ void __launch_bounds__(kThreads) fc_gather_kernel(DecodeParams p, con
 // tile's candidates are selected.
 // ---------------------------------------------------------------------------
 template <int G, int TPS, int NGR>
-__global__ void __launch_bounds__(kThreads, 1) tip_chunk_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(DecodeParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   constexpr int ST = kThreads * TPS;
   const int W = 2 * p.nfc;
@@ -407,12 +348,7 @@ __global__ void __launch_bounds__(kThreads, 1) tip_chunk_kernel(DecodeParams p) 
     __syncthreads();
 
     // Scores: a float32 FMA chain per (token, head) over the columns in order.  Thread tid takes
-    // tokens tid + 256 u of each slab; its j-th key of the chunk (j = slab TPS + u) joins group j / 4.
-    uint32_t gmax[G][NGR];
-#pragma unroll
-    for (int hh = 0; hh < G; ++hh)
-#pragma unroll
-      for (int r = 0; r < NGR; ++r) gmax[hh][r] = 0u;
+    // tokens tid + 256 u of each slab.
     for (int sl = 0; sl < nsl; ++sl, ++consumed) {
       const int stg = consumed % NS;
       if (!wait_parity_bounded((uint32_t)__cvta_generic_to_shared(&bars[stg]), (consumed / NS) & 1)) lost = 1;
@@ -455,33 +391,59 @@ __global__ void __launch_bounds__(kThreads, 1) tip_chunk_kernel(DecodeParams p) 
 #pragma unroll
       for (int u = 0; u < TPS; ++u) {
         const int t = sl * ST + u * kThreads + tid;
-        const int grp = (sl * TPS + u) >> 2;
         if (t < n) {
 #pragma unroll
-          for (int hh = 0; hh < G; ++hh) {
-            const uint32_t key = order_key(acc[u][hh]);
-            keys[(size_t)hh * C + t] = key;
-#pragma unroll
-            for (int r = 0; r < NGR; ++r)
-              if (r == grp) gmax[hh][r] = max(gmax[hh][r], key);
-          }
+          for (int hh = 0; hh < G; ++hh) keys[(size_t)hh * C + t] = order_key(acc[u][hh]);
         }
       }
       __syncthreads();  // stage consumed
       if (tid == 0) issue_next();
     }
 
-    // Per head, a lower bound LB of the chunk's k-th largest key: a value with at least k of the
-    // 256 NGR group maxima (each a distinct key, or 0) at or above it, when k <= 256 NGR.  Every
-    // token of the row's top k has a key >= the row's k-th largest >= the chunk's k-th largest
-    // >= LB, so keys below LB are dropped.
-    uint32_t LB[G];
-    if (p.k <= kThreads * NGR) {
-      block_lower_bound<G, NGR, 16>(gmax, p.k, LB, scratch);
-    } else {
+    // Per head, a lower bound LB of the chunk's k-th largest key, by warp h alone: the maxima
+    // of the C / 4 groups of 4 consecutive keys (0 past the end of the chunk), then a bisection
+    // over them in registers.  Any value with at least k group maxima at or above it is at most
+    // the chunk's k-th largest (each maximum is a distinct key), so stopping the bisection
+    // early still gives a valid bound.  Every token of the row's top k has a key >= the row's
+    // k-th largest >= the chunk's k-th largest >= LB, so keys below LB are dropped.
+    {
+      const int lane = tid & 31, warp = tid >> 5;
+      constexpr int NGPL = 8 * NGR;  // groups per lane: C / 4 / 32
+      if (warp < G) {
+        uint32_t LBw = 0u;
+        if (p.k <= 32 * NGPL) {
+          const uint32_t* hk = keys + (size_t)warp * C;
+          uint32_t gm[NGPL];
+          uint32_t mn = 0xFFFFFFFFu, mx = 0u;
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) LB[hh] = 0u;
+          for (int j = 0; j < NGPL; ++j) {
+            const int t = 4 * (j * 32 + lane);
+            const uint4 v = *reinterpret_cast<const uint4*>(hk + t);
+            const uint32_t m0 = t < n ? v.x : 0u, m1 = t + 1 < n ? v.y : 0u;
+            const uint32_t m2 = t + 2 < n ? v.z : 0u, m3 = t + 3 < n ? v.w : 0u;
+            gm[j] = max(max(m0, m1), max(m2, m3));
+            mn = min(mn, gm[j]);
+            mx = max(mx, gm[j]);
+          }
+          mn = __reduce_min_sync(0xffffffffu, mn);
+          mx = __reduce_max_sync(0xffffffffu, mx);
+          uint64_t lo = mn, hi = (uint64_t)mx + 1;  // #{>= lo} >= k, #{>= hi} < k
+          for (int it = 0; it < 24 && hi - lo > 1; ++it) {
+            const uint32_t mid = (uint32_t)(lo + ((hi - lo) >> 1));
+            int c = 0;
+#pragma unroll
+            for (int j = 0; j < NGPL; ++j) c += gm[j] >= mid ? 1 : 0;
+            if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= p.k) lo = mid; else hi = mid;
+          }
+          LBw = (uint32_t)lo;
+        }
+        if (lane == 0) scratch[warp] = (int)LBw;
+      }
+      __syncthreads();
     }
+    uint32_t LB[G];
+#pragma unroll
+    for (int hh = 0; hh < G; ++hh) LB[hh] = (uint32_t)scratch[hh];
     // Candidates in token order: warp w scans its contiguous range [w S, w S + S) of the chunk
     // and writes its own segment of the slot; counts per (slot, warp).
     const int bad = lost;
