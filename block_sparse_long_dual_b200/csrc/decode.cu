@@ -494,6 +494,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
 // candidates than fit use the block radix select over global memory.
 // ---------------------------------------------------------------------------
 constexpr int kMergeSmem = 12288;
+constexpr int kWarpSel = 64;  // survivors per lane for the single-warp exact threshold (2048 in all)
 constexpr int kMaxChunks = 512;
 
 __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
@@ -553,10 +554,14 @@ __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
     int* st = reinterpret_cast<int*>(sk + n);             // [n] token indices
     int* sv = st + n;                                     // [n] survivor positions
     uint32_t* gk = reinterpret_cast<uint32_t*>(sv + n);   // [n] survivor keys
-    for (int i = tid; i < n; i += kThreads) {
-      const size_t o = locate(i);
-      sk[i] = __ldg(ck + o);
-      st[i] = __ldg(ci + o);
+    // segment-wise copies: warp w takes segments w, w + 8, ...; lanes stride each segment
+    for (int sg = warp; sg < nseg; sg += kWarps) {
+      const int o = off[sg], cnt = off[sg + 1] - o;
+      const size_t src = (size_t)sg * S;
+      for (int r = lane; r < cnt; r += 32) {
+        sk[o + r] = __ldg(ck + src + r);
+        st[o + r] = __ldg(ci + src + r);
+      }
     }
     __syncthreads();
     if (p.k >= n) {
@@ -581,7 +586,41 @@ __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
       for (int j = tid; j < ns; j += kThreads) gk[j] = sk[sv[j]];
       __syncthreads();
       int gt = 0;
-      const uint32_t T = block_kth_largest_smem(gk, ns, p.k, sh, &gt);
+      uint32_t T;
+      if (ns <= 32 * kWarpSel) {
+        // few survivors: one warp finds the k-th largest in registers, no barriers per step
+        if (warp == 0) {
+          uint32_t v[kWarpSel];
+          uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+          for (int j = 0; j < kWarpSel; ++j) {
+            const int q = j * 32 + lane;
+            v[j] = q < ns ? gk[q] : 0u;
+            if (q < ns) { mn = min(mn, v[j]); mx = max(mx, v[j]); }
+          }
+          mn = __reduce_min_sync(0xffffffffu, mn);
+          mx = __reduce_max_sync(0xffffffffu, mx);
+          uint64_t lo = mn, hi = (uint64_t)mx + 1;  // #{>= lo} >= k, #{>= hi} < k (padding 0 < mn)
+          while (hi - lo > 1) {
+            const uint32_t mid = (uint32_t)(lo + ((hi - lo) >> 1));
+            int c = 0;
+#pragma unroll
+            for (int j = 0; j < kWarpSel; ++j) c += (j * 32 + lane < ns && v[j] >= mid) ? 1 : 0;
+            if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= p.k) lo = mid; else hi = mid;
+          }
+          int g2 = 0;
+#pragma unroll
+          for (int j = 0; j < kWarpSel; ++j) g2 += (j * 32 + lane < ns && v[j] > (uint32_t)lo) ? 1 : 0;
+          g2 = (int)__reduce_add_sync(0xffffffffu, (unsigned)g2);
+          if (lane == 0) { sh[30] = (int)(uint32_t)lo; sh[31] = g2; }
+        }
+        __syncthreads();
+        T = (uint32_t)sh[30];
+        gt = sh[31];
+        __syncthreads();
+      } else {
+        T = block_kth_largest_smem(gk, ns, p.k, sh, &gt);
+      }
       const int take = p.k - gt;
       // ordered emission over the survivors with ties by index
       const unsigned lt = (1u << lane) - 1u;
