@@ -126,6 +126,20 @@ def _cuda(t: torch.Tensor, name: str):
         raise ValueError(f"{name} must be contiguous")
 
 
+def _expect(t, name: str, shape, dtype, device=None):
+    """The library takes raw pointers, so every buffer's shape, dtype, layout and device is checked
+    here before a kernel can read or write past it."""
+    if t is None:
+        return
+    if tuple(t.shape) != tuple(int(x) for x in shape):
+        raise ValueError(f"{name} must have shape {tuple(int(x) for x in shape)}, got {tuple(t.shape)}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    _cuda(t, name)
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+
+
 def make_shape(Q: torch.Tensor, K: torch.Tensor) -> Shape:
     if Q.dim() != 4 or K.dim() != 4:
         raise ValueError("Q and K must be [B, H, L, d]")
@@ -171,6 +185,21 @@ def workspace_views(ws: torch.Tensor, shape: Shape, block: int):
             view(3, B * Hq * 2, torch.float64, (B, Hq, 2)))
 
 
+def _check_score_buffers(Q, K, cos, sin, apply_rope, Q_rot, K_rot, probs, workspace, nb):
+    dev = Q.device
+    _expect(K, "K", K.shape, Q.dtype, dev)
+    if apply_rope:
+        half = Q.shape[-1] // 2
+        _expect(cos, "cos", (Q.shape[2], half), torch.float32, dev)
+        _expect(sin, "sin", (Q.shape[2], half), torch.float32, dev)
+        _expect(Q_rot, "Q_rot", Q.shape, Q.dtype, dev)
+        _expect(K_rot, "K_rot", K.shape, K.dtype, dev)
+    _expect(probs, "probs", (Q.shape[0], Q.shape[1], nb, nb), torch.float32, dev)
+    if workspace.dtype != torch.uint8 or workspace.dim() != 1:
+        raise ValueError("workspace must be a 1-D uint8 tensor")
+    _cuda(workspace, "workspace")
+
+
 def block_scores(Q, K, cos, sin, *, band_split: int, block: int, flags: int = 0, apply_rope: bool = True,
                  Q_rot=None, K_rot=None, probs=None, workspace=None, store_q_rot: bool = True, stream=None):
     """sfa_block_scores: returns (Q_rot, K_rot, probs, workspace).
@@ -190,6 +219,7 @@ def block_scores(Q, K, cos, sin, *, band_split: int, block: int, flags: int = 0,
         probs = torch.empty((shape.batch, shape.heads_q, nb, nb), dtype=torch.float32, device=Q.device)
     if workspace is None:
         workspace = torch.empty(max(workspace_bytes(shape, block), 256), dtype=torch.uint8, device=Q.device)
+    _check_score_buffers(Q, K, cos, sin, apply_rope, Q_rot, K_rot, probs, workspace, nb)
     rope = Rope(cos.data_ptr() if apply_rope else None, sin.data_ptr() if apply_rope else None,
                 1 if apply_rope else 0)
     _check(lib.sfa_block_scores(ctypes.byref(shape), _ptr(Q), _ptr(K), ctypes.byref(rope), band_split, block,
@@ -225,6 +255,11 @@ def block_scores_select(Q, K, cos, sin, *, band_split: int, block: int, k: int |
         idx = torch.empty((shape.batch, shape.heads_q, nb, max(kmax, 1)), dtype=torch.int32, device=Q.device)
     if workspace is None:
         workspace = torch.empty(max(workspace_bytes(shape, block), 256), dtype=torch.uint8, device=Q.device)
+    _check_score_buffers(Q, K, cos, sin, apply_rope, Q_rot, K_rot, probs, workspace, nb)
+    _expect(counts, "counts", (shape.batch, shape.heads_q, nb), torch.int32, Q.device)
+    _expect(idx, "idx", (shape.batch, shape.heads_q, nb, idx.shape[-1]), torch.int32, Q.device)
+    if idx.shape[-1] < kmax:
+        raise ValueError(f"idx rows hold {idx.shape[-1]} entries, kmax = {kmax}")
     rope = Rope(cos.data_ptr() if apply_rope else None, sin.data_ptr() if apply_rope else None,
                 1 if apply_rope else 0)
     _check(lib.sfa_block_scores_select(ctypes.byref(shape), _ptr(Q), _ptr(K), ctypes.byref(rope), band_split,
@@ -256,10 +291,26 @@ def select(probs, shape: Shape, *, block: int, k: int | None = None, mass: float
         counts = torch.empty((shape.batch, shape.heads_q, nb), dtype=torch.int32, device=probs.device)
     if idx is None:
         idx = torch.empty((shape.batch, shape.heads_q, nb, kmax), dtype=torch.int32, device=probs.device)
+    _expect(probs, "probs", (shape.batch, shape.heads_q, nb, nb), torch.float32)
+    _expect(counts, "counts", (shape.batch, shape.heads_q, nb), torch.int32, probs.device)
+    _expect(idx, "idx", (shape.batch, shape.heads_q, nb, kmax), torch.int32, probs.device)
     _check(lib.sfa_select(ctypes.byref(shape), block, _ptr(probs), -1 if k is None else int(k),
                           0.0 if mass is None else float(mass), flags, _ptr(counts), _ptr(idx), kmax,
                           _stream(stream)), "sfa_select")
     return counts, idx
+
+
+def _check_attn_buffers(Q, K, V, counts, idx, O, lse, status, block):
+    dev = Q.device
+    B, Hq, L, _ = Q.shape
+    nb = L // block if block > 0 else 0
+    _expect(V, "V", K.shape, K.dtype, dev)
+    _expect(counts, "counts", (B, Hq, nb), torch.int32, dev)
+    _expect(idx, "idx", (B, Hq, nb, idx.shape[-1]), torch.int32, dev)
+    _expect(O, "O", Q.shape, Q.dtype, dev)
+    _expect(lse, "lse", (B, Hq, L), torch.float32, dev)
+    if status is not None and (status.dtype != torch.int32 or status.numel() < 1):
+        raise ValueError("status must be an int32 tensor with at least one element")
 
 
 def block_sparse_attn(Q, K, V, counts, idx, *, block: int, causal: bool = True, scale: float = 0.0,
@@ -272,6 +323,7 @@ def block_sparse_attn(Q, K, V, counts, idx, *, block: int, causal: bool = True, 
     if V.shape != K.shape or V.dtype != K.dtype:
         raise ValueError("V must match K")
     O = torch.empty_like(Q) if O is None else O
+    _check_attn_buffers(Q, K, V, counts, idx, O, lse, status, block)
     _check(lib.sfa_block_sparse_attn(ctypes.byref(shape), block, _ptr(Q), _ptr(K), _ptr(V), _ptr(counts),
                                      _ptr(idx), idx.shape[-1], 1 if causal else 0, float(scale), _ptr(O),
                                      _ptr(lse), _ptr(status), _stream(stream)), "sfa_block_sparse_attn")
@@ -289,6 +341,9 @@ def block_sparse_attn_rope(Q, cos, sin, K_rot, V, counts, idx, *, block: int, ca
     if V.shape != K_rot.shape or V.dtype != K_rot.dtype:
         raise ValueError("V must match K_rot")
     O = torch.empty_like(Q) if O is None else O
+    _expect(cos, "cos", (Q.shape[2], Q.shape[-1] // 2), torch.float32, Q.device)
+    _expect(sin, "sin", (Q.shape[2], Q.shape[-1] // 2), torch.float32, Q.device)
+    _check_attn_buffers(Q, K_rot, V, counts, idx, O, lse, status, block)
     rope = Rope(cos.data_ptr(), sin.data_ptr(), 1)
     _check(lib.sfa_block_sparse_attn_rope(ctypes.byref(shape), block, _ptr(Q), ctypes.byref(rope), _ptr(K_rot),
                                           _ptr(V), _ptr(counts), _ptr(idx), idx.shape[-1], 1 if causal else 0,
@@ -404,6 +459,7 @@ def decode_fc_gather(K_cache, fc, *, K_fc=None, pos0: int = 0, npos: int | None 
     shape = Shape(B, Hkv, Hkv, L, d, _dtype_code(K_cache))
     if K_fc is None:
         K_fc = torch.empty((B, Hkv, L, 2 * nfc), dtype=K_cache.dtype, device=K_cache.device)
+    _expect(K_fc, "K_fc", (B, Hkv, L, 2 * nfc), K_cache.dtype, K_cache.device)
     npos = L - pos0 if npos is None else npos
     _check(lib.sfa_decode_fc_gather(ctypes.byref(shape), _ptr(K_cache), fch, nfc, pos0, npos, _ptr(K_fc),
                                     _stream(stream)), "sfa_decode_fc_gather")
@@ -422,6 +478,8 @@ def decode_select(q, K_fc, fc, L: int, *, k: int, idx=None, workspace=None, stat
     if workspace is None:
         workspace = torch.empty(max(lib.sfa_decode_workspace(ctypes.byref(shape), k), 256), dtype=torch.uint8,
                                 device=q.device)
+    _expect(K_fc, "K_fc", (B, K_fc.shape[1], L, 2 * nfc), q.dtype, q.device)
+    _expect(idx, "idx", (B, Hq, k), torch.int32, q.device)
     _check(lib.sfa_decode_select(ctypes.byref(shape), _ptr(q), _ptr(K_fc), fch, nfc, k, _ptr(idx),
                                  _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
            "sfa_decode_select")
@@ -435,6 +493,13 @@ def decode_attn(q, K_cache, V_cache, idx, *, scale: float = 0.0, o=None, lse=Non
         _cuda(t, n)
     shape = decode_shape(q, K_cache)
     o = torch.empty_like(q) if o is None else o
+    B, Hq, d = q.shape
+    if K_cache.dim() != 4 or K_cache.shape[0] != B or K_cache.shape[3] != d:
+        raise ValueError("K_cache must be [B, Hkv, L, d] matching q [B, Hq, d]")
+    _expect(V_cache, "V_cache", K_cache.shape, K_cache.dtype, q.device)
+    _expect(idx, "idx", (B, Hq, idx.shape[-1]), torch.int32, q.device)
+    _expect(o, "o", q.shape, q.dtype, q.device)
+    _expect(lse, "lse", (B, Hq), torch.float32, q.device)
     _check(lib.sfa_decode_attn(ctypes.byref(shape), _ptr(q), _ptr(K_cache), _ptr(V_cache), _ptr(idx),
                                idx.shape[-1], float(scale), _ptr(o), _ptr(lse), _ptr(status), _stream(stream)),
            "sfa_decode_attn")

@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from block_sparse_long_dual_b200 import build as sfa_build
 from block_sparse_long_dual_b200 import sfa
@@ -219,3 +220,15 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(sfa, "_lib", None)
     with pytest.raises(ImportError):
         sfa.load()
+
+
+def test_binding_checks_buffer_shapes_before_any_call():
+    """The binding rejects a buffer of the wrong shape or dtype before the library sees its pointer."""
+    t = torch.zeros((1, 2, 256, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="shape"):
+        sfa._expect(torch.zeros((1, 2, 128, 64), dtype=torch.bfloat16), "Q_rot", t.shape, t.dtype)
+    with pytest.raises(ValueError, match="float32"):
+        sfa._expect(torch.zeros((4, 4), dtype=torch.float64), "probs", (4, 4), torch.float32)
+    with pytest.raises(ValueError, match="CUDA"):
+        sfa._expect(torch.zeros((4, 4), dtype=torch.float32), "probs", (4, 4), torch.float32)
+    sfa._expect(None, "lse", (1,), torch.float32)  # optional buffers may be absent
