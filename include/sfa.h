@@ -7,7 +7,10 @@
  *      per block, split into a high- and a low-frequency band and calibrated
  *      by an energy (RMS) temperature, followed by a block-level score matrix
  *      and a per-query-block selection (§1, §2, §3.1, §3.2, §5);
- *   2. exact softmax attention over the kept key blocks only (§1).
+ *   2. exact softmax attention over the kept key blocks only (§1);
+ * and the decode-side analogue of "FASA: Frequency-aware Sparse Attention"
+ * (§2B): token importance of a KV cache from dominant rotary pairs, the top-k
+ * tokens, and exact attention of one query token over them (sfa_decode_*).
  *
  * Conventions shared by every entry point:
  *   - Tensors are contiguous, row-major, layout [B, H, L, d] (batch, head,
@@ -23,8 +26,9 @@
  *     (bounded waits that ran out, bad index lists) are written into the
  *     optional `status_word` (a device int, first error wins; 0 = ok) and the
  *     kernel returns without hanging.  No C++ exception crosses this ABI.
- *   - Sizes: L % block == 0; block in {64, 128}; d in {64, 128};
- *     heads_q % heads_kv == 0; nb = L / block <= 2048.
+ *   - Sizes (prefill calls): L % block == 0; block in {64, 128}; d in {64, 128};
+ *     heads_q % heads_kv == 0; nb = L / block <= 2048.  The decode calls state
+ *     their own rules below.
  */
 #ifndef SFA_H_
 #define SFA_H_
