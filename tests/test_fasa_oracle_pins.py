@@ -183,3 +183,20 @@ def test_ranked_float32_score_is_within_the_recursive_summation_bound():
     qi = np.round(q * 4) / 4
     Ki = np.round(K * 4) / 4
     np.testing.assert_array_equal(fo.tip_keys(qi, Ki, fc).astype(np.float64), fo.tip_scores(qi, Ki, fc))
+
+
+def test_ranked_score_is_the_left_to_right_float32_sum():
+    """Products 2^24, 1, -2^24 in column order: float32 left to right gives 2^24 + 1 -> 2^24 (ties to
+    even), then 0; the exact sum is 1.  Pins the order and the precision of the ranked value."""
+    d = 16
+    fc = np.array([[0, 1, 2, 3]])          # columns: dims 0, 1, 2, 3, then 8, 9, 10, 11
+    q = np.zeros((1, 1, d))
+    K = np.zeros((1, 1, 1, d))
+    q[0, 0, [0, 1, 2]] = 1.0
+    K[0, 0, 0, [0, 1, 2]] = [2.0 ** 24, 1.0, -(2.0 ** 24)]
+    assert fo.tip_scores(q, K, fc)[0, 0, 0] == 1.0
+    assert fo.tip_keys(q, K, fc)[0, 0, 0] == 0.0
+    K[0, 0, 0, [0, 1, 2]] = [1.0, 2.0 ** 24, -(2.0 ** 24)]   # 1 + 2^24 -> 2^24 as well
+    assert fo.tip_keys(q, K, fc)[0, 0, 0] == 0.0
+    K[0, 0, 0, [0, 1, 2]] = [2.0 ** 24, -(2.0 ** 24), 1.0]   # cancellation first: exact
+    assert fo.tip_keys(q, K, fc)[0, 0, 0] == 1.0

@@ -529,3 +529,25 @@ def test_band_max_single_band_is_default():
         a = po.prism_scores(Q, K, beta, bs, flags | po.FLAG_BAND_MAX, (cos, sin))
         b = po.prism_scores(Q, K, beta, bs, flags, (cos, sin))
         np.testing.assert_array_equal(a.probs, b.probs)
+
+
+def test_block_tau_logit_closed_form_with_different_q_and_k_amplitudes():
+    """Constant Q in rotary pair 0 only; constant K in pairs 0 and 8 (one band).  Every block of Q
+    keeps rho_Q = D_0 and every block of K rho_K = sqrt((D_0^2 b^2 + D_8^2 c^2) / (b^2 + c^2))
+    (golden Dirichlet factors, beta = 64, base 1e4, d = 64), and only pair 0 meets in the dot
+    product, so s_ij = D_0 a b cos(64 (i - j)) / (rho_K sqrt(d))."""
+    rows = {(r[2], r[3]): r for r in _golden_rows() if r[0] == 1e4 and r[1] == 64}
+    D0, D8 = rows[(0, 64)][5], rows[(8, 64)][5]
+    beta, d, L, a, b, c = 64, 64, 64 * 6, 1.3, 0.7, 2.1
+    cos, sin = po.rope_tables(1e4, L, d)
+    Q = np.zeros((1, 1, L, d))
+    K = np.zeros((1, 1, L, d))
+    Q[..., 0] = a
+    K[..., 0] = b
+    K[..., 8] = c
+    sc = po.prism_scores(Q, K, beta, 0, po.FLAG_BLOCK_TAU | po.FLAG_SINGLE_BAND, (cos, sin))
+    rho_k = math.sqrt((D0 ** 2 * b ** 2 + D8 ** 2 * c ** 2) / (b ** 2 + c ** 2))
+    nb = L // beta
+    i, j = np.meshgrid(np.arange(nb), np.arange(nb), indexing="ij")
+    want = D0 * a * b * np.cos(64.0 * (i - j)) / (rho_k * math.sqrt(d))
+    np.testing.assert_allclose(sc.logits[0, 0], want, rtol=0, atol=2e-5)
