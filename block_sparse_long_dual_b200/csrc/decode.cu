@@ -777,8 +777,9 @@ DecodeGeometry decode_geometry(int group, int nfc) {
   const int W = 2 * nfc;
   d.tps = W <= 32 ? 2 : 1;
   const size_t slab = (size_t)kThreads * d.tps * W * 2;
-  // Two CTAs per SM when the keys and a two-stage ring fit in half the shared memory.
-  size_t budget = 110 * 1024;
+  // Two CTAs per SM when the keys and a two-stage ring fit in half the shared memory (228 KB per
+  // SM, 1 KB reserved per CTA, under 1 KB of static shared memory per CTA).
+  size_t budget = 113 * 1024;
   if ((size_t)group * 4096 * 4 + 2 * slab > budget) budget = 200 * 1024;
   d.chunk = 4096;
   while (d.chunk > 1024 && (size_t)group * d.chunk * 4 + 2 * slab > budget) d.chunk /= 2;
@@ -806,6 +807,8 @@ static cudaError_t launch_tip_chunk_t(const DecodeParams& p, cudaStream_t st) {
   const DecodeGeometry d = decode_geometry(G, p.nfc);
   auto kern = tip_chunk_kernel<G, TPS, NGR>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)d.smem);
+  if (e != cudaSuccess) return e;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
   if (e != cudaSuccess) return e;
   int dev = 0, sms = 148;
   cudaGetDevice(&dev);
