@@ -200,6 +200,18 @@ def oracle_head_sample(w: wl.Workload, Q, K, V, h: int = 0, attn_blocks: int | N
     return flops / secs / 1e12, secs, text
 
 
+def cpu_model() -> str:
+    """The host CPU's model name (from /proc/cpuinfo), for the oracle timings."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
 def blas_threads():
     try:
         from threadpoolctl import threadpool_info
@@ -258,7 +270,7 @@ def run_decode(args, w: wl.DecodeWorkload, rank, world):
                 "data": "synthetic", "impl": "reference",
                 "config": {"workload": w.name},
                 "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": blas_threads() or
-                                 len(os.sched_getaffinity(0)), "kind": "oracle", "sample": text},
+                                 len(os.sched_getaffinity(0)), "kind": "oracle", "sample": text, "cpu_model": cpu_model()},
                 "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
         return
@@ -364,7 +376,7 @@ def run_decode(args, w: wl.DecodeWorkload, rank, world):
             v, secs, text = oracle_decode_sample(w, q, K, V, fc)
             line["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": blas_threads() or
                                     len(os.sched_getaffinity(0)), "kind": "oracle", "sample": text,
-                                    "seconds": secs}
+                                    "seconds": secs, "cpu_model": cpu_model()}
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
@@ -393,7 +405,7 @@ def run_reference(args, w, rank, world):
             "config": {"workload": w.name, "layer": f"B={w.batch} Hq={w.heads_q} Hkv={w.heads_kv} "
                        f"L={w.seq_len} d={w.head_dim} block={w.block}"},
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads() or cores,
-                             "kind": "oracle", "sample": text},
+                             "kind": "oracle", "sample": text, "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -530,7 +542,7 @@ def main():
             v, secs, text = oracle_head_sample(w, Q, K, V, h=0)
             line["cpu_baseline"] = {"value": v, "unit": "TFLOP/s",
                                     "cores": blas_threads() or len(os.sched_getaffinity(0)),
-                                    "kind": "oracle", "sample": text, "seconds": secs}
+                                    "kind": "oracle", "sample": text, "seconds": secs, "cpu_model": cpu_model()}
         print(json.dumps(line), flush=True)
     if dist:
         dist.barrier()
