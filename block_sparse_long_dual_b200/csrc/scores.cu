@@ -5,10 +5,14 @@
 // Three kernels, launched in order on one stream:
 //   rope_pool_energy  HBM stream over Q and K: RoPE, rotated copy, per-block
 //                     mean vectors and per-band energies (one CTA per block
-//                     and head, the block staged by bulk asynchronous copies).
+//                     and group of heads, each head's block staged by bulk
+//                     asynchronous copies).
 //   band_temperature  per (batch, Q head): reduce the energies to tau^H, tau^L.
 //   block_score_softmax  calibrated block logits (float64 tensor-core MMAs)
-//                     and the causal row softmax, both in float64.
+//                     and the causal row softmax, both in float64; in the
+//                     FUSED instantiation each row's selection follows in the
+//                     same warp (select_row.cuh), so the probabilities need
+//                     not reach device memory.
 #include <math.h>
 
 #include "common.cuh"
