@@ -455,6 +455,10 @@ sfa_status sfa_decode_attn(const sfa_shape* shape, const void* q, const void* K_
 
 }  // extern "C"
 
+namespace sfa {
+cudaError_t launch_bounded_wait_selftest(int* status, uint64_t limit_ns, int arrive, cudaStream_t st);  // selftest.cu
+}  // namespace sfa
+
 extern "C" {
 
 sfa_status sfa_selftest_bounded_wait(int* status_word, unsigned limit_ms, int complete, void* stream) {

@@ -107,7 +107,6 @@ int decode_max_chunks();
 cudaError_t launch_fc_gather(const DecodeParams& p, const void* Kc, void* Kfc, int pos0, int npos, cudaStream_t st);
 cudaError_t launch_decode_select(const DecodeParams& p, cudaStream_t st);
 cudaError_t launch_decode_attn(const DecodeParams& p, cudaStream_t st);
-cudaError_t launch_bounded_wait_selftest(int* status, uint64_t limit_ns, int arrive, cudaStream_t st);
 cudaError_t launch_attn_tcgen05(const AttnParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
                                 const CUtensorMap& tmV, cudaStream_t st);
 
