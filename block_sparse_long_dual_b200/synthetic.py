@@ -22,7 +22,10 @@ vector's rotation is again random).  Dominant pairs ``fc`` [Hkv, nfc]: nfc
 distinct pairs per KV head drawn with seed 5 (a stand-in for the offline
 calibration the page describes).  Needles: round(needle_frac * L) tokens per
 (b, KV head), drawn with seed 6, get 2 x the group's mean query added on that
-head's dominant dims, so the estimate has real winners to find.
+head's dominant dims, so the estimate has real winners to find.  With
+``dominant_gain`` != 1 the dominant dims of q and K are scaled by it (a cache
+whose attention scores are carried mostly by a few frequency pairs, the
+premise of the page's §2A); the bench inputs use 1.
 """
 
 from __future__ import annotations
@@ -100,14 +103,20 @@ def make_decode_inputs(w: DecodeWorkload, seed: int = 0, device: str | torch.dev
     g = torch.Generator().manual_seed(seed)
     fc = decode_fc(w)
     q = torch.randn((w.batch, w.heads_q, w.head_dim), generator=g)
+    half = w.head_dim // 2
+    if w.dominant_gain != 1.0:
+        for h in range(w.heads_q):
+            dims = torch.cat([torch.as_tensor(fc[h // w.group]), torch.as_tensor(fc[h // w.group]) + half])
+            q[:, h, dims] *= w.dominant_gain
     K = torch.empty((w.batch, w.heads_kv, w.seq_len, w.head_dim), dtype=torch.bfloat16, device=device)
     V = torch.empty_like(K)
     gn = torch.Generator().manual_seed(6)
     nneedle = int(round(w.needle_frac * w.seq_len))
-    half = w.head_dim // 2
     for b in range(w.batch):
         for h in range(w.heads_kv):
             x = torch.randn((w.seq_len, w.head_dim), generator=g)
+            if w.dominant_gain != 1.0:
+                x[:, torch.cat([torch.as_tensor(fc[h]), torch.as_tensor(fc[h]) + half])] *= w.dominant_gain
             if nneedle:
                 dims = torch.cat([torch.as_tensor(fc[h]), torch.as_tensor(fc[h]) + half])
                 qm = q[b, h * w.group:(h + 1) * w.group].mean(0)

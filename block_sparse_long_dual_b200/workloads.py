@@ -123,6 +123,7 @@ class DecodeWorkload:
     nfc: int          # dominant rotary pairs per KV head
     k: int            # token budget
     needle_frac: float = 0.01   # fraction of cache tokens aligned with the query on the dominant pairs
+    dominant_gain: float = 1.0  # amplitude of q and K on the dominant pairs' dims (1: plain N(0, 1))
 
     @property
     def group(self) -> int:
