@@ -269,10 +269,12 @@ sfa_status sfa_block_sparse_attn_rope(const sfa_shape* shape, int block, const v
  * ---------------------------------------------------------------------------
  * Decode step ("FASA: Frequency-aware Sparse Attention" §2B): one query token
  * per (batch, Q head) against a KV cache.  shape->seq_len is the cache length
- * L; shape->dtype must be SFA_BF16 (SFA_ERR_DTYPE otherwise); heads_q /
- * heads_kv in {1, 2, 4, 8} and L <= 2^21 (SFA_ERR_UNSUPPORTED otherwise).  q [B, heads_q, d] is the newest token's query, already
- * rotated at its position; K_cache, V_cache [B, heads_kv, L, d] hold the
- * rotated keys and the values at their original positions.
+ * L; shape->dtype must be SFA_BF16 (SFA_ERR_DTYPE otherwise).  heads_q /
+ * heads_kv in {1, 2, 4, 8}, and L at most 512 chunks of the selection kernel
+ * (4096 tokens each, fewer for long pair lists: L <= 2^21 when 2 nfc <= 32),
+ * else SFA_ERR_UNSUPPORTED.  q [B, heads_q, d] is the newest token's query,
+ * already rotated at its position; K_cache, V_cache [B, heads_kv, L, d] hold
+ * the rotated keys and the values at their original positions.
  *
  * fc: HOST array [heads_kv][nfc] of each KV head's dominant rotary pairs
  * (pair m = dims m and m + d/2; found by an offline calibration that this
@@ -298,8 +300,9 @@ size_t sfa_decode_workspace(const sfa_shape* shape, int k);
 /*
  * Token Importance Predictor (§2B.1): for Q head h of KV group g,
  *   s_t = sum_{m in fc[g]} q_m k_{t,m} + q_{m+d/2} k_{t,m+d/2}
- * from K_fc, summed in float64 and rounded once to float32; then the first
- * min(k, L) tokens by (s desc, index asc).  idx [B, heads_q, k] int32: the kept
+ * from K_fc, as a float32 sum over the compact columns in order (column 0
+ * first, one rounding per step; each bf16 x bf16 product is exact), then the
+ * first min(k, L) tokens by (s desc, index asc).  idx [B, heads_q, k] int32: the kept
  * token indices ascending, padded with -1.  k >= 1.  workspace: device, at
  * least sfa_decode_workspace() bytes, 256-byte aligned (SFA_ERR_WORKSPACE).
  * status_word (device, nullable): SFA_ERR_TIMEOUT if a copy of the compact
