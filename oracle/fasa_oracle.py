@@ -3,7 +3,8 @@
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
 module.  It shares no code with the CUDA library and computes in float64 from
-the same seeded host arrays the GPU receives.
+the same seeded host arrays the GPU receives, except the ranked token score,
+which reading D2 below defines as a float32 sum.
 
 What it restates (source: "FASA: Frequency-aware Sparse Attention", §2):
 

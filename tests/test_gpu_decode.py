@@ -2,7 +2,7 @@
 against the CPU oracle ("FASA: Frequency-aware Sparse Attention" §2B), through the C ABI.
 
 The compact key copy and the index lists are compared bit for bit (both sides rank the same
-float32 rounding of an exact float64 score); outputs within the bf16 tolerance."""
+float32 column-order sum of exact bf16 products); outputs within the bf16 tolerance."""
 
 import numpy as np
 import pytest
