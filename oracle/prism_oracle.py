@@ -73,8 +73,14 @@ attention.  R4c: per-block rho equal to the golden Dirichlet factor for a
 constant pair, the 1e-3 floor on a full turn per block, restoration of each
 block's token RMS, block size 1 giving token softmax.  R5b: mirrored bands
 giving the half-logit softmax, a one-hot branch against a uniform branch in
-closed form, and a single band reducing to R5/R6.  Parity of the *selection rule itself* with the pages' own
-selections is unpinned: the pages print no worked example.
+closed form, and a single band reducing to R5/R6.  Also: the RoPE tables as
+float32 roundings of the exact angles, per-block band energies of a rotated
+constant vector, tau = 1 for a band with no energy, the array form of a
+selection, and the attention reading the rounded Q_r / K_r.  Every pin's power
+is itself checked: tests/test_oracle_mutations.py plants mistakes in a copy of
+this module and requires a pin to fail for each.  Parity of the *selection
+rule itself* with the pages' own selections is unpinned: the pages print no
+worked example.
 """
 
 from __future__ import annotations

@@ -253,7 +253,9 @@ def test_selection_matches_bruteforce(seed, flags):
     # dyadic values with many exact ties: sums are exact in float64
     P = rng.integers(0, 6, size=(nb, nb)).astype(np.float64) / 64.0
     for i in range(nb):
-        forced = po.forced_blocks(i, flags)
+        # reading R7: the diagonal is always kept, and block 0 too with KEEP_SINK
+        forced = (0, i) if (flags & po.FLAG_KEEP_SINK) and i > 0 else (i,)
+        assert set(po.forced_blocks(i, flags)) == set(forced)
         cand = [j for j in range(i + 1) if j not in forced]
         for k in range(0, nb + 1):
             r = po.select_row(P[i], i, flags, k=k)
@@ -285,12 +287,13 @@ def test_selection_invariants_on_softmax_rows():
         sel0 = po.select_blocks(p, flags, k=0)
         all1 = po.select_blocks(p, flags, mass=1.0)
         for i in range(nb):
-            assert set(sel0[0][0][i].kept.tolist()) == set(po.forced_blocks(i, flags))
+            forced = {0, i} if flags & po.FLAG_KEEP_SINK else {i}
+            assert set(sel0[0][0][i].kept.tolist()) == forced
             assert list(all1[0][0][i].kept) == list(range(i + 1))
             for kk in (1, 3, 50):
                 r = po.select_row(p[0, 0, i], i, flags, k=kk)
                 assert i in r.kept
-                assert len(r.kept) == min(i + 1, kk + len(po.forced_blocks(i, flags)))
+                assert len(r.kept) == min(i + 1, kk + len(forced))
 
 
 # ---------------------------------------------------------------------------
@@ -373,6 +376,90 @@ def test_tiny_path_structure():
         assert i in kept and (i == 0 or 0 in kept)
         assert len(kept) == min(i + 1, w.k + (2 if i else 1))
     assert np.all(np.isfinite(r.out))
+
+
+def test_f32_rounding_matches_torch():
+    rng = np.random.default_rng(13)
+    x = rng.normal(size=20000) * np.exp(rng.normal(size=20000) * 4)
+    ref = torch.from_numpy(x).to(torch.float32).to(torch.float64).numpy()
+    np.testing.assert_array_equal(po.round_to_dtype(x, "f32"), ref)
+
+
+def test_rope_tables_are_float32_roundings_of_the_exact_angles():
+    """R1: the tables hold cos/sin of the float64 angle, each rounded once to float32 (checked
+    against the standard library's cos/sin at a sample of entries, to half a float32 ulp)."""
+    base, L, d = 5e5, 4096, 128
+    cos, sin = po.rope_tables(base, L, d)
+    assert cos.dtype == np.float32 and sin.dtype == np.float32 and cos.shape == (L, d // 2)
+    rng = np.random.default_rng(14)
+    for p, m in zip(rng.integers(0, L, 200), rng.integers(0, d // 2, 200)):
+        ang = float(p) * base ** (-2.0 * float(m) / d)
+        for table, exact in ((cos, math.cos(ang)), (sin, math.sin(ang))):
+            v = float(table[p, m])
+            assert abs(v - exact) <= 0.5 * float(np.spacing(np.float32(abs(v)))) * (1 + 1e-9)
+
+
+def test_selection_arrays_layout():
+    """The array form of a selection: counts = number kept, idx = the kept ids ascending, then -1."""
+    rng = np.random.default_rng(15)
+    nb = 7
+    p = po.causal_block_softmax(rng.normal(size=(1, 2, nb, nb)))
+    for flags in (0, po.FLAG_KEEP_SINK):
+        sel = po.select_blocks(p, flags, k=2)
+        counts, idx = po.selection_to_arrays(sel, kmax=5)
+        for h in range(2):
+            for i in range(nb):
+                kept = sorted(set(sel[0][h][i].kept.tolist()))
+                assert counts[0, h, i] == len(kept)
+                assert idx[0, h, i].tolist() == kept + [-1] * (5 - len(kept))
+
+
+def test_zero_energy_band_has_unit_temperature():
+    """R4: a band with no energy anywhere retains nothing to restore, so its tau is exactly 1
+    (and its logits are 0, so the other band alone decides)."""
+    rng = np.random.default_rng(16)
+    d, bs, L, beta = 16, 3, 64, 8
+    Q = rng.normal(size=(1, 2, L, d))
+    K = rng.normal(size=(1, 1, L, d))
+    hmask = np.zeros(d, dtype=bool)
+    hmask[:bs] = True
+    hmask[d // 2:d // 2 + bs] = True
+    Q[..., hmask] = 0.0
+    K[..., hmask] = 0.0
+    sc = po.prism_scores(Q, K, beta, bs, 0, rope=po.rope_tables(1e4, L, d))
+    assert np.all(sc.tau[..., 0] == 1.0)
+    assert np.all(sc.tau[..., 1] < 1.0)
+
+
+def test_block_token_energy_closed_form():
+    """R3/R4 energies: a constant vector under RoPE keeps each pair's norm, so every block holds
+    beta times the vector's squared norm in each band."""
+    d, bs, L, beta = 16, 3, 64, 8
+    rng = np.random.default_rng(17)
+    x = rng.normal(size=d)
+    X = np.broadcast_to(x, (1, 1, L, d)).copy()
+    xr = po.apply_rope(X, *po.rope_tables(1e4, L, d))
+    e = po.block_token_energy(xr, beta, bs, 0)
+    h = np.r_[x[:bs], x[d // 2:d // 2 + bs]]
+    lo = np.r_[x[bs:d // 2], x[d // 2 + bs:]]
+    # the float32 tables give c^2 + s^2 = 1 only to about 2^-23
+    np.testing.assert_allclose(e[0, 0, :, 0], beta * np.sum(h ** 2), rtol=1e-7)
+    np.testing.assert_allclose(e[0, 0, :, 1], beta * np.sum(lo ** 2), rtol=1e-7)
+
+
+def test_path_attention_reads_the_rounded_rotated_values():
+    """R1/R8: the attention step reads Q_r, K_r rounded to the input dtype, as the GPU stores them."""
+    from block_sparse_long_dual_b200.workloads import TINY
+    from block_sparse_long_dual_b200.synthetic import make_inputs
+    w = TINY.scaled(seq_len=256)
+    Q, K, V = (t.numpy() for t in make_inputs(w))
+    rope = po.rope_tables(w.rope_base, w.seq_len, w.head_dim)
+    for dtype, tdt in (("bf16", torch.bfloat16), ("f32", torch.float32)):
+        r = po.prism_path(Q, K, V, block=w.block, band_split=w.band_split, flags=w.flags, k=w.k,
+                          rope=rope, dtype=dtype)
+        for got, exact in ((r.q_attn, r.scores.q_rot), (r.k_attn, r.scores.k_rot)):
+            ref = torch.from_numpy(exact).to(tdt).to(torch.float64).numpy()
+            np.testing.assert_array_equal(got, ref)
 
 
 # ---------------------------------------------------------------------------

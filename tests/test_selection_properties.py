@@ -31,7 +31,7 @@ def test_prism_topk_selection(levels, k, sink):
     i = nb - 1
     flags = po.FLAG_KEEP_SINK if sink else 0
     r = po.select_row(p, i, flags, k=k)
-    forced = set(po.forced_blocks(i, flags))
+    forced = {0, i} if sink else {i}
     cand = [j for j in range(i + 1) if j not in forced]
     want = _brute(p, cand, min(k, len(cand))) | forced
     assert set(r.kept.tolist()) == want
