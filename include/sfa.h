@@ -27,8 +27,10 @@
  *     optional `status_word` (a device int, first error wins; 0 = ok) and the
  *     kernel returns without hanging.  No C++ exception crosses this ABI.
  *   - Sizes (prefill calls): L % block == 0; block in {64, 128}; d in {64, 128};
- *     heads_q % heads_kv == 0; nb = L / block <= 2048.  The decode calls state
- *     their own rules below.
+ *     heads_q % heads_kv == 0 (SFA_ERR_SHAPE otherwise); nb = L / block <= 2048
+ *     and batch * heads_q * L < 2^31, so that every row of the [B*H*L, d] views
+ *     has an int32 index (SFA_ERR_UNSUPPORTED otherwise).  The decode calls
+ *     state their own rules below.
  */
 #ifndef SFA_H_
 #define SFA_H_

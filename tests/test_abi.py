@@ -63,6 +63,7 @@ def S(B=1, Hq=4, Hkv=2, L=1024, d=128, dt=sfa.BF16):
     (S(Hq=6, Hkv=4), 128, 2),      # heads_q % heads_kv
     (S(dt=7), 128, 3),             # dtype
     (S(L=128 * 4096), 128, 4),     # nb > 2048
+    (S(B=256, Hq=32, Hkv=8, L=1 << 18), 128, 4),   # B * Hq * L = 2^31 rows: past int32
     (S(B=0), 128, 2),
 ])
 def test_shape_validation(lib, shape, block, code):
@@ -78,6 +79,13 @@ def test_shape_validation(lib, shape, block, code):
                                        None, None, None, dummy, dummy, 64, dummy, 1 << 30, None) == code
     assert lib.sfa_block_sparse_attn(ctypes.byref(shape), block, dummy, dummy, dummy, dummy, dummy, 8, 1, 0.0,
                                      dummy, None, None, None) == code
+
+
+def test_row_limit_is_exclusive_at_2_to_the_31(lib):
+    below = S(B=255, Hq=32, Hkv=8, L=1 << 18)          # 255 * 32 * 2^18 rows < 2^31
+    nb = (1 << 18) // 128
+    want = 255 * 32 * nb * 128 * 8                        # Qbar alone, float64
+    assert lib.sfa_block_scores_workspace(ctypes.byref(below), 128) > want
 
 
 def test_workspace_layout_matches_documented_sizes(lib):
