@@ -200,7 +200,7 @@ __global__ void __launch_bounds__(256, 1) rope_pool_energy_kernel(RopePoolParams
 
 // ---------------------------------------------------------------------------
 // band_temperature: tau^b = max(rho^b(Q_h) * rho^b(K_g), 1e-6),
-// rho = sqrt(mean_j ||xbar_j^b||^2 / mean_t ||x_t^b||^2), 1 for an empty band;
+// rho = sqrt(mean_j ||xbar_j^b||^2 / mean_t ||x_t^b||^2), 1 for a band without energy;
 // with SFA_RELATIVE_CALIB tau^H / tau^L and 1.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) band_temperature_kernel(TauParams p) {

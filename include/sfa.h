@@ -127,7 +127,7 @@ sfa_status sfa_workspace_layout(const sfa_shape* shape, int block, size_t offset
  * Per (batch, Q head, band b in {H, L}), with band H = rotary pairs
  * m < band_split (dims m and m + d/2), band L = the other dims:
  *   xbar_j  = mean of the rotated vectors of block j
- *   rho^b   = sqrt(mean_j ||xbar_j^b||^2 / mean_t ||x_t^b||^2)   (1 if the band is empty)
+ *   rho^b   = sqrt(mean_j ||xbar_j^b||^2 / mean_t ||x_t^b||^2)   (1 if the band has no energy)
  *   tau^b   = max(rho^b(Q_h) * rho^b(K_g), 1e-6)   (1 with SFA_NO_CALIB)
  *   s_ij    = sum_b (qbar_i^b . kbar_j^b) / (tau^b * sqrt(d)),  j <= i
  *   probs_ij = exp(s_ij) / sum_{j' <= i} exp(s_ij'), and 0 for j > i.
