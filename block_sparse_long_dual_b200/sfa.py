@@ -107,8 +107,12 @@ def _ptr(t):
 
 
 def _stream(stream=None):
-    s = stream if stream is not None else torch.cuda.current_stream()
-    return ctypes.c_void_p(s.cuda_stream)
+    if stream is None:
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    cur = torch.cuda.current_device()
+    if stream.device.index != cur:
+        raise ValueError(f"stream belongs to {stream.device} but the current CUDA device is cuda:{cur}")
+    return ctypes.c_void_p(stream.cuda_stream)
 
 
 def _dtype_code(t: torch.Tensor) -> int:
@@ -120,10 +124,31 @@ def _dtype_code(t: torch.Tensor) -> int:
 
 
 def _cuda(t: torch.Tensor, name: str):
+    """A contiguous tensor on the current CUDA device: the library launches every kernel on the
+    calling thread's current device, so a buffer of another device would be read through a foreign
+    pointer."""
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+    cur = torch.cuda.current_device()
+    if t.device.index != cur:
+        raise ValueError(f"{name} is on {t.device} but the current CUDA device is cuda:{cur}")
+
+
+def _status(status):
+    """The optional device status word: an int32 CUDA tensor with at least one element."""
+    if status is None:
+        return
+    if status.dtype != torch.int32 or status.numel() < 1:
+        raise ValueError("status must be an int32 tensor with at least one element")
+    _cuda(status, "status")
+
+
+def _workspace(workspace):
+    if workspace.dtype != torch.uint8 or workspace.dim() != 1:
+        raise ValueError("workspace must be a 1-D uint8 tensor")
+    _cuda(workspace, "workspace")
 
 
 def _expect(t, name: str, shape, dtype, device=None):
@@ -195,9 +220,7 @@ def _check_score_buffers(Q, K, cos, sin, apply_rope, Q_rot, K_rot, probs, worksp
         _expect(Q_rot, "Q_rot", Q.shape, Q.dtype, dev)
         _expect(K_rot, "K_rot", K.shape, K.dtype, dev)
     _expect(probs, "probs", (Q.shape[0], Q.shape[1], nb, nb), torch.float32, dev)
-    if workspace.dtype != torch.uint8 or workspace.dim() != 1:
-        raise ValueError("workspace must be a 1-D uint8 tensor")
-    _cuda(workspace, "workspace")
+    _workspace(workspace)
 
 
 def block_scores(Q, K, cos, sin, *, band_split: int, block: int, flags: int = 0, apply_rope: bool = True,
@@ -309,8 +332,7 @@ def _check_attn_buffers(Q, K, V, counts, idx, O, lse, status, block):
     _expect(idx, "idx", (B, Hq, nb, idx.shape[-1]), torch.int32, dev)
     _expect(O, "O", Q.shape, Q.dtype, dev)
     _expect(lse, "lse", (B, Hq, L), torch.float32, dev)
-    if status is not None and (status.dtype != torch.int32 or status.numel() < 1):
-        raise ValueError("status must be an int32 tensor with at least one element")
+    _status(status)
 
 
 def block_sparse_attn(Q, K, V, counts, idx, *, block: int, causal: bool = True, scale: float = 0.0,
@@ -480,6 +502,8 @@ def decode_select(q, K_fc, fc, L: int, *, k: int, idx=None, workspace=None, stat
                                 device=q.device)
     _expect(K_fc, "K_fc", (B, K_fc.shape[1], L, 2 * nfc), q.dtype, q.device)
     _expect(idx, "idx", (B, Hq, k), torch.int32, q.device)
+    _workspace(workspace)
+    _status(status)
     _check(lib.sfa_decode_select(ctypes.byref(shape), _ptr(q), _ptr(K_fc), fch, nfc, k, _ptr(idx),
                                  _ptr(workspace), workspace.numel(), _ptr(status), _stream(stream)),
            "sfa_decode_select")
@@ -500,6 +524,7 @@ def decode_attn(q, K_cache, V_cache, idx, *, scale: float = 0.0, o=None, lse=Non
     _expect(idx, "idx", (B, Hq, idx.shape[-1]), torch.int32, q.device)
     _expect(o, "o", q.shape, q.dtype, q.device)
     _expect(lse, "lse", (B, Hq), torch.float32, q.device)
+    _status(status)
     _check(lib.sfa_decode_attn(ctypes.byref(shape), _ptr(q), _ptr(K_cache), _ptr(V_cache), _ptr(idx),
                                idx.shape[-1], float(scale), _ptr(o), _ptr(lse), _ptr(status), _stream(stream)),
            "sfa_decode_attn")
@@ -549,6 +574,7 @@ def selftest_bounded_wait(limit_ms: int, complete: bool, device="cuda", stream=N
     """sfa_selftest_bounded_wait: returns the device status word (0 or SFA_ERR_TIMEOUT)."""
     lib = load()
     status = torch.full((1,), -1, dtype=torch.int32, device=device)
+    _status(status)
     _check(lib.sfa_selftest_bounded_wait(_ptr(status), int(limit_ms), 1 if complete else 0, _stream(stream)),
            "sfa_selftest_bounded_wait")
     return int(status.item())

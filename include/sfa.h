@@ -16,10 +16,12 @@
  *   - Tensors are contiguous, row-major, layout [B, H, L, d] (batch, head,
  *     token, head dim).  Q has heads_q heads, K and V have heads_kv heads;
  *     Q head h reads KV head h / (heads_q / heads_kv) (grouped-query attention).
- *   - All tensor pointers are DEVICE pointers owned by the caller.  The
- *     library never allocates or frees device memory and never synchronises
- *     the stream; every launch goes on `stream` (a cudaStream_t passed as
- *     void*, NULL = legacy default stream).
+ *   - All tensor pointers are DEVICE pointers owned by the caller, into the
+ *     memory of the calling thread's current CUDA device: every kernel is
+ *     launched there.  The library never allocates or frees device memory and
+ *     never synchronises the stream; every launch goes on `stream` (a
+ *     cudaStream_t of that device passed as void*, NULL = legacy default
+ *     stream).
  *   - Arguments are validated on the host before anything is launched; a
  *     validation failure returns an error status and launches nothing.  A
  *     failed launch returns SFA_ERR_CUDA.  Faults detected on the device

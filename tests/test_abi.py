@@ -5,6 +5,7 @@ import ctypes
 import os
 import re
 
+import numpy as np
 import pytest
 import torch
 
@@ -240,3 +241,56 @@ def test_binding_checks_buffer_shapes_before_any_call():
     with pytest.raises(ValueError, match="CUDA"):
         sfa._expect(torch.zeros((4, 4), dtype=torch.float32), "probs", (4, 4), torch.float32)
     sfa._expect(None, "lse", (1,), torch.float32)  # optional buffers may be absent
+
+
+class _FakeCuda:
+    """Stands in for a CUDA tensor on a CPU-only host: only what the binding's checks read."""
+
+    def __init__(self, index, shape=(1,), dtype=torch.int32):
+        self.is_cuda = True
+        self.device = torch.device("cuda", index)
+        self.shape = torch.Size(shape)
+        self.dtype = dtype
+
+    def is_contiguous(self):
+        return True
+
+    def numel(self):
+        return int(np.prod(self.shape))
+
+    def dim(self):
+        return len(self.shape)
+
+
+def test_binding_rejects_buffers_of_another_device(lib, monkeypatch):
+    """Every kernel launches on the current device, so a buffer, status word or stream of another
+    device is refused before its pointer reaches the library."""
+    monkeypatch.setattr(torch.cuda, "current_device", lambda: 0)
+    sfa._cuda(_FakeCuda(0), "q")
+    with pytest.raises(ValueError, match="current CUDA device"):
+        sfa._cuda(_FakeCuda(1), "q")
+    with pytest.raises(ValueError, match="current CUDA device"):
+        sfa._expect(_FakeCuda(1, (4,), torch.float32), "lse", (4,), torch.float32)
+    sfa._status(None)
+    sfa._status(_FakeCuda(0))
+    with pytest.raises(ValueError, match="int32"):
+        sfa._status(_FakeCuda(0, dtype=torch.float32))
+    with pytest.raises(ValueError, match="current CUDA device"):
+        sfa._status(_FakeCuda(1))
+    sfa._workspace(_FakeCuda(0, (256,), torch.uint8))
+    with pytest.raises(ValueError, match="uint8"):
+        sfa._workspace(_FakeCuda(0, (64,), torch.int32))
+    with pytest.raises(ValueError, match="current CUDA device"):
+        sfa._workspace(_FakeCuda(1, (256,), torch.uint8))
+
+    class OtherStream:
+        device = torch.device("cuda", 1)
+        cuda_stream = 0
+
+    with pytest.raises(ValueError, match="current CUDA device"):
+        sfa._stream(OtherStream())
+    q = _FakeCuda(0, (1, 4, 128), torch.bfloat16)
+    cache = _FakeCuda(1, (1, 1, 64, 128), torch.bfloat16)
+    idx = _FakeCuda(0, (1, 4, 8), torch.int32)
+    with pytest.raises(ValueError, match="current CUDA device"):
+        sfa.decode_attn(q, cache, cache, idx)
