@@ -6,9 +6,9 @@ chunk's k-th largest key (any value with at least k of the chunk's 4-key group m
 it; the bisection may stop early, so any such value is allowed), keep the tokens with key >= LB in
 token order, and a merge picks the first k of the candidates by (key desc, index asc).  This model
 checks that the strategy never drops a token of the exact top k, for exact and deliberately loose
-bounds, including the distributions that send every token to the merge (identical keys).  The merge's own bound (the
-least of its threads' candidate maxima) is modelled too, with 256 threads as in the kernel and with 8
-so that it cuts deep."""
+bounds, including the distributions that send every token to the merge (identical keys).  The
+merge's own bound (the least of its threads' candidate maxima) is modelled too, with 256 threads as
+in the kernel and with 8 so that it cuts deep."""
 
 import numpy as np
 import pytest
