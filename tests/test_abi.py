@@ -192,7 +192,6 @@ def test_decode_validation(lib):
     ws = lib.sfa_decode_workspace(ctypes.byref(sh), 256)
     assert ws >= 2 * 8 * 2 * 256 * 8
     g = lib.sfa_decode_fc_gather
-    assert g(ctypes.byref(sh), d, fc, 4, 0, 5000, d, None) != 1                    # valid (no GPU: not 1)
     assert g(ctypes.byref(S(B=2, Hq=8, Hkv=2, L=5000, dt=sfa.F32)), d, fc, 4, 0, 5000, d, None) == 3
     assert g(ctypes.byref(S(B=1, Hq=18, Hkv=2, L=50)), d, fc, 4, 0, 50, d, None) == 4  # group 9
     assert g(ctypes.byref(sh), d, fc, 3, 0, 5000, d, None) == 1                    # nfc % 4
