@@ -37,15 +37,32 @@ def uncertain_candidates(sel: po.RowSelection, p_row: np.ndarray, mass: float | 
     return U
 
 
+def threshold_alone(sel: po.RowSelection, p_row: np.ndarray, mass: float | None, rel=NEAR_TIE_REL) -> bool:
+    """True when the only candidate the near-tie rule excuses is the threshold candidate itself (no
+    other candidate within the window and, in mass mode, no running sum near the target): the
+    literal rule still excuses that candidate, but no float32/float64 difference can move it."""
+    order, n = sel.order, sel.n_taken
+    if order.size == 0 or n == 0:
+        return False
+    t = p_row[order[n - 1]]
+    if sum(1 for c in order if abs(p_row[c] - t) <= rel * t) > 1:
+        return False
+    if mass is not None and (abs(sel.cum_before_last - mass) <= rel or abs(sel.cum_final - mass) <= rel):
+        return False
+    return True
+
+
 def compare_masks(sel, probs_oracle, counts, idx, mass=None):
     """Row-by-row comparison of the GPU's kept sets with the oracle's.
 
     Returns (stats, exact) where exact[b][h][i] is True when the GPU row equals
-    the oracle row exactly (those rows are the ones whose outputs are compared)."""
+    the oracle row exactly (those rows are the ones whose outputs are compared).
+    stats["threshold_only_rows"] counts rows excused only because the rule, read
+    literally, excuses the threshold candidate itself (see threshold_alone)."""
     counts = counts.cpu().numpy()
     idx = idx.cpu().numpy()
     B, H, nb = counts.shape
-    stats = dict(rows=0, uncertain_rows=0, mismatches=0, bad_rows=[])
+    stats = dict(rows=0, uncertain_rows=0, mismatches=0, bad_rows=[], threshold_only_rows=0)
     exact = np.zeros((B, H, nb), dtype=bool)
     for b in range(B):
         for h in range(H):
@@ -66,6 +83,8 @@ def compare_masks(sel, probs_oracle, counts, idx, mass=None):
                 if (gs - U) != (os_ - U):
                     stats["mismatches"] += 1
                     stats["bad_rows"].append((b, h, i, sorted(gs ^ os_)))
+                elif threshold_alone(r, probs_oracle[b, h, i], mass):
+                    stats["threshold_only_rows"] += 1
     return stats, exact
 
 

@@ -65,6 +65,8 @@ def test_full_size_sampled(w):
         sel = po.select_blocks(sc.probs, w.flags, k=w.k, mass=mass)
         stats, exact = compare_masks(sel, sc.probs, model.counts[b:b + 1, h:h + 1], model.idx[b:b + 1, h:h + 1],
                                      mass)
+        print(f"{w.name} b={b} h={h}: near-tie rows {stats['uncertain_rows']}, "
+              f"threshold-only excusals {stats['threshold_only_rows']}")
         assert stats["mismatches"] == 0, stats["bad_rows"][:5]
         # outputs of a few query blocks whose masks agree exactly
         want = [i for i in (0, 1, nb // 2, nb - 1) if exact[0, 0, i]]

@@ -106,6 +106,8 @@ def test_path_matches_oracle(w):
 
     # a5: masks identical except near-ties at the row threshold
     stats, exact = compare_masks(ref.selection, sc.probs, model.counts, model.idx, mass)
+    print(f"{w.name}: rows {stats['rows']}, near-tie rows {stats['uncertain_rows']}, "
+          f"threshold-only excusals {stats['threshold_only_rows']}")
     assert stats["mismatches"] == 0, stats["bad_rows"][:5]
 
     # a6: outputs on rows whose kept set equals the oracle's
