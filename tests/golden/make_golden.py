@@ -26,15 +26,18 @@ CASES = [
 ]
 
 
-def main():
-    out = pathlib.Path(__file__).with_name("dirichlet_factors.txt")
+def render() -> str:
     lines = ["# Prism: Spectral-Aware Block-Sparse Attention, §2 (mean pooling under RoPE, blind spot)",
              "# D = |sin(beta*theta/2)| / (beta*|sin(theta/2)|), theta = base**(-2m/d); written by make_golden.py",
              "# base head_dim m beta theta D"]
     for base, d, m, beta in CASES:
         theta = base ** (-2.0 * m / d)
         lines.append(f"{base:g} {d} {m} {beta} {theta:.17g} {dirichlet(theta, beta):.12f}")
-    out.write_text("\n".join(lines) + "\n")
+    return "\n".join(lines) + "\n"
+
+
+def main():
+    pathlib.Path(__file__).with_name("dirichlet_factors.txt").write_text(render())
 
 
 if __name__ == "__main__":

@@ -33,6 +33,18 @@ def _golden_rows():
 # ---------------------------------------------------------------------------
 # §2: amplitude collapse of mean pooling under RoPE (closed-form Dirichlet factor)
 # ---------------------------------------------------------------------------
+def test_golden_file_is_what_its_generator_writes():
+    """The stored Dirichlet factors come from tests/golden/make_golden.py (closed form, standard
+    library only) and nothing else has edited them."""
+    import importlib.util
+    spec = importlib.util.spec_from_file_location("make_golden", os.path.join(os.path.dirname(GOLDEN),
+                                                                              "make_golden.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    with open(GOLDEN) as f:
+        assert f.read() == mod.render()
+
+
 @pytest.mark.parametrize("row", _golden_rows())
 def test_pooled_pair_amplitude_is_dirichlet_factor(row):
     base, d, m, beta, theta, D = row
