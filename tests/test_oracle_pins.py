@@ -218,6 +218,46 @@ def test_no_calib_is_plain_mean_pool_matmul():
     np.testing.assert_allclose(sc.probs, ref.numpy(), rtol=0, atol=1e-12)
 
 
+def test_estimate_scale_invariances():
+    """R4/R5: rho is a ratio of energies, so scaling Q (or K) by c leaves tau unchanged and scales
+    every calibrated block logit by c."""
+    B, Hq, Hkv, L, d, beta = 1, 2, 1, 96, 16, 8
+    rope = po.rope_tables(1e4, L, d)
+    rng = np.random.default_rng(18)
+    Q = rng.normal(size=(B, Hq, L, d))
+    K = rng.normal(size=(B, Hkv, L, d))
+    for flags in (0, po.FLAG_RELATIVE_CALIB, po.FLAG_SINGLE_BAND):
+        a = po.prism_scores(Q, K, beta, 3, flags, rope)
+        b = po.prism_scores(2.5 * Q, K, beta, 3, flags, rope)
+        c = po.prism_scores(Q, -0.75 * K, beta, 3, flags, rope)
+        np.testing.assert_allclose(b.tau, a.tau, rtol=1e-12)
+        np.testing.assert_allclose(c.tau, a.tau, rtol=1e-12)
+        np.testing.assert_allclose(b.logits, 2.5 * a.logits, rtol=1e-10, atol=1e-12)
+        np.testing.assert_allclose(c.logits, -0.75 * a.logits, rtol=1e-10, atol=1e-12)
+
+
+def test_rows_see_later_key_blocks_only_through_tau():
+    """R5/R6: row i's probabilities use key blocks j <= i; later keys enter only through the
+    sequence-wide temperature (reading R4), so with tau held fixed (or SFA_NO_CALIB) the first rows
+    do not change when the later key blocks do."""
+    B, Hq, Hkv, L, d, beta, bs = 1, 2, 1, 96, 16, 8, 3
+    rope = po.rope_tables(1e4, L, d)
+    rng = np.random.default_rng(19)
+    Q = rng.normal(size=(B, Hq, L, d))
+    K = rng.normal(size=(B, Hkv, L, d))
+    K2 = K.copy()
+    i = 5
+    K2[:, :, (i + 1) * beta:] = 3.0 * rng.normal(size=K2[:, :, (i + 1) * beta:].shape)
+    a = po.prism_scores(Q, K, beta, bs, po.FLAG_NO_CALIB, rope)
+    b = po.prism_scores(Q, K2, beta, bs, po.FLAG_NO_CALIB, rope)
+    np.testing.assert_array_equal(b.probs[..., :i + 1, :], a.probs[..., :i + 1, :])
+    a = po.prism_scores(Q, K, beta, bs, 0, rope)
+    b = po.prism_scores(Q, K2, beta, bs, 0, rope)
+    assert not np.allclose(b.tau, a.tau)                  # the temperature is sequence-wide
+    s_fixed = po.block_logits(b.qbar, b.kbar, a.tau, bs, 0, Hq // Hkv)
+    np.testing.assert_array_equal(po.causal_block_softmax(s_fixed)[..., :i + 1, :], a.probs[..., :i + 1, :])
+
+
 def test_band_bookkeeping_equivalences():
     B, Hq, Hkv, L, d, beta = 1, 2, 1, 64, 16, 8
     cos, sin = po.rope_tables(1e4, L, d)
