@@ -200,3 +200,25 @@ def test_ranked_score_is_the_left_to_right_float32_sum():
     assert fo.tip_keys(q, K, fc)[0, 0, 0] == 0.0
     K[0, 0, 0, [0, 1, 2]] = [2.0 ** 24, -(2.0 ** 24), 1.0]   # cancellation first: exact
     assert fo.tip_keys(q, K, fc)[0, 0, 0] == 1.0
+
+
+def test_power_of_two_query_scaling_scales_the_keys_exactly():
+    """Scaling q by 2^e scales every float32 product and partial sum by 2^e exactly (no overflow or
+    underflow here), so the ranked keys scale exactly and the kept tokens do not change; negating q
+    reverses the ranking of distinct keys."""
+    q, K, _ = _inputs(seed=9)
+    fc = np.array([[1, 5, 6, 7], [0, 2, 3, 4]])
+    k = 5
+    base = fo.tip_keys(q, K, fc)
+    for e in (-3, 1, 4):
+        scaled = fo.tip_keys(q * 2.0 ** e, K, fc)
+        np.testing.assert_array_equal(scaled, base * np.float32(2.0 ** e))
+        np.testing.assert_array_equal(fo.select_tokens(scaled, k), fo.select_tokens(base, k))
+    neg = fo.tip_keys(-q, K, fc)
+    np.testing.assert_array_equal(neg, -base)
+    for b in range(q.shape[0]):
+        for h in range(q.shape[1]):
+            row = base[b, h].astype(np.float64)
+            if np.unique(row).size == row.size:
+                lowest = np.sort(np.argsort(row, kind="stable")[:k])
+                np.testing.assert_array_equal(fo.select_row(neg[b, h], k), lowest)
