@@ -3,8 +3,7 @@
 TEST INFRASTRUCTURE ONLY.  Only ``tests/``, ``__graft_entry__.smoke()`` and the
 ``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
 module.  It shares no code with the CUDA library and computes in float64 from
-the same seeded host arrays the GPU receives, except the ranked token score,
-which reading D2 below defines as a float32 sum.
+the same seeded host arrays the GPU receives.
 
 What it restates (source: "FASA: Frequency-aware Sparse Attention", §2):
 
@@ -29,11 +28,12 @@ D1  A frequency chunk is one rotary pair (m, m + d/2) of the rotate-half
 D2  TIP score of Q head h for cached token t:
         s_t = sum_{m in fc[g(h)]} q_m k_{t,m} + q_{m+d/2} k_{t,m+d/2}
     from the rotated query (at the newest position) and the rotated cache.
-    The page fixes no precision, so the ranked value takes the kernel's: a
-    float32 sum taken left to right over the compact copy's columns (D5
-    order), each step one rounding of (running sum + product).  A product of
-    two bf16 values is exact in float32, so this value is reproducible
-    bit for bit; ``tip_scores`` keeps the exact float64 sum for the pins.
+    The page fixes no precision and no summation order, so the ranked value
+    is the dot product itself: ``tip_scores`` in float64 (each bf16 x bf16
+    product is exact there, and so is the sum of the few dozen products
+    unless their magnitudes span more than ~30 binades).  ``tip_keys``, a
+    float32 running sum in column order, is a diagnostic only (the error a
+    float32 estimate makes), not what is ranked.
 D3  T_t = the first min(k, L) tokens in the order (score desc, index asc),
     output ascending, padded with -1.  No forced tokens (the page names none).
 D4  FAC: o = sum_{t in T_t} softmax_t(scale * q . k_t) v_t over all d dims,
@@ -85,8 +85,8 @@ def tip_scores(q: np.ndarray, K: np.ndarray, fc: np.ndarray) -> np.ndarray:
 
 
 def tip_keys(q: np.ndarray, K: np.ndarray, fc: np.ndarray) -> np.ndarray:
-    """D2: the float32 values the selection ranks [B, Hq, L]: running float32 sum over the
-    compact columns in order, starting from 0, each step rounding (sum + q_c * k_c) once."""
+    """Diagnostic, not ranked: the TIP score as a float32 running sum over the compact columns in
+    order [B, Hq, L], starting from 0, each step rounding (sum + q_c * k_c) once."""
     q = np.asarray(q, dtype=np.float32)
     K = np.asarray(K, dtype=np.float32)
     B, Hq, d = q.shape
@@ -103,7 +103,7 @@ def tip_keys(q: np.ndarray, K: np.ndarray, fc: np.ndarray) -> np.ndarray:
 
 
 def select_row(keys: np.ndarray, k: int) -> np.ndarray:
-    """D3 for one row: ascending indices of the first min(k, L) tokens by (key desc, index asc)."""
+    """D3 for one row: ascending indices of the first min(k, L) tokens by (score desc, index asc)."""
     L = keys.shape[0]
     n = min(k, L)
     order = sorted(range(L), key=lambda t: (-float(keys[t]), t))
@@ -146,9 +146,8 @@ def focused_attention(q, K, V, idx, scale=None):
 
 
 def decode_step(q, K, V, fc, k, scale=None):
-    """TIP -> select -> FAC for one decode step: (scores64, keys32, idx, o, lse)."""
+    """TIP -> select -> FAC for one decode step: (scores, idx, o, lse), scores float64 [B, Hq, L]."""
     s = tip_scores(q, K, fc)
-    keys = tip_keys(q, K, fc)
-    idx = select_tokens(keys, k)
+    idx = select_tokens(s, k)
     o, lse = focused_attention(q, K, V, idx, scale)
-    return s, keys, idx, o, lse
+    return s, idx, o, lse

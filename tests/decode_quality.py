@@ -54,7 +54,7 @@ def measure(w: DecodeWorkload, seed=0):
     allp = np.tile(np.arange(half), (w.heads_kv, 1))
     res = {}
     for name, pairs in (("all pairs (exact top-k)", allp), ("dominant pairs", fc), ("other pairs", other)):
-        idx = fo.select_tokens(fo.tip_keys(q, K, pairs), w.k)
+        idx = fo.select_tokens(fo.tip_scores(q, K, pairs), w.k)
         res[name] = mass_recall(q, K, idx)
     recent = np.tile(np.arange(w.seq_len - w.k, w.seq_len), (w.batch, w.heads_q, 1))
     res["most recent k (no estimate)"] = mass_recall(q, K, recent)

@@ -160,7 +160,7 @@ def test_decode_step_top1_picks_planted_key():
     d = 16
     dims = fo.fc_dims(fc[0], d)
     K[0, 0, 11, dims] = 50.0 * q[0, 0, dims]
-    _, _, idx, o, _ = fo.decode_step(q, K, V, fc, 1)
+    _, idx, o, _ = fo.decode_step(q, K, V, fc, 1)
     assert idx[0, 0, 0] == 11
     np.testing.assert_array_equal(o[0, 0], V[0, 0, 11])
 
@@ -185,9 +185,9 @@ def test_ranked_float32_score_is_within_the_recursive_summation_bound():
     np.testing.assert_array_equal(fo.tip_keys(qi, Ki, fc).astype(np.float64), fo.tip_scores(qi, Ki, fc))
 
 
-def test_ranked_score_is_the_left_to_right_float32_sum():
-    """Products 2^24, 1, -2^24 in column order: float32 left to right gives 2^24 + 1 -> 2^24 (ties to
-    even), then 0; the exact sum is 1.  Pins the order and the precision of the ranked value."""
+def test_float32_diagnostic_is_the_left_to_right_sum():
+    """The float32 diagnostic (not ranked): products 2^24, 1, -2^24 in column order give 2^24 + 1 ->
+    2^24 (ties to even), then 0, where the exact sum is 1; with the cancellation first it is exact."""
     d = 16
     fc = np.array([[0, 1, 2, 3]])          # columns: dims 0, 1, 2, 3, then 8, 9, 10, 11
     q = np.zeros((1, 1, d))
@@ -200,6 +200,46 @@ def test_ranked_score_is_the_left_to_right_float32_sum():
     assert fo.tip_keys(q, K, fc)[0, 0, 0] == 0.0
     K[0, 0, 0, [0, 1, 2]] = [2.0 ** 24, -(2.0 ** 24), 1.0]   # cancellation first: exact
     assert fo.tip_keys(q, K, fc)[0, 0, 0] == 1.0
+
+
+def test_ranked_score_is_the_exact_dot_product():
+    """The selection ranks the dot product itself, not a float32 running sum: token 0's products
+    2^24, 1, -2^24 sum to 1 (a float32 column-order sum gives 0), token 1's to 1/2, token 2's to
+    -1; top-1 is token 0 and top-2 is {0, 1}."""
+    d = 16
+    fc = np.array([[0, 1, 2, 3]])
+    q = np.zeros((1, 1, d))
+    q[0, 0, [0, 1, 2]] = 1.0
+    K = np.zeros((1, 1, 3, d))
+    V = np.arange(3 * d, dtype=np.float64).reshape(1, 1, 3, d)
+    K[0, 0, 0, [0, 1, 2]] = [2.0 ** 24, 1.0, -(2.0 ** 24)]
+    K[0, 0, 1, 1] = 0.5
+    K[0, 0, 2, 0] = -1.0
+    s, idx, o, _ = fo.decode_step(q, K, V, fc, 1)
+    np.testing.assert_array_equal(s[0, 0], [1.0, 0.5, -1.0])
+    assert idx[0, 0].tolist() == [0]
+    np.testing.assert_array_equal(o[0, 0], V[0, 0, 0])
+    assert fo.decode_step(q, K, V, fc, 2)[1][0, 0].tolist() == [0, 1]
+
+
+def test_scores_of_bf16_inputs_equal_the_exact_rational_sum():
+    """bf16 x bf16 products and their sum over a few dozen columns are exact in float64 when the
+    magnitudes stay within a few binades: the float64 score equals the exact rational dot product
+    (fractions), so the ranked value carries no summation-order rounding."""
+    from fractions import Fraction
+    rng = np.random.default_rng(11)
+    d, L = 32, 25
+    q = torch.from_numpy(rng.normal(size=(1, 2, d))).to(torch.bfloat16).double().numpy()
+    K = torch.from_numpy(rng.uniform(0.25, 4.0, size=(1, 1, L, d)) * rng.choice([-1, 1], size=(1, 1, L, d))
+                         ).to(torch.bfloat16).double().numpy()
+    q = np.where(np.abs(q) < 0.25, 0.25, q)                  # keep every product within 2^-4 .. 2^4
+    fc = np.array([[0, 3, 5, 6, 9, 12, 14, 15]])
+    s = fo.tip_scores(q, K, fc)
+    dims = fo.fc_dims(fc[0], d)
+    for h in range(2):
+        for t in range(L):
+            exact = sum(Fraction(float(q[0, h, c])) * Fraction(float(K[0, 0, t, c])) for c in dims)
+            assert s[0, h, t] == float(exact)
 
 
 def test_power_of_two_query_scaling_scales_the_keys_exactly():

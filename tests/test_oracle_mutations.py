@@ -148,6 +148,10 @@ FASA_MUTANTS = [
     ("select: padded with 0", "idx = -np.ones((B, H, k), dtype=np.int64)", "idx = np.zeros((B, H, k), dtype=np.int64)"),
     ("select: output in rank order", "return np.sort(np.asarray(order[:n], dtype=np.int64))",
      "return np.asarray(order[:n], dtype=np.int64)"),
+    ("decode step: ranks the float32 running sum", "idx = select_tokens(s, k)",
+     "idx = select_tokens(tip_keys(q, K, fc), k)"),
+    ("tip: float32 dot product", "out[:, h] = np.einsum(\"bd,btd->bt\", q[:, h][:, dims], K[:, g][..., dims])",
+     "out[:, h] = np.einsum(\"bd,btd->bt\", q[:, h][:, dims].astype(np.float32), K[:, g][..., dims].astype(np.float32))"),
 ]
 
 PIN_MODULES = [test_oracle_pins, test_fasa_oracle_pins, test_selection_properties]

@@ -108,7 +108,7 @@ def run_decode_units(us, q, K, V, fc):
     out = {}
     for b, g in us:
         hs = list(sharding.q_heads(g, DW.heads_q, DW.heads_kv))
-        _, _, idx, o, _ = fo.decode_step(q[b:b + 1, hs].double().numpy(), K[b:b + 1, g:g + 1].double().numpy(),
+        _, idx, o, _ = fo.decode_step(q[b:b + 1, hs].double().numpy(), K[b:b + 1, g:g + 1].double().numpy(),
                                          V[b:b + 1, g:g + 1].double().numpy(), fc[g:g + 1], DW.k)
         out[(b, g)] = (idx[0], o[0])
     return out
@@ -144,7 +144,7 @@ def test_two_rank_gloo_decode_split_equals_single_process():
         p.join(timeout=60)
         assert p.exitcode == 0
     qq, K, V, fc = make_decode_inputs(DW, seed=0)
-    _, _, idx, o, _ = fo.decode_step(qq.double().numpy(), K.double().numpy(), V.double().numpy(), fc, DW.k)
+    _, idx, o, _ = fo.decode_step(qq.double().numpy(), K.double().numpy(), V.double().numpy(), fc, DW.k)
     assert sorted(merged) == sharding.units(DW.batch, DW.heads_kv)
     for (b, g), (ii, oo) in merged.items():
         hs = list(sharding.q_heads(g, DW.heads_q, DW.heads_kv))
