@@ -106,9 +106,12 @@ def test_path_matches_oracle(w):
 
     # a5: masks identical except near-ties at the row threshold
     stats, exact = compare_masks(ref.selection, sc.probs, model.counts, model.idx, mass)
-    print(f"{w.name}: rows {stats['rows']}, near-tie rows {stats['uncertain_rows']}, "
-          f"threshold-only excusals {stats['threshold_only_rows']}")
+    print(f"{w.name}: rows {stats['rows']}, near-tie rows excused {stats['excused_rows']} "
+          f"(count differs {stats['count_diff_rows']})")
     assert stats["mismatches"] == 0, stats["bad_rows"][:5]
+    assert stats["threshold_only_rows"] == 0
+    if w.k is not None:
+        assert stats["count_diff_rows"] == 0
 
     # a6: outputs on rows whose kept set equals the oracle's
     O = to_np(model.O).astype(np.float64)
