@@ -12,8 +12,9 @@ replica of the layer (the path has no exchange step between layers' units;
 
 value  = attention FLOPs over the kept blocks (causal diagonal counted half),
          summed over ranks, / the slowest rank's device time for K steps -> TFLOP/s.
-e2e    = the same metric through PrismAttention.run_host from pinned host
-         tensors: H2D of Q, K, V and D2H of O inside every timed step.
+e2e    = the same metric through sfa.HostPipeline from pinned host tensors:
+         H2D of Q, K, V and D2H of O for every timed step, on two copy streams
+         overlapping the path of the neighbouring steps (double-buffered).
 --impl reference times the CPU oracle (the slow fp64 restatement) on a
 bounded sample of the same workload (see cpu_baseline.sample).
 
@@ -200,6 +201,15 @@ def oracle_head_sample(w: wl.Workload, Q, K, V, h: int = 0, attn_blocks: int | N
     return flops / secs / 1e12, secs, text
 
 
+def layer_config(w: wl.Workload, world: int) -> dict:
+    """The config keys both arms report for a prefill workload."""
+    return {"workload": w.name,
+            "layer": f"B={w.batch} Hq={w.heads_q} Hkv={w.heads_kv} L={w.seq_len} d={w.head_dim} "
+                     f"block={w.block} rope_base={w.rope_base:g} band_split={w.band_split}",
+            "budget": (f"top-{w.k} + diagonal" if w.k is not None else f"mass {w.mass}"),
+            "parallelism": f"replicas x{world}"}
+
+
 def cpu_model() -> str:
     """The host CPU's model name (from /proc/cpuinfo), for the oracle timings."""
     try:
@@ -245,7 +255,7 @@ def oracle_decode_sample(w: wl.DecodeWorkload, q, K, V, fc, b=0, h=0):
     secs = time.perf_counter() - t0
     # a step is batch x heads_q such rows for batch tokens
     value = w.batch / (secs * w.batch * w.heads_q)
-    text = (f"one (sequence, Q head) row of {w.batch} x {w.heads_q}: float32 importance over the {w.seq_len}-token "
+    text = (f"one (sequence, Q head) row of {w.batch} x {w.heads_q}: float64 importance over the {w.seq_len}-token "
             f"cache, top-{w.k}, float64 attention; scaled to the full step")
     return value, secs, text
 
@@ -391,19 +401,22 @@ def run_reference(args, w, rank, world):
     per_step = []
     blocks = max(4, min(64, w.nb // 16))
     text = ""
+    wall = []
     for s in range(args.warmup + args.steps):
+        t0 = time.perf_counter()
         v, secs, text = oracle_head_sample(w, Q, K, V, h=s % w.heads_q, attn_blocks=blocks)
         if s >= args.warmup:
             per_step.append((v, secs))
+            wall.append(time.perf_counter() - t0)
     value = float(np.mean([v for v, _ in per_step]))
     ms = float(np.mean([s for _, s in per_step]) * 1e3)
     cores = len(os.sched_getaffinity(0))
     line = {"metric": "prefill attention effective TFLOP/s over kept blocks (whole path)", "value": value,
             "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": w.name, "layer": f"B={w.batch} Hq={w.heads_q} Hkv={w.heads_kv} "
-                       f"L={w.seq_len} d={w.head_dim} block={w.block}"},
+            "dtype": "f64", "data": "synthetic", "impl": "reference", "extrapolated": True,
+            "measured_ms_per_step": float(np.mean(wall)) * 1e3,
+            "config": layer_config(w, world),
             "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads() or cores,
                              "kind": "oracle", "sample": text, "cpu_model": cpu_model()},
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -473,25 +486,33 @@ def main():
     flops_step = attention_flops(counts, w.block, w.head_dim)
     kept_frac = float(counts.sum()) / (w.batch * w.heads_q * w.nb * (w.nb + 1) / 2)
 
-    # e2e: the public API from pinned host buffers, copies inside the timed region
+    # e2e: the public API from pinned host buffers, every step's copies inside the timed region
+    # (uploads and downloads on their own streams, overlapping the neighbouring steps' path)
     e2e_steps = args.e2e_steps or K_
     Qh, Kh, Vh = (t.pin_memory() for t in (Q, K, V))
-    Oh = torch.empty(model.O.shape, dtype=model.O.dtype).pin_memory()
-    dev_in = (torch.empty_like(Qd), torch.empty_like(Kd), torch.empty_like(Vd))
-    model.run_host(Qh, Kh, Vh, Oh, dev_in=dev_in)
+    Oh = [torch.empty(model.O.shape, dtype=model.O.dtype).pin_memory() for _ in range(2)]
+    pipe = sfa.HostPipeline(model, Qd, Kd, Vd)
+    for i in range(2):
+        pipe.submit(Qh, Kh, Vh, Oh[i])
+    pipe.drain()
     torch.cuda.synchronize(dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
         dist.barrier()
     torch.cuda.synchronize(dev)
     e0.record(stream)
-    for _ in range(e2e_steps):
-        model.run_host(Qh, Kh, Vh, Oh, dev_in=dev_in)
+    pipe.up.wait_stream(stream)
+    pipe.down.wait_stream(stream)
+    for i in range(e2e_steps):
+        pipe.submit(Qh, Kh, Vh, Oh[i % 2])
+    pipe.drain(stream)
     e1.record(stream)
     torch.cuda.synchronize(dev)
     e2e_ms = e0.elapsed_time(e1)
+    if int(model.status.item()) != 0:
+        raise RuntimeError(f"device status {int(model.status.item())}")
     h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh))
-    d2h = Oh.numel() * Oh.element_size()
+    d2h = Oh[0].numel() * Oh[0].element_size()
 
     vals = torch.tensor([total_ms, e2e_ms, float(np.mean(t_attn)), float(np.mean(t_scores)),
                          float(np.mean(t_select))], dtype=torch.float64, device=dev)
@@ -515,11 +536,7 @@ def main():
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K_, "warmup": args.warmup,
             "ms_per_step": total_ms / K_, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic",
-            "config": {"workload": w.name,
-                       "layer": f"B={w.batch} Hq={w.heads_q} Hkv={w.heads_kv} L={w.seq_len} d={w.head_dim} "
-                                f"block={w.block} rope_base={w.rope_base:g} band_split={w.band_split}",
-                       "budget": (f"top-{w.k} + diagonal" if w.k is not None else f"mass {w.mass}"),
-                       "kept_fraction": round(kept_frac, 5), "parallelism": f"replicas x{world}",
+            "config": {**layer_config(w, world), "kept_fraction": round(kept_frac, 5),
                        "l2": "inputs larger than L2 (Q 1.07 GB, K 0.27 GB, V 0.27 GB at 128K); no flush"},
             "stages_ms": {"block_scores": scores_ms, "select": select_ms, "attention": attn_ms},
             "scoring": {"bytes": sb + selb, "GB_s": (sb + selb) / ((scores_ms + select_ms) * 1e-3) / 1e9,
@@ -534,6 +551,7 @@ def main():
                                           if tr else "no capture for the current kernel source"),
                          "flops_per_launch": flops_step},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "copies": "upload and download streams, double-buffered device inputs and outputs",
                     "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
             "gpu_launches": KERNELS_PER_STEP * K_,
             "clocks": clk.summary(),

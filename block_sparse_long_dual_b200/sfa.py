@@ -445,7 +445,8 @@ class PrismAttention:
         return self.O
 
     def run_host(self, Q_host, K_host, V_host, O_host, dev_in=None, stream=None):
-        """End to end from pinned host tensors: H2D copies, the path, D2H copy of O."""
+        """End to end from pinned host tensors: H2D copies, the path, D2H copy of O, all on one
+        stream (each step's copies serialise with its kernels; HostPipeline overlaps them)."""
         if dev_in is None:
             dev_in = tuple(torch.empty(t.shape, dtype=t.dtype, device=self.O.device) for t in (Q_host, K_host, V_host))
         for d, h in zip(dev_in, (Q_host, K_host, V_host)):
@@ -453,6 +454,60 @@ class PrismAttention:
         self(*dev_in, stream=stream)
         O_host.copy_(self.O, non_blocking=True)
         return O_host
+
+
+class HostPipeline:
+    """Layers fed from and returned to pinned host memory, with the copies overlapped.
+
+    Step n's inputs go host -> device on an upload stream and its output device -> host on a
+    download stream, while step n - 1's path runs on the compute stream: device inputs and
+    outputs are double-buffered and events order each buffer's reuse (an upload waits until the
+    path of the step two back has read that input buffer; a path waits until the download of the
+    step two back has read that output buffer).  The library's kernels are the ones PrismAttention
+    launches; only the copies and events are added here."""
+
+    def __init__(self, model: PrismAttention, like_q, like_k, like_v):
+        dev = model.O.device
+        self.model = model
+        self.dev_in = [tuple(torch.empty(t.shape, dtype=t.dtype, device=dev) for t in (like_q, like_k, like_v))
+                       for _ in range(2)]
+        self.dev_out = [model.O, torch.empty_like(model.O)]
+        self.up = torch.cuda.Stream(dev)
+        self.down = torch.cuda.Stream(dev)
+        ev = lambda: [torch.cuda.Event() for _ in range(2)]
+        self.in_ready, self.in_free, self.out_ready, self.out_free = ev(), ev(), ev(), ev()
+        self.n = 0
+
+    def submit(self, Q_host, K_host, V_host, O_host, stream=None):
+        """Enqueue one step; O_host is written once the download stream reaches it."""
+        comp = torch.cuda.current_stream(self.model.O.device) if stream is None else stream
+        s = self.n % 2
+        if self.n >= 2:
+            self.up.wait_event(self.in_free[s])
+        with torch.cuda.stream(self.up):
+            for d, h in zip(self.dev_in[s], (Q_host, K_host, V_host)):
+                d.copy_(h, non_blocking=True)
+            self.in_ready[s].record(self.up)
+        comp.wait_event(self.in_ready[s])
+        if self.n >= 2:
+            comp.wait_event(self.out_free[s])
+        self.model.O = self.dev_out[s]
+        with torch.cuda.stream(comp):
+            self.model(*self.dev_in[s], stream=comp)
+            self.in_free[s].record(comp)
+            self.out_ready[s].record(comp)
+        self.down.wait_event(self.out_ready[s])
+        with torch.cuda.stream(self.down):
+            O_host.copy_(self.dev_out[s], non_blocking=True)
+            self.out_free[s].record(self.down)
+        self.n += 1
+        return O_host
+
+    def drain(self, stream=None):
+        """Make ``stream`` (default: the current one) wait for every copy submitted so far."""
+        comp = torch.cuda.current_stream(self.model.O.device) if stream is None else stream
+        comp.wait_stream(self.up)
+        comp.wait_stream(self.down)
 
 
 # ---------------------------------------------------------------------------
