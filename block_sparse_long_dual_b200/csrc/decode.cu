@@ -7,23 +7,34 @@
 //   tip_chunk      Token Importance Predictor, persistent (one or two CTAs per
 //                  SM) over tiles (chunk of C tokens, b, KV head): the chunk's
 //                  K_fc rows stream through a bulk-copy ring once for all Q
-//                  heads of the group; each score is a float32 FMA chain over
-//                  the compact columns in order (a bf16 x bf16 product is exact
-//                  in float32, so every step rounds once and the value is
-//                  reproducible); then per head a lower bound of the chunk's
-//                  k-th largest score (from group maxima) and the tokens at or
-//                  above it, written per warp segment in token order.
-//   tip_merge      CTA per (b, h): the candidates staged in shared memory,
-//                  bounded again, exact k-th largest by block bisection, ties
-//                  by index; ascending index list, -1 padded (radix select over
-//                  global memory when the candidates do not fit).
+//                  heads of the group; each token's score is first taken as a
+//                  float32 FMA chain (a filter), then per head a lower bound
+//                  of the chunk's k-th largest score (from group maxima),
+//                  lowered by twice the float32 chain's rounding bound, and
+//                  the tokens at or above it (token order, per warp segment)
+//                  get their exact score recomputed in float64.
+//   tip_merge      CTA per (b, h): the candidates' float64 keys staged in
+//                  shared memory, bounded again, exact k-th largest by radix
+//                  select, ties by index; ascending index list, -1 padded (the
+//                  same select over global memory when the candidates do not
+//                  fit).
 //   fac            Focused Attention Computation: CTA per (b, h), 16 warps,
 //                  each warp gathers the K / V rows of its share of the kept
 //                  tokens (eight tokens' loads in flight per lane), float32
 //                  online softmax, warps merged through shared memory.
 //
-// Ranking: key = order-preserving uint32 of the float32 score (+0 for both
-// zeros); the first k by (key desc, index asc).
+// Ranking: the token score is the dot product over the dominant pairs' dims;
+// it is ranked by its float64 value (key = order-preserving uint64 of the
+// double, +0 for both zeros); the first k by (key desc, index asc).
+//
+// Why the float32 filter loses no token of the top k (finite inputs): each
+// bf16 x bf16 product is exact in float32, so a chain of n = 2 nfc FMAs is off
+// the exact score by at most M = n u sum_c |q_c k_c| + n 2^-150 (u = 2^-24;
+// the second term covers subnormal partial sums), and sum_c |q_c k_c| <=
+// ||q||_1 A, A = the largest |k| in the chunk's compact rows.  If at least k
+// tokens of a chunk have float32 scores >= x, they have exact scores >= x - M,
+// so the row's k-th largest exact score is >= x - M, and every token of the
+// row's top k has a float32 score >= x - 2M.
 #include <math.h>
 
 #include "common.cuh"
@@ -36,19 +47,27 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kWarps = kThreads / 32;
 
+// Order-preserving unsigned keys of float32 (filter) and float64 (ranked) scores.
 __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+__device__ __forceinline__ float key_value(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+__device__ __forceinline__ uint64_t order_key64(double f) {
+  const uint64_t u = (uint64_t)__double_as_longlong(f == 0.0 ? 0.0 : f);
+  return (u >> 63) ? ~u : (u | 0x8000000000000000ull);
+}
 
 // The k-th largest of n keys (1 <= k <= n) by MSB-first 8-bit radix select over a
 // block of kThreads threads: returns T and sets *gt = #{key > T}.
-template <typename KeyAt>
-__device__ uint32_t block_kth_largest(KeyAt key_at, int n, int k, uint32_t* hist, int* sh, int* gt) {
+template <typename Key, typename KeyAt>
+__device__ Key block_kth_largest(KeyAt key_at, int n, int k, uint32_t* hist, int* sh, int* gt) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  uint32_t prefix = 0, pmask = 0;
+  Key prefix = 0, pmask = 0;
   int krem = k;
-  for (int shift = 24; shift >= 0; shift -= 8) {
+  for (int shift = 8 * (int)sizeof(Key) - 8; shift >= 0; shift -= 8) {
     for (int i = tid; i < 256; i += kThreads) hist[i] = 0;
     __syncthreads();
     // Warp-aggregated increments: keys cluster in a few digits (float exponents), so lanes with
@@ -57,7 +76,7 @@ __device__ uint32_t block_kth_largest(KeyAt key_at, int n, int k, uint32_t* hist
       const int i = i0 + tid;
       int bin = -1;
       if (i < n) {
-        const uint32_t u = key_at(i);
+        const Key u = key_at(i);
         if ((u & pmask) == prefix) bin = (int)((u >> shift) & 255u);
       }
       const unsigned same = __match_any_sync(0xffffffffu, bin);
@@ -93,10 +112,10 @@ __device__ uint32_t block_kth_largest(KeyAt key_at, int n, int k, uint32_t* hist
       }
     }
     __syncthreads();
-    const uint32_t digit = (uint32_t)sh[0];
+    const Key digit = (Key)sh[0];
     krem -= sh[1];
     prefix |= digit << shift;
-    pmask |= 0xFFu << shift;
+    pmask |= (Key)0xFF << shift;
     __syncthreads();
   }
   *gt = k - krem;
@@ -124,16 +143,16 @@ __device__ int warp_exclusive_sum(int v, int* sh, int* total) {
 // emit(rank, i) for the kept i in ascending i, rank = 0, 1, ...  Returns the kept count.
 // Warp w owns a contiguous range of 32-key groups; lane j takes key 32 g + j of each group, so
 // shared-memory reads are conflict-free and global reads coalesced; ranks come from ballots.
-template <typename KeyAt, typename Emit>
+template <typename Key, typename KeyAt, typename Emit>
 __device__ int block_select_ordered(KeyAt key_at, int n, int k, Emit emit, uint32_t* hist, int* sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned lt = (1u << lane) - 1u;
-  uint32_t T = 0;
+  Key T = 0;
   int take = n;  // ties at T to keep (all when every key is kept)
   const bool all = k >= n;
   if (!all) {
     int gt = 0;
-    T = block_kth_largest(key_at, n, k, hist, sh, &gt);
+    T = block_kth_largest<Key>(key_at, n, k, hist, sh, &gt);
     take = k - gt;
   }
   const int S = ((n + kWarps * 32 - 1) / (kWarps * 32)) * 32;
@@ -149,7 +168,7 @@ __device__ int block_select_ordered(KeyAt key_at, int n, int k, Emit emit, uint3
   int nk = 0, tr = tie_base;
   for (int b = w0; b < w1; b += 32) {
     const int i = b + lane;
-    const uint32_t u = (i < w1 && !all) ? key_at(i) : 0u;
+    const Key u = (i < w1 && !all) ? key_at(i) : (Key)0;
     const bool tie = i < w1 && !all && u == T;
     const unsigned tb = __ballot_sync(0xffffffffu, tie);
     const bool keep = i < w1 && (all || u > T || (tie && tr + __popc(tb & lt) < take));
@@ -161,7 +180,7 @@ __device__ int block_select_ordered(KeyAt key_at, int n, int k, Emit emit, uint3
   tr = tie_base;
   for (int b = w0; b < w1; b += 32) {
     const int i = b + lane;
-    const uint32_t u = (i < w1 && !all) ? key_at(i) : 0u;
+    const Key u = (i < w1 && !all) ? key_at(i) : (Key)0;
     const bool tie = i < w1 && !all && u == T;
     const unsigned tb = __ballot_sync(0xffffffffu, tie);
     const bool keep = i < w1 && (all || u > T || (tie && tr + __popc(tb & lt) < take));
@@ -175,8 +194,8 @@ __device__ int block_select_ordered(KeyAt key_at, int n, int k, Emit emit, uint3
 
 // Block-wide: emit(rank, i) for every i in [0, n) with key_at(i) >= LB, in ascending i; returns
 // the count.  Warp-contiguous ranges of 32-key groups, ranks from ballots.
-template <typename KeyAt, typename Emit>
-__device__ int block_filter_ordered(KeyAt key_at, int n, uint32_t LB, Emit emit, int* sh) {
+template <typename Key, typename KeyAt, typename Emit>
+__device__ int block_filter_ordered(KeyAt key_at, int n, Key LB, Emit emit, int* sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned lt = (1u << lane) - 1u;
   const int S = ((n + kWarps * 32 - 1) / (kWarps * 32)) * 32;
@@ -196,50 +215,6 @@ __device__ int block_filter_ordered(KeyAt key_at, int n, uint32_t LB, Emit emit,
     pos += __popc(kb);
   }
   return total;
-}
-
-// Block-wide bisection over n values in shared memory (1 <= k <= n): the k-th largest T and
-// *gt = #{> T}.  Bracketed by the values' minimum and maximum.
-__device__ uint32_t block_kth_largest_smem(const uint32_t* vals, int n, int k, int* sh, int* gt) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-  for (int i = threadIdx.x; i < n; i += kThreads) {
-    mn = min(mn, vals[i]);
-    mx = max(mx, vals[i]);
-  }
-  mn = __reduce_min_sync(0xffffffffu, mn);
-  mx = __reduce_max_sync(0xffffffffu, mx);
-  if (lane == 0) { sh[warp] = (int)mn; sh[kWarps + warp] = (int)mx; }
-  __syncthreads();
-  for (int w = 0; w < kWarps; ++w) {
-    mn = min(mn, (uint32_t)sh[w]);
-    mx = max(mx, (uint32_t)sh[kWarps + w]);
-  }
-  __syncthreads();
-  uint64_t lo = mn, hi = (uint64_t)mx + 1;
-  while (hi - lo > 1) {  // uniform across the block
-    const uint32_t mid = (uint32_t)(lo + ((hi - lo) >> 1));
-    int c = 0;
-    for (int i = threadIdx.x; i < n; i += kThreads) c += vals[i] >= mid ? 1 : 0;
-    c = (int)__reduce_add_sync(0xffffffffu, (unsigned)c);
-    if (lane == 0) sh[warp] = c;
-    __syncthreads();
-    int t = 0;
-    for (int w = 0; w < kWarps; ++w) t += sh[w];
-    __syncthreads();
-    if (t >= k) lo = mid; else hi = mid;
-  }
-  const uint32_t T = (uint32_t)lo;
-  int g = 0;
-  for (int i = threadIdx.x; i < n; i += kThreads) g += vals[i] > T ? 1 : 0;
-  g = (int)__reduce_add_sync(0xffffffffu, (unsigned)g);
-  if (lane == 0) sh[warp] = g;
-  __syncthreads();
-  int t = 0;
-  for (int w = 0; w < kWarps; ++w) t += sh[w];
-  __syncthreads();
-  *gt = t;
-  return T;
 }
 
 // ---------------------------------------------------------------------------
@@ -274,12 +249,12 @@ __global__ void __launch_bounds__(kThreads) fc_gather_kernel(DecodeParams p, con
 }
 
 // ---------------------------------------------------------------------------
-// tip_chunk: persistent, one CTA per SM, looping over tiles (chunk, b, KV head);
-// G = Q heads per KV head, TPS = tokens per thread per slab, NGR = groups of 4
-// keys per thread per chunk.  The chunk's compact key rows stream through an
-// NS-stage ring of slabs (ST = 256 TPS tokens) filled by bulk copies; the ring
-// runs across tiles, so the next tile's first slabs are in flight while this
-// tile's candidates are selected.
+// tip_chunk: persistent, one or two CTAs per SM, looping over tiles (chunk, b,
+// KV head); G = Q heads per KV head, TPS = tokens per thread per slab, NGR =
+// groups of 4 keys per thread per chunk.  The chunk's compact key rows stream
+// through an NS-stage ring of slabs (ST = 256 TPS tokens) filled by bulk
+// copies; the ring runs across tiles, so the next tile's first slabs are in
+// flight while this tile's candidates are selected.
 // ---------------------------------------------------------------------------
 template <int G, int TPS, int NGR>
 __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(DecodeParams p) {
@@ -347,23 +322,30 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
     }
     __syncthreads();
 
-    // Scores: a float32 FMA chain per (token, head) over the columns in order.  Thread tid takes
-    // tokens tid + 256 u of each slab.
+    // Filter scores: a float32 FMA chain per (token, head) over the columns in order.  Thread tid
+    // takes tokens tid + 256 u of each slab.  am: the largest |k| bit patterns of the chunk's
+    // compact values seen by this thread (two bf16 lanes; |x| orders like its bits for finite x).
+    uint32_t am = 0u;
     for (int sl = 0; sl < nsl; ++sl, ++consumed) {
       const int stg = consumed % NS;
       if (!wait_parity_bounded((uint32_t)__cvta_generic_to_shared(&bars[stg]), (consumed / NS) & 1)) lost = 1;
       const __nv_bfloat16* slab = reinterpret_cast<const __nv_bfloat16*>(ring + (size_t)stg * SB);
       float acc[TPS][G];
+      uint32_t vmask[TPS];
 #pragma unroll
-      for (int u = 0; u < TPS; ++u)
+      for (int u = 0; u < TPS; ++u) {
+        vmask[u] = sl * ST + u * kThreads + tid < n ? 0x7FFF7FFFu : 0u;
 #pragma unroll
         for (int hh = 0; hh < G; ++hh) acc[u][hh] = 0.f;
+      }
       for (int q8 = 0; q8 < W / 8; ++q8) {
         uint32_t w4[TPS][4];
 #pragma unroll
         for (int u = 0; u < TPS; ++u) {
           const uint4 v = reinterpret_cast<const uint4*>(slab + (size_t)(u * kThreads + tid) * W)[q8];
           w4[u][0] = v.x; w4[u][1] = v.y; w4[u][2] = v.z; w4[u][3] = v.w;
+#pragma unroll
+          for (int e = 0; e < 4; ++e) am = __vmaxu2(am, w4[u][e] & vmask[u]);
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
@@ -399,13 +381,19 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
       __syncthreads();  // stage consumed
       if (tid == 0) issue_next();
     }
+    {
+      const uint32_t a16 = __reduce_max_sync(0xffffffffu, max(am & 0xFFFFu, am >> 16));
+      if ((tid & 31) == 0) scratch[64 + (tid >> 5)] = (int)a16;
+    }
+    __syncthreads();
 
     // Per head, a lower bound LB of the chunk's k-th largest key, by warp h alone: the maxima
     // of the C / 4 groups of 4 consecutive keys (0 past the end of the chunk), then a bisection
     // over them in registers.  Any value with at least k group maxima at or above it is at most
-    // the chunk's k-th largest (each maximum is a distinct key), so stopping the bisection
-    // early still gives a valid bound.  Every token of the row's top k has a key >= the row's
-    // k-th largest >= the chunk's k-th largest >= LB, so keys below LB are dropped.
+    // the chunk's k-th largest float32 score (each maximum is a distinct token), so stopping the
+    // bisection early still gives a valid bound; the bound is then lowered by twice the float32
+    // chain's rounding bound M (see the top of this file), so that no token of the row's top k
+    // by exact score is dropped.
     {
       const int lane = tid & 31, warp = tid >> 5;
       constexpr int NGPL = 8 * NGR;  // groups per lane: C / 4 / 32
@@ -436,6 +424,17 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
             if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= p.k) lo = mid; else hi = mid;
           }
           LBw = (uint32_t)lo;
+          // M = n u ||q||_1 A + n 2^-150, every operation rounded up; then LB - 2M rounded down.
+          float q1 = 0.f;
+          for (int c = lane; c < W; c += 32) q1 = __fadd_ru(q1, fabsf(qd[c * G + warp]));
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) q1 = __fadd_ru(q1, __shfl_xor_sync(0xffffffffu, q1, off));
+          uint32_t a16 = 0u;
+#pragma unroll
+          for (int w = 0; w < kWarps; ++w) a16 = max(a16, (uint32_t)scratch[64 + w]);
+          const float A = __uint_as_float(a16 << 16);
+          const float M = __fadd_ru(__fmul_ru(__fmul_ru((float)W * 0x1p-24f, q1), A), (float)W * 0x1p-149f);
+          if (LBw > 0u) LBw = order_key(__fsub_rd(key_value(LBw), __fmul_ru(2.f, M)));
         }
         if (lane == 0) scratch[warp] = (int)LBw;
       }
@@ -445,32 +444,97 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) LB[hh] = (uint32_t)scratch[hh];
     // Candidates in token order: warp w scans its contiguous range [w S, w S + S) of the chunk
-    // and writes its own segment of the slot; counts per (slot, warp).
+    // and writes its own segment of each head's slot (token indices); then it computes its
+    // candidates' exact scores in float64, all heads together and four candidates per lane at a
+    // time so that their compact rows (just streamed, so read from L2) are in flight together;
+    // counts per (slot, warp).
     const int bad = lost;
     {
       const int lane = tid & 31, warp = tid >> 5;
       const unsigned lt = (1u << lane) - 1u;
       const int S = C / kWarps;
       const int w0 = min(n, warp * S), w1 = min(n, w0 + S);
+      const __nv_bfloat16* kfc_rows = kfc_all + (size_t)bg * p.L * W;
+      int cnt[G];
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
         const size_t slot = ((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk;
-        uint32_t* ck = p.cand_key + slot * C + (size_t)warp * S;
         int* ci = p.cand_idx + slot * C + (size_t)warp * S;
         const uint32_t* hk = keys + (size_t)hh * C;
-        int cnt = 0;
+        int c = 0;
         for (int b0 = w0; b0 < w1; b0 += 32) {
           const int i = b0 + lane;
-          const uint32_t u = i < w1 ? hk[i] : 0u;
-          const bool keep = i < w1 && u >= LB[hh];
+          const bool keep = i < w1 && hk[i] >= LB[hh];
           const unsigned kb = __ballot_sync(0xffffffffu, keep);
-          if (keep) {
-            ck[cnt + __popc(kb & lt)] = u;
-            ci[cnt + __popc(kb & lt)] = t0 + i;
-          }
-          cnt += __popc(kb);
+          if (keep) ci[c + __popc(kb & lt)] = t0 + i;
+          c += __popc(kb);
         }
-        if (lane == 0) p.cand_count[slot * kWarps + warp] = bad ? 0 : cnt;
+        cnt[hh] = c;
+        if (lane == 0) p.cand_count[slot * kWarps + warp] = bad ? 0 : c;
+      }
+      __syncwarp();
+      int tot = 0;
+#pragma unroll
+      for (int hh = 0; hh < G; ++hh) tot += cnt[hh];
+      constexpr int kBatch = 4;
+      for (int q0 = 0; q0 < tot; q0 += 32 * kBatch) {
+        int hs[kBatch], rs[kBatch];
+        uint4 rows[kBatch][4];  // compact rows of up to 32 columns (W <= 32 here; longer rows loop below)
+        const int W8 = W / 8;
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          int q = q0 + u * 32 + lane, hh = 0;
+          hs[u] = -1;
+          if (q < tot) {
+#pragma unroll
+            for (int h2 = 0; h2 < G; ++h2) {
+              if (hs[u] < 0) {
+                if (q < cnt[h2]) { hs[u] = h2; rs[u] = q; } else { q -= cnt[h2]; }
+              }
+            }
+            (void)hh;
+          }
+          if (hs[u] >= 0 && W8 <= 4) {
+            const size_t slot = ((size_t)b * p.Hq + g * G + hs[u]) * p.nchunks + chunk;
+            const int t = p.cand_idx[slot * C + (size_t)warp * S + rs[u]];
+            const uint4* kr = reinterpret_cast<const uint4*>(kfc_rows + (size_t)t * W);
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8)
+              if (q8 < W8) rows[u][q8] = __ldg(kr + q8);
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < kBatch; ++u) {
+          if (hs[u] < 0) continue;
+          const int hh = hs[u];
+          const size_t slot = ((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk;
+          double sc = 0.0;
+          if (W8 <= 4) {
+#pragma unroll
+            for (int q8 = 0; q8 < 4; ++q8) {
+              if (q8 >= W8) break;
+              const uint32_t w[4] = {rows[u][q8].x, rows[u][q8].y, rows[u][q8].z, rows[u][q8].w};
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float kv = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+                sc = fma((double)qd[(q8 * 8 + e) * G + hh], (double)kv, sc);
+              }
+            }
+          } else {
+            const int t = p.cand_idx[slot * C + (size_t)warp * S + rs[u]];
+            const uint4* kr = reinterpret_cast<const uint4*>(kfc_rows + (size_t)t * W);
+            for (int q8 = 0; q8 < W8; ++q8) {
+              const uint4 v = __ldg(kr + q8);
+              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float kv = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
+                sc = fma((double)qd[(q8 * 8 + e) * G + hh], (double)kv, sc);
+              }
+            }
+          }
+          p.cand_key[slot * C + (size_t)warp * S + rs[u]] = order_key64(sc);
+        }
       }
     }
     if (bad && tid == 0) report(p.status, SFA_ERR_TIMEOUT);
@@ -486,15 +550,15 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
 }
 
 // ---------------------------------------------------------------------------
-// tip_merge: CTA per (b, h).  The chunks' candidates (token order, counts per
-// chunk) are staged in shared memory when they fit (kMergeSmem); bounded again
-// (with k <= 256, the least of the 256 threads' maxima is at most the k-th
-// largest), compacted, and the exact k-th largest found by block bisection;
-// the first k by (key desc, index asc) are written ascending.  More
-// candidates than fit use the block radix select over global memory.
+// tip_merge: CTA per (b, h).  The chunks' candidates (token order, float64
+// keys, counts per warp segment) are staged in shared memory when they fit
+// (kMergeSmem); with k <= 256 the least of the 256 threads' maxima is at most
+// the k-th largest key (each maximum is a distinct candidate), so only keys at
+// or above it survive; the exact k-th largest of the survivors by radix
+// select; the first k by (key desc, index asc) are written ascending.  More
+// candidates than fit use the same select over global memory.
 // ---------------------------------------------------------------------------
 constexpr int kMergeSmem = 12288;
-constexpr int kWarpSel = 64;  // survivors per lane for the single-warp exact threshold (2048 in all)
 constexpr int kMaxChunks = 512;
 
 __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
@@ -505,7 +569,7 @@ __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nseg = p.nchunks * kWarps;
   const int S = p.chunk / kWarps;
-  const uint32_t* ck = p.cand_key + row * p.nchunks * p.chunk;
+  const uint64_t* ck = p.cand_key + row * p.nchunks * p.chunk;
   const int* ci = p.cand_idx + row * p.nchunks * p.chunk;
   const int* cc = p.cand_count + row * nseg;
   int* out = p.idx + row * p.k;
@@ -550,10 +614,9 @@ __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
   int kept;
   const int ob = (nseg + 1 + 3) & ~3;  // keys start after the offsets (16-byte aligned)
   if (n <= kMergeSmem) {
-    uint32_t* sk = msm + ob;                              // [n] keys
-    int* st = reinterpret_cast<int*>(sk + n);             // [n] token indices
-    int* sv = st + n;                                     // [n] survivor positions
-    uint32_t* gk = reinterpret_cast<uint32_t*>(sv + n);   // [n] survivor keys
+    uint64_t* sk = reinterpret_cast<uint64_t*>(msm + ob);  // [n] keys
+    int* st = reinterpret_cast<int*>(sk + n);              // [n] token indices
+    int* sv = st + n;                                      // [n] survivor positions
     // segment-wise copies: warp w takes segments w, w + 8, ...; lanes stride each segment
     for (int sg = warp; sg < nseg; sg += kWarps) {
       const int o = off[sg], cnt = off[sg + 1] - o;
@@ -568,98 +631,33 @@ __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
       for (int i = tid; i < n; i += kThreads) out[i] = st[i];
       kept = n;
     } else {
-      uint32_t LB = 0u;
+      uint64_t LB = 0u;
       if (p.k <= kThreads) {
-        // the least of the 256 threads' maxima is at most the k-th largest when k <= 256
-        uint32_t m = 0u;
+        uint64_t m = 0u;
         for (int i = tid; i < n; i += kThreads) m = max(m, sk[i]);
-        m = __reduce_min_sync(0xffffffffu, m);
-        if (lane == 0) sh[warp] = (int)m;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = min(m, __shfl_xor_sync(0xffffffffu, m, o));
         __syncthreads();
-        LB = 0xFFFFFFFFu;
-        for (int w = 0; w < kWarps; ++w) LB = min(LB, (uint32_t)sh[w]);
+        if (lane == 0) reinterpret_cast<uint64_t*>(hist)[warp] = m;
+        __syncthreads();
+        LB = ~0ull;
+        for (int w = 0; w < kWarps; ++w) LB = min(LB, reinterpret_cast<const uint64_t*>(hist)[w]);
         __syncthreads();
       }
-      const int ns = block_filter_ordered([&](int i) { return sk[i]; }, n, LB, [&](int r, int i) { sv[r] = i; },
-                                          sh + 16);
-      __syncthreads();
-      for (int j = tid; j < ns; j += kThreads) gk[j] = sk[sv[j]];
-      __syncthreads();
-      int gt = 0;
-      uint32_t T;
-      if (ns <= 32 * kWarpSel) {
-        // few survivors: one warp finds the k-th largest in registers, no barriers per step
-        if (warp == 0) {
-          uint32_t v[kWarpSel];
-          uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-#pragma unroll
-          for (int j = 0; j < kWarpSel; ++j) {
-            const int q = j * 32 + lane;
-            v[j] = q < ns ? gk[q] : 0u;
-            if (q < ns) { mn = min(mn, v[j]); mx = max(mx, v[j]); }
-          }
-          mn = __reduce_min_sync(0xffffffffu, mn);
-          mx = __reduce_max_sync(0xffffffffu, mx);
-          uint64_t lo = mn, hi = (uint64_t)mx + 1;  // #{>= lo} >= k, #{>= hi} < k (padding 0 < mn)
-          while (hi - lo > 1) {
-            const uint32_t mid = (uint32_t)(lo + ((hi - lo) >> 1));
-            int c = 0;
-#pragma unroll
-            for (int j = 0; j < kWarpSel; ++j) c += (j * 32 + lane < ns && v[j] >= mid) ? 1 : 0;
-            if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= p.k) lo = mid; else hi = mid;
-          }
-          int g2 = 0;
-#pragma unroll
-          for (int j = 0; j < kWarpSel; ++j) g2 += (j * 32 + lane < ns && v[j] > (uint32_t)lo) ? 1 : 0;
-          g2 = (int)__reduce_add_sync(0xffffffffu, (unsigned)g2);
-          if (lane == 0) { sh[30] = (int)(uint32_t)lo; sh[31] = g2; }
-        }
-        __syncthreads();
-        T = (uint32_t)sh[30];
-        gt = sh[31];
-        __syncthreads();
+      int ns = n;
+      if (LB > 0u) {
+        ns = block_filter_ordered<uint64_t>([&](int i) { return sk[i]; }, n, LB, [&](int r, int i) { sv[r] = i; },
+                                            sh + 16);
       } else {
-        T = block_kth_largest_smem(gk, ns, p.k, sh, &gt);
+        for (int i = tid; i < n; i += kThreads) sv[i] = i;
       }
-      const int take = p.k - gt;
-      // ordered emission over the survivors with ties by index
-      const unsigned lt = (1u << lane) - 1u;
-      const int SW = ((ns + kWarps * 32 - 1) / (kWarps * 32)) * 32;
-      const int w0 = min(ns, warp * SW), w1 = min(ns, w0 + SW);
-      int nt = 0;
-      for (int b = w0; b < w1; b += 32) {
-        const int j = b + lane;
-        nt += __popc(__ballot_sync(0xffffffffu, j < w1 && gk[j] == T));
-      }
-      int tot = 0;
-      const int tie_base = warp_exclusive_sum(nt, sh + 16, &tot);
-      int nk = 0, tr = tie_base;
-      for (int b = w0; b < w1; b += 32) {
-        const int j = b + lane;
-        const uint32_t u = j < w1 ? gk[j] : 0u;
-        const bool tie = j < w1 && u == T;
-        const unsigned tb = __ballot_sync(0xffffffffu, tie);
-        const bool keep = j < w1 && (u > T || (tie && tr + __popc(tb & lt) < take));
-        nk += __popc(__ballot_sync(0xffffffffu, keep));
-        tr += __popc(tb);
-      }
-      int pos = warp_exclusive_sum(nk, sh + 16, &kept);
-      tr = tie_base;
-      for (int b = w0; b < w1; b += 32) {
-        const int j = b + lane;
-        const uint32_t u = j < w1 ? gk[j] : 0u;
-        const bool tie = j < w1 && u == T;
-        const unsigned tb = __ballot_sync(0xffffffffu, tie);
-        const bool keep = j < w1 && (u > T || (tie && tr + __popc(tb & lt) < take));
-        const unsigned kb = __ballot_sync(0xffffffffu, keep);
-        if (keep) out[pos + __popc(kb & lt)] = st[sv[j]];
-        pos += __popc(kb);
-        tr += __popc(tb);
-      }
+      __syncthreads();
+      kept = block_select_ordered<uint64_t>([&](int j) { return sk[sv[j]]; }, ns, p.k,
+                                            [&](int r, int j) { out[r] = st[sv[j]]; }, hist, sh);
     }
   } else {
-    kept = block_select_ordered([&](int i) { return __ldg(ck + locate(i)); }, n, p.k,
-                                [&](int r, int i) { out[r] = __ldg(ci + locate(i)); }, hist, sh);
+    kept = block_select_ordered<uint64_t>([&](int i) { return __ldg(ck + locate(i)); }, n, p.k,
+                                          [&](int r, int i) { out[r] = __ldg(ci + locate(i)); }, hist, sh);
   }
   for (int r = kept + tid; r < p.k; r += kThreads) out[r] = -1;
 }

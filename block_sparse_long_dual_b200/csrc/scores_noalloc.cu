@@ -19,9 +19,22 @@ constexpr int kMaxDevices = 64;
 
 static __device__ __align__(256) unsigned char g_scores_scratch[kScratchBytes];
 
-std::once_flag g_once[kMaxDevices];
-void* g_scratch_ptr[kMaxDevices];
-cudaError_t g_scratch_err[kMaxDevices];
+std::mutex g_lock;
+void* g_scratch_ptr[kMaxDevices];  // set once a lookup on that device succeeded
+
+// The scratch array's device address on the current device `dev`, looked up on first use.  Only a
+// successful lookup is cached, so a lookup that failed (for instance a first call made while the
+// stream was being captured, which is refused before any lookup) is retried by the next call.
+void* scratch_address(int dev, cudaStream_t stream) {
+  std::lock_guard<std::mutex> guard(g_lock);
+  if (g_scratch_ptr[dev] != nullptr) return g_scratch_ptr[dev];
+  cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(stream, &cap) != cudaSuccess || cap != cudaStreamCaptureStatusNone) return nullptr;
+  void* ptr = nullptr;
+  if (cudaGetSymbolAddress(&ptr, g_scores_scratch) != cudaSuccess) return nullptr;
+  g_scratch_ptr[dev] = ptr;
+  return ptr;
+}
 
 }  // namespace
 
@@ -35,12 +48,10 @@ extern "C" sfa_status sfa_block_scores_noalloc(const sfa_shape* shape, const voi
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return SFA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return SFA_ERR_UNSUPPORTED;
-  std::call_once(g_once[dev], [dev] {
-    g_scratch_err[dev] = cudaGetSymbolAddress(&g_scratch_ptr[dev], g_scores_scratch);
-  });
-  if (g_scratch_err[dev] != cudaSuccess || g_scratch_ptr[dev] == nullptr) return SFA_ERR_CUDA;
+  void* scratch = scratch_address(dev, static_cast<cudaStream_t>(stream));
+  if (scratch == nullptr) return SFA_ERR_CUDA;
   // Every scratch region (block means, energies, temperatures) is fully written by the
   // kernels before it is read, so nothing left by an earlier call needs clearing.
-  return sfa_block_scores(shape, Q, K, rope, band_split, block, flags, Q_rot, K_rot, probs, g_scratch_ptr[dev],
+  return sfa_block_scores(shape, Q, K, rope, band_split, block, flags, Q_rot, K_rot, probs, scratch,
                           kScratchBytes, stream);
 }

@@ -110,6 +110,8 @@ sfa_status sfa_rope_table(double base, int seq_len, int head_dim, float* cos, fl
  *              sum_t ||x_t^H||^2, sum_t ||x_t^L||^2, ||xbar^H||^2, ||xbar^L||^2
  *              (Q heads first, then KV heads)
  *   [3] tau    [B, heads_q, 2] float64  (band H, band L)
+ * followed, for head_dim 128, by internal scratch of the tensor-core block
+ * logits (int8 digit slices of the block means; not part of the layout).
  */
 size_t sfa_block_scores_workspace(const sfa_shape* shape, int block);
 
@@ -146,9 +148,13 @@ sfa_status sfa_workspace_layout(const sfa_shape* shape, int block, size_t offset
  * band's part of s_ij gets its own causal softmax p^b; then
  * probs_ij = max_b p^b_ij / sum_{j' <= i} max_b p^b_ij'.  With one band (band
  * H or L empty, or SFA_SINGLE_BAND) it changes nothing.
- * RoPE is applied in float32; block means, energies, temperatures, logits and
- * the softmax are float64 (the 1/tau calibration amplifies pooled logits, so
+ * RoPE is applied in float32; block means, energies, temperatures and the
+ * softmax are float64 (the 1/tau calibration amplifies pooled logits, so
  * float32 sums would move probabilities by ~1e-6), rounded once to float32.
+ * Logits are float64 products of the means, or, for head_dim 128 without
+ * SFA_BAND_MAX / SFA_BLOCK_TAU, exact int8 tensor-core products of five 7-bit
+ * digit slices of the means (a power-of-two scale per block), within 2^-26 of
+ * the product of the two blocks' scales.
  *
  * workspace: device buffer of at least sfa_block_scores_workspace() bytes,
  * 256-byte aligned; its contents are documented above and may be read back.
@@ -188,18 +194,20 @@ sfa_status sfa_block_scores_select(const sfa_shape* shape, const void* Q, const 
  * latency-bound loops that must not risk the implicit device synchronisation
  * an allocation can cause.  This entry point takes the same arguments minus
  * the workspace; it uses a fixed scratch array of SFA_NOALLOC_SCRATCH_BYTES
- * (16 MiB) that the library declares in device memory, so every GPU that
- * loads the library holds those 16 MiB until the process exits.  It calls no
+ * (32 MiB) that the library declares in device memory, so every GPU that
+ * loads the library holds those 32 MiB until the process exits.  It calls no
  * cudaMalloc, cudaFree or allocating library routine.
  *
  * Limit: shapes whose sfa_block_scores_workspace() exceeds
  * SFA_NOALLOC_SCRATCH_BYTES are rejected with SFA_ERR_WORKSPACE (e.g. the
- * 32 query / 8 KV head, d = 128, block = 128 layer fits up to L = 32768 per
+ * 32 query / 8 KV head, d = 128, block = 128 layer fits up to L = 61440 per
  * batch element).  The caller still passes Q, K, Q_rot, K_rot and probs.
  *
  * The first call on a device looks up the scratch array's device address
- * (cudaGetSymbolAddress, with that device current) and caches it; make that
- * first call before any stream capture.  All calls on a device share the one
+ * (cudaGetSymbolAddress, with that device current) and caches it once the
+ * lookup succeeds; make that first call before any stream capture (a first
+ * call on a stream that is being captured returns SFA_ERR_CUDA and launches
+ * nothing; the lookup is tried again by the next call).  All calls on a device share the one
  * scratch array and it keeps the last call's contents: calls whose kernels
  * overlap on the GPU (different streams, no ordering between them) race on it
  * and give wrong results.  Serialise such calls, e.g. issue them on one stream.
@@ -207,7 +215,7 @@ sfa_status sfa_block_scores_select(const sfa_shape* shape, const void* Q, const 
  * clearing between calls.  Errors: as sfa_block_scores, plus SFA_ERR_WORKSPACE
  * for shapes over the limit and SFA_ERR_UNSUPPORTED for device ordinals >= 64.
  */
-#define SFA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
+#define SFA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
 sfa_status sfa_block_scores_noalloc(const sfa_shape* shape, const void* Q, const void* K,
                                     const sfa_rope* rope, int band_split, int block, unsigned flags,
                                     void* Q_rot, void* K_rot, float* probs, void* stream);
@@ -304,15 +312,17 @@ size_t sfa_decode_workspace(const sfa_shape* shape, int k);
 /*
  * Token Importance Predictor (§2B.1): for Q head h of KV group g,
  *   s_t = sum_{m in fc[g]} q_m k_{t,m} + q_{m+d/2} k_{t,m+d/2}
- * from K_fc, as a float32 sum over the compact columns in order (column 0
- * first, one rounding per step; each bf16 x bf16 product is exact), then the
- * first min(k, L) tokens by (s desc, index asc).  idx [B, heads_q, k] int32: the kept
- * token indices ascending, padded with -1.  k >= 1.  workspace: device, at
- * least sfa_decode_workspace() bytes, 256-byte aligned (SFA_ERR_WORKSPACE).
- * status_word (device, nullable): SFA_ERR_TIMEOUT if a copy of the compact
- * keys did not land within about 2 s (that chunk then contributes no tokens).
- * Launches 2 kernels: a persistent one (per chunk of the cache: scores, a
- * lower bound of the chunk's k-th largest, the tokens above it) and a merge
+ * from K_fc, ranked by its float64 value (each bf16 x bf16 product is exact
+ * in float64), then the first min(k, L) tokens by (s desc, index asc).  A
+ * float32 copy of s serves only as a filter, with a margin of twice its
+ * rounding bound, so it never drops a token of the top k (finite inputs).
+ * idx [B, heads_q, k] int32: the kept token indices ascending, padded with -1.
+ * k >= 1.  workspace: device, at least sfa_decode_workspace() bytes, 256-byte
+ * aligned (SFA_ERR_WORKSPACE).  status_word (device, nullable):
+ * SFA_ERR_TIMEOUT if a copy of the compact keys did not land within about 2 s
+ * (that chunk then contributes no tokens).  Launches 2 kernels: a persistent
+ * one (per chunk of the cache: float32 scores, a lower bound of the chunk's
+ * k-th largest, the tokens above it with their float64 scores) and a merge
  * (exact top k of the candidates).
  */
 sfa_status sfa_decode_select(const sfa_shape* shape, const void* q, const void* K_fc, const int* fc,

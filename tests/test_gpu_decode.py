@@ -1,8 +1,10 @@
 """GPU decode step (token importance on dominant rotary pairs -> top-k -> focused attention)
 against the CPU oracle ("FASA: Frequency-aware Sparse Attention" §2B), through the C ABI.
 
-The compact key copy and the index lists are compared bit for bit (both sides rank the same
-float32 column-order sum of exact bf16 products); outputs within the bf16 tolerance."""
+The compact key copy is compared bit for bit.  Both sides rank the float64 dot product over the
+dominant pairs (each bf16 x bf16 product exact); index lists must equal the oracle's, tokens
+within 1e-6 relative of a row's k-th score being interchangeable (counted and bounded); outputs
+within the bf16 tolerance on rows whose lists are identical."""
 
 import numpy as np
 import pytest
@@ -12,6 +14,7 @@ from block_sparse_long_dual_b200 import sfa
 from block_sparse_long_dual_b200.synthetic import make_decode_inputs
 from block_sparse_long_dual_b200.workloads import FASA_DECODE_128K_B4, DecodeWorkload
 from oracle import fasa_oracle as fo
+from tests.parity import compare_token_lists
 
 pytestmark = pytest.mark.gpu
 
@@ -35,8 +38,8 @@ CASES = [
 ]
 
 
-def run(w: DecodeWorkload, seed=0):
-    q, K, V, fc = make_decode_inputs(w, seed=seed)
+def run(w: DecodeWorkload, seed=0, inputs=None):
+    q, K, V, fc = make_decode_inputs(w, seed=seed) if inputs is None else inputs
     dev = torch.device("cuda")
     m = sfa.FasaDecode(batch=w.batch, heads_q=w.heads_q, heads_kv=w.heads_kv, seq_len=w.seq_len,
                        head_dim=w.head_dim, fc=fc, k=w.k, device=dev)
@@ -47,22 +50,38 @@ def run(w: DecodeWorkload, seed=0):
     return m, q, K, V, fc
 
 
+def check_against_oracle(m, q, K, V, fc, k, max_excused_frac=0.01):
+    qn, Kn, Vn = (t.to(torch.float64).numpy() for t in (q, K, V))
+    s, idx, o, lse = fo.decode_step(qn, Kn, Vn, fc, k)
+    got = m.idx.cpu().numpy()
+    stats = compare_token_lists(got, s, k)
+    print(f"rows {stats['rows']}, near-tie rows excused {stats['excused_rows']}")
+    assert stats["mismatches"] == 0, stats["bad_rows"][:5]
+    assert stats["excused_rows"] <= max_excused_frac * stats["rows"]
+    same = (got == idx).all(-1)
+    assert int(m.status.item()) == 0
+    np.testing.assert_allclose(m.o.cpu().to(torch.float64).numpy()[same], o[same], rtol=0, atol=TOL_O)
+    np.testing.assert_allclose(m.lse.cpu().numpy()[same], lse[same], rtol=0, atol=1e-3)
+
+
 @pytest.mark.parametrize("w", CASES, ids=lambda w: w.name)
 def test_decode_matches_oracle(w):
     m, q, K, V, fc = run(w)
-    qn, Kn, Vn = (t.to(torch.float64).numpy() for t in (q, K, V))
     # compact key copy: exact
     np.testing.assert_array_equal(m.K_fc.cpu().view(torch.int16).numpy(),
                                   fo.gather_fc(K.view(torch.int16).numpy(), fc))
-    # selection: bit-exact
-    s, keys, idx, o, lse = fo.decode_step(qn, Kn, Vn, fc, w.k)
-    got = m.idx.cpu().numpy()
-    mism = np.argwhere((got != idx).any(-1))
-    assert mism.size == 0, f"rows differ: {mism[:5].tolist()}"
-    # attention over the kept tokens
-    assert int(m.status.item()) == 0
-    np.testing.assert_allclose(m.o.cpu().to(torch.float64).numpy(), o, rtol=0, atol=TOL_O)
-    np.testing.assert_allclose(m.lse.cpu().numpy(), lse, rtol=0, atol=1e-3)
+    check_against_oracle(m, q, K, V, fc, w.k)
+
+
+def test_identical_keys_merge_over_global_memory():
+    """Every cached key identical: all scores of a row tie, every token of every chunk is a
+    candidate (more than the merge stages in shared memory), and the first k by index win."""
+    w = D("identical-keys", heads_q=4, heads_kv=1, seq_len=20000, nfc=8, k=100, needle_frac=0.0)
+    q, K, V, fc = make_decode_inputs(w, seed=4)
+    K = K[:, :, :1].expand_as(K).contiguous()
+    m, q, K, V, fc = run(w, inputs=(q, K, V, fc))
+    assert np.all(m.idx.cpu().numpy() == np.arange(w.k)[None, None, :])
+    check_against_oracle(m, q, K, V, fc, w.k, max_excused_frac=0.0)
 
 
 def test_fc_gather_range_touches_only_that_range():
@@ -102,12 +121,15 @@ def test_decode_full_size_sampled_rows():
     w = FASA_DECODE_128K_B4
     m, q, K, V, fc = run(w, seed=3)
     rng = np.random.default_rng(0)
-    for _ in range(4):
+    for _ in range(6):
         b, h = int(rng.integers(w.batch)), int(rng.integers(w.heads_q))
         g = h // w.group
         qn = q[b:b + 1, h:h + 1].to(torch.float64).numpy()
         Kn = K[b:b + 1, g:g + 1].to(torch.float64).numpy()
         Vn = V[b:b + 1, g:g + 1].to(torch.float64).numpy()
-        s, keys, idx, o, lse = fo.decode_step(qn, Kn, Vn, fc[g:g + 1], w.k)
-        np.testing.assert_array_equal(m.idx[b, h].cpu().numpy(), idx[0, 0])
-        np.testing.assert_allclose(m.o[b, h].cpu().to(torch.float64).numpy(), o[0, 0], rtol=0, atol=TOL_O)
+        s, idx, o, lse = fo.decode_step(qn, Kn, Vn, fc[g:g + 1], w.k)
+        stats = compare_token_lists(m.idx[b:b + 1, h:h + 1].cpu().numpy(), s, w.k)
+        print(f"b={b} h={h}: near-tie excused {stats['excused_rows']}")
+        assert stats["mismatches"] == 0, stats["bad_rows"]
+        if np.array_equal(m.idx[b, h].cpu().numpy(), idx[0, 0]):
+            np.testing.assert_allclose(m.o[b, h].cpu().to(torch.float64).numpy(), o[0, 0], rtol=0, atol=TOL_O)

@@ -3,11 +3,12 @@
 Plugin code hosted by a runtime that owns all device memory, or code in a
 process whose memory another allocator has already reserved, cannot hand the
 library a scratch workspace.  The no-allocation variant keeps its scratch in a
-fixed 16 MiB device array inside the library.  This test calls it through the
-C ABI twice in a row (two different shapes, so the second call runs on
-scratch left over from the first) and checks each result against the
-workspace-taking sfa_block_scores, within the parity tolerances the other
-tests use, and checks that shapes over the limit are refused.
+fixed 32 MiB device array inside the library.  This test calls it through the
+C ABI twice in a row (a small shape, then a larger one, so the second call
+reads scratch regions the first did not cover and runs on what the first left)
+and checks each result against the workspace-taking sfa_block_scores: the
+same kernels on the same inputs, so the outputs must be identical bit for bit.
+It also checks that shapes over the limit are refused.
 
 The file name sorts last so that a run stopping at the first failure has
 already run every other test.
@@ -16,7 +17,6 @@ already run every other test.
 import ctypes
 from ctypes import POINTER, c_int, c_uint, c_void_p
 
-import numpy as np
 import pytest
 import torch
 
@@ -48,7 +48,7 @@ def test_no_alloc_matches_workspace_entry_point_twice():
     fn = _noalloc(lib)
     dev = torch.device("cuda")
     stream = torch.cuda.current_stream()
-    for w in (LLAMA_32K, TINY):   # two calls in a row, different shapes
+    for w in (TINY, LLAMA_32K):   # two calls in a row, the larger shape second
         Q, K, _ = make_inputs(w, seed=3)
         Qd, Kd = Q.to(dev), K.to(dev)
         cos, sin = sfa.rope_table(w.rope_base, w.seq_len, w.head_dim, device=dev)
@@ -63,11 +63,7 @@ def test_no_alloc_matches_workspace_entry_point_twice():
         assert rc == 0, lib.sfa_status_string(rc)
         torch.cuda.synchronize()
         assert torch.equal(Qr, Qr_ref) and torch.equal(Kr, Kr_ref)
-        a = P.double().cpu().numpy()
-        b = P_ref.double().cpu().numpy()
-        m = b > 1e-35
-        assert np.array_equal(a == 0, b == 0)
-        assert np.max(np.abs(a[m] - b[m]) / b[m]) <= 1e-6   # the probability tolerance of the parity tests
+        assert torch.equal(P, P_ref)
 
 
 def test_no_alloc_refuses_shapes_over_the_limit():
@@ -75,8 +71,8 @@ def test_no_alloc_refuses_shapes_over_the_limit():
         pytest.skip("no CUDA device")
     lib = sfa.load()
     fn = _noalloc(lib)
-    shape = sfa.Shape(1, 32, 8, 65536, 128, sfa.BF16)   # needs ~21 MiB of scratch
-    assert lib.sfa_block_scores_workspace(ctypes.byref(shape), 128) > (16 << 20)
+    shape = sfa.Shape(1, 32, 8, 65536, 128, sfa.BF16)   # needs ~33 MiB of scratch
+    assert lib.sfa_block_scores_workspace(ctypes.byref(shape), 128) > (32 << 20)
     d = ctypes.c_void_p(1 << 20)
     rope = sfa.Rope(d, d, 1)
     assert fn(ctypes.byref(shape), d, d, ctypes.byref(rope), 32, 128, 0, d, d, d, None) == SFA_ERR_WORKSPACE
