@@ -46,7 +46,7 @@ from block_sparse_long_dual_b200 import workloads as wl  # noqa: E402
 from block_sparse_long_dual_b200.synthetic import make_inputs  # noqa: E402
 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_STEP = 5  # rope_pool_energy, band_temperature, block_score_softmax, select, attention
+KERNELS_PER_STEP = 5  # rope_pool_energy, band_temperature, block_score_softmax, select, attention (4 when fused)
 
 
 def parse():
@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--workload", default=wl.LLAMA_128K.name, choices=sorted(wl.ALL) + sorted(wl.DECODE))
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=None)
+    ap.add_argument("--fused", action="store_true",
+                    help="estimate and selection in one call (sfa_block_scores_select; probabilities not stored)")
     return ap.parse_args()
 
 
@@ -77,20 +79,21 @@ def attention_flops(counts: np.ndarray, block: int, d: int) -> float:
     return float(4.0 * d * (block * block * (n - diag) + block * (block + 1) / 2.0 * diag).sum())
 
 
-def scoring_bytes(w: wl.Workload) -> float:
+def scoring_bytes(w: wl.Workload, store_probs: bool = True) -> float:
     """Algorithmic HBM bytes of sfa_block_scores: read Q, K; write Q_r, K_r; read the cos/sin
-    table once; write the float64 block means; write probs [B, Hq, nb, nb]."""
+    table once; write the float64 block means; write probs [B, Hq, nb, nb] (unless the selection
+    is fused and the probabilities are not stored)."""
     e = 2 if w.dtype == "bf16" else 4
     qk = w.batch * (w.heads_q + w.heads_kv) * w.seq_len * w.head_dim * e
     table = 2 * w.seq_len * (w.head_dim // 2) * 4
     means = w.batch * (w.heads_q + w.heads_kv) * w.nb * w.head_dim * 8
-    probs = w.batch * w.heads_q * w.nb * w.nb * 4
+    probs = w.batch * w.heads_q * w.nb * w.nb * 4 if store_probs else 0
     return float(2 * qk + table + means + probs)
 
 
-def select_bytes(w: wl.Workload, kmax: int) -> float:
-    """Read the causal triangle of probs, write counts and idx."""
-    tri = w.batch * w.heads_q * w.nb * (w.nb + 1) / 2 * 4
+def select_bytes(w: wl.Workload, kmax: int, read_probs: bool = True) -> float:
+    """Read the causal triangle of probs (unless the selection is fused), write counts and idx."""
+    tri = w.batch * w.heads_q * w.nb * (w.nb + 1) / 2 * 4 if read_probs else 0
     return float(tri + w.batch * w.heads_q * w.nb * (1 + kmax) * 4)
 
 
@@ -448,7 +451,8 @@ def main():
     Q, K, V = make_inputs(w, seed=rank)
     model = sfa.PrismAttention(batch=w.batch, heads_q=w.heads_q, heads_kv=w.heads_kv, seq_len=w.seq_len,
                                head_dim=w.head_dim, dtype=w.dtype, block=w.block, rope_base=w.rope_base,
-                               band_split=w.band_split, k=w.k, mass=w.mass, flags=w.flags, device=dev)
+                               band_split=w.band_split, k=w.k, mass=w.mass, flags=w.flags, device=dev,
+                               fused=args.fused)
     Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
@@ -467,9 +471,13 @@ def main():
         start.record(stream)
         for s in range(K_):
             ev[s][0].record(stream)
-            model.scores(Qd, Kd)
+            if args.fused:
+                model.scores_select(Qd, Kd)
+            else:
+                model.scores(Qd, Kd)
             ev[s][1].record(stream)
-            model.select()
+            if not args.fused:
+                model.select()
             ev[s][2].record(stream)
             model.attend(Vd)
             ev[s][3].record(stream)
@@ -530,13 +538,15 @@ def main():
         achieved = flops_step / (attn_ms * 1e-3) / 1e12
         peak = float(pk["bf16_tflops"])
         tr = traffic_record("block_sparse_long_dual_b200/csrc/attn_tc.cu")
-        sb, selb = scoring_bytes(w), select_bytes(w, model.kmax)
+        sb, selb = scoring_bytes(w, not args.fused), select_bytes(w, model.kmax, not args.fused)
         line = {
             "metric": "prefill attention effective TFLOP/s over kept blocks (whole path)",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K_, "warmup": args.warmup,
             "ms_per_step": total_ms / K_, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": w.dtype, "data": "synthetic",
             "config": {**layer_config(w, world), "kept_fraction": round(kept_frac, 5),
+                       "estimate": ("fused with the selection (sfa_block_scores_select, probabilities not stored)"
+                                    if args.fused else "sfa_block_scores then sfa_select"),
                        "l2": "inputs larger than L2 (Q 1.07 GB, K 0.27 GB, V 0.27 GB at 128K); no flush"},
             "stages_ms": {"block_scores": scores_ms, "select": select_ms, "attention": attn_ms},
             "scoring": {"bytes": sb + selb, "GB_s": (sb + selb) / ((scores_ms + select_ms) * 1e-3) / 1e9,
@@ -553,7 +563,7 @@ def main():
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "copies": "upload and download streams, double-buffered device inputs and outputs",
                     "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
-            "gpu_launches": KERNELS_PER_STEP * K_,
+            "gpu_launches": (KERNELS_PER_STEP - (1 if args.fused else 0)) * K_,
             "clocks": clk.summary(),
         }
         if world == 1 and not args.no_cpu_baseline:

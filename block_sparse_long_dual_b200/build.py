@@ -20,8 +20,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD_DIR = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libsfa.so")
 
-SOURCES = ["api.cu", "scores.cu", "score_i8.cu", "scores_noalloc.cu", "select.cu", "attn_simt.cu", "attn_tc.cu",
-           "decode.cu", "selftest.cu"]
+SOURCES = ["api.cu", "scores.cu", "scores_noalloc.cu", "select.cu", "attn_simt.cu", "attn_tc.cu", "decode.cu",
+           "selftest.cu"]
 HEADERS = ["common.cuh", "kernels.h", "tc_ptx.cuh", "select_row.cuh"]
 
 NVCC_FLAGS = [

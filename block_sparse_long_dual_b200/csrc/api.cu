@@ -44,12 +44,8 @@ sfa_status check_shape(const sfa_shape* s, int block, int* nb_out) {
   return SFA_OK;
 }
 
-// Workspace: the four arrays the header documents, then (head dim 128) the int8 digit slices
-// of the calibrated block means that the tensor-core block GEMM reads: query digits
-// [B, Hq, 5, nb, 128], key digits [B, Hkv, 5, nb, 128], int32 row exponents [B, Hq, nb] and
-// [B, Hkv, nb].
 struct WsLayout {
-  size_t off[8];
+  size_t off[4];
   size_t total;
 };
 
@@ -65,15 +61,6 @@ WsLayout ws_layout(const sfa_shape* s, int nb) {
   o = align256(o + (size_t)s->batch * (s->heads_q + s->heads_kv) * nb * 4 * sizeof(double));
   w.off[3] = o;
   o = align256(o + (size_t)s->batch * s->heads_q * 2 * sizeof(double));
-  const size_t dig = d == 128 ? 5 * d : 0, ex = d == 128 ? sizeof(int) : 0;
-  w.off[4] = o;
-  o = align256(o + (size_t)s->batch * s->heads_q * nb * dig);
-  w.off[5] = o;
-  o = align256(o + (size_t)s->batch * s->heads_kv * nb * dig);
-  w.off[6] = o;
-  o = align256(o + (size_t)s->batch * s->heads_q * nb * ex);
-  w.off[7] = o;
-  o = align256(o + (size_t)s->batch * s->heads_kv * nb * ex);
   w.total = o;
   return w;
 }
@@ -107,20 +94,6 @@ bool make_tile_map(CUtensorMap* m, const void* base, uint64_t rows) {
   const cuuint32_t box[2] = {64, 128};
   const cuuint32_t estr[2] = {1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// 3D int8 view [planes, rows, 128] of digit slices with 128-byte rows, boxes of box_rows rows of one
-// plane, 128-byte swizzle; rows past the plane's end read as zeros.
-bool make_digit_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t planes, uint32_t box_rows) {
-  EncodeTiledFn fn = encode_fn();
-  if (fn == nullptr) return false;
-  const cuuint64_t dims[3] = {128, rows, planes};
-  const cuuint64_t strides[2] = {128, rows * 128};
-  const cuuint32_t box[3] = {128, box_rows, 1};
-  const cuuint32_t estr[3] = {1, 1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
@@ -265,26 +238,6 @@ sfa_status run_block_scores(const sfa_shape* shape, const void* Q, const void* K
   tp.B = rp.B; tp.Hq = rp.Hq; tp.Hkv = rp.Hkv; tp.L = rp.L; tp.nb = nb; tp.flags = flags;
   st = cuda_status(launch_band_temperature(tp, cs));
   if (st != SFA_OK) return st;
-
-  // Head dim 128, one calibrated logit per block pair, probabilities stored: block logits on the
-  // int8 tensor cores from digit slices of the means.  The per-band-softmax and per-block
-  // temperature readings and the fused selection keep the float64 kernel.
-  if (D == 128 && fused == nullptr && !(flags & (SFA_BAND_MAX | SFA_BLOCK_TAU))) {
-    ScoreSliceParams sl;
-    sl.qbar = rp.qbar; sl.kbar = rp.kbar; sl.tau = tp.tau; sl.probs = probs; sl.status = nullptr;
-    sl.qd = reinterpret_cast<int8_t*>(ws + w.off[4]);
-    sl.kd = reinterpret_cast<int8_t*>(ws + w.off[5]);
-    sl.qe = reinterpret_cast<int*>(ws + w.off[6]);
-    sl.ke = reinterpret_cast<int*>(ws + w.off[7]);
-    sl.B = rp.B; sl.Hq = rp.Hq; sl.Hkv = rp.Hkv; sl.nb = nb; sl.band_pairs = band_pairs;
-    CUtensorMap tq, tk;
-    if (!make_digit_map(&tq, sl.qd, (uint64_t)nb, (uint64_t)rp.B * rp.Hq * 5, 128) ||
-        !make_digit_map(&tk, sl.kd, (uint64_t)nb, (uint64_t)rp.B * rp.Hkv * 5, 48))
-      return SFA_ERR_CUDA;
-    st = cuda_status(launch_score_slices(sl, cs));
-    if (st != SFA_OK) return st;
-    return cuda_status(launch_score_i8(sl, tq, tk, cs));
-  }
 
   ScoreParams sp;
   sp.qbar = rp.qbar; sp.kbar = rp.kbar; sp.tau = tp.tau; sp.energy = rp.energy; sp.probs = probs;

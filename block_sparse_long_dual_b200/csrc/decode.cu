@@ -7,8 +7,8 @@
 //   tip_chunk      Token Importance Predictor, persistent (one or two CTAs per
 //                  SM) over tiles (chunk of C tokens, b, KV head): the chunk's
 //                  K_fc rows stream through a bulk-copy ring once for all Q
-//                  heads of the group; each token's score is first taken as a
-//                  float32 FMA chain (a filter), then per head a lower bound
+//                  heads of the group; each token's score is first taken on
+//                  the tensor cores in float32 (a filter), then per head a lower bound
 //                  of the chunk's k-th largest score (from group maxima),
 //                  lowered by twice the float32 chain's rounding bound, and
 //                  the tokens at or above it (token order, per warp segment)
@@ -27,14 +27,16 @@
 // it is ranked by its float64 value (key = order-preserving uint64 of the
 // double, +0 for both zeros); the first k by (key desc, index asc).
 //
-// Why the float32 filter loses no token of the top k (finite inputs): each
-// bf16 x bf16 product is exact in float32, so a chain of n = 2 nfc FMAs is off
-// the exact score by at most M = n u sum_c |q_c k_c| + n 2^-150 (u = 2^-24;
-// the second term covers subnormal partial sums), and sum_c |q_c k_c| <=
-// ||q||_1 A, A = the largest |k| in the chunk's compact rows.  If at least k
-// tokens of a chunk have float32 scores >= x, they have exact scores >= x - M,
-// so the row's k-th largest exact score is >= x - M, and every token of the
-// row's top k has a float32 score >= x - 2M.
+// Why the float32 filter loses no token of the top k (finite inputs): the
+// filter score is a tensor-core sum of n = 2 nfc products, each exact (bf16 x
+// bf16); whatever the order and rounding of its float32 accumulation (even
+// truncation to 22 bits per addition), it is off the exact score by at most
+// n 2^-21 sum_c |q_c k_c| + n 2^-126 (the second term covers flushed
+// subnormals), below M = 2^-16 ||q||_1 A + n 2^-126 for n <= 128, where
+// sum_c |q_c k_c| <= ||q||_1 A and A = the largest |k| in the chunk's compact
+// rows.  If at least k tokens of a chunk have filter scores >= x, they have
+// exact scores >= x - M, so the row's k-th largest exact score is >= x - M,
+// and every token of the row's top k has a filter score >= x - 2M.
 #include <math.h>
 
 #include "common.cuh"
@@ -322,64 +324,60 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
     }
     __syncthreads();
 
-    // Filter scores: a float32 FMA chain per (token, head) over the columns in order.  Thread tid
-    // takes tokens tid + 256 u of each slab.  am: the largest |k| bit patterns of the chunk's
-    // compact values seen by this thread (two bf16 lanes; |x| orders like its bits for finite x).
+    // Filter scores on the tensor cores: per slab, warp w takes 16-token tiles of its share, the
+    // compact columns in k-steps of 8 (mma.sync m16n8k8, bf16 in, float32 out; A = tokens x
+    // columns straight from the slab, B = columns x heads, heads >= G zero).  The products are
+    // exact and the margin (see the top of this file) covers the accumulation's rounding.
+    // am: the largest |k| bit patterns of the chunk's compact values seen by this lane (two bf16
+    // halves; |x| orders like its bits for finite x).
     uint32_t am = 0u;
-    for (int sl = 0; sl < nsl; ++sl, ++consumed) {
-      const int stg = consumed % NS;
-      if (!wait_parity_bounded((uint32_t)__cvta_generic_to_shared(&bars[stg]), (consumed / NS) & 1)) lost = 1;
-      const __nv_bfloat16* slab = reinterpret_cast<const __nv_bfloat16*>(ring + (size_t)stg * SB);
-      float acc[TPS][G];
-      uint32_t vmask[TPS];
+    {
+      const int lane = tid & 31, warp = tid >> 5, gq = lane >> 2, tq = lane & 3;
+      const int KS = W / 8;
+      uint32_t qb[16];  // B fragments: {q[8 ks + 2 tq][gq], q[8 ks + 2 tq + 1][gq]} as bf16 pairs
 #pragma unroll
-      for (int u = 0; u < TPS; ++u) {
-        vmask[u] = sl * ST + u * kThreads + tid < n ? 0x7FFF7FFFu : 0u;
-#pragma unroll
-        for (int hh = 0; hh < G; ++hh) acc[u][hh] = 0.f;
+      for (int ks = 0; ks < 16; ++ks) {
+        qb[ks] = 0u;
+        if (ks < KS && gq < G)
+          qb[ks] = pack_bf16x2(qd[(8 * ks + 2 * tq) * G + gq], qd[(8 * ks + 2 * tq + 1) * G + gq]);
       }
-      for (int q8 = 0; q8 < W / 8; ++q8) {
-        uint32_t w4[TPS][4];
+      constexpr int MT = ST / 16 / kWarps;  // 16-token tiles per warp per slab
+      for (int sl = 0; sl < nsl; ++sl, ++consumed) {
+        const int stg = consumed % NS;
+        if (!wait_parity_bounded((uint32_t)__cvta_generic_to_shared(&bars[stg]), (consumed / NS) & 1)) lost = 1;
+        const unsigned char* slab = ring + (size_t)stg * SB;
 #pragma unroll
-        for (int u = 0; u < TPS; ++u) {
-          const uint4 v = reinterpret_cast<const uint4*>(slab + (size_t)(u * kThreads + tid) * W)[q8];
-          w4[u][0] = v.x; w4[u][1] = v.y; w4[u][2] = v.z; w4[u][3] = v.w;
+        for (int mt = 0; mt < MT; ++mt) {
+          const int r0 = (warp * MT + mt) * 16 + gq;  // slab rows r0 and r0 + 8
+          const int t0s = sl * ST + r0;               // their tokens in the chunk
+          const uint32_t m0 = t0s < n ? 0x7FFF7FFFu : 0u, m1 = t0s + 8 < n ? 0x7FFF7FFFu : 0u;
+          float c[4] = {0.f, 0.f, 0.f, 0.f};
+          const unsigned char* row0 = slab + (size_t)r0 * (2 * W) + 4 * tq;
+          const unsigned char* row1 = row0 + (size_t)8 * (2 * W);
 #pragma unroll
-          for (int e = 0; e < 4; ++e) am = __vmaxu2(am, w4[u][e] & vmask[u]);
-        }
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const int c = q8 * 8 + e;
-          float qv[G];
-          if constexpr (G % 4 == 0) {
-#pragma unroll
-            for (int h4 = 0; h4 < G; h4 += 4) {
-              const float4 f = *reinterpret_cast<const float4*>(qd + c * G + h4);
-              qv[h4] = f.x; qv[h4 + 1] = f.y; qv[h4 + 2] = f.z; qv[h4 + 3] = f.w;
-            }
-          } else {
-#pragma unroll
-            for (int hh = 0; hh < G; ++hh) qv[hh] = qd[c * G + hh];
+          for (int ks = 0; ks < 16; ++ks) {
+            if (ks >= KS) break;
+            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(row0 + 16 * ks);
+            const uint32_t a1 = *reinterpret_cast<const uint32_t*>(row1 + 16 * ks);
+            am = __vmaxu2(am, a0 & m0);
+            am = __vmaxu2(am, a1 & m1);
+            asm volatile(
+                "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+                "{%0, %1, %2, %3};"
+                : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                : "r"(a0), "r"(a1), "r"(qb[ks]));
           }
+          // c = scores of tokens (r0, r0 + 8) x heads (2 tq, 2 tq + 1)
 #pragma unroll
-          for (int u = 0; u < TPS; ++u) {
-            const uint32_t w = w4[u][e >> 1];
-            const float kv = __uint_as_float((e & 1) ? (w & 0xFFFF0000u) : (w << 16));
-#pragma unroll
-            for (int hh = 0; hh < G; ++hh) acc[u][hh] = fmaf(qv[hh], kv, acc[u][hh]);
+          for (int e = 0; e < 4; ++e) {
+            const int hh = 2 * tq + (e & 1);
+            const int t = t0s + (e >> 1) * 8;
+            if (hh < G && t < n) keys[(size_t)hh * C + t] = order_key(c[e]);
           }
         }
+        __syncthreads();  // stage consumed
+        if (tid == 0) issue_next();
       }
-#pragma unroll
-      for (int u = 0; u < TPS; ++u) {
-        const int t = sl * ST + u * kThreads + tid;
-        if (t < n) {
-#pragma unroll
-          for (int hh = 0; hh < G; ++hh) keys[(size_t)hh * C + t] = order_key(acc[u][hh]);
-        }
-      }
-      __syncthreads();  // stage consumed
-      if (tid == 0) issue_next();
     }
     {
       const uint32_t a16 = __reduce_max_sync(0xffffffffu, max(am & 0xFFFFu, am >> 16));
@@ -424,7 +422,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
             if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= p.k) lo = mid; else hi = mid;
           }
           LBw = (uint32_t)lo;
-          // M = n u ||q||_1 A + n 2^-150, every operation rounded up; then LB - 2M rounded down.
+          // M = 2^-16 ||q||_1 A + n 2^-126, every operation rounded up; then LB - 2M rounded down.
           float q1 = 0.f;
           for (int c = lane; c < W; c += 32) q1 = __fadd_ru(q1, fabsf(qd[c * G + warp]));
 #pragma unroll
@@ -433,7 +431,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
 #pragma unroll
           for (int w = 0; w < kWarps; ++w) a16 = max(a16, (uint32_t)scratch[64 + w]);
           const float A = __uint_as_float(a16 << 16);
-          const float M = __fadd_ru(__fmul_ru(__fmul_ru((float)W * 0x1p-24f, q1), A), (float)W * 0x1p-149f);
+          const float M = __fadd_ru(__fmul_ru(__fmul_ru(0x1p-16f, q1), A), (float)W * 0x1p-126f);
           if (LBw > 0u) LBw = order_key(__fsub_rd(key_value(LBw), __fmul_ru(2.f, M)));
         }
         if (lane == 0) scratch[warp] = (int)LBw;

@@ -48,21 +48,6 @@ struct ScoreParams {
   unsigned flags;
 };
 
-// Int8-slice block logits (score_i8.cu).
-struct ScoreSliceParams {
-  const double* qbar;
-  const double* kbar;
-  const double* tau;
-  int8_t* qd;    // [B, Hq, 5, nb, 128] digits of the calibrated query block means
-  int8_t* kd;    // [B, Hkv, 5, nb, 128] digits of the key block means
-  int* qe;       // [B, Hq, nb] row scale exponents
-  int* ke;       // [B, Hkv, nb]
-  float* probs;  // [B, Hq, nb, nb]
-  int* status;   // nullable
-  int B, Hq, Hkv, nb;
-  int band_pairs;
-};
-
 struct SelectParams {
   const float* probs;
   int* counts;
@@ -112,9 +97,6 @@ cudaError_t launch_band_temperature(const TauParams& p, cudaStream_t st);
 cudaError_t launch_block_score_softmax(const ScoreParams& p, int D, cudaStream_t st);
 size_t score_smem_bytes(int nb, int D, bool band_max);
 cudaError_t launch_select(const SelectParams& p, cudaStream_t st);
-cudaError_t launch_score_slices(const ScoreSliceParams& p, cudaStream_t st);
-cudaError_t launch_score_i8(const ScoreSliceParams& p, const CUtensorMap& tmQ, const CUtensorMap& tmK,
-                            cudaStream_t st);
 cudaError_t launch_attn_simt(const AttnParams& p, int dtype, int D, cudaStream_t st);
 struct DecodeGeometry {
   int chunk, tps, nstages, ctas_per_sm;

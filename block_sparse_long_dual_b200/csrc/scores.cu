@@ -28,16 +28,16 @@ namespace sfa {
 // K of each head (contiguous, 32 KB for bf16 d = 128) stream through an
 // NS-stage shared-memory ring filled by bulk asynchronous copies (mbarrier per
 // stage), so HBM reads stay in flight without holding registers.  Per head:
-// CH = D/16 threads cover one token (each owns 8 rotary pairs), NTH / CH
-// tokens per pass (NTH threads per CTA); RoPE in float32, the rotated row written back (input dtype,
+// CH = D/16 threads cover one token (each owns 8 rotary pairs), 256 / CH
+// tokens per pass; RoPE in float32, the rotated row written back (input dtype,
 // round to nearest even), per-thread partial sums reduced across threads in
 // float64 to the block mean and the per-band energies.
 // ---------------------------------------------------------------------------
-template <typename T, int D, int PASSES, int NS, int NTH>
-__global__ void __launch_bounds__(NTH, 1) rope_pool_energy_kernel(RopePoolParams p, int heads_per_cta) {
+template <typename T, int D, int PASSES, int NS>
+__global__ void __launch_bounds__(256, 1) rope_pool_energy_kernel(RopePoolParams p, int heads_per_cta) {
   constexpr int CH = D / 16;
-  constexpr int TPP = NTH / CH;  // tokens per pass
-  constexpr int NW = NTH / 32;
+  constexpr int TPP = 256 / CH;  // tokens per pass
+  constexpr int NW = 8;
   constexpr int BLK = TPP * PASSES;
   constexpr uint32_t XBYTES = BLK * D * sizeof(T);
   __shared__ double red[NW][D];
@@ -484,11 +484,11 @@ __global__ void __launch_bounds__(256, 1) block_score_softmax_kernel(ScoreParams
 // ---------------------------------------------------------------------------
 // Launchers
 // ---------------------------------------------------------------------------
-template <typename T, int D, int PASSES, int NTH>
+template <typename T, int D, int PASSES>
 static cudaError_t launch_rope_pool_tdp(const RopePoolParams& p, cudaStream_t st) {
   constexpr int NS = sizeof(T) == 2 ? 3 : 2;  // ring stages of one head's block rows
-  const size_t smem = (size_t)NS * (NTH / (D / 16)) * PASSES * D * sizeof(T);
-  auto kern = rope_pool_energy_kernel<T, D, PASSES, NS, NTH>;
+  const size_t smem = (size_t)NS * (256 / (D / 16)) * PASSES * D * sizeof(T);
+  auto kern = rope_pool_energy_kernel<T, D, PASSES, NS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   // Enough CTAs for about four waves of 148 SMs; each CTA reads the table slice once for its heads.
@@ -499,21 +499,15 @@ static cudaError_t launch_rope_pool_tdp(const RopePoolParams& p, cudaStream_t st
   const int per = (heads + groups - 1) / groups;
   groups = (heads + per - 1) / per;
   const unsigned grid = (unsigned)(blocks * groups);
-  kern<<<grid, NTH, smem, st>>>(p, per);
+  kern<<<grid, 256, smem, st>>>(p, per);
   return cudaGetLastError();
 }
 
 template <typename T>
 static cudaError_t launch_rope_pool_t(const RopePoolParams& p, int D, cudaStream_t st) {
-  // tokens per pass: NTH / (D / 16).  bf16, d = 128, block 128 (the long-context layers) runs
-  // 512 threads, two passes: twice the warps of a 256-thread CTA to hide the per-head
-  // reductions, half the table slice held per thread.
-  if (D == 128) {
-    if (p.block == 128)
-      return sizeof(T) == 2 ? launch_rope_pool_tdp<T, 128, 2, 512>(p, st) : launch_rope_pool_tdp<T, 128, 4, 256>(p, st);
-    return launch_rope_pool_tdp<T, 128, 2, 256>(p, st);
-  }
-  return p.block == 128 ? launch_rope_pool_tdp<T, 64, 2, 256>(p, st) : launch_rope_pool_tdp<T, 64, 1, 256>(p, st);
+  // tokens per pass: 256 / (D / 16) = 32 (D = 128) or 64 (D = 64)
+  if (D == 128) return p.block == 128 ? launch_rope_pool_tdp<T, 128, 4>(p, st) : launch_rope_pool_tdp<T, 128, 2>(p, st);
+  return p.block == 128 ? launch_rope_pool_tdp<T, 64, 2>(p, st) : launch_rope_pool_tdp<T, 64, 1>(p, st);
 }
 
 cudaError_t launch_rope_pool_energy(const RopePoolParams& p, int dtype, int D, cudaStream_t st) {

@@ -110,8 +110,6 @@ sfa_status sfa_rope_table(double base, int seq_len, int head_dim, float* cos, fl
  *              sum_t ||x_t^H||^2, sum_t ||x_t^L||^2, ||xbar^H||^2, ||xbar^L||^2
  *              (Q heads first, then KV heads)
  *   [3] tau    [B, heads_q, 2] float64  (band H, band L)
- * followed, for head_dim 128, by internal scratch of the tensor-core block
- * logits (int8 digit slices of the block means; not part of the layout).
  */
 size_t sfa_block_scores_workspace(const sfa_shape* shape, int block);
 
@@ -148,13 +146,9 @@ sfa_status sfa_workspace_layout(const sfa_shape* shape, int block, size_t offset
  * band's part of s_ij gets its own causal softmax p^b; then
  * probs_ij = max_b p^b_ij / sum_{j' <= i} max_b p^b_ij'.  With one band (band
  * H or L empty, or SFA_SINGLE_BAND) it changes nothing.
- * RoPE is applied in float32; block means, energies, temperatures and the
- * softmax are float64 (the 1/tau calibration amplifies pooled logits, so
+ * RoPE is applied in float32; block means, energies, temperatures, logits and
+ * the softmax are float64 (the 1/tau calibration amplifies pooled logits, so
  * float32 sums would move probabilities by ~1e-6), rounded once to float32.
- * Logits are float64 products of the means, or, for head_dim 128 without
- * SFA_BAND_MAX / SFA_BLOCK_TAU, exact int8 tensor-core products of five 7-bit
- * digit slices of the means (a power-of-two scale per block), within 2^-26 of
- * the product of the two blocks' scales.
  *
  * workspace: device buffer of at least sfa_block_scores_workspace() bytes,
  * 256-byte aligned; its contents are documented above and may be read back.
@@ -194,13 +188,13 @@ sfa_status sfa_block_scores_select(const sfa_shape* shape, const void* Q, const 
  * latency-bound loops that must not risk the implicit device synchronisation
  * an allocation can cause.  This entry point takes the same arguments minus
  * the workspace; it uses a fixed scratch array of SFA_NOALLOC_SCRATCH_BYTES
- * (32 MiB) that the library declares in device memory, so every GPU that
- * loads the library holds those 32 MiB until the process exits.  It calls no
+ * (16 MiB) that the library declares in device memory, so every GPU that
+ * loads the library holds those 16 MiB until the process exits.  It calls no
  * cudaMalloc, cudaFree or allocating library routine.
  *
  * Limit: shapes whose sfa_block_scores_workspace() exceeds
  * SFA_NOALLOC_SCRATCH_BYTES are rejected with SFA_ERR_WORKSPACE (e.g. the
- * 32 query / 8 KV head, d = 128, block = 128 layer fits up to L = 61440 per
+ * 32 query / 8 KV head, d = 128, block = 128 layer fits up to L = 32768 per
  * batch element).  The caller still passes Q, K, Q_rot, K_rot and probs.
  *
  * The first call on a device looks up the scratch array's device address
@@ -215,7 +209,7 @@ sfa_status sfa_block_scores_select(const sfa_shape* shape, const void* Q, const 
  * clearing between calls.  Errors: as sfa_block_scores, plus SFA_ERR_WORKSPACE
  * for shapes over the limit and SFA_ERR_UNSUPPORTED for device ordinals >= 64.
  */
-#define SFA_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+#define SFA_NOALLOC_SCRATCH_BYTES ((size_t)16 << 20)
 sfa_status sfa_block_scores_noalloc(const sfa_shape* shape, const void* Q, const void* K,
                                     const sfa_rope* rope, int band_split, int block, unsigned flags,
                                     void* Q_rot, void* K_rot, float* probs, void* stream);
