@@ -14,7 +14,7 @@
 //   warps 0 .. 8 KT - 1  softmax of tile w / 8: two threads per query row r
 //                    (TMEM lane r; warps w and w+4 share lanes), each owning 64
 //                    of the 128 key columns, row maxima exchanged through shared
-//                    memory; reads S_t from TMEM, online softmax with a lazily
+//                    memory (one barrier per warp pair); reads S_t from TMEM, online softmax with a lazily
 //                    rescaled O_t, writes P_t (bf16) back into the S_t columns of
 //                    TMEM, final O_t / l epilogue.  Two softmax warps per SM
 //                    sub-partition work on a tile at once, hiding each other's
@@ -47,9 +47,10 @@ constexpr int kHD = 128;
 constexpr uint32_t kSub = 16384;       // 128 rows x 64 bf16 (one 128B-swizzle box)
 constexpr uint32_t kTile = 2 * kSub;   // 128 x 128 bf16
 // Barriers, two of each (one per tile) except DRAIN and QR.
-enum { B_Q = 0, B_KF = 2, B_VF = 4, B_KE = 6, B_VE = 8, B_SF = 10, B_PF = 12, B_OD = 14, B_X = 16, B_DRAIN = 20,
-       B_QR = 21, NBAR = 22 };  // B_X: [tile][parity] row-max / row-sum exchange of the two column halves;
-                                // B_QR: the CTA's Q tiles rotated in shared memory (RoPE on load)
+enum { B_Q = 0, B_KF = 2, B_VF = 4, B_KE = 6, B_VE = 8, B_SF = 10, B_PF = 12, B_OD = 14, B_X = 16, B_DRAIN = 32,
+       B_QR = 33, NBAR = 34 };  // B_X: [tile][warp pair][parity] row-max / row-sum exchange of the two
+                                // column halves (warps w and w + 4, 64 arrivals); B_QR: the CTA's Q tiles
+                                // rotated in shared memory (RoPE on load)
 constexpr int kMaxList = 2048;  // nb <= 2048, so a valid list has <= 2048 entries
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
@@ -260,7 +261,7 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
       *cx.abort_flag = 0;
       for (int k = 0; k < NBAR; ++k)
         tc::mbar_init(cx.bar(k), k == B_QR ? KT * 256
-                                 : (k == B_PF || k == B_PF + 1 || (k >= B_X && k < B_X + 4)) ? 256 : 1);
+                                 : (k == B_PF || k == B_PF + 1) ? 256 : (k >= B_X && k < B_X + 16) ? 64 : 1);
       tc::fence_mbar_init();
     }
   } else if (warp == L::kProducerWarp && lane == 0) {
@@ -407,12 +408,13 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
     const uint32_t tP = tmem + lane_base + L::col_s(t) + 64 * hf;     // this half's P columns (2 bf16 each)
     const uint32_t tO = tmem + lane_base + L::col_o(t) + 64 * hf;     // this half's O columns
     float* xchg = reinterpret_cast<float*>(sm + L::OFF_XCHG) + t * 512;  // [parity][half][row]
-    // Exchange with the other half of the row: write, arrive on the tile's parity barrier (256
-    // arrivals), bounded wait, read.  Use u of parity q waits for phase parity (u / 2) & 1.
+    // Exchange with the other half of the row: write, arrive on the barrier of this warp pair
+    // (warps w and w + 4, 64 arrivals) and parity, bounded wait, read.  Use u of parity q waits for
+    // phase parity (u / 2) & 1.  A pair waits only for itself, not for the tile's other warps.
     auto exchange = [&](int use, float v) -> float {
       float* xc = xchg + (use & 1) * 256;
       xc[hf * 128 + r] = v;
-      const uint32_t xb = cx.bar(B_X + t * 2 + (use & 1));
+      const uint32_t xb = cx.bar(B_X + t * 8 + (warp & 3) * 2 + (use & 1));
       tc::mbar_arrive(xb);
       if (!wait_bar(cx, xb, (use >> 1) & 1)) return NAN;
       return xc[(1 - hf) * 128 + r];

@@ -141,22 +141,15 @@ __device__ int warp_exclusive_sum(int v, int* sh, int* total) {
   return before;
 }
 
-// Stable compaction of the first k keys by (key desc, index asc) out of n (k >= n keeps all):
-// emit(rank, i) for the kept i in ascending i, rank = 0, 1, ...  Returns the kept count.
+// Ordered emission of the first k keys by (key desc, index asc), given the k-th largest key T
+// and take = k - #{key > T} (the number of keys equal to T to keep, lowest index first); all keys
+// when all.  emit(rank, i) for the kept i in ascending i, rank = 0, 1, ...  Returns the kept count.
 // Warp w owns a contiguous range of 32-key groups; lane j takes key 32 g + j of each group, so
 // shared-memory reads are conflict-free and global reads coalesced; ranks come from ballots.
 template <typename Key, typename KeyAt, typename Emit>
-__device__ int block_select_ordered(KeyAt key_at, int n, int k, Emit emit, uint32_t* hist, int* sh) {
+__device__ int block_emit_ordered(KeyAt key_at, int n, bool all, Key T, int take, Emit emit, int* sh) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned lt = (1u << lane) - 1u;
-  Key T = 0;
-  int take = n;  // ties at T to keep (all when every key is kept)
-  const bool all = k >= n;
-  if (!all) {
-    int gt = 0;
-    T = block_kth_largest<Key>(key_at, n, k, hist, sh, &gt);
-    take = k - gt;
-  }
   const int S = ((n + kWarps * 32 - 1) / (kWarps * 32)) * 32;
   const int w0 = min(n, warp * S), w1 = min(n, w0 + S);
   int nt = 0;
@@ -166,7 +159,7 @@ __device__ int block_select_ordered(KeyAt key_at, int n, int k, Emit emit, uint3
       nt += __popc(__ballot_sync(0xffffffffu, i < w1 && key_at(i) == T));
     }
   int tot = 0;
-  const int tie_base = warp_exclusive_sum(nt, sh + 4, &tot);
+  const int tie_base = warp_exclusive_sum(nt, sh, &tot);
   int nk = 0, tr = tie_base;
   for (int b = w0; b < w1; b += 32) {
     const int i = b + lane;
@@ -178,7 +171,7 @@ __device__ int block_select_ordered(KeyAt key_at, int n, int k, Emit emit, uint3
     tr += __popc(tb);
   }
   int kept = 0;
-  int pos = warp_exclusive_sum(nk, sh + 4, &kept);
+  int pos = warp_exclusive_sum(nk, sh, &kept);
   tr = tie_base;
   for (int b = w0; b < w1; b += 32) {
     const int i = b + lane;
@@ -192,6 +185,81 @@ __device__ int block_select_ordered(KeyAt key_at, int n, int k, Emit emit, uint3
     tr += __popc(tb);
   }
   return kept;
+}
+
+// Stable compaction of the first k keys by (key desc, index asc) out of n (k >= n keeps all), the
+// threshold found by the block radix select.  Returns the kept count.
+template <typename Key, typename KeyAt, typename Emit>
+__device__ int block_select_ordered(KeyAt key_at, int n, int k, Emit emit, uint32_t* hist, int* sh) {
+  Key T = 0;
+  int take = n;
+  const bool all = k >= n;
+  if (!all) {
+    int gt = 0;
+    T = block_kth_largest<Key>(key_at, n, k, hist, sh, &gt);
+    take = k - gt;
+  }
+  return block_emit_ordered<Key>(key_at, n, all, T, take, emit, sh + 4);
+}
+
+// One warp, keys in registers (n <= 2048, 64 per lane): the k-th largest of n 64-bit keys
+// (1 <= k <= n) by bisection on their high 32 bits, then on the low 32 bits of the keys whose
+// high half equals the threshold's.  Returns T and sets *gt = #{key > T}.  All lanes must call it.
+template <typename KeyAt>
+__device__ uint64_t warp_kth_largest64(KeyAt key_at, int n, int k, int* gt) {
+  constexpr int V = 64;
+  const int lane = threadIdx.x & 31;
+  uint32_t v[V];
+  uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll
+  for (int q = 0; q < V; ++q) {
+    const int j = q * 32 + lane;
+    v[q] = j < n ? (uint32_t)(key_at(j) >> 32) : 0u;
+    if (j < n) { mn = min(mn, v[q]); mx = max(mx, v[q]); }
+  }
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  uint64_t lo = mn, hi = (uint64_t)mx + 1;  // #{high >= lo} >= k, #{high >= hi} < k
+  while (hi - lo > 1) {
+    const uint32_t mid = (uint32_t)(lo + ((hi - lo) >> 1));
+    int c = 0;
+#pragma unroll
+    for (int q = 0; q < V; ++q) c += (q * 32 + lane < n && v[q] >= mid) ? 1 : 0;
+    if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= k) lo = mid; else hi = mid;
+  }
+  const uint32_t th = (uint32_t)lo;
+  int g = 0;
+#pragma unroll
+  for (int q = 0; q < V; ++q) g += (q * 32 + lane < n && v[q] > th) ? 1 : 0;
+  g = (int)__reduce_add_sync(0xffffffffu, (unsigned)g);
+  const int need = k - g;  // >= 1 keys with high half th
+  // Low halves of the keys whose high half is th; the rest drop out of the second bisection.
+  bool in[V];
+  mn = 0xFFFFFFFFu;
+  mx = 0u;
+#pragma unroll
+  for (int q = 0; q < V; ++q) {
+    const int j = q * 32 + lane;
+    in[q] = j < n && v[q] == th;
+    v[q] = in[q] ? (uint32_t)key_at(j) : 0u;
+    if (in[q]) { mn = min(mn, v[q]); mx = max(mx, v[q]); }
+  }
+  mn = __reduce_min_sync(0xffffffffu, mn);
+  mx = __reduce_max_sync(0xffffffffu, mx);
+  lo = mn;
+  hi = (uint64_t)mx + 1;
+  while (hi - lo > 1) {
+    const uint32_t mid = (uint32_t)(lo + ((hi - lo) >> 1));
+    int c = 0;
+#pragma unroll
+    for (int q = 0; q < V; ++q) c += (in[q] && v[q] >= mid) ? 1 : 0;
+    if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= need) lo = mid; else hi = mid;
+  }
+  int g2 = 0;
+#pragma unroll
+  for (int q = 0; q < V; ++q) g2 += (in[q] && v[q] > (uint32_t)lo) ? 1 : 0;
+  *gt = g + (int)__reduce_add_sync(0xffffffffu, (unsigned)g2);
+  return ((uint64_t)th << 32) | (uint32_t)lo;
 }
 
 // Block-wide: emit(rank, i) for every i in [0, n) with key_at(i) >= LB, in ascending i; returns
@@ -267,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
   const int NS = p.nstages;
   const uint32_t SB = (uint32_t)ST * W * 2;                                                // slab bytes
   unsigned char* ring = smem_raw;                                                           // [NS][SB]
-  uint32_t* keys = reinterpret_cast<uint32_t*>(ring + (size_t)NS * SB);                   // [G][C]
+  uint16_t* keys = reinterpret_cast<uint16_t*>(ring + (size_t)NS * SB);                   // [G][C]
   float* qd = reinterpret_cast<float*>(keys + (size_t)G * C);                              // [W][G]
   __shared__ __align__(8) uint64_t bars[4];
   __shared__ int scratch[128];
@@ -372,7 +440,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
           for (int e = 0; e < 4; ++e) {
             const int hh = 2 * tq + (e & 1);
             const int t = t0s + (e >> 1) * 8;
-            if (hh < G && t < n) keys[(size_t)hh * C + t] = order_key(c[e]);
+            if (hh < G && t < n) keys[(size_t)hh * C + t] = (uint16_t)(order_key(c[e]) >> 16);
           }
         }
         __syncthreads();  // stage consumed
@@ -398,15 +466,15 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
       if (warp < G) {
         uint32_t LBw = 0u;
         if (p.k <= 32 * NGPL) {
-          const uint32_t* hk = keys + (size_t)warp * C;
+          const uint16_t* hk = keys + (size_t)warp * C;
           uint32_t gm[NGPL];
           uint32_t mn = 0xFFFFFFFFu, mx = 0u;
 #pragma unroll
           for (int j = 0; j < NGPL; ++j) {
             const int t = 4 * (j * 32 + lane);
-            const uint4 v = *reinterpret_cast<const uint4*>(hk + t);
-            const uint32_t m0 = t < n ? v.x : 0u, m1 = t + 1 < n ? v.y : 0u;
-            const uint32_t m2 = t + 2 < n ? v.z : 0u, m3 = t + 3 < n ? v.w : 0u;
+            const uint2 v = *reinterpret_cast<const uint2*>(hk + t);
+            const uint32_t m0 = t < n ? (v.x & 0xFFFFu) : 0u, m1 = t + 1 < n ? (v.x >> 16) : 0u;
+            const uint32_t m2 = t + 2 < n ? (v.y & 0xFFFFu) : 0u, m3 = t + 3 < n ? (v.y >> 16) : 0u;
             gm[j] = max(max(m0, m1), max(m2, m3));
             mn = min(mn, gm[j]);
             mx = max(mx, gm[j]);
@@ -432,7 +500,10 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
           for (int w = 0; w < kWarps; ++w) a16 = max(a16, (uint32_t)scratch[64 + w]);
           const float A = __uint_as_float(a16 << 16);
           const float M = __fadd_ru(__fmul_ru(__fmul_ru(0x1p-16f, q1), A), (float)W * 0x1p-126f);
-          if (LBw > 0u) LBw = order_key(__fsub_rd(key_value(LBw), __fmul_ru(2.f, M)));
+          // The stored keys are the high 16 bits of the float32 keys (rounded down), so LBw << 16
+          // bounds the true keys of those group maxima from below; the lowered bound is rounded
+          // down to 16 bits again for the comparison with the stored keys.
+          if (LBw > 0u) LBw = order_key(__fsub_rd(key_value(LBw << 16), __fmul_ru(2.f, M))) >> 16;
         }
         if (lane == 0) scratch[warp] = (int)LBw;
       }
@@ -441,7 +512,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
     uint32_t LB[G];
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) LB[hh] = (uint32_t)scratch[hh];
-    // Candidates in token order: warp w scans its contiguous range [w S, w S + S) of the chunk
+    // Candidates in token order (16-bit key at or above the 16-bit bound: a superset of the tokens
+    // whose float32 key reaches the bound): warp w scans its contiguous range [w S, w S + S) of the chunk
     // and writes its own segment of each head's slot (token indices); then it computes its
     // candidates' exact scores in float64, all heads together and four candidates per lane at a
     // time so that their compact rows (just streamed, so read from L2) are in flight together;
@@ -458,7 +530,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
       for (int hh = 0; hh < G; ++hh) {
         const size_t slot = ((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk;
         int* ci = p.cand_idx + slot * C + (size_t)warp * S;
-        const uint32_t* hk = keys + (size_t)hh * C;
+        const uint16_t* hk = keys + (size_t)hh * C;
         int c = 0;
         for (int b0 = w0; b0 < w1; b0 += 32) {
           const int i = b0 + lane;
@@ -615,13 +687,27 @@ __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
     uint64_t* sk = reinterpret_cast<uint64_t*>(msm + ob);  // [n] keys
     int* st = reinterpret_cast<int*>(sk + n);              // [n] token indices
     int* sv = st + n;                                      // [n] survivor positions
-    // segment-wise copies: warp w takes segments w, w + 8, ...; lanes stride each segment
-    for (int sg = warp; sg < nseg; sg += kWarps) {
-      const int o = off[sg], cnt = off[sg + 1] - o;
-      const size_t src = (size_t)sg * S;
-      for (int r = lane; r < cnt; r += 32) {
-        sk[o + r] = __ldg(ck + src + r);
-        st[o + r] = __ldg(ci + src + r);
+    // Flat copy: thread tid takes candidates tid, tid + 256, ... (segment by binary search), four
+    // at a time, so that hundreds of independent loads are in flight instead of one segment's.
+    for (int i0 = tid; i0 < n; i0 += 4 * kThreads) {
+      uint64_t kv[4];
+      int iv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kThreads;
+        if (i < n) {
+          const size_t at = locate(i);
+          kv[u] = __ldg(ck + at);
+          iv[u] = __ldg(ci + at);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int i = i0 + u * kThreads;
+        if (i < n) {
+          sk[i] = kv[u];
+          st[i] = iv[u];
+        }
       }
     }
     __syncthreads();
@@ -650,8 +736,26 @@ __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
         for (int i = tid; i < n; i += kThreads) sv[i] = i;
       }
       __syncthreads();
-      kept = block_select_ordered<uint64_t>([&](int j) { return sk[sv[j]]; }, ns, p.k,
-                                            [&](int r, int j) { out[r] = st[sv[j]]; }, hist, sh);
+      auto key_s = [&](int j) { return sk[sv[j]]; };
+      auto emit_s = [&](int r, int j) { out[r] = st[sv[j]]; };
+      if (ns <= 2048) {
+        // few survivors: one warp finds the k-th largest in registers, no block barriers per step
+        if (warp == 0) {
+          int gt = 0;
+          const uint64_t T = warp_kth_largest64(key_s, ns, p.k, &gt);
+          if (lane == 0) {
+            reinterpret_cast<uint64_t*>(hist)[0] = T;
+            sh[1] = p.k - gt;
+          }
+        }
+        __syncthreads();
+        const uint64_t T = reinterpret_cast<const uint64_t*>(hist)[0];
+        const int take = sh[1];
+        __syncthreads();
+        kept = block_emit_ordered<uint64_t>(key_s, ns, false, T, take, emit_s, sh + 4);
+      } else {
+        kept = block_select_ordered<uint64_t>(key_s, ns, p.k, emit_s, hist, sh);
+      }
     }
   } else {
     kept = block_select_ordered<uint64_t>([&](int i) { return __ldg(ck + locate(i)); }, n, p.k,
@@ -767,7 +871,7 @@ __global__ void __launch_bounds__(kFacWarps * 32) fac_kernel(DecodeParams p) {
 }  // namespace
 
 // Chunk geometry for a group size and compact row width: C tokens per chunk, TPS tokens per
-// thread per slab, NS ring stages; shared memory = NS slabs + G C keys + the query table.
+// thread per slab, NS ring stages; shared memory = NS slabs + G C 16-bit filter keys + the query table.
 DecodeGeometry decode_geometry(int group, int nfc) {
   DecodeGeometry d;
   const int W = 2 * nfc;
@@ -776,13 +880,13 @@ DecodeGeometry decode_geometry(int group, int nfc) {
   // Two CTAs per SM when the keys and a two-stage ring fit in half the shared memory (228 KB per
   // SM, 1 KB reserved per CTA, under 1 KB of static shared memory per CTA).
   size_t budget = 113 * 1024;
-  if ((size_t)group * 4096 * 4 + 2 * slab > budget) budget = 200 * 1024;
+  if ((size_t)group * 4096 * 2 + 2 * slab > budget) budget = 200 * 1024;
   d.chunk = 4096;
-  while (d.chunk > 1024 && (size_t)group * d.chunk * 4 + 2 * slab > budget) d.chunk /= 2;
-  d.nstages = (int)((budget - (size_t)group * d.chunk * 4) / slab);
+  while (d.chunk > 1024 && (size_t)group * d.chunk * 2 + 2 * slab > budget) d.chunk /= 2;
+  d.nstages = (int)((budget - (size_t)group * d.chunk * 2) / slab);
   d.nstages = d.nstages > 4 ? 4 : d.nstages;
   d.ctas_per_sm = budget < 150 * 1024 ? 2 : 1;
-  d.smem = d.nstages * slab + (size_t)group * d.chunk * 4 + (size_t)group * W * 4;
+  d.smem = d.nstages * slab + (size_t)group * d.chunk * 2 + (size_t)group * W * 4;
   return d;
 }
 
