@@ -395,7 +395,8 @@ size_t decode_ws_bytes(const DecodeParams& p, int /*k*/) {
   const size_t rows = (size_t)p.B * p.Hq;
   const size_t slots = rows * (((size_t)p.L + 4095) / 4096) * 4096;
   const size_t counts = rows * (((size_t)p.L + 1023) / 1024) * 8;
-  return align256(slots * sizeof(uint64_t)) + align256(slots * sizeof(int)) + align256(counts * sizeof(int));
+  const size_t margins = rows * (((size_t)p.L + 1023) / 1024);
+  return align256(slots * sizeof(uint32_t)) + align256(counts * sizeof(int)) + align256(margins * sizeof(float));
 }
 
 }  // namespace
@@ -432,9 +433,10 @@ sfa_status sfa_decode_select(const sfa_shape* shape, const void* q, const void* 
   const size_t n = (size_t)p.B * p.Hq * p.nchunks * p.chunk;
   unsigned char* ws = static_cast<unsigned char*>(workspace);
   p.q = q; p.Kfc = K_fc; p.idx = idx; p.k = k; p.status = status_word;
-  p.cand_key = reinterpret_cast<uint64_t*>(ws);
-  p.cand_idx = reinterpret_cast<int*>(ws + align256(n * sizeof(uint64_t)));
-  p.cand_count = reinterpret_cast<int*>(ws + align256(n * sizeof(uint64_t)) + align256(n * sizeof(int)));
+  const size_t cnts = (size_t)p.B * p.Hq * (((size_t)p.L + 1023) / 1024) * 8;
+  p.cand = reinterpret_cast<uint32_t*>(ws);
+  p.cand_count = reinterpret_cast<int*>(ws + align256(n * sizeof(uint32_t)));
+  p.cand_margin = reinterpret_cast<float*>(ws + align256(n * sizeof(uint32_t)) + align256(cnts * sizeof(int)));
   return cuda_status(launch_decode_select(p, as_stream(stream)));
 }
 

@@ -10,14 +10,17 @@
 //                  heads of the group; each token's score is first taken on
 //                  the tensor cores in float32 (a filter), then per head a lower bound
 //                  of the chunk's k-th largest score (from group maxima),
-//                  lowered by twice the float32 chain's rounding bound, and
-//                  the tokens at or above it (token order, per warp segment)
-//                  get their exact score recomputed in float64.
-//   tip_merge      CTA per (b, h): the candidates' float64 keys staged in
-//                  shared memory, bounded again, exact k-th largest by radix
-//                  select, ties by index; ascending index list, -1 padded (the
-//                  same select over global memory when the candidates do not
-//                  fit).
+//                  lowered by twice the filter's error bound M, and the tokens
+//                  at or above it (token order, per warp segment) as one word
+//                  each: 16-bit filter key << 16 | offset in the chunk; M is
+//                  recorded per (row, chunk).
+//   tip_merge      CTA per (b, h): the candidate words staged in shared memory,
+//                  the k-th largest filter key found by bisection and the
+//                  candidates bounded again with it, the survivors' exact
+//                  scores recomputed in float64 from the compact rows and
+//                  ranked (key desc, index asc); ascending index list, -1
+//                  padded (a radix select with scores recomputed on the fly
+//                  when the candidates do not fit).
 //   fac            Focused Attention Computation: CTA per (b, h), 16 warps,
 //                  each warp gathers the K / V rows of its share of the kept
 //                  tokens (eight tokens' loads in flight per lane), float32
@@ -262,31 +265,6 @@ __device__ uint64_t warp_kth_largest64(KeyAt key_at, int n, int k, int* gt) {
   return ((uint64_t)th << 32) | (uint32_t)lo;
 }
 
-// Block-wide: emit(rank, i) for every i in [0, n) with key_at(i) >= LB, in ascending i; returns
-// the count.  Warp-contiguous ranges of 32-key groups, ranks from ballots.
-template <typename Key, typename KeyAt, typename Emit>
-__device__ int block_filter_ordered(KeyAt key_at, int n, Key LB, Emit emit, int* sh) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const unsigned lt = (1u << lane) - 1u;
-  const int S = ((n + kWarps * 32 - 1) / (kWarps * 32)) * 32;
-  const int w0 = min(n, warp * S), w1 = min(n, w0 + S);
-  int nk = 0;
-  for (int b = w0; b < w1; b += 32) {
-    const int i = b + lane;
-    nk += __popc(__ballot_sync(0xffffffffu, i < w1 && key_at(i) >= LB));
-  }
-  int total = 0;
-  int pos = warp_exclusive_sum(nk, sh, &total);
-  for (int b = w0; b < w1; b += 32) {
-    const int i = b + lane;
-    const bool keep = i < w1 && key_at(i) >= LB;
-    const unsigned kb = __ballot_sync(0xffffffffu, keep);
-    if (keep) emit(pos + __popc(kb & lt), i);
-    pos += __popc(kb);
-  }
-  return total;
-}
-
 // ---------------------------------------------------------------------------
 // fc_gather
 // ---------------------------------------------------------------------------
@@ -464,6 +442,17 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
       const int lane = tid & 31, warp = tid >> 5;
       constexpr int NGPL = 8 * NGR;  // groups per lane: C / 4 / 32
       if (warp < G) {
+        // M = 2^-16 ||q||_1 A + n 2^-126, every operation rounded up (also recorded for the merge).
+        float q1 = 0.f;
+        for (int c = lane; c < W; c += 32) q1 = __fadd_ru(q1, fabsf(qd[c * G + warp]));
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) q1 = __fadd_ru(q1, __shfl_xor_sync(0xffffffffu, q1, off));
+        uint32_t a16 = 0u;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) a16 = max(a16, (uint32_t)scratch[64 + w]);
+        const float A = __uint_as_float(a16 << 16);
+        const float M = __fadd_ru(__fmul_ru(__fmul_ru(0x1p-16f, q1), A), (float)W * 0x1p-126f);
+        if (lane == 0) p.cand_margin[((size_t)b * p.Hq + g * G + warp) * p.nchunks + chunk] = M;
         uint32_t LBw = 0u;
         if (p.k <= 32 * NGPL) {
           const uint16_t* hk = keys + (size_t)warp * C;
@@ -490,20 +479,11 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
             if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= p.k) lo = mid; else hi = mid;
           }
           LBw = (uint32_t)lo;
-          // M = 2^-16 ||q||_1 A + n 2^-126, every operation rounded up; then LB - 2M rounded down.
-          float q1 = 0.f;
-          for (int c = lane; c < W; c += 32) q1 = __fadd_ru(q1, fabsf(qd[c * G + warp]));
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) q1 = __fadd_ru(q1, __shfl_xor_sync(0xffffffffu, q1, off));
-          uint32_t a16 = 0u;
-#pragma unroll
-          for (int w = 0; w < kWarps; ++w) a16 = max(a16, (uint32_t)scratch[64 + w]);
-          const float A = __uint_as_float(a16 << 16);
-          const float M = __fadd_ru(__fmul_ru(__fmul_ru(0x1p-16f, q1), A), (float)W * 0x1p-126f);
           // The stored keys are the high 16 bits of the float32 keys (rounded down), so LBw << 16
           // bounds the true keys of those group maxima from below; the lowered bound is rounded
           // down to 16 bits again for the comparison with the stored keys.
-          if (LBw > 0u) LBw = order_key(__fsub_rd(key_value(LBw << 16), __fmul_ru(2.f, M))) >> 16;
+          // (Keys under 0x0080 hold no finite score: no bound then.)
+          LBw = LBw >= 0x80u ? order_key(__fsub_rd(key_value(LBw << 16), __fmul_ru(2.f, M))) >> 16 : 0u;
         }
         if (lane == 0) scratch[warp] = (int)LBw;
       }
@@ -513,98 +493,41 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) LB[hh] = (uint32_t)scratch[hh];
     // Candidates in token order (16-bit key at or above the 16-bit bound: a superset of the tokens
-    // whose float32 key reaches the bound): warp w scans its contiguous range [w S, w S + S) of the chunk
-    // and writes its own segment of each head's slot (token indices); then it computes its
-    // candidates' exact scores in float64, all heads together and four candidates per lane at a
-    // time so that their compact rows (just streamed, so read from L2) are in flight together;
-    // counts per (slot, warp).
+    // whose float32 key reaches the bound): warp w scans its contiguous range [w S, w S + S) of the
+    // chunk, two tokens per lane per step and all heads at once, and writes its own segment of
+    // each head's slot (16-bit filter key << 16 | token offset in the chunk); counts per (slot,
+    // warp).  The merge rescores the candidates that survive its own bound.
     const int bad = lost;
     {
       const int lane = tid & 31, warp = tid >> 5;
       const unsigned lt = (1u << lane) - 1u;
       const int S = C / kWarps;
       const int w0 = min(n, warp * S), w1 = min(n, w0 + S);
-      const __nv_bfloat16* kfc_rows = kfc_all + (size_t)bg * p.L * W;
-      int cnt[G];
+      uint32_t* cw[G];
+      int c[G];
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
-        const size_t slot = ((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk;
-        int* ci = p.cand_idx + slot * C + (size_t)warp * S;
-        const uint16_t* hk = keys + (size_t)hh * C;
-        int c = 0;
-        for (int b0 = w0; b0 < w1; b0 += 32) {
-          const int i = b0 + lane;
-          const bool keep = i < w1 && hk[i] >= LB[hh];
-          const unsigned kb = __ballot_sync(0xffffffffu, keep);
-          if (keep) ci[c + __popc(kb & lt)] = t0 + i;
-          c += __popc(kb);
-        }
-        cnt[hh] = c;
-        if (lane == 0) p.cand_count[slot * kWarps + warp] = bad ? 0 : c;
+        cw[hh] = p.cand + (((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk) * C + (size_t)warp * S;
+        c[hh] = 0;
       }
-      __syncwarp();
-      int tot = 0;
+      for (int b0 = w0; b0 < w1; b0 += 64) {
+        const int i = b0 + 2 * lane;  // tokens i and i + 1 (w0 is even; the second is masked past w1)
 #pragma unroll
-      for (int hh = 0; hh < G; ++hh) tot += cnt[hh];
-      constexpr int kBatch = 4;
-      for (int q0 = 0; q0 < tot; q0 += 32 * kBatch) {
-        int hs[kBatch], rs[kBatch];
-        uint4 rows[kBatch][4];  // compact rows of up to 32 columns (W <= 32 here; longer rows loop below)
-        const int W8 = W / 8;
-#pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-          int q = q0 + u * 32 + lane, hh = 0;
-          hs[u] = -1;
-          if (q < tot) {
-#pragma unroll
-            for (int h2 = 0; h2 < G; ++h2) {
-              if (hs[u] < 0) {
-                if (q < cnt[h2]) { hs[u] = h2; rs[u] = q; } else { q -= cnt[h2]; }
-              }
-            }
-            (void)hh;
-          }
-          if (hs[u] >= 0 && W8 <= 4) {
-            const size_t slot = ((size_t)b * p.Hq + g * G + hs[u]) * p.nchunks + chunk;
-            const int t = p.cand_idx[slot * C + (size_t)warp * S + rs[u]];
-            const uint4* kr = reinterpret_cast<const uint4*>(kfc_rows + (size_t)t * W);
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8)
-              if (q8 < W8) rows[u][q8] = __ldg(kr + q8);
-          }
+        for (int hh = 0; hh < G; ++hh) {
+          const uint32_t pr = i < w1 ? *reinterpret_cast<const uint32_t*>(keys + (size_t)hh * C + i) : 0u;
+          const uint32_t u0 = pr & 0xFFFFu, u1 = pr >> 16;
+          const bool k0 = i < w1 && u0 >= LB[hh], k1 = i + 1 < w1 && u1 >= LB[hh];
+          const unsigned m0 = __ballot_sync(0xffffffffu, k0), m1 = __ballot_sync(0xffffffffu, k1);
+          const int at = c[hh] + __popc(m0 & lt) + __popc(m1 & lt);
+          if (k0) cw[hh][at] = (u0 << 16) | (uint32_t)i;
+          if (k1) cw[hh][at + (k0 ? 1 : 0)] = (u1 << 16) | (uint32_t)(i + 1);
+          c[hh] += __popc(m0) + __popc(m1);
         }
+      }
+      if (lane == 0) {
 #pragma unroll
-        for (int u = 0; u < kBatch; ++u) {
-          if (hs[u] < 0) continue;
-          const int hh = hs[u];
-          const size_t slot = ((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk;
-          double sc = 0.0;
-          if (W8 <= 4) {
-#pragma unroll
-            for (int q8 = 0; q8 < 4; ++q8) {
-              if (q8 >= W8) break;
-              const uint32_t w[4] = {rows[u][q8].x, rows[u][q8].y, rows[u][q8].z, rows[u][q8].w};
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float kv = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
-                sc = fma((double)qd[(q8 * 8 + e) * G + hh], (double)kv, sc);
-              }
-            }
-          } else {
-            const int t = p.cand_idx[slot * C + (size_t)warp * S + rs[u]];
-            const uint4* kr = reinterpret_cast<const uint4*>(kfc_rows + (size_t)t * W);
-            for (int q8 = 0; q8 < W8; ++q8) {
-              const uint4 v = __ldg(kr + q8);
-              const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-              for (int e = 0; e < 8; ++e) {
-                const float kv = __uint_as_float((e & 1) ? (w[e >> 1] & 0xFFFF0000u) : (w[e >> 1] << 16));
-                sc = fma((double)qd[(q8 * 8 + e) * G + hh], (double)kv, sc);
-              }
-            }
-          }
-          p.cand_key[slot * C + (size_t)warp * S + rs[u]] = order_key64(sc);
-        }
+        for (int hh = 0; hh < G; ++hh)
+          p.cand_count[(((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk) * kWarps + warp] = bad ? 0 : c[hh];
       }
     }
     if (bad && tid == 0) report(p.status, SFA_ERR_TIMEOUT);
@@ -620,30 +543,57 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
 }
 
 // ---------------------------------------------------------------------------
-// tip_merge: CTA per (b, h).  The chunks' candidates (token order, float64
-// keys, counts per warp segment) are staged in shared memory when they fit
-// (kMergeSmem); with k <= 256 the least of the 256 threads' maxima is at most
-// the k-th largest key (each maximum is a distinct candidate), so only keys at
-// or above it survive; the exact k-th largest of the survivors by radix
-// select; the first k by (key desc, index asc) are written ascending.  More
-// candidates than fit use the same select over global memory.
+// tip_merge: CTA per (b, h).  The chunks' candidate words (token order, counts
+// per warp segment) are staged in shared memory when they fit (kMergeSmem), a
+// warp per segment, and their 16-bit filter keys held in registers.  The k-th
+// largest filter key X (a four-way bisection between the least and largest
+// key) bounds the row's exact k-th largest score from below by value(X) - M
+// (at least k candidates have filter scores >= value(X), each within M of its
+// exact score, M = the largest margin of the row's chunks), so only candidates
+// whose filter key reaches value(X) - 2 M can be in the top k.  Those
+// survivors (in token order) get their exact score in float64 from the
+// compact key rows; up to kMergeRank of them are ranked by counting (key desc,
+// index asc), up to kMergeExact by a bisection in one warp's registers, more
+// by a block radix select with the scores recomputed on the fly, as when the
+// candidates do not fit in shared memory.  Output ascending, -1 padded.
 // ---------------------------------------------------------------------------
-constexpr int kMergeSmem = 12288;
+constexpr int kMergeSmem = 12288;                  // candidates staged in shared memory
+constexpr int kMergeKeys = kMergeSmem / kThreads;  // filter keys per thread (48)
+constexpr int kMergeExact = 2048;                  // survivors rescored into shared memory
+constexpr int kMergeRank = 512;                    // survivors ranked by counting
+constexpr int kSegBatch = 16;                      // segments a warp stages with their loads in flight
 constexpr int kMaxChunks = 512;
 
 __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
   extern __shared__ __align__(16) uint32_t msm[];
   __shared__ uint32_t hist[256];
   __shared__ int sh[64];
+  __shared__ int bred[2][3][kWarps];
+  __shared__ uint32_t mnx[2][kWarps];
+  __shared__ float qf[256];  // this row's query on its KV head's compact columns
+  __shared__ float red[kWarps];
+  __shared__ int nlose;
   const size_t row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const unsigned lt = (1u << lane) - 1u;
+  const int b = (int)(row / p.Hq), h = (int)(row % p.Hq), g = h / (p.Hq / p.Hkv);
+  const int W = 2 * p.nfc;
   const int nseg = p.nchunks * kWarps;
   const int S = p.chunk / kWarps;
-  const uint64_t* ck = p.cand_key + row * p.nchunks * p.chunk;
-  const int* ci = p.cand_idx + row * p.nchunks * p.chunk;
+  const uint32_t* cw = p.cand + row * p.nchunks * p.chunk;
   const int* cc = p.cand_count + row * nseg;
   int* out = p.idx + row * p.k;
   int* off = reinterpret_cast<int*>(msm);  // [nseg + 1] prefix of the segment counts
+  if (tid == 0) nlose = 0;
+  for (int c = tid; c < W; c += kThreads) {
+    const int dim = c < p.nfc ? p.fc[g * p.nfc + c] : p.fc[g * p.nfc + c - p.nfc] + p.D / 2;
+    qf[c] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.q)[row * p.D + dim]);
+  }
+  float mg = 0.f;  // the row's largest chunk margin
+  for (int c = tid; c < p.nchunks; c += kThreads) mg = fmaxf(mg, p.cand_margin[row * p.nchunks + c]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mg = fmaxf(mg, __shfl_xor_sync(0xffffffffu, mg, o));
+  if (lane == 0) red[warp] = mg;
   {
     // block scan of the segment counts, kThreads segments at a time
     int carry = 0;
@@ -671,78 +621,281 @@ __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
     if (tid == 0) off[nseg] = carry;
     __syncthreads();
   }
+  float M = 0.f;
+  for (int w = 0; w < kWarps; ++w) M = fmaxf(M, red[w]);
   const int n = off[nseg];
-  // flat candidate position -> offset in the slot array (segment by binary search)
-  auto locate = [&](int i) -> size_t {
+  // segment of candidate position i (binary search over the offsets); token of a word of segment sg
+  auto seg_of = [&](int i) -> int {
     int lo = 0, hi = nseg;  // off[lo] <= i < off[hi]
     while (hi - lo > 1) {
       const int mid = (lo + hi) >> 1;
       if (off[mid] <= i) lo = mid; else hi = mid;
     }
-    return (size_t)lo * S + (i - off[lo]);
+    return lo;
   };
-  int kept;
-  const int ob = (nseg + 1 + 3) & ~3;  // keys start after the offsets (16-byte aligned)
-  if (n <= kMergeSmem) {
-    uint64_t* sk = reinterpret_cast<uint64_t*>(msm + ob);  // [n] keys
-    int* st = reinterpret_cast<int*>(sk + n);              // [n] token indices
-    int* sv = st + n;                                      // [n] survivor positions
-    // Flat copy: thread tid takes candidates tid, tid + 256, ... (segment by binary search), four
-    // at a time, so that hundreds of independent loads are in flight instead of one segment's.
-    for (int i0 = tid; i0 < n; i0 += 4 * kThreads) {
-      uint64_t kv[4];
-      int iv[4];
+  auto token_of = [&](int sg, uint32_t w) -> int { return (sg / kWarps) * p.chunk + (int)(w & 0xFFFFu); };
+  auto token_global = [&](int i) -> int {
+    const int sg = seg_of(i);
+    return token_of(sg, __ldg(cw + (size_t)sg * S + (i - off[sg])));
+  };
+  // Exact score of tokens t0 and t1 (t1 < 0: none): the float64 dot product over the compact
+  // columns in order, both rows' sixteen-byte groups loaded (four at a time) before the sums.
+  const __nv_bfloat16* kfc_rows = static_cast<const __nv_bfloat16*>(p.Kfc) + (size_t)(b * p.Hkv + g) * p.L * W;
+  auto rescore2 = [&](int t0, int t1, uint64_t* k0, uint64_t* k1) {
+    const uint4* r0 = reinterpret_cast<const uint4*>(kfc_rows + (size_t)t0 * W);
+    const uint4* r1 = reinterpret_cast<const uint4*>(kfc_rows + (size_t)(t1 < 0 ? t0 : t1) * W);
+    double s0 = 0.0, s1 = 0.0;
+    for (int q0 = 0; q0 < W / 8; q0 += 4) {
+      uint4 v0[4], v1[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * kThreads;
-        if (i < n) {
-          const size_t at = locate(i);
-          kv[u] = __ldg(ck + at);
-          iv[u] = __ldg(ci + at);
-        }
+        const bool in = q0 + u < W / 8;
+        v0[u] = in ? __ldg(r0 + q0 + u) : make_uint4(0u, 0u, 0u, 0u);
+        v1[u] = in ? __ldg(r1 + q0 + u) : make_uint4(0u, 0u, 0u, 0u);
       }
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
-        const int i = i0 + u * kThreads;
-        if (i < n) {
-          sk[i] = kv[u];
-          st[i] = iv[u];
+        if (q0 + u >= W / 8) break;
+        const uint32_t a[4] = {v0[u].x, v0[u].y, v0[u].z, v0[u].w};
+        const uint32_t c[4] = {v1[u].x, v1[u].y, v1[u].z, v1[u].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const double qv = (double)qf[(q0 + u) * 8 + e];
+          const float ka = __uint_as_float((e & 1) ? (a[e >> 1] & 0xFFFF0000u) : (a[e >> 1] << 16));
+          const float kc = __uint_as_float((e & 1) ? (c[e >> 1] & 0xFFFF0000u) : (c[e >> 1] << 16));
+          s0 = fma(qv, (double)ka, s0);
+          s1 = fma(qv, (double)kc, s1);
         }
+      }
+    }
+    *k0 = order_key64(s0);
+    *k1 = order_key64(s1);
+  };
+  auto rescore = [&](int t) -> uint64_t {
+    uint64_t k0, k1;
+    rescore2(t, -1, &k0, &k1);
+    return k0;
+  };
+  int kept;
+  const int ob = (nseg + 1 + 3) & ~3;  // arrays start after the offsets (16-byte aligned)
+  if (n <= kMergeSmem) {
+    uint64_t* gk = reinterpret_cast<uint64_t*>(msm + ob);  // [kMergeExact] survivors' exact keys
+    int* stok = reinterpret_cast<int*>(gk + kMergeExact);   // [kMergeExact] survivors' tokens
+    int* sv = stok + kMergeExact;                            // [n] survivor positions (then losers)
+    int* wc = sv + kMergeSmem;                               // [kMergeKeys][kWarps] counts
+    uint32_t* sc = reinterpret_cast<uint32_t*>(wc + kMergeKeys * kWarps);  // [n] candidate words
+    // Warp w stages segments kSegBatch at a time (w kSegBatch + 8 kSegBatch j ...): lane l takes words
+    // 2 l and 2 l + 1 of each segment in one load (a segment starts 8-byte aligned and both words
+    // lie in its slots), all of the batch's loads issued before any store; words past 64 one by one.
+    for (int s0 = warp * kSegBatch; s0 < nseg; s0 += kWarps * kSegBatch) {
+      uint2 kv[kSegBatch];
+#pragma unroll
+      for (int u = 0; u < kSegBatch; ++u) {
+        const int sg = s0 + u;
+        const int cnt = sg < nseg ? off[sg + 1] - off[sg] : 0;
+        kv[u] = 2 * lane < cnt ? __ldg(reinterpret_cast<const uint2*>(cw + (size_t)sg * S) + lane) : make_uint2(0u, 0u);
+      }
+#pragma unroll
+      for (int u = 0; u < kSegBatch; ++u) {
+        const int sg = s0 + u;
+        const int base = sg < nseg ? off[sg] : 0;
+        const int cnt = sg < nseg ? off[sg + 1] - base : 0;
+        if (2 * lane < cnt) sc[base + 2 * lane] = kv[u].x;
+        if (2 * lane + 1 < cnt) sc[base + 2 * lane + 1] = kv[u].y;
+        for (int j = 64 + lane; j < cnt; j += 32) sc[base + j] = __ldg(cw + (size_t)sg * S + j);
       }
     }
     __syncthreads();
     if (p.k >= n) {
-      for (int i = tid; i < n; i += kThreads) out[i] = st[i];
+      for (int i = tid; i < n; i += kThreads) out[i] = token_of(seg_of(i), sc[i]);
       kept = n;
     } else {
-      uint64_t LB = 0u;
-      if (p.k <= kThreads) {
-        uint64_t m = 0u;
-        for (int i = tid; i < n; i += kThreads) m = max(m, sk[i]);
+      // Filter keys in registers, candidate i = tid + kThreads q, two per word (0 past the end).
+      uint32_t kp[kMergeKeys / 2];
+      uint32_t kmin = 0xFFFFu, kmax = 0u;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) m = min(m, __shfl_xor_sync(0xffffffffu, m, o));
-        __syncthreads();
-        if (lane == 0) reinterpret_cast<uint64_t*>(hist)[warp] = m;
-        __syncthreads();
-        LB = ~0ull;
-        for (int w = 0; w < kWarps; ++w) LB = min(LB, reinterpret_cast<const uint64_t*>(hist)[w]);
-        __syncthreads();
+      for (int q2 = 0; q2 < kMergeKeys / 2; ++q2) {
+        const int i0 = 2 * q2 * kThreads + tid, i1 = i0 + kThreads;
+        const uint32_t a = i0 < n ? sc[i0] >> 16 : 0u, c = i1 < n ? sc[i1] >> 16 : 0u;
+        kp[q2] = a | (c << 16);
+        if (i0 < n) { kmin = min(kmin, a); kmax = max(kmax, a); }
+        if (i1 < n) { kmin = min(kmin, c); kmax = max(kmax, c); }
       }
-      int ns = n;
-      if (LB > 0u) {
-        ns = block_filter_ordered<uint64_t>([&](int i) { return sk[i]; }, n, LB, [&](int r, int i) { sv[r] = i; },
-                                            sh + 16);
-      } else {
-        for (int i = tid; i < n; i += kThreads) sv[i] = i;
+      kmin = __reduce_min_sync(0xffffffffu, kmin);
+      kmax = __reduce_max_sync(0xffffffffu, kmax);
+      if (lane == 0) {
+        mnx[0][warp] = kmin;
+        mnx[1][warp] = kmax;
       }
       __syncthreads();
-      auto key_s = [&](int j) { return sk[sv[j]]; };
-      auto emit_s = [&](int r, int j) { out[r] = st[sv[j]]; };
-      if (ns <= 2048) {
-        // few survivors: one warp finds the k-th largest in registers, no block barriers per step
+      // X = the k-th largest filter key: #{key >= lo} >= k > #{key >= hi}, the span cut in four per
+      // step (a threshold of 0 counts every candidate; keys past the end are 0 and never count
+      // against a threshold >= 1).
+      uint32_t lo = 0xFFFFu, hi = 0u;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) {
+        lo = min(lo, mnx[0][w]);
+        hi = max(hi, mnx[1][w]);
+      }
+      hi += 1u;
+      for (int it = 0; hi - lo > 1u; ++it) {
+        const uint32_t span = hi - lo;
+        const uint32_t m1 = lo + (span >> 2), m2 = lo + (span >> 1), m3 = lo + ((3u * span) >> 2);
+        const uint32_t t1 = m1 | (m1 << 16), t2 = m2 | (m2 << 16), t3 = m3 | (m3 << 16);
+        uint32_t a1 = 0u, a2 = 0u, a3 = 0u;  // per-halfword counts (at most kMergeKeys / 2 each)
+#pragma unroll
+        for (int q2 = 0; q2 < kMergeKeys / 2; ++q2) {
+          a1 += __vsetgeu2(kp[q2], t1);
+          a2 += __vsetgeu2(kp[q2], t2);
+          a3 += __vsetgeu2(kp[q2], t3);
+        }
+        const uint32_t c1 = __reduce_add_sync(0xffffffffu, (a1 & 0xFFFFu) + (a1 >> 16));
+        const uint32_t c2 = __reduce_add_sync(0xffffffffu, (a2 & 0xFFFFu) + (a2 >> 16));
+        const uint32_t c3 = __reduce_add_sync(0xffffffffu, (a3 & 0xFFFFu) + (a3 >> 16));
+        if (lane == 0) {
+          bred[it & 1][0][warp] = (int)c1;
+          bred[it & 1][1][warp] = (int)c2;
+          bred[it & 1][2][warp] = (int)c3;
+        }
+        __syncthreads();
+        int s1 = 0, s2 = 0, s3 = 0;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) {
+          s1 += bred[it & 1][0][w];
+          s2 += bred[it & 1][1][w];
+          s3 += bred[it & 1][2][w];
+        }
+        if (m1 == 0u) s1 = n;
+        if (s3 >= p.k) {
+          lo = m3;
+        } else if (s2 >= p.k) {
+          lo = m2;
+          hi = m3;
+        } else if (s1 >= p.k) {
+          lo = m1;
+          hi = m2;
+        } else {
+          hi = m1;
+        }
+      }
+      // Survivors: filter key >= thr (keys under 0x0080 hold no finite score: no bound then),
+      // compacted in candidate order from per-(q, warp) ballot counts.
+      const uint32_t X = lo;
+      const uint32_t thr = X >= 0x80u ? order_key(__fsub_rd(key_value(X << 16), __fmul_ru(2.f, M))) >> 16 : 0u;
+      const uint32_t tt = thr | (thr << 16);
+      auto survives = [&](int q) {
+        const uint32_t ge = __vsetgeu2(kp[q >> 1], tt);
+        return ((q & 1) ? (ge >> 16) : (ge & 0xFFFFu)) != 0u && q * kThreads + tid < n;
+      };
+#pragma unroll
+      for (int q = 0; q < kMergeKeys; ++q) {
+        const unsigned kb = __ballot_sync(0xffffffffu, survives(q));
+        if (lane == 0) wc[q * kWarps + warp] = __popc(kb);
+      }
+      __syncthreads();
+      if (warp == 0) {
+        constexpr int PL = kMergeKeys * kWarps / 32;  // counts per lane
+        int v[PL];
+        int sum = 0;
+#pragma unroll
+        for (int e = 0; e < PL; ++e) {
+          v[e] = wc[lane * PL + e];
+          sum += v[e];
+        }
+        int incl = sum;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        int run = incl - sum;
+#pragma unroll
+        for (int e = 0; e < PL; ++e) {
+          wc[lane * PL + e] = run;
+          run += v[e];
+        }
+        if (lane == 31) sh[0] = incl;
+      }
+      __syncthreads();
+      const int ns = sh[0];
+#pragma unroll
+      for (int q = 0; q < kMergeKeys; ++q) {
+        const bool keep = survives(q);
+        const unsigned kb = __ballot_sync(0xffffffffu, keep);
+        if (keep) sv[wc[q * kWarps + warp] + __popc(kb & lt)] = q * kThreads + tid;
+      }
+      __syncthreads();
+      // The survivors' tokens and exact keys (the first kMergeExact), two per thread at a time.
+      const int nr = min(ns, kMergeExact);
+      for (int j0 = tid; j0 < nr; j0 += 2 * kThreads) {
+        const int j1 = j0 + kThreads;
+        const int i0 = sv[j0];
+        const int t0 = token_of(seg_of(i0), sc[i0]);
+        int t1 = -1;
+        if (j1 < nr) {
+          const int i1 = sv[j1];
+          t1 = token_of(seg_of(i1), sc[i1]);
+        }
+        uint64_t k0, k1;
+        rescore2(t0, t1, &k0, &k1);
+        stok[j0] = t0;
+        gk[j0] = k0;
+        if (j1 < nr) {
+          stok[j1] = t1;
+          gk[j1] = k1;
+        }
+      }
+      __syncthreads();
+      auto emit_s = [&](int r, int j) { out[r] = stok[j]; };
+      if (ns <= kMergeRank) {
+        // rank of survivor j = #{i : key_i > key_j, or key_i == key_j and i < j} (survivors are in
+        // token order): warp w ranks eight survivors at a time, lanes splitting the i range two
+        // keys per step, and records those ranked k or later (the ns - k losers); a kept
+        // survivor's place in the output is j minus the losers before it
+        constexpr int RJ = 8;
+        for (int j0 = warp * RJ; j0 < ns; j0 += kWarps * RJ) {
+          uint64_t kj[RJ];
+          int r[RJ];
+#pragma unroll
+          for (int u = 0; u < RJ; ++u) {
+            kj[u] = gk[min(j0 + u, ns - 1)];
+            r[u] = 0;
+          }
+          for (int i = lane; i < ns; i += 64) {
+            const int i2 = i + 32;
+            const uint64_t ka = gk[i], kb = i2 < ns ? gk[i2] : 0ull;  // 0: no finite score's key
+#pragma unroll
+            for (int u = 0; u < RJ; ++u) {
+              r[u] += (ka > kj[u] || (ka == kj[u] && i < j0 + u)) ? 1 : 0;
+              r[u] += (kb > kj[u] || (kb == kj[u] && i2 < j0 + u)) ? 1 : 0;
+            }
+          }
+          int rr = 0;
+#pragma unroll
+          for (int u = 0; u < RJ; ++u) {
+            const int t = (int)__reduce_add_sync(0xffffffffu, (unsigned)r[u]);
+            if (lane == u) rr = t;
+          }
+          if (lane < RJ && j0 + lane < ns && rr >= p.k) sv[atomicAdd(&nlose, 1)] = j0 + lane;
+        }
+        __syncthreads();
+        const int L = nlose;
+        for (int j = tid; j < ns; j += kThreads) {
+          int below = 0;
+          bool lose = false;
+          for (int e = 0; e < L; ++e) {
+            const int x = sv[e];
+            below += x < j ? 1 : 0;
+            lose = lose || x == j;
+          }
+          if (!lose) out[j - below] = stok[j];
+        }
+        kept = ns - L;
+      } else if (ns <= kMergeExact) {
+        // one warp finds the k-th largest exact key in registers, no block barriers per step
         if (warp == 0) {
           int gt = 0;
-          const uint64_t T = warp_kth_largest64(key_s, ns, p.k, &gt);
+          const uint64_t T = warp_kth_largest64([&](int j) { return gk[j]; }, ns, p.k, &gt);
           if (lane == 0) {
             reinterpret_cast<uint64_t*>(hist)[0] = T;
             sh[1] = p.k - gt;
@@ -752,14 +905,16 @@ __global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
         const uint64_t T = reinterpret_cast<const uint64_t*>(hist)[0];
         const int take = sh[1];
         __syncthreads();
-        kept = block_emit_ordered<uint64_t>(key_s, ns, false, T, take, emit_s, sh + 4);
+        kept = block_emit_ordered<uint64_t>([&](int j) { return gk[j]; }, ns, false, T, take, emit_s, sh + 4);
       } else {
-        kept = block_select_ordered<uint64_t>(key_s, ns, p.k, emit_s, hist, sh);
+        auto tok = [&](int j) { const int i = sv[j]; return token_of(seg_of(i), sc[i]); };
+        kept = block_select_ordered<uint64_t>([&](int j) { return rescore(tok(j)); }, ns, p.k,
+                                              [&](int r, int j) { out[r] = tok(j); }, hist, sh);
       }
     }
   } else {
-    kept = block_select_ordered<uint64_t>([&](int i) { return __ldg(ck + locate(i)); }, n, p.k,
-                                          [&](int r, int i) { out[r] = __ldg(ci + locate(i)); }, hist, sh);
+    kept = block_select_ordered<uint64_t>([&](int i) { return rescore(token_global(i)); }, n, p.k,
+                                          [&](int r, int i) { out[r] = token_global(i); }, hist, sh);
   }
   for (int r = kept + tid; r < p.k; r += kThreads) out[r] = -1;
 }
@@ -936,7 +1091,9 @@ cudaError_t launch_decode_select(const DecodeParams& p, cudaStream_t st) {
                   : G == 4 ? launch_tip_chunk<4>(p, st)
                            : launch_tip_chunk<8>(p, st);
   if (e != cudaSuccess) return e;
-  const size_t msmem = ((size_t)p.nchunks * kWarps + 8 + (size_t)4 * kMergeSmem) * sizeof(uint32_t);
+  // offsets, survivors' keys and tokens, survivor positions, compaction counts, candidate words
+  const size_t msmem = ((size_t)p.nchunks * kWarps + 4 + (size_t)3 * kMergeExact + kMergeSmem +
+                        (size_t)kMergeKeys * kWarps + kMergeSmem) * sizeof(uint32_t);
   e = cudaFuncSetAttribute(tip_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
   if (e != cudaSuccess) return e;
   tip_merge_kernel<<<p.B * p.Hq, kThreads, msmem, st>>>(p);

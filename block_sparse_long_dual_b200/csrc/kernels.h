@@ -80,9 +80,10 @@ struct DecodeParams {
   const void* Kfc;   // [B, Hkv, L, 2 nfc] bf16 compact dominant-pair keys
   const void* Kc;    // [B, Hkv, L, D] bf16 rotated key cache
   const void* Vc;    // [B, Hkv, L, D] bf16 value cache
-  uint64_t* cand_key;  // [B * Hq, nchunks, chunk] float64 order keys of each chunk's candidates, token order
-  int* cand_idx;
+  uint32_t* cand;      // [B * Hq, nchunks, chunk] each chunk's candidates in token order per warp segment:
+                       // 16-bit filter key << 16 | token offset in the chunk
   int* cand_count;     // [B * Hq, nchunks, 8] per warp segment of each chunk
+  float* cand_margin;  // [B * Hq, nchunks] error bound of the chunk's filter scores
   int* idx;          // [B, Hq, k]
   void* o;           // [B, Hq, D] bf16
   float* lse;        // [B, Hq] (nullable)
