@@ -112,14 +112,20 @@ __device__ __forceinline__ void arm_and_load(uint32_t bar, uint32_t dst, const v
   bulk_load(dst, src, bytes, bar);
 }
 
+__device__ __forceinline__ bool try_wait_parity(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+               "selp.u32 %0, 1, 0, p;\n\t}" : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0u;
+}
+
+// The clock is read only once the phase is found incomplete, then every 64 polls.
 __device__ __forceinline__ bool wait_parity_bounded(uint32_t bar, uint32_t parity) {
+  if (try_wait_parity(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
-  for (;;) {
-    uint32_t ok;
-    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                 "selp.u32 %0, 1, 0, p;\n\t}" : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-    if (ok) return true;
-    if (globaltimer_ns() - t0 > 2000000000ull) return false;
+  for (uint32_t it = 1;; ++it) {
+    if (try_wait_parity(bar, parity)) return true;
+    if ((it & 63u) == 0u && globaltimer_ns() - t0 > 2000000000ull) return false;
   }
 }
 

@@ -57,6 +57,12 @@ __device__ __forceinline__ uint32_t order_key(float f) {
   uint32_t u = __float_as_uint(f == 0.f ? 0.f : f);
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
+// The same order without merging the zeros (-0 keys just below +0): for the filter keys, whose
+// bounds are always lowered by a positive margin first.
+__device__ __forceinline__ uint32_t order_key_signed_zero(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return u ^ ((uint32_t)((int32_t)u >> 31) | 0x80000000u);
+}
 __device__ __forceinline__ float key_value(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
@@ -322,25 +328,29 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
   const int tid = threadIdx.x;
   const int ntiles = p.nchunks * p.B * p.Hkv;
   const __nv_bfloat16* kfc_all = static_cast<const __nv_bfloat16*>(p.Kfc);
-  auto slabs_of = [&](int tile) {
-    const int n = min(C, p.L - (tile % p.nchunks) * C);
-    return (n + ST - 1) / ST;
-  };
-  // Producer state (thread 0): next (tile, slab) to copy and the stage it goes to.
-  int ptile = blockIdx.x, pslab = 0, issued = 0;
+  // Producer state (thread 0): the next (chunk, group, slab) to copy, advanced by the grid size
+  // without divisions, and the stage it goes to.
+  const int nbg = p.B * p.Hkv;
+  const int dq = (int)gridDim.x / p.nchunks, dr = (int)gridDim.x % p.nchunks;
+  int pchunk = (int)blockIdx.x % p.nchunks, pbg = (int)blockIdx.x / p.nchunks, pslab = 0, issued = 0;
+  int pn = min(C, p.L - pchunk * C);  // tokens of the producer's chunk
   auto issue_next = [&]() {
-    if (ptile >= ntiles) return;
-    const int chunk = ptile % p.nchunks, bg = ptile / p.nchunks;
-    const int n = min(C, p.L - chunk * C);
-    const int rows = min(ST, n - pslab * ST);
-    const __nv_bfloat16* src = kfc_all + ((size_t)bg * p.L + (size_t)chunk * C + (size_t)pslab * ST) * W;
+    if (pbg >= nbg) return;
+    const int rows = min(ST, pn - pslab * ST);
+    const __nv_bfloat16* src = kfc_all + ((size_t)pbg * p.L + (size_t)pchunk * C + (size_t)pslab * ST) * W;
     const int stg = issued % NS;
     arm_and_load((uint32_t)__cvta_generic_to_shared(&bars[stg]), (uint32_t)__cvta_generic_to_shared(ring + (size_t)stg * SB),
                  src, (uint32_t)rows * W * 2);
     ++issued;
-    if (++pslab == slabs_of(ptile)) {
+    if (++pslab * ST >= pn) {
       pslab = 0;
-      ptile += gridDim.x;
+      pchunk += dr;
+      pbg += dq;
+      if (pchunk >= p.nchunks) {
+        pchunk -= p.nchunks;
+        ++pbg;
+      }
+      pn = min(C, p.L - pchunk * C);
     }
   };
   if (tid == 0) {
@@ -391,34 +401,48 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
       for (int sl = 0; sl < nsl; ++sl, ++consumed) {
         const int stg = consumed % NS;
         if (!wait_parity_bounded((uint32_t)__cvta_generic_to_shared(&bars[stg]), (consumed / NS) & 1)) lost = 1;
-        const unsigned char* slab = ring + (size_t)stg * SB;
+        // Fragment rows gq and gq + 8 of tile mt take slab rows r0 and r0 + 1, so that a lane's two
+        // tokens are adjacent and their keys of one head go out in one word; the tiles' k-steps are
+        // interleaved so that their mma chains overlap.
+        const int rb = warp * MT * 16 + 2 * gq;  // tile 0's r0
+        const unsigned char* rowb = ring + (size_t)stg * SB + (size_t)rb * (2 * W) + 4 * tq;
+        uint32_t m0[MT], m1[MT];
+        float c[MT][4];
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-          const int r0 = (warp * MT + mt) * 16 + gq;  // slab rows r0 and r0 + 8
-          const int t0s = sl * ST + r0;               // their tokens in the chunk
-          const uint32_t m0 = t0s < n ? 0x7FFF7FFFu : 0u, m1 = t0s + 8 < n ? 0x7FFF7FFFu : 0u;
-          float c[4] = {0.f, 0.f, 0.f, 0.f};
-          const unsigned char* row0 = slab + (size_t)r0 * (2 * W) + 4 * tq;
-          const unsigned char* row1 = row0 + (size_t)8 * (2 * W);
+          const int t0s = sl * ST + rb + 16 * mt;
+          m0[mt] = t0s < n ? 0x7FFF7FFFu : 0u;
+          m1[mt] = t0s + 1 < n ? 0x7FFF7FFFu : 0u;
+          c[mt][0] = c[mt][1] = c[mt][2] = c[mt][3] = 0.f;
+        }
 #pragma unroll
-          for (int ks = 0; ks < 16; ++ks) {
-            if (ks >= KS) break;
-            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(row0 + 16 * ks);
-            const uint32_t a1 = *reinterpret_cast<const uint32_t*>(row1 + 16 * ks);
-            am = __vmaxu2(am, a0 & m0);
-            am = __vmaxu2(am, a1 & m1);
-            asm volatile(
-                "mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
+        for (int ks = 0; ks < 16; ++ks) {
+          if (ks >= KS) break;
+#pragma unroll
+          for (int mt = 0; mt < MT; ++mt) {
+            const unsigned char* row0 = rowb + (size_t)(16 * mt) * (2 * W) + 16 * ks;
+            const uint32_t a0 = *reinterpret_cast<const uint32_t*>(row0);
+            const uint32_t a1 = *reinterpret_cast<const uint32_t*>(row0 + 2 * W);
+            am = __vmaxu2(am, a0 & m0[mt]);
+            am = __vmaxu2(am, a1 & m1[mt]);
+            asm("mma.sync.aligned.m16n8k8.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5}, {%6}, "
                 "{%0, %1, %2, %3};"
-                : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+                : "+f"(c[mt][0]), "+f"(c[mt][1]), "+f"(c[mt][2]), "+f"(c[mt][3])
                 : "r"(a0), "r"(a1), "r"(qb[ks]));
           }
-          // c = scores of tokens (r0, r0 + 8) x heads (2 tq, 2 tq + 1)
+        }
+        // c[mt] = scores of tokens (t0s, t0s + 1) x heads (2 tq, 2 tq + 1); past the end of the chunk
+        // the second token's key is left for the readers to mask
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int hh = 2 * tq + (e & 1);
-            const int t = t0s + (e >> 1) * 8;
-            if (hh < G && t < n) keys[(size_t)hh * C + t] = (uint16_t)(order_key(c[e]) >> 16);
+        for (int mt = 0; mt < MT; ++mt) {
+          const int t0s = sl * ST + rb + 16 * mt;
+          if (t0s < n) {
+            if (2 * tq < G)
+              *reinterpret_cast<uint32_t*>(keys + (size_t)(2 * tq) * C + t0s) =
+                  __byte_perm(order_key_signed_zero(c[mt][0]), order_key_signed_zero(c[mt][2]), 0x7632);
+            if (2 * tq + 1 < G)
+              *reinterpret_cast<uint32_t*>(keys + (size_t)(2 * tq + 1) * C + t0s) =
+                  __byte_perm(order_key_signed_zero(c[mt][1]), order_key_signed_zero(c[mt][3]), 0x7632);
           }
         }
         __syncthreads();  // stage consumed
@@ -470,13 +494,18 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
           }
           mn = __reduce_min_sync(0xffffffffu, mn);
           mx = __reduce_max_sync(0xffffffffu, mx);
-          uint64_t lo = mn, hi = (uint64_t)mx + 1;  // #{>= lo} >= k, #{>= hi} < k
-          for (int it = 0; it < 24 && hi - lo > 1; ++it) {
-            const uint32_t mid = (uint32_t)(lo + ((hi - lo) >> 1));
-            int c = 0;
+          // two maxima per word, counted per halfword
+          uint32_t gp[NGPL / 2];
 #pragma unroll
-            for (int j = 0; j < NGPL; ++j) c += gm[j] >= mid ? 1 : 0;
-            if ((int)__reduce_add_sync(0xffffffffu, (unsigned)c) >= p.k) lo = mid; else hi = mid;
+          for (int j = 0; j < NGPL / 2; ++j) gp[j] = gm[2 * j] | (gm[2 * j + 1] << 16);
+          uint32_t lo = mn, hi = mx + 1;  // #{>= lo} >= k, #{>= hi} < k
+          while (hi - lo > 1u) {
+            const uint32_t mid = lo + ((hi - lo) >> 1);
+            const uint32_t mm = mid | (mid << 16);
+            uint32_t a = 0u;
+#pragma unroll
+            for (int j = 0; j < NGPL / 2; ++j) a += __vsetgeu2(gp[j], mm);
+            if ((int)__reduce_add_sync(0xffffffffu, (a & 0xFFFFu) + (a >> 16)) >= p.k) lo = mid; else hi = mid;
           }
           LBw = (uint32_t)lo;
           // The stored keys are the high 16 bits of the float32 keys (rounded down), so LBw << 16
@@ -493,41 +522,55 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
 #pragma unroll
     for (int hh = 0; hh < G; ++hh) LB[hh] = (uint32_t)scratch[hh];
     // Candidates in token order (16-bit key at or above the 16-bit bound: a superset of the tokens
-    // whose float32 key reaches the bound): warp w scans its contiguous range [w S, w S + S) of the
-    // chunk, two tokens per lane per step and all heads at once, and writes its own segment of
-    // each head's slot (16-bit filter key << 16 | token offset in the chunk); counts per (slot,
-    // warp).  The merge rescores the candidates that survive its own bound.
+    // whose float32 key reaches the bound): warp w takes its contiguous range [w S, w S + S) of the
+    // chunk, lane l the run of R = S / 32 tokens at w S + l R; per head a lane marks its run's
+    // candidates in a bit mask (two keys per compare), a warp scan of the counts places them, and
+    // the lane writes its own (16-bit filter key << 16 | token offset in the chunk) into the warp's
+    // segment of the head's slot; counts per (slot, warp).  The merge rescores the candidates that
+    // survive its own bound.
     const int bad = lost;
     {
+      constexpr int R = 4 * NGR;  // tokens per lane: C / 8 warps / 32 lanes
       const int lane = tid & 31, warp = tid >> 5;
-      const unsigned lt = (1u << lane) - 1u;
       const int S = C / kWarps;
-      const int w0 = min(n, warp * S), w1 = min(n, w0 + S);
-      uint32_t* cw[G];
-      int c[G];
+      const int r0 = warp * S + lane * R;                 // the lane's run (8-byte aligned keys)
+      const int nv = max(0, min(R, n - r0));              // its tokens inside the chunk
+      const uint32_t vmask = nv >= 32 ? 0xFFFFFFFFu : ((1u << nv) - 1u);
 #pragma unroll
       for (int hh = 0; hh < G; ++hh) {
-        cw[hh] = p.cand + (((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk) * C + (size_t)warp * S;
-        c[hh] = 0;
-      }
-      for (int b0 = w0; b0 < w1; b0 += 64) {
-        const int i = b0 + 2 * lane;  // tokens i and i + 1 (w0 is even; the second is masked past w1)
+        const uint16_t* hk = keys + (size_t)hh * C + r0;
+        uint32_t kk[R / 2];
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh) {
-          const uint32_t pr = i < w1 ? *reinterpret_cast<const uint32_t*>(keys + (size_t)hh * C + i) : 0u;
-          const uint32_t u0 = pr & 0xFFFFu, u1 = pr >> 16;
-          const bool k0 = i < w1 && u0 >= LB[hh], k1 = i + 1 < w1 && u1 >= LB[hh];
-          const unsigned m0 = __ballot_sync(0xffffffffu, k0), m1 = __ballot_sync(0xffffffffu, k1);
-          const int at = c[hh] + __popc(m0 & lt) + __popc(m1 & lt);
-          if (k0) cw[hh][at] = (u0 << 16) | (uint32_t)i;
-          if (k1) cw[hh][at + (k0 ? 1 : 0)] = (u1 << 16) | (uint32_t)(i + 1);
-          c[hh] += __popc(m0) + __popc(m1);
+        for (int v = 0; v < R / 4; ++v) {
+          const uint2 x = *reinterpret_cast<const uint2*>(hk + 4 * v);
+          kk[2 * v] = x.x;
+          kk[2 * v + 1] = x.y;
         }
-      }
-      if (lane == 0) {
+        const uint32_t lb2 = LB[hh] | (LB[hh] << 16);
+        uint32_t mask = 0u;
 #pragma unroll
-        for (int hh = 0; hh < G; ++hh)
-          p.cand_count[(((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk) * kWarps + warp] = bad ? 0 : c[hh];
+        for (int j = 0; j < R / 2; ++j) {
+          const uint32_t ge = __vsetgeu2(kk[j], lb2);
+          mask |= ((ge & 1u) | ((ge >> 15) & 2u)) << (2 * j);
+        }
+        mask &= vmask;
+        const int cnt = __popc(mask);
+        int incl = cnt;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int y = __shfl_up_sync(0xffffffffu, incl, o);
+          if (lane >= o) incl += y;
+        }
+        uint32_t* cw = p.cand + (((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk) * C + (size_t)warp * S;
+        int at = incl - cnt;
+        while (mask) {
+          const int j = __ffs(mask) - 1;
+          mask &= mask - 1u;
+          cw[at++] = ((uint32_t)hk[j] << 16) | (uint32_t)(r0 + j);
+        }
+        const int total = __shfl_sync(0xffffffffu, incl, 31);
+        if (lane == 0)
+          p.cand_count[(((size_t)b * p.Hq + g * G + hh) * p.nchunks + chunk) * kWarps + warp] = bad ? 0 : total;
       }
     }
     if (bad && tid == 0) report(p.status, SFA_ERR_TIMEOUT);
