@@ -607,7 +607,7 @@ constexpr int kMergeRank = 512;                    // survivors ranked by counti
 constexpr int kSegBatch = 16;                      // segments a warp stages with their loads in flight
 constexpr int kMaxChunks = 512;
 
-__global__ void __launch_bounds__(kThreads) tip_merge_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 1) tip_merge_kernel(DecodeParams p) {
   extern __shared__ __align__(16) uint32_t msm[];
   __shared__ uint32_t hist[256];
   __shared__ int sh[64];
