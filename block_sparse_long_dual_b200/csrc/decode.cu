@@ -330,12 +330,15 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
   const __nv_bfloat16* kfc_all = static_cast<const __nv_bfloat16*>(p.Kfc);
   // Producer state (thread 0): the next (chunk, group, slab) to copy, advanced by the grid size
   // without divisions, and the stage it goes to.
-  const int nbg = p.B * p.Hkv;
-  const int dq = (int)gridDim.x / p.nchunks, dr = (int)gridDim.x % p.nchunks;
-  int pchunk = (int)blockIdx.x % p.nchunks, pbg = (int)blockIdx.x / p.nchunks, pslab = 0, issued = 0;
+  // This CTA's tiles: a contiguous range (consecutive chunks of one (b, KV head), mostly), the
+  // ranges as even as the grid allows.
+  const int per_cta = ntiles / (int)gridDim.x, extra = ntiles % (int)gridDim.x;
+  const int t_begin = (int)blockIdx.x * per_cta + min((int)blockIdx.x, extra);
+  const int t_end = t_begin + per_cta + ((int)blockIdx.x < extra ? 1 : 0);
+  int ptile = t_begin, pchunk = t_begin % p.nchunks, pbg = t_begin / p.nchunks, pslab = 0, issued = 0;
   int pn = min(C, p.L - pchunk * C);  // tokens of the producer's chunk
   auto issue_next = [&]() {
-    if (pbg >= nbg) return;
+    if (ptile >= t_end) return;
     const int rows = min(ST, pn - pslab * ST);
     const __nv_bfloat16* src = kfc_all + ((size_t)pbg * p.L + (size_t)pchunk * C + (size_t)pslab * ST) * W;
     const int stg = issued % NS;
@@ -344,10 +347,9 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
     ++issued;
     if (++pslab * ST >= pn) {
       pslab = 0;
-      pchunk += dr;
-      pbg += dq;
-      if (pchunk >= p.nchunks) {
-        pchunk -= p.nchunks;
+      ++ptile;
+      if (++pchunk == p.nchunks) {
+        pchunk = 0;
         ++pbg;
       }
       pn = min(C, p.L - pchunk * C);
@@ -364,7 +366,12 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
   __syncthreads();
 
   int consumed = 0;
-  for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x) {
+  // The bound carried to the next chunk of the same rows (warp h keeps head h's): the raw k-th
+  // group maximum of the run's first chunk and that chunk's margin.
+  int run_bg = -1;
+  uint32_t run_lb = 0u;
+  float run_m = 0.f;
+  for (int tile = t_begin; tile < t_end; ++tile) {
     const int chunk = tile % p.nchunks, bg = tile / p.nchunks;
     const int b = bg / p.Hkv, g = bg % p.Hkv;
     const int t0 = chunk * C;
@@ -461,7 +468,9 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
     // the chunk's k-th largest float32 score (each maximum is a distinct token), so stopping the
     // bisection early still gives a valid bound; the bound is then lowered by twice the float32
     // chain's rounding bound M (see the top of this file), so that no token of the row's top k
-    // by exact score is dropped.
+    // by exact score is dropped.  A bound found in one chunk holds for the whole row: the next
+    // chunks of the same rows in this CTA's range reuse it (lowered by that chunk's margin plus
+    // their own) instead of searching again.
     {
       const int lane = tid & 31, warp = tid >> 5;
       constexpr int NGPL = 8 * NGR;  // groups per lane: C / 4 / 32
@@ -478,7 +487,11 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
         const float M = __fadd_ru(__fmul_ru(__fmul_ru(0x1p-16f, q1), A), (float)W * 0x1p-126f);
         if (lane == 0) p.cand_margin[((size_t)b * p.Hq + g * G + warp) * p.nchunks + chunk] = M;
         uint32_t LBw = 0u;
-        if (p.k <= 32 * NGPL) {
+        if (p.k <= 32 * NGPL && run_bg == bg) {
+          LBw = run_lb >= 0x80u
+                    ? order_key(__fsub_rd(key_value(run_lb << 16), __fadd_ru(run_m, M))) >> 16
+                    : 0u;
+        } else if (p.k <= 32 * NGPL) {
           const uint16_t* hk = keys + (size_t)warp * C;
           uint32_t gm[NGPL];
           uint32_t mn = 0xFFFFFFFFu, mx = 0u;
@@ -507,12 +520,13 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
             for (int j = 0; j < NGPL / 2; ++j) a += __vsetgeu2(gp[j], mm);
             if ((int)__reduce_add_sync(0xffffffffu, (a & 0xFFFFu) + (a >> 16)) >= p.k) lo = mid; else hi = mid;
           }
-          LBw = (uint32_t)lo;
-          // The stored keys are the high 16 bits of the float32 keys (rounded down), so LBw << 16
+          // The stored keys are the high 16 bits of the float32 keys (rounded down), so lo << 16
           // bounds the true keys of those group maxima from below; the lowered bound is rounded
           // down to 16 bits again for the comparison with the stored keys.
           // (Keys under 0x0080 hold no finite score: no bound then.)
-          LBw = LBw >= 0x80u ? order_key(__fsub_rd(key_value(LBw << 16), __fmul_ru(2.f, M))) >> 16 : 0u;
+          run_lb = lo;
+          run_m = M;
+          LBw = lo >= 0x80u ? order_key(__fsub_rd(key_value(lo << 16), __fmul_ru(2.f, M))) >> 16 : 0u;
         }
         if (lane == 0) scratch[warp] = (int)LBw;
       }
@@ -574,6 +588,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
       }
     }
     if (bad && tid == 0) report(p.status, SFA_ERR_TIMEOUT);
+    run_bg = bg;
     __syncthreads();  // keys / qd free for the next tile
   }
   // After a wait that gave up, let this CTA's copies land (bounded) before it exits.
