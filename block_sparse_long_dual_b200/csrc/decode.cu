@@ -630,7 +630,7 @@ __global__ void __launch_bounds__(kThreads, 1) tip_merge_kernel(DecodeParams p) 
   __shared__ uint32_t mnx[2][kWarps];
   __shared__ float qf[256];  // this row's query on its KV head's compact columns
   __shared__ float red[kWarps];
-  __shared__ int nlose;
+  __shared__ int nlose, nabove, nband;
   const size_t row = blockIdx.x;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const unsigned lt = (1u << lane) - 1u;
@@ -642,7 +642,11 @@ __global__ void __launch_bounds__(kThreads, 1) tip_merge_kernel(DecodeParams p) 
   const int* cc = p.cand_count + row * nseg;
   int* out = p.idx + row * p.k;
   int* off = reinterpret_cast<int*>(msm);  // [nseg + 1] prefix of the segment counts
-  if (tid == 0) nlose = 0;
+  if (tid == 0) {
+    nlose = 0;
+    nabove = 0;
+    nband = 0;
+  }
   for (int c = tid; c < W; c += kThreads) {
     const int dim = c < p.nfc ? p.fc[g * p.nfc + c] : p.fc[g * p.nfc + c - p.nfc] + p.D / 2;
     qf[c] = __bfloat162float(static_cast<const __nv_bfloat16*>(p.q)[row * p.D + dim]);
@@ -906,35 +910,77 @@ __global__ void __launch_bounds__(kThreads, 1) tip_merge_kernel(DecodeParams p) 
       __syncthreads();
       auto emit_s = [&](int r, int j) { out[r] = stok[j]; };
       if (ns <= kMergeRank) {
-        // rank of survivor j = #{i : key_i > key_j, or key_i == key_j and i < j} (survivors are in
-        // token order): warp w ranks eight survivors at a time, lanes splitting the i range two
-        // keys per step, and records those ranked k or later (the ns - k losers); a kept
-        // survivor's place in the output is j minus the losers before it
-        constexpr int RJ = 8;
-        for (int j0 = warp * RJ; j0 < ns; j0 += kWarps * RJ) {
-          uint64_t kj[RJ];
-          int r[RJ];
-#pragma unroll
-          for (int u = 0; u < RJ; ++u) {
-            kj[u] = gk[min(j0 + u, ns - 1)];
-            r[u] = 0;
-          }
-          for (int i = lane; i < ns; i += 64) {
-            const int i2 = i + 32;
-            const uint64_t ka = gk[i], kb = i2 < ns ? gk[i2] : 0ull;  // 0: no finite score's key
-#pragma unroll
-            for (int u = 0; u < RJ; ++u) {
-              r[u] += (ka > kj[u] || (ka == kj[u] && i < j0 + u)) ? 1 : 0;
-              r[u] += (kb > kj[u] || (kb == kj[u] && i2 < j0 + u)) ? 1 : 0;
+        // The band: with X the k-th largest filter key, at least k candidates have exact scores
+        // >= v_lo = value(X) - M, and fewer than k have exact scores >= v_hi = value(X + 1) + M
+        // (such a score means a filter score >= value(X + 1), i.e. a key above X).  So survivors
+        // scoring >= v_hi are all kept, those below v_lo all dropped, and only the band between is
+        // ranked, for the k - (number above) places left.  Checked at run time (counts and the
+        // key range); otherwise every survivor is ranked.
+        bool band = X >= 0x80u && X < 0xFF80u;
+        uint64_t klo = 0ull, khi = 0ull;
+        if (band) {
+          klo = order_key64((double)__fsub_rd(key_value(X << 16), M));
+          khi = order_key64((double)__fadd_ru(key_value((X + 1u) << 16), M));
+          for (int j = tid; j < ns; j += kThreads) {
+            const uint64_t e = gk[j];
+            if (e >= khi) atomicAdd(&nabove, 1);
+            else if (e >= klo) {
+              const int t = atomicAdd(&nband, 1);
+              if (t < kMergeKeys * kWarps) wc[t] = j;
             }
           }
-          int rr = 0;
-#pragma unroll
-          for (int u = 0; u < RJ; ++u) {
-            const int t = (int)__reduce_add_sync(0xffffffffu, (unsigned)r[u]);
-            if (lane == u) rr = t;
+        }
+        __syncthreads();
+        const int na = nabove, nb = nband;
+        band = band && na < p.k && na + nb >= p.k && nb <= kMergeKeys * kWarps;
+        if (band) {
+          // rank within the band (key desc, position asc); the band's last ones and everything
+          // below it are the losers
+          const int left = p.k - na;
+          for (int t = tid; t < nb; t += kThreads) {
+            const int j = wc[t];
+            const uint64_t e = gk[j];
+            int r = 0;
+            for (int u = 0; u < nb; ++u) {
+              const int j2 = wc[u];
+              const uint64_t e2 = gk[j2];
+              r += (e2 > e || (e2 == e && j2 < j)) ? 1 : 0;
+            }
+            if (r >= left) sv[atomicAdd(&nlose, 1)] = j;
           }
-          if (lane < RJ && j0 + lane < ns && rr >= p.k) sv[atomicAdd(&nlose, 1)] = j0 + lane;
+          for (int j = tid; j < ns; j += kThreads)
+            if (gk[j] < klo) sv[atomicAdd(&nlose, 1)] = j;
+        } else {
+          // rank of survivor j = #{i : key_i > key_j, or key_i == key_j and i < j} (survivors are in
+          // token order): warp w ranks eight survivors at a time, lanes splitting the i range two
+          // keys per step, and records those ranked k or later (the ns - k losers); a kept
+          // survivor's place in the output is j minus the losers before it
+          constexpr int RJ = 8;
+          for (int j0 = warp * RJ; j0 < ns; j0 += kWarps * RJ) {
+            uint64_t kj[RJ];
+            int r[RJ];
+#pragma unroll
+            for (int u = 0; u < RJ; ++u) {
+              kj[u] = gk[min(j0 + u, ns - 1)];
+              r[u] = 0;
+            }
+            for (int i = lane; i < ns; i += 64) {
+              const int i2 = i + 32;
+              const uint64_t ka = gk[i], kb = i2 < ns ? gk[i2] : 0ull;  // 0: no finite score's key
+#pragma unroll
+              for (int u = 0; u < RJ; ++u) {
+                r[u] += (ka > kj[u] || (ka == kj[u] && i < j0 + u)) ? 1 : 0;
+                r[u] += (kb > kj[u] || (kb == kj[u] && i2 < j0 + u)) ? 1 : 0;
+              }
+            }
+            int rr = 0;
+#pragma unroll
+            for (int u = 0; u < RJ; ++u) {
+              const int t = (int)__reduce_add_sync(0xffffffffu, (unsigned)r[u]);
+              if (lane == u) rr = t;
+            }
+            if (lane < RJ && j0 + lane < ns && rr >= p.k) sv[atomicAdd(&nlose, 1)] = j0 + lane;
+          }
         }
         __syncthreads();
         const int L = nlose;

@@ -35,6 +35,10 @@ CASES = [
     D("single-token-cache", heads_q=4, heads_kv=2, seq_len=1, head_dim=64, nfc=4, k=3),
     D("k-above-chunk", heads_q=2, heads_kv=1, seq_len=10000, head_dim=64, nfc=8, k=5000),
     D("no-needles-many-ties", heads_q=4, heads_kv=1, seq_len=7000, nfc=4, k=100, needle_frac=0.0),
+    # more tiles (chunk, b, KV head) than the persistent grid holds: some CTAs take two
+    # consecutive chunks of the same rows, the second one (a ragged last chunk among them) with
+    # the bound carried from the first and its candidates taken straight from the scores
+    D("multi-tile-runs", batch=8, heads_q=32, heads_kv=8, seq_len=20000),
 ]
 
 
