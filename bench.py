@@ -521,6 +521,26 @@ def main():
         raise RuntimeError(f"device status {int(model.status.item())}")
     h2d = sum(t.numel() * t.element_size() for t in (Qh, Kh, Vh))
     d2h = Oh[0].numel() * Oh[0].element_size()
+    # The host links alone (no layer): the same uploads, then uploads and downloads together.
+    link_ms = []
+    for both in (False, True):
+        l0, l1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        l0.record(stream)
+        pipe.up.wait_stream(stream)
+        pipe.down.wait_stream(stream)
+        for i in range(3):
+            with torch.cuda.stream(pipe.up):
+                for d, hst in zip(pipe.dev_in[i % 2], (Qh, Kh, Vh)):
+                    d.copy_(hst, non_blocking=True)
+            if both:
+                with torch.cuda.stream(pipe.down):
+                    Oh[i % 2].copy_(pipe.dev_out[(i + 1) % 2], non_blocking=True)
+        stream.wait_stream(pipe.up)
+        stream.wait_stream(pipe.down)
+        l1.record(stream)
+        torch.cuda.synchronize(dev)
+        link_ms.append(l0.elapsed_time(l1) / 3)
 
     vals = torch.tensor([total_ms, e2e_ms, float(np.mean(t_attn)), float(np.mean(t_scores)),
                          float(np.mean(t_select))], dtype=torch.float64, device=dev)
@@ -562,7 +582,9 @@ def main():
                          "flops_per_launch": flops_step},
             "e2e": {"value": e2e_value, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "copies": "upload and download streams, double-buffered device inputs and outputs",
-                    "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps},
+                    "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                    "links_alone": {"h2d_GBps": h2d / (link_ms[0] * 1e-3) / 1e9,
+                                    "ms_per_step_copies_both_ways": link_ms[1]}},
             "gpu_launches": (KERNELS_PER_STEP - (1 if args.fused else 0)) * K_,
             "clocks": clk.summary(),
         }
