@@ -624,6 +624,28 @@ class FasaDecode:
         self.attend(q, K_cache, V_cache, stream)
         return self.o
 
+    def step(self, q, K_cache, V_cache, pos: int):
+        """One decode step for the token at position ``pos`` (its compact key row, select, attend)
+        replayed as a CUDA graph: captured on the first call for these buffers and this position,
+        replayed on later calls (new values in the same q / cache tensors are picked up; the
+        kernels, their arguments and the buffers are fixed at capture).  Runs on the current
+        stream; returns ``self.o``."""
+        key = (q.data_ptr(), K_cache.data_ptr(), V_cache.data_ptr(), int(pos))
+        if getattr(self, "_graph_key", None) != key:
+            side = torch.cuda.Stream(q.device)
+            side.wait_stream(torch.cuda.current_stream(q.device))
+            with torch.cuda.stream(side):  # one eager step before capture
+                self.refresh_keys(K_cache, pos0=pos, npos=1)
+                self(q, K_cache, V_cache)
+            torch.cuda.current_stream(q.device).wait_stream(side)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                self.refresh_keys(K_cache, pos0=pos, npos=1)
+                self(q, K_cache, V_cache)
+            self._graph, self._graph_key = graph, key
+        self._graph.replay()
+        return self.o
+
 
 def selftest_bounded_wait(limit_ms: int, complete: bool, device="cuda", stream=None) -> int:
     """sfa_selftest_bounded_wait: returns the device status word (0 or SFA_ERR_TIMEOUT)."""

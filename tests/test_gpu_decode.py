@@ -137,3 +137,27 @@ def test_decode_full_size_sampled_rows():
         assert stats["mismatches"] == 0, stats["bad_rows"]
         if np.array_equal(m.idx[b, h].cpu().numpy(), idx[0, 0]):
             np.testing.assert_allclose(m.o[b, h].cpu().to(torch.float64).numpy(), o[0, 0], rtol=0, atol=TOL_O)
+
+
+def test_graph_step_matches_eager():
+    """FasaDecode.step (the step's kernels captured once as a CUDA graph, then replayed) gives the
+    eager step's index lists and outputs bit for bit, also after new query values are written into
+    the captured q buffer."""
+    w = D("graph-step", batch=2, heads_q=8, heads_kv=2, seq_len=9000)
+    m, q, K, V, fc = run(w)
+    dev = torch.device("cuda")
+    qd, Kd, Vd = q.to(dev), K.to(dev), V.to(dev)
+    pos = w.seq_len - 1
+    for qv in (qd.clone(), (qd * -0.5).contiguous()):
+        qd.copy_(qv)
+        m.refresh_keys(Kd, pos0=pos, npos=1)
+        m(qd, Kd, Vd)
+        torch.cuda.synchronize()
+        idx_e, o_e = m.idx.clone(), m.o.clone()
+        for _ in range(2):
+            m.idx.fill_(-7)
+            m.step(qd, Kd, Vd, pos)
+            torch.cuda.synchronize()
+            assert torch.equal(m.idx, idx_e)
+            assert torch.equal(m.o, o_e)
+    assert int(m.status.item()) == 0
