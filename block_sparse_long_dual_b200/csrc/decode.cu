@@ -1027,7 +1027,7 @@ __global__ void __launch_bounds__(kThreads, 1) tip_merge_kernel(DecodeParams p) 
 // fac: CTA per (b, h), 16 warps
 // ---------------------------------------------------------------------------
 constexpr int kFacWarps = 16;
-constexpr int kFacBatch = 8;  // tokens per warp with loads in flight
+constexpr int kFacBatch = 16;  // tokens per warp with loads in flight
 
 template <int D>
 __global__ void __launch_bounds__(kFacWarps * 32) fac_kernel(DecodeParams p) {
@@ -1056,39 +1056,44 @@ __global__ void __launch_bounds__(kFacWarps * 32) fac_kernel(DecodeParams p) {
   for (int e = 0; e < DPL; ++e) acc[e] = 0.f;
 
   for (int base = warp * kFacBatch; base < p.k; base += kFacWarps * kFacBatch) {
+    // The batch's token indices (lane u < kFacBatch loads index base + u), broadcast, then all
+    // the batch's K / V row slices loaded before any is used.
+    int tl = -1;
+    if (lane < kFacBatch && base + lane < p.k) {
+      tl = __ldg(list + base + lane);
+      if (tl >= p.L || tl < -1) {  // out of range (-1 is padding): record, skip the row
+        bad = 1;
+        tl = -1;
+      }
+    }
     int tok[kFacBatch];
-    float kv[kFacBatch][DPL], vv[kFacBatch][DPL];
+    uint2 ku[kFacBatch], vu[kFacBatch];  // this lane's DPL bf16 of the token's K and V rows
 #pragma unroll
     for (int u = 0; u < kFacBatch; ++u) {
-      const int r = base + u;
-      int t = r < p.k ? __ldg(list + r) : -1;
-      if (t >= p.L || t < -1) {  // out of range (-1 is padding): record, skip the row
-        if (lane == 0) bad = 1;
-        t = -1;
-      }
-      tok[u] = t;
-      const int ts = t < 0 ? 0 : t;
+      tok[u] = __shfl_sync(0xffffffffu, tl, u);
+      const int ts = tok[u] < 0 ? 0 : tok[u];
       const __nv_bfloat16* kr = kbase + (size_t)ts * D + lane * DPL;
       const __nv_bfloat16* vr = vbase + (size_t)ts * D + lane * DPL;
       if constexpr (DPL == 4) {
-        const uint2 ku = __ldg(reinterpret_cast<const uint2*>(kr));
-        const uint2 vu = __ldg(reinterpret_cast<const uint2*>(vr));
-        kv[u][0] = __uint_as_float(ku.x << 16); kv[u][1] = __uint_as_float(ku.x & 0xFFFF0000u);
-        kv[u][2] = __uint_as_float(ku.y << 16); kv[u][3] = __uint_as_float(ku.y & 0xFFFF0000u);
-        vv[u][0] = __uint_as_float(vu.x << 16); vv[u][1] = __uint_as_float(vu.x & 0xFFFF0000u);
-        vv[u][2] = __uint_as_float(vu.y << 16); vv[u][3] = __uint_as_float(vu.y & 0xFFFF0000u);
+        ku[u] = __ldg(reinterpret_cast<const uint2*>(kr));
+        vu[u] = __ldg(reinterpret_cast<const uint2*>(vr));
       } else {
-        const uint32_t ku = __ldg(reinterpret_cast<const uint32_t*>(kr));
-        const uint32_t vu = __ldg(reinterpret_cast<const uint32_t*>(vr));
-        kv[u][0] = __uint_as_float(ku << 16); kv[u][1] = __uint_as_float(ku & 0xFFFF0000u);
-        vv[u][0] = __uint_as_float(vu << 16); vv[u][1] = __uint_as_float(vu & 0xFFFF0000u);
+        ku[u] = make_uint2(__ldg(reinterpret_cast<const uint32_t*>(kr)), 0u);
+        vu[u] = make_uint2(__ldg(reinterpret_cast<const uint32_t*>(vr)), 0u);
       }
     }
 #pragma unroll
     for (int u = 0; u < kFacBatch; ++u) {
+      float kv[DPL], vv[DPL];
+      kv[0] = __uint_as_float(ku[u].x << 16); kv[1] = __uint_as_float(ku[u].x & 0xFFFF0000u);
+      vv[0] = __uint_as_float(vu[u].x << 16); vv[1] = __uint_as_float(vu[u].x & 0xFFFF0000u);
+      if constexpr (DPL == 4) {
+        kv[2] = __uint_as_float(ku[u].y << 16); kv[3] = __uint_as_float(ku[u].y & 0xFFFF0000u);
+        vv[2] = __uint_as_float(vu[u].y << 16); vv[3] = __uint_as_float(vu[u].y & 0xFFFF0000u);
+      }
       float s = 0.f;
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) s = fmaf(q[e], kv[u][e], s);
+      for (int e = 0; e < DPL; ++e) s = fmaf(q[e], kv[e], s);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
       if (tok[u] < 0) continue;  // padding (warp-uniform)
@@ -1096,7 +1101,7 @@ __global__ void __launch_bounds__(kFacWarps * 32) fac_kernel(DecodeParams p) {
       const float f = expf(m - mn), pe = expf(s - mn);
       l = l * f + pe;
 #pragma unroll
-      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(acc[e], f, pe * vv[u][e]);
+      for (int e = 0; e < DPL; ++e) acc[e] = fmaf(acc[e], f, pe * vv[e]);
       m = mn;
     }
   }
