@@ -313,22 +313,31 @@ def run_decode(args, w: wl.DecodeWorkload, rank, world):
     torch.cuda.synchronize(dev)
     if int(m.status.item()) != 0:
         raise RuntimeError(f"device status {int(m.status.item())}")
+    # stage times: each stage captured as a CUDA graph of its own and replayed back to back, so
+    # that host launch costs do not show up as device time
+    def graph_ms(fn, reps):
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fn()
+        stream.wait_stream(side)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        g.replay()
+        torch.cuda.synchronize(dev)
+        g0, g1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        g0.record(stream)
+        for _ in range(reps):
+            g.replay()
+        g1.record(stream)
+        torch.cuda.synchronize(dev)
+        return g0.elapsed_time(g1) / reps
+
     K_ = max(args.steps, 50)
-    # stage times: the step's kernels launched one by one with events between them
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_)]
-    torch.cuda.synchronize(dev)
-    for s_ in range(K_):
-        ev[s_][0].record(stream)
-        m.refresh_keys(Kd, pos0=w.seq_len - 1, npos=1)
-        ev[s_][1].record(stream)
-        m.select(qd)
-        ev[s_][2].record(stream)
-        m.attend(qd, Kd, Vd)
-        ev[s_][3].record(stream)
-    torch.cuda.synchronize(dev)
-    t_sel = float(np.mean([ev[s_][1].elapsed_time(ev[s_][2]) for s_ in range(K_)]))
-    t_att = float(np.mean([ev[s_][2].elapsed_time(ev[s_][3]) for s_ in range(K_)]))
-    t_app = float(np.mean([ev[s_][0].elapsed_time(ev[s_][1]) for s_ in range(K_)]))
+    t_app = graph_ms(lambda: m.refresh_keys(Kd, pos0=w.seq_len - 1, npos=1), K_)
+    t_sel = graph_ms(lambda: m.select(qd), K_)
+    t_att = graph_ms(lambda: m.attend(qd, Kd, Vd), K_)
     # the timed steps: graph replays back to back
     start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if dist:
