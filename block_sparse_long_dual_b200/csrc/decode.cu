@@ -602,7 +602,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
 
 // ---------------------------------------------------------------------------
 // tip_merge: CTA per (b, h).  The chunks' candidate words (token order, counts
-// per warp segment) are staged in shared memory when they fit (kMergeSmem), a
+// per warp segment) are staged in shared memory when they fit (merge_cap <=
+// kMergeSmem, set per launch from the number of chunks), a
 // warp per segment, and their 16-bit filter keys held in registers.  The k-th
 // largest filter key X (a four-way bisection between the least and largest
 // key) bounds the row's exact k-th largest score from below by value(X) - M
@@ -622,7 +623,7 @@ constexpr int kMergeRank = 512;                    // survivors ranked by counti
 constexpr int kSegBatch = 16;                      // segments a warp stages with their loads in flight
 constexpr int kMaxChunks = 512;
 
-__global__ void __launch_bounds__(kThreads, 1) tip_merge_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 2) tip_merge_kernel(DecodeParams p) {
   extern __shared__ __align__(16) uint32_t msm[];
   __shared__ uint32_t hist[256];
   __shared__ int sh[64];
@@ -740,11 +741,12 @@ __global__ void __launch_bounds__(kThreads, 1) tip_merge_kernel(DecodeParams p) 
   };
   int kept;
   const int ob = (nseg + 1 + 3) & ~3;  // arrays start after the offsets (16-byte aligned)
-  if (n <= kMergeSmem) {
+  const int cap = p.merge_cap;
+  if (n <= cap) {
     uint64_t* gk = reinterpret_cast<uint64_t*>(msm + ob);  // [kMergeExact] survivors' exact keys
     int* stok = reinterpret_cast<int*>(gk + kMergeExact);   // [kMergeExact] survivors' tokens
     int* sv = stok + kMergeExact;                            // [n] survivor positions (then losers)
-    int* wc = sv + kMergeSmem;                               // [kMergeKeys][kWarps] counts
+    int* wc = sv + cap;                                      // [kMergeKeys][kWarps] counts
     uint32_t* sc = reinterpret_cast<uint32_t*>(wc + kMergeKeys * kWarps);  // [n] candidate words
     // Warp w stages segments kSegBatch at a time (w kSegBatch + 8 kSegBatch j ...): lane l takes words
     // 2 l and 2 l + 1 of each segment in one load (a segment starts 8-byte aligned and both words
@@ -1201,11 +1203,15 @@ cudaError_t launch_decode_select(const DecodeParams& p, cudaStream_t st) {
                            : launch_tip_chunk<8>(p, st);
   if (e != cudaSuccess) return e;
   // offsets, survivors' keys and tokens, survivor positions, compaction counts, candidate words
-  const size_t msmem = ((size_t)p.nchunks * kWarps + 4 + (size_t)3 * kMergeExact + kMergeSmem +
-                        (size_t)kMergeKeys * kWarps + kMergeSmem) * sizeof(uint32_t);
+  // Candidate capacity: all of them for a few chunks (about k + 10% per chunk), so that two or three
+  // CTAs share an SM when there are many rows; the full kMergeSmem otherwise.
+  DecodeParams q = p;
+  q.merge_cap = p.nchunks <= 8 ? 4096 : kMergeSmem;
+  const size_t msmem = ((size_t)p.nchunks * kWarps + 4 + (size_t)3 * kMergeExact + q.merge_cap +
+                        (size_t)kMergeKeys * kWarps + q.merge_cap) * sizeof(uint32_t);
   e = cudaFuncSetAttribute(tip_merge_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
   if (e != cudaSuccess) return e;
-  tip_merge_kernel<<<p.B * p.Hq, kThreads, msmem, st>>>(p);
+  tip_merge_kernel<<<p.B * p.Hq, kThreads, msmem, st>>>(q);
   return cudaGetLastError();
 }
 

@@ -89,6 +89,7 @@ struct DecodeParams {
   float* lse;        // [B, Hq] (nullable)
   int* status;
   int B, Hq, Hkv, L, D, nfc, k, chunk, nchunks, tps, nstages;
+  int merge_cap;     // candidates a merge CTA stages in shared memory (set at launch)
   float scale;
   uint8_t fc[1024];  // [Hkv][nfc] dominant pair indices
 };
