@@ -21,10 +21,12 @@
 //                  ranked (key desc, index asc); ascending index list, -1
 //                  padded (a radix select with scores recomputed on the fly
 //                  when the candidates do not fit).
-//   fac            Focused Attention Computation: CTA per (b, h), 16 warps,
-//                  each warp gathers the K / V rows of its share of the kept
-//                  tokens (eight tokens' loads in flight per lane), float32
-//                  online softmax, warps merged through shared memory.
+//   fac            Focused Attention Computation: CTA per (b, h), 16 warps (8
+//                  when the rows fill two CTAs per SM); each warp gathers the
+//                  K / V rows of its share of the kept tokens (sixteen tokens'
+//                  loads in flight per lane, their indices loaded once and
+//                  broadcast), float32 online softmax, warps merged through
+//                  shared memory.
 //
 // Ranking: the token score is the dot product over the dominant pairs' dims;
 // it is ranked by its float64 value (key = order-preserving uint64 of the
@@ -1026,12 +1028,11 @@ __global__ void __launch_bounds__(kThreads, 2) tip_merge_kernel(DecodeParams p) 
 }
 
 // ---------------------------------------------------------------------------
-// fac: CTA per (b, h), 16 warps
+// fac: CTA per (b, h), 16 or 8 warps
 // ---------------------------------------------------------------------------
-constexpr int kFacWarps = 16;
 constexpr int kFacBatch = 16;  // tokens per warp with loads in flight
 
-template <int D>
+template <int D, int kFacWarps>
 __global__ void __launch_bounds__(kFacWarps * 32) fac_kernel(DecodeParams p) {
   constexpr int DPL = D / 32;  // dims per lane (4 for d = 128, 2 for d = 64)
   __shared__ float wm[kFacWarps], wl[kFacWarps];
@@ -1215,11 +1216,20 @@ cudaError_t launch_decode_select(const DecodeParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// 16 warps per row while the rows fill fewer than two CTAs per SM, else 8 (two CTAs per SM).
 cudaError_t launch_decode_attn(const DecodeParams& p, cudaStream_t st) {
-  if (p.D == 128)
-    fac_kernel<128><<<p.B * p.Hq, kFacWarps * 32, 0, st>>>(p);
-  else
-    fac_kernel<64><<<p.B * p.Hq, kFacWarps * 32, 0, st>>>(p);
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int rows = p.B * p.Hq;
+  const bool many = rows >= 2 * sms;
+  if (p.D == 128) {
+    if (many) fac_kernel<128, 8><<<rows, 256, 0, st>>>(p);
+    else fac_kernel<128, 16><<<rows, 512, 0, st>>>(p);
+  } else {
+    if (many) fac_kernel<64, 8><<<rows, 256, 0, st>>>(p);
+    else fac_kernel<64, 16><<<rows, 512, 0, st>>>(p);
+  }
   return cudaGetLastError();
 }
 

@@ -39,6 +39,8 @@ CASES = [
     # consecutive chunks of the same rows, the second one (a ragged last chunk among them) with
     # the bound carried from the first and its candidates taken straight from the scores
     D("multi-tile-runs", batch=8, heads_q=32, heads_kv=8, seq_len=20000),
+    # rows enough for two attention CTAs per SM: the eight-warp attention kernel
+    D("many-rows-eight-warp-attention", batch=10, heads_q=32, heads_kv=8, seq_len=3000),
 ]
 
 
