@@ -315,9 +315,13 @@ size_t sfa_decode_workspace(const sfa_shape* shape, int k);
  * aligned (SFA_ERR_WORKSPACE).  status_word (device, nullable):
  * SFA_ERR_TIMEOUT if a copy of the compact keys did not land within about 2 s
  * (that chunk then contributes no tokens).  Launches 2 kernels: a persistent
- * one (per chunk of the cache: float32 scores, a lower bound of the chunk's
- * k-th largest, the tokens above it with their float64 scores) and a merge
- * (exact top k of the candidates).
+ * one (per chunk of the cache: float32 filter scores, a lower bound of the
+ * row's k-th largest score found in the chunk or carried from an earlier
+ * chunk of the same rows, the tokens above it with their 16-bit filter keys
+ * and the chunk's filter error bound) and a merge per row (a tighter bound
+ * from the candidates' filter keys, float64 scores of the survivors, exact top
+ * k).  The calls of one step may be captured in a CUDA graph (all buffers
+ * fixed at capture), as FasaDecode.step does.
  */
 sfa_status sfa_decode_select(const sfa_shape* shape, const void* q, const void* K_fc, const int* fc,
                              int nfc, int k, int* idx, void* workspace, size_t workspace_bytes,
