@@ -7,7 +7,8 @@
 //   tip_chunk      Token Importance Predictor, persistent (one or two CTAs per
 //                  SM) over tiles (chunk of C tokens, b, KV head): the chunk's
 //                  K_fc rows stream through a bulk-copy ring once for all Q
-//                  heads of the group; each token's score is first taken on
+//                  heads of the group (a ninth warp refills each stage as soon
+//                  as the eight consumer warps release it); each token's score is first taken on
 //                  the tensor cores in float32 (a filter), then per head a lower bound
 //                  of the chunk's k-th largest score (from group maxima),
 //                  lowered by twice the filter's error bound M, and the tokens
@@ -313,7 +314,7 @@ __global__ void __launch_bounds__(kThreads) fc_gather_kernel(DecodeParams p, con
 // flight while this tile's candidates are selected.
 // ---------------------------------------------------------------------------
 template <int G, int TPS, int NGR>
-__global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(DecodeParams p) {
+__global__ void __launch_bounds__(kThreads + 32, G <= 4 ? 2 : 1) tip_chunk_kernel(DecodeParams p) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   constexpr int ST = kThreads * TPS;
   const int W = 2 * p.nfc;
@@ -323,7 +324,8 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
   unsigned char* ring = smem_raw;                                                           // [NS][SB]
   uint16_t* keys = reinterpret_cast<uint16_t*>(ring + (size_t)NS * SB);                   // [G][C]
   float* qd = reinterpret_cast<float*>(keys + (size_t)G * C);                              // [W][G]
-  __shared__ __align__(8) uint64_t bars[4];
+  __shared__ __align__(8) uint64_t bars[4];   // stage filled (one arrival + the copy's bytes)
+  __shared__ __align__(8) uint64_t ebars[4];  // stage consumed (one arrival per consumer warp)
   __shared__ int scratch[128];
   __shared__ int lost;
 
@@ -359,13 +361,32 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
   };
   if (tid == 0) {
     lost = 0;
-    for (int st = 0; st < NS; ++st)
+    for (int st = 0; st < NS; ++st) {
       asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"((uint32_t)__cvta_generic_to_shared(&bars[st]))
                    : "memory");
+      asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"((uint32_t)__cvta_generic_to_shared(&ebars[st])),
+                   "r"(kWarps)
+                   : "memory");
+    }
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int st = 0; st < NS; ++st) issue_next();
   }
   __syncthreads();
+  // Warp 8 is the producer: it refills each stage as soon as the eight consumer warps have
+  // released it, so no consumer waits on a copy being issued.  The consumers synchronise among
+  // themselves on named barrier 1 from here on.
+  if (tid >= kThreads) {
+    if (tid == kThreads) {
+      while (ptile < t_end) {
+        const int i = issued;
+        if (i >= NS &&
+            !wait_parity_bounded((uint32_t)__cvta_generic_to_shared(&ebars[i % NS]), ((i / NS) - 1) & 1))
+          lost = 1;
+        issue_next();
+      }
+    }
+    return;
+  }
+  auto consumers_sync = [] { asm volatile("bar.sync 1, %0;" ::"n"(kThreads) : "memory"); };
 
   int consumed = 0;
   // The bound carried to the next chunk of the same rows (warp h keeps head h's): the raw k-th
@@ -387,7 +408,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
       const __nv_bfloat16* qrow = static_cast<const __nv_bfloat16*>(p.q) + ((size_t)b * p.Hq + g * G + hh) * p.D;
       qd[c * G + hh] = __bfloat162float(qrow[dim]);
     }
-    __syncthreads();
+    consumers_sync();
 
     // Filter scores on the tensor cores: per slab, warp w takes 16-token tiles of its share, the
     // compact columns in k-steps of 8 (mma.sync m16n8k8, bf16 in, float32 out; A = tokens x
@@ -454,15 +475,18 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
                   __byte_perm(order_key_signed_zero(c[mt][1]), order_key_signed_zero(c[mt][3]), 0x7632);
           }
         }
-        __syncthreads();  // stage consumed
-        if (tid == 0) issue_next();
+        __syncwarp();  // stage consumed by this warp
+        if ((tid & 31) == 0)
+          asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(
+                           (uint32_t)__cvta_generic_to_shared(&ebars[stg]))
+                       : "memory");
       }
     }
     {
       const uint32_t a16 = __reduce_max_sync(0xffffffffu, max(am & 0xFFFFu, am >> 16));
       if ((tid & 31) == 0) scratch[64 + (tid >> 5)] = (int)a16;
     }
-    __syncthreads();
+    consumers_sync();
 
     // Per head, a lower bound LB of the chunk's k-th largest key, by warp h alone: the maxima
     // of the C / 4 groups of 4 consecutive keys (0 past the end of the chunk), then a bisection
@@ -532,7 +556,7 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
         }
         if (lane == 0) scratch[warp] = (int)LBw;
       }
-      __syncthreads();
+      consumers_sync();
     }
     uint32_t LB[G];
 #pragma unroll
@@ -591,12 +615,13 @@ __global__ void __launch_bounds__(kThreads, G <= 4 ? 2 : 1) tip_chunk_kernel(Dec
     }
     if (bad && tid == 0) report(p.status, SFA_ERR_TIMEOUT);
     run_bg = bg;
-    __syncthreads();  // keys / qd free for the next tile
+    consumers_sync();  // keys / qd free for the next tile
   }
-  // After a wait that gave up, let this CTA's copies land (bounded) before it exits.
+  // After a wait that gave up, let this CTA's copies land (bounded) before it exits: every copy
+  // the producer issued completes a phase of its stage's barrier (consumed counts them all).
   if (tid == 0 && lost) {
-    for (int st = 0; st < NS && st < issued; ++st) {
-      const int uses = (issued - st + NS - 1) / NS;
+    for (int st = 0; st < NS && st < consumed; ++st) {
+      const int uses = (consumed - st + NS - 1) / NS;
       wait_parity_bounded((uint32_t)__cvta_generic_to_shared(&bars[st]), (uses - 1) & 1);
     }
   }
@@ -1182,7 +1207,7 @@ static cudaError_t launch_tip_chunk_t(const DecodeParams& p, cudaStream_t st) {
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int ntiles = p.nchunks * p.B * p.Hkv;
   const int grid = sms * d.ctas_per_sm;
-  kern<<<ntiles < grid ? ntiles : grid, kThreads, d.smem, st>>>(p);
+  kern<<<ntiles < grid ? ntiles : grid, kThreads + 32, d.smem, st>>>(p);
   return cudaGetLastError();
 }
 
