@@ -26,7 +26,9 @@
 //                    memory), M = N = 128, K = 16 steps; completion tracked with
 //                    tcgen05.commit -> mbarriers.  A commit covers every MMA the
 //                    thread issued before it, so the commit that signals S_t(j)
-//                    also means O_t has absorbed P_t(j-1).
+//                    also means O_t has absorbed P_t(j-1).  The softmax threads
+//                    signal P_t in two parts (chunks 0-1, then 2-3 of each column
+//                    half), so half of P_t.V_t runs while they compute the rest.
 // TMEM (256 KT columns): S_t at [128 t, 128 t + 128), O_t at [128 (KT + t), +128);
 // P_t aliases S_t (two bf16 per column): keys [0,64) in S columns [0,32), keys
 // [64,128) in S columns [64,96), each half written by the threads that read it.
@@ -48,9 +50,10 @@ constexpr uint32_t kSub = 16384;       // 128 rows x 64 bf16 (one 128B-swizzle b
 constexpr uint32_t kTile = 2 * kSub;   // 128 x 128 bf16
 // Barriers, two of each (one per tile) except DRAIN and QR.
 enum { B_Q = 0, B_KF = 2, B_VF = 4, B_KE = 6, B_VE = 8, B_SF = 10, B_PF = 12, B_OD = 14, B_X = 16, B_DRAIN = 32,
-       B_QR = 33, NBAR = 34 };  // B_X: [tile][warp pair][parity] row-max / row-sum exchange of the two
-                                // column halves (warps w and w + 4, 64 arrivals); B_QR: the CTA's Q tiles
-                                // rotated in shared memory (RoPE on load)
+       B_QR = 33, B_PH = 34, NBAR = 36 };  // B_X: [tile][warp pair][parity] row-max / row-sum exchange of
+                                           // the two column halves (warps w and w + 4, 64 arrivals); B_QR:
+                                           // the CTA's Q tiles rotated in shared memory (RoPE on load);
+                                           // B_PH: the first half of P_t written (B_PF: all of it)
 constexpr int kMaxList = 2048;  // nb <= 2048, so a valid list has <= 2048 entries
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
@@ -261,7 +264,8 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
       *cx.abort_flag = 0;
       for (int k = 0; k < NBAR; ++k)
         tc::mbar_init(cx.bar(k), k == B_QR ? KT * 256
-                                 : (k == B_PF || k == B_PF + 1) ? 256 : (k >= B_X && k < B_X + 16) ? 64 : 1);
+                                 : (k == B_PF || k == B_PF + 1 || k == B_PH || k == B_PH + 1) ? 256
+                                 : (k >= B_X && k < B_X + 16) ? 64 : 1);
       tc::fence_mbar_init();
     }
   } else if (warp == L::kProducerWarp && lane == 0) {
@@ -359,18 +363,33 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
 #pragma unroll
         for (int t = 0; t < KT; ++t) {
           if (!ok || it >= tl[t].n) continue;
-          // O_t += P_t(it) V_t(it)
-          if (!wait_bar(cx, cx.bar(B_PF + t), it & 1) || !wait_bar(cx, cx.bar(B_VF + t), it & 1)) {
+          // O_t += P_t(it) V_t(it), in two parts: the key steps whose P chunks the softmax threads
+          // store first (chunks 0 and 1 of each column half) as soon as those are written, while
+          // the threads still compute the rest; then the others.
+          if (!wait_bar(cx, cx.bar(B_PH + t), it & 1) || !wait_bar(cx, cx.bar(B_VF + t), it & 1)) {
             ok = false;
             break;
           }
           tc::tc_fence_after();
           const uint32_t sV = cx.sbase + L::off_v(t);
-#pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            // P keys [16 kk, 16 kk + 16): half kk / 4 wrote them into its own S columns
+          // P keys [16 kk, 16 kk + 16): half kk / 4 wrote them into its own S columns (chunk kk % 4)
+          auto pv = [&](int kk, uint32_t acc) {
             tc::mma_bf16_ts(tmem + L::col_o(t), tmem + L::col_s(t) + (kk >> 2) * 64 + (kk & 3) * 8,
-                            tc::sw128_desc(sV + kk * 2048, kSub, 1024), id_pv, (it > 0 || kk > 0) ? 1u : 0u);
+                            tc::sw128_desc(sV + kk * 2048, kSub, 1024), id_pv, acc);
+          };
+          pv(0, it > 0 ? 1u : 0u);
+          pv(1, 1u);
+          pv(4, 1u);
+          pv(5, 1u);
+          if (!wait_bar(cx, cx.bar(B_PF + t), it & 1)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          pv(2, 1u);
+          pv(3, 1u);
+          pv(6, 1u);
+          pv(7, 1u);
           tc::mma_commit(cx.bar(B_VE + t));
           if (it + 1 < tl[t].n) {
             // S_t(it + 1) = Q_t K_t(it + 1)^T overwrites the TMEM columns holding P_t(it): issue it
@@ -508,6 +527,11 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
         tc::tmem_st8(tP + c * 8, pk);
+        if (c == 1) {  // chunks 0 and 1 written: the tensor core may start on them
+          tc::tmem_wait_st();
+          tc::tc_fence_before();
+          tc::mbar_arrive(cx.bar(B_PH + t));
+        }
         if (c < 3) tc::tmem_wait_ld();
       }
       float rs0, rs1, rs2, rs3;
