@@ -11,27 +11,25 @@
 // CTA's prologue (barriers, tensor memory, Q) and epilogue (O) hide behind the
 // other's main loop.
 //
-//   warps 0 .. 8 KT - 1  softmax of tile w / 8: two threads per query row r
-//                    (TMEM lane r; warps w and w+4 share lanes), each owning 64
-//                    of the 128 key columns, row maxima exchanged through shared
-//                    memory (one barrier per warp pair); reads S_t from TMEM, online softmax with a lazily
-//                    rescaled O_t, writes P_t (bf16) back into the S_t columns of
-//                    TMEM, final O_t / l epilogue.  Two softmax warps per SM
-//                    sub-partition work on a tile at once, hiding each other's
-//                    latency.
-//   warp 8 KT        producer: TMA loads of Q_t and of K_t(j), V_t(j) for every
+//   warps 0 .. 4 KT - 1  softmax of tile w / 4: one thread per query row r
+//                    (TMEM lane r = 32 (w % 4) + lane).  The thread loads its
+//                    whole row of S_t (128 columns) into registers, takes the
+//                    row maximum with no exchange, rescales O_t lazily, computes
+//                    P_t from the same registers and writes it (bf16) back into
+//                    the S_t columns of TMEM; final O_t / l epilogue.
+//   warp 4 KT        producer: TMA loads of Q_t and of K_t(j), V_t(j) for every
 //                    kept block j of each tile (one K and one V slot per tile).
-//   warp 8 KT + 1    MMA issuer: S_t = Q_t K_t^T (A, B from shared memory) and
+//   warp 4 KT + 1    MMA issuer: S_t = Q_t K_t^T (A, B from shared memory) and
 //                    O_t += P_t V_t (A = P_t from TMEM, B = V_t from shared
 //                    memory), M = N = 128, K = 16 steps; completion tracked with
 //                    tcgen05.commit -> mbarriers.  A commit covers every MMA the
 //                    thread issued before it, so the commit that signals S_t(j)
 //                    also means O_t has absorbed P_t(j-1).  The softmax threads
-//                    signal P_t in two parts (chunks 0-1, then 2-3 of each column
-//                    half), so half of P_t.V_t runs while they compute the rest.
+//                    signal P_t in two parts (keys [0, 64), then [64, 128)), so
+//                    half of P_t.V_t runs while they compute the rest.
 // TMEM (256 KT columns): S_t at [128 t, 128 t + 128), O_t at [128 (KT + t), +128);
-// P_t aliases S_t (two bf16 per column): keys [0,64) in S columns [0,32), keys
-// [64,128) in S columns [64,96), each half written by the threads that read it.
+// P_t aliases S_t (two bf16 per column): keys [16 c, 16 c + 16) in S columns
+// [8 c, 8 c + 8), written once the whole row of S_t is in registers.
 // Every mbarrier wait is bounded (about 2 s); a wait that runs out writes
 // SFA_ERR_TIMEOUT to the status word, raises a CTA-wide abort flag, drains the
 // copies / MMAs this CTA issued and frees its tensor memory.
@@ -49,11 +47,9 @@ constexpr int kHD = 128;
 constexpr uint32_t kSub = 16384;       // 128 rows x 64 bf16 (one 128B-swizzle box)
 constexpr uint32_t kTile = 2 * kSub;   // 128 x 128 bf16
 // Barriers, two of each (one per tile) except DRAIN and QR.
-enum { B_Q = 0, B_KF = 2, B_VF = 4, B_KE = 6, B_VE = 8, B_SF = 10, B_PF = 12, B_OD = 14, B_X = 16, B_DRAIN = 32,
-       B_QR = 33, B_PH = 34, NBAR = 36 };  // B_X: [tile][warp pair][parity] row-max / row-sum exchange of
-                                           // the two column halves (warps w and w + 4, 64 arrivals); B_QR:
-                                           // the CTA's Q tiles rotated in shared memory (RoPE on load);
-                                           // B_PH: the first half of P_t written (B_PF: all of it)
+enum { B_Q = 0, B_KF = 2, B_VF = 4, B_KE = 6, B_VE = 8, B_SF = 10, B_PF = 12, B_OD = 14, B_PH = 16, B_DRAIN = 18,
+       B_QR = 19, NBAR = 20 };  // B_PH: the first half of P_t written (B_PF: all of it); B_QR: the CTA's
+                                // Q tiles rotated in shared memory (RoPE on load)
 constexpr int kMaxList = 2048;  // nb <= 2048, so a valid list has <= 2048 entries
 constexpr uint64_t kTimeoutNs = 2000000000ull;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units: rescale O only when the max grows by > 2^8
@@ -70,13 +66,13 @@ struct Layout {
   static __host__ __device__ constexpr uint32_t off_v(int t) { return 2 * KT * kTile + t * kTile; }
   static constexpr uint32_t OFF_BAR = 3 * KT * kTile;
   static constexpr uint32_t OFF_MISC = OFF_BAR + NBAR * 8;
-  static constexpr uint32_t OFF_XCHG = OFF_MISC + 32;  // [KT tiles][2 parities][2 halves][128 rows] float
-  static constexpr uint32_t OFF_LIST = OFF_XCHG + KT * 2 * 2 * 128 * 4;  // per tile: the validated index list
+  static constexpr uint32_t OFF_LIST = OFF_MISC + 32;  // per tile: the validated index list
   static constexpr uint32_t SMEM_BYTES = OFF_LIST + KT * kMaxList * 4 + 1024;
-  // Warps 0 .. 8 KT - 1: softmax of tile w / 8 (two threads per query row: warps w and w + 4
-  // share TMEM lanes and split the 128 key columns); then the TMA producer and the MMA issuer.
-  static constexpr int kThreads = KT * 256 + 64;
-  static constexpr int kProducerWarp = KT * 8, kMmaWarp = KT * 8 + 1;
+  // Warps 0 .. 4 KT - 1: softmax of tile w / 4 (one thread per query row, warp w on TMEM lanes
+  // [32 (w % 4), +32)); then the TMA producer and the MMA issuer.
+  static constexpr int kSoftmaxThreads = KT * 128;
+  static constexpr int kThreads = kSoftmaxThreads + 64;
+  static constexpr int kProducerWarp = KT * 4, kMmaWarp = KT * 4 + 1;
   static constexpr uint32_t TMEM_COLS = KT * 256;
   static __host__ __device__ constexpr uint32_t col_s(int t) { return t * 128; }
   static __host__ __device__ constexpr uint32_t col_o(int t) { return KT * 128 + t * 128; }
@@ -139,18 +135,19 @@ __device__ Tile decode_tile(const AttnParams& p, int t) {
   return x;
 }
 
-// RoPE on load: the 256 KT softmax threads rotate the CTA's Q tiles in shared
+// RoPE on load: the 128 KT softmax threads rotate the CTA's Q tiles in shared
 // memory once their TMA copies have landed (bounded waits on the tiles' B_Q
 // barriers); returns false if a wait gave up.  Work unit = (row, 16-byte
 // chunk c) of a tile: chunk c of box 0 holds dims [8c, 8c + 8) and the same
 // offset of box 1 holds their rotary partners [64 + 8c, 64 + 8c + 8) (chunk c of
 // row r is stored at chunk c ^ (r & 7) of the 128-byte row).  Thread st takes
-// chunk st & 7 of rows st / 8 + 32 KT j (j < 4 / KT), so a warp touches four whole
-// rows: conflict-free in shared memory, and each row's table entries are one
-// contiguous 256-byte run.  The two tiles usually share the query block (two
-// heads of a GQA group), so the table entries are fetched once, before the
-// waits, and their latency hides behind the copies.  Kept out of line: it runs
-// once per CTA and must not add to the register pressure of the softmax loop.
+// chunk st & 7 of rows st / 8 + 16 KT k (k < 8 / KT), so a warp touches four
+// whole rows: conflict-free in shared memory, and each row's table entries are
+// one contiguous 256-byte run.  Rows go four at a time; the first four rows'
+// table entries are fetched before the waits, so their latency hides behind
+// the copies.  The two tiles usually share the query block (two heads of a GQA
+// group): the entries then serve both.  Kept out of line: it runs once per CTA
+// and must not add to the register pressure of the softmax loop.
 template <int KT>
 __device__ __noinline__ bool rope_q_on_load(volatile int* abort_flag, int* status, uint32_t bar_q0,
                                             unsigned char* sm, const float* cos_t, const float* sin_t, int i0,
@@ -160,51 +157,57 @@ __device__ __noinline__ bool rope_q_on_load(volatile int* abort_flag, int* statu
   cx.bars = 0;
   cx.abort_flag = abort_flag;
   cx.status = status;
-  constexpr int RPT = 4 / KT, RS = 32 * KT;  // rows per thread, row stride between them
+  constexpr int RS = 16 * KT, RPT = 128 / RS, GR = 4;  // row stride, rows per thread, rows per group
+  static_assert(RPT % GR == 0, "whole groups of rows");
   const int c = st & 7;
   const bool two = KT == 2 && n0 > 0 && n1 > 0 && i1 != i0;  // tiles at different query blocks: two slices
   const int ia = n0 > 0 ? i0 : i1;
-  float ca[RPT][8], sa[RPT][8], cb[RPT][8], sb[RPT][8];
+#pragma unroll 1
+  for (int g0 = 0; g0 < RPT; g0 += GR) {
+    float ca[GR][8], sa[GR][8], cb[GR][8], sb[GR][8];
 #pragma unroll
-  for (int k = 0; k < RPT; ++k) {
-    const int row = (st >> 3) + RS * k;
-    load8(cos_t + ((size_t)ia * 128 + row) * 64 + c * 8, ca[k]);
-    load8(sin_t + ((size_t)ia * 128 + row) * 64 + c * 8, sa[k]);
-    if (two) {
-      load8(cos_t + ((size_t)i1 * 128 + row) * 64 + c * 8, cb[k]);
-      load8(sin_t + ((size_t)i1 * 128 + row) * 64 + c * 8, sb[k]);
-    }
-  }
-  bool ok = true;
-  if (n0 > 0) ok = wait_bar(cx, bar_q0, 0);
-  if (ok && KT == 2 && n1 > 0) ok = wait_bar(cx, bar_q0 + 8, 0);  // B_Q + 1
-  if (!__all_sync(0xffffffffu, ok)) return false;
-#pragma unroll
-  for (int t = 0; t < KT; ++t) {
-    if ((t == 0 ? n0 : n1) == 0) continue;
-    const bool use_b = t == 1 && two;
-#pragma unroll
-    for (int k = 0; k < RPT; ++k) {
-      const int row = (st >> 3) + RS * k;
-      unsigned char* rp = sm + Layout<KT>::off_q(t) + row * 128 + ((c ^ (row & 7)) << 4);
-      uint4* plo = reinterpret_cast<uint4*>(rp);
-      uint4* phi = reinterpret_cast<uint4*>(rp + kSub);
-      const uint4 ulo = *plo, uhi = *phi;
-      const uint32_t wl[4] = {ulo.x, ulo.y, ulo.z, ulo.w}, wh[4] = {uhi.x, uhi.y, uhi.z, uhi.w};
-      uint32_t ol[4], oh[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float c0 = use_b ? cb[k][2 * e] : ca[k][2 * e], s0 = use_b ? sb[k][2 * e] : sa[k][2 * e];
-        const float c1 = use_b ? cb[k][2 * e + 1] : ca[k][2 * e + 1];
-        const float s1 = use_b ? sb[k][2 * e + 1] : sa[k][2 * e + 1];
-        float l0, l1, h0, h1;
-        rope_pair(__uint_as_float(wl[e] << 16), __uint_as_float(wh[e] << 16), c0, s0, l0, h0);
-        rope_pair(__uint_as_float(wl[e] & 0xFFFF0000u), __uint_as_float(wh[e] & 0xFFFF0000u), c1, s1, l1, h1);
-        ol[e] = pack_bf16x2(l0, l1);
-        oh[e] = pack_bf16x2(h0, h1);
+    for (int k = 0; k < GR; ++k) {
+      const int row = (st >> 3) + RS * (g0 + k);
+      load8(cos_t + ((size_t)ia * 128 + row) * 64 + c * 8, ca[k]);
+      load8(sin_t + ((size_t)ia * 128 + row) * 64 + c * 8, sa[k]);
+      if (two) {
+        load8(cos_t + ((size_t)i1 * 128 + row) * 64 + c * 8, cb[k]);
+        load8(sin_t + ((size_t)i1 * 128 + row) * 64 + c * 8, sb[k]);
       }
-      *plo = make_uint4(ol[0], ol[1], ol[2], ol[3]);
-      *phi = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+    }
+    if (g0 == 0) {
+      bool ok = true;
+      if (n0 > 0) ok = wait_bar(cx, bar_q0, 0);
+      if (ok && KT == 2 && n1 > 0) ok = wait_bar(cx, bar_q0 + 8, 0);  // B_Q + 1
+      if (!__all_sync(0xffffffffu, ok)) return false;
+    }
+#pragma unroll
+    for (int t = 0; t < KT; ++t) {
+      if ((t == 0 ? n0 : n1) == 0) continue;
+      const bool use_b = t == 1 && two;
+#pragma unroll
+      for (int k = 0; k < GR; ++k) {
+        const int row = (st >> 3) + RS * (g0 + k);
+        unsigned char* rp = sm + Layout<KT>::off_q(t) + row * 128 + ((c ^ (row & 7)) << 4);
+        uint4* plo = reinterpret_cast<uint4*>(rp);
+        uint4* phi = reinterpret_cast<uint4*>(rp + kSub);
+        const uint4 ulo = *plo, uhi = *phi;
+        const uint32_t wl[4] = {ulo.x, ulo.y, ulo.z, ulo.w}, wh[4] = {uhi.x, uhi.y, uhi.z, uhi.w};
+        uint32_t ol[4], oh[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float c0 = use_b ? cb[k][2 * e] : ca[k][2 * e], s0 = use_b ? sb[k][2 * e] : sa[k][2 * e];
+          const float c1 = use_b ? cb[k][2 * e + 1] : ca[k][2 * e + 1];
+          const float s1 = use_b ? sb[k][2 * e + 1] : sa[k][2 * e + 1];
+          float l0, l1, h0, h1;
+          rope_pair(__uint_as_float(wl[e] << 16), __uint_as_float(wh[e] << 16), c0, s0, l0, h0);
+          rope_pair(__uint_as_float(wl[e] & 0xFFFF0000u), __uint_as_float(wh[e] & 0xFFFF0000u), c1, s1, l1, h1);
+          ol[e] = pack_bf16x2(l0, l1);
+          oh[e] = pack_bf16x2(h0, h1);
+        }
+        *plo = make_uint4(ol[0], ol[1], ol[2], ol[3]);
+        *phi = make_uint4(oh[0], oh[1], oh[2], oh[3]);
+      }
     }
   }
   tc::fence_proxy_async_smem();  // the generic-proxy writes become visible to the MMAs
@@ -237,9 +240,9 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
   tl[1] = decode_tile(p, KT == 2 ? 2 * blockIdx.x + 1 : KT * blockIdx.x);
   if (KT == 1) tl[1].valid = false;
 
-  if (warp == 0 || (KT == 2 && warp == 8)) {
+  if (warp == 0 || (KT == 2 && warp == 4)) {
     // Validate one tile's index list: count in [0, kmax], entries ascending in [0, nb), <= i if causal.
-    const int t = warp >> 3;
+    const int t = warp >> 2;
     const Tile x = t == 0 ? tl[0] : tl[1];
     int n = 0;
     if (x.valid) {
@@ -263,9 +266,8 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
     if (warp == 0 && lane == 0) {
       *cx.abort_flag = 0;
       for (int k = 0; k < NBAR; ++k)
-        tc::mbar_init(cx.bar(k), k == B_QR ? KT * 256
-                                 : (k == B_PF || k == B_PF + 1 || k == B_PH || k == B_PH + 1) ? 256
-                                 : (k >= B_X && k < B_X + 16) ? 64 : 1);
+        tc::mbar_init(cx.bar(k), k == B_QR ? L::kSoftmaxThreads
+                                 : (k == B_PF || k == B_PF + 1 || k == B_PH || k == B_PH + 1) ? 128 : 1);
       tc::fence_mbar_init();
     }
   } else if (warp == L::kProducerWarp && lane == 0) {
@@ -363,31 +365,30 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
 #pragma unroll
         for (int t = 0; t < KT; ++t) {
           if (!ok || it >= tl[t].n) continue;
-          // O_t += P_t(it) V_t(it), in two parts: the key steps whose P chunks the softmax threads
-          // store first (chunks 0 and 1 of each column half) as soon as those are written, while
-          // the threads still compute the rest; then the others.
+          // O_t += P_t(it) V_t(it), in two parts: keys [0, 64) as soon as the softmax threads have
+          // written them, while they still compute the rest; then keys [64, 128).
           if (!wait_bar(cx, cx.bar(B_PH + t), it & 1) || !wait_bar(cx, cx.bar(B_VF + t), it & 1)) {
             ok = false;
             break;
           }
           tc::tc_fence_after();
           const uint32_t sV = cx.sbase + L::off_v(t);
-          // P keys [16 kk, 16 kk + 16): half kk / 4 wrote them into its own S columns (chunk kk % 4)
+          // P keys [16 kk, 16 kk + 16) as bf16 pairs in S columns [8 kk, 8 kk + 8)
           auto pv = [&](int kk, uint32_t acc) {
-            tc::mma_bf16_ts(tmem + L::col_o(t), tmem + L::col_s(t) + (kk >> 2) * 64 + (kk & 3) * 8,
+            tc::mma_bf16_ts(tmem + L::col_o(t), tmem + L::col_s(t) + kk * 8,
                             tc::sw128_desc(sV + kk * 2048, kSub, 1024), id_pv, acc);
           };
           pv(0, it > 0 ? 1u : 0u);
           pv(1, 1u);
-          pv(4, 1u);
-          pv(5, 1u);
+          pv(2, 1u);
+          pv(3, 1u);
           if (!wait_bar(cx, cx.bar(B_PF + t), it & 1)) {
             ok = false;
             break;
           }
           tc::tc_fence_after();
-          pv(2, 1u);
-          pv(3, 1u);
+          pv(4, 1u);
+          pv(5, 1u);
           pv(6, 1u);
           pv(7, 1u);
           tc::mma_commit(cx.bar(B_VE + t));
@@ -418,34 +419,20 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
     }
   } else {
     // ------------------------------ softmax -------------------------------
-    const int t = warp >> 3;                 // tile of this warp
-    const int hf = (warp >> 2) & 1;          // key-column half: [64 hf, 64 hf + 64)
+    const int t = warp >> 2;                 // tile of this warp
     const int r = ((warp & 3) << 5) | lane;  // query row = TMEM lane
     const Tile x = t == 0 ? tl[0] : tl[1];
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + L::col_s(t) + 64 * hf;     // this half's S columns
-    const uint32_t tP = tmem + lane_base + L::col_s(t) + 64 * hf;     // this half's P columns (2 bf16 each)
-    const uint32_t tO = tmem + lane_base + L::col_o(t) + 64 * hf;     // this half's O columns
-    float* xchg = reinterpret_cast<float*>(sm + L::OFF_XCHG) + t * 512;  // [parity][half][row]
-    // Exchange with the other half of the row: write, arrive on the barrier of this warp pair
-    // (warps w and w + 4, 64 arrivals) and parity, bounded wait, read.  Use u of parity q waits for
-    // phase parity (u / 2) & 1.  A pair waits only for itself, not for the tile's other warps.
-    auto exchange = [&](int use, float v) -> float {
-      float* xc = xchg + (use & 1) * 256;
-      xc[hf * 128 + r] = v;
-      const uint32_t xb = cx.bar(B_X + t * 8 + (warp & 3) * 2 + (use & 1));
-      tc::mbar_arrive(xb);
-      if (!wait_bar(cx, xb, (use >> 1) & 1)) return NAN;
-      return xc[(1 - hf) * 128 + r];
-    };
+    const uint32_t tS = tmem + lane_base + L::col_s(t);  // row r of S_t; P_t in its first 64 columns
+    const uint32_t tO = tmem + lane_base + L::col_o(t);  // row r of O_t
     const int qt = x.i * 128 + r;
     const float sl2 = p.scale * 1.4426950408889634f;
-    float m = -INFINITY, l = 0.f;  // l: this half's share of the row sum
+    float m = -INFINITY, l = 0.f;
     bool ok = true;
     if (p.rope_cos != nullptr && nmax > 0) {
       // RoPE on load: all softmax threads rotate the CTA's Q tiles, then one arrival each on B_QR.
       ok = rope_q_on_load<KT>(cx.abort_flag, cx.status, cx.bar(B_Q), sm, p.rope_cos, p.rope_sin, tl[0].i, tl[1].i,
-                          tl[0].n, tl[1].n, warp * 32 + lane);
+                              tl[0].n, tl[1].n, warp * 32 + lane);
       tc::mbar_arrive(cx.bar(B_QR));
     }
     for (int it = 0; ok && it < x.n; ++it) {
@@ -453,45 +440,42 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
       if (!ok) break;
       tc::tc_fence_after();
       const int j = slist[t * kMaxList + it];
-      // keys c (0..127 of the block) with c <= lim are visible; this half holds c = 64 hf + cc
-      const int lim = ((p.causal && j * 128 + 127 > qt) ? qt - j * 128 : 127) - 64 * hf;
-      // Pass 1: max over this half, then the row max through shared memory.
-      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-      {
-        uint32_t sv[2][32];
-        tc::tmem_ld32(tS, sv[0]);
-        tc::tmem_ld32(tS + 32, sv[1]);
-        tc::tmem_wait_ld();
-        if (lim < 63) {  // causal diagonal: keys beyond the query row are masked
+      // keys c (0..127 of the block) with c <= lim are visible
+      const int lim = (p.causal && j * 128 + 127 > qt) ? qt - j * 128 : 127;
+      // The whole row of S_t in registers: its maximum, then P from the same registers.
+      uint32_t sv[4][32];
 #pragma unroll
-          for (int c = 0; c < 2; ++c)
+      for (int q = 0; q < 4; ++q) tc::tmem_ld32(tS + 32 * q, sv[q]);
+      tc::tmem_wait_ld();
+      if (lim < 127) {  // causal diagonal: keys beyond the query row are masked
 #pragma unroll
-            for (int e = 0; e < 32; ++e)
-              if (c * 32 + e > lim) sv[c][e] = __float_as_uint(-INFINITY);
-        }
+        for (int q = 0; q < 4; ++q)
 #pragma unroll
-        for (int c = 0; c < 2; ++c)
-#pragma unroll
-          for (int e = 0; e < 32; e += 8)
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              mq[q] = tc::max3(mq[q], __uint_as_float(sv[c][e + 2 * q]), __uint_as_float(sv[c][e + 2 * q + 1]));
+          for (int e = 0; e < 32; ++e)
+            if (32 * q + e > lim) sv[q][e] = __float_as_uint(-INFINITY);
       }
-      const float mhalf = tc::max3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
-      const float mx = fmaxf(mhalf, exchange(it, mhalf));
+      float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+#pragma unroll
+        for (int e = 0; e < 32; e += 8)
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            mq[u] = tc::max3(mq[u], __uint_as_float(sv[q][e + 2 * u]), __uint_as_float(sv[q][e + 2 * u + 1]));
+      const float mx = tc::max3(mq[0], mq[1], fmaxf(mq[2], mq[3]));
       const float mnew = fmaxf(m, mx * sl2);
       const bool need = mnew > m + kRescaleThreshold || (m == -INFINITY && mnew != -INFINITY);
       // O_t is stable here: PV_t(it-1) completed before S_t(it) was signalled.
       if (__any_sync(0xffffffffu, need) && it > 0) {
         const float f = need ? exp2f(m - mnew) : 1.f;
 #pragma unroll 1
-        for (int c = 0; c < 2; ++c) {
-          uint32_t v[32];
-          tc::tmem_ld32(tO + c * 32, v);
+        for (int c = 0; c < 8; ++c) {  // 16 columns at a time: the row of S_t is live in registers
+          uint32_t v[16];
+          tc::tmem_ld16(tO + c * 16, v);
           tc::tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
-          tc::tmem_st32(tO + c * 32, v);
+          for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * f);
+          tc::tmem_st16(tO + c * 16, v);
         }
       }
       if (need) {
@@ -499,23 +483,14 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
         m = mnew;
       }
       const float nmu = (m == -INFINITY) ? 0.f : -m;
-      // Pass 2: P = 2^(s * scale * log2e - m) as bf16 pairs, 16 columns at a time
-      // (double-buffered TMEM loads).  P chunk c of this half lands in S columns
-      // [64 hf + 8 c, +8), which this thread has already read.
+      // P = 2^(s * scale * log2e - m) as bf16 pairs, 16 keys at a time: keys [16 c, 16 c + 16) into
+      // S columns [8 c, 8 c + 8) (the whole row is already in registers).  Keys [0, 64) are
+      // signalled on their own (B_PH) so that the tensor core starts on them.
       const uint64_t sl2x2 = tc::f2_pack(sl2, sl2), nmux2 = tc::f2_pack(nmu, nmu);
       uint64_t acc[4] = {0, 0, 0, 0};  // packed (even, odd) column partial row sums
-      uint32_t buf[2][16];
-      tc::tmem_ld16(tS, buf[0]);
-      tc::tmem_wait_ld();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t (&cur)[16] = buf[c & 1];
-        if (c < 3) tc::tmem_ld16(tS + (c + 1) * 16, buf[(c + 1) & 1]);
-        if (lim < 63) {
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            if (c * 16 + e > lim) cur[e] = __float_as_uint(-INFINITY);
-        }
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t* cur = &sv[c >> 1][(c & 1) * 16];
         uint32_t pk[8];
 #pragma unroll
         for (int e = 0; e < 16; e += 2) {
@@ -526,13 +501,12 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
           acc[(e >> 1) & 3] = tc::f2_add(acc[(e >> 1) & 3], tc::f2_pack(p0, p1));
           pk[e >> 1] = pack_bf16x2(p0, p1);
         }
-        tc::tmem_st8(tP + c * 8, pk);
-        if (c == 1) {  // chunks 0 and 1 written: the tensor core may start on them
+        tc::tmem_st8(tS + c * 8, pk);
+        if (c == 3) {  // keys [0, 64) written: the tensor core may start on them
           tc::tmem_wait_st();
           tc::tc_fence_before();
           tc::mbar_arrive(cx.bar(B_PH + t));
         }
-        if (c < 3) tc::tmem_wait_ld();
       }
       float rs0, rs1, rs2, rs3;
       tc::f2_unpack(tc::f2_add(acc[0], acc[1]), rs0, rs1);
@@ -543,17 +517,14 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
       tc::mbar_arrive(cx.bar(B_PF + t));
     }
     if (x.n > 0 && ok) ok = __all_sync(0xffffffffu, wait_bar(cx, cx.bar(B_OD + t), 0));
-    // Both halves of a row take the same branch: ok and x.n are uniform over the tile.
+    // ok and x.n are uniform over the tile's warps.
     if (x.valid && (x.n == 0 || ok)) {
-      __nv_bfloat16* orow =
-          static_cast<__nv_bfloat16*>(p.O) + ((size_t)(x.b * p.Hq + x.h) * p.L + qt) * kHD + 64 * hf;
-      float ltot = 0.f;
+      __nv_bfloat16* orow = static_cast<__nv_bfloat16*>(p.O) + ((size_t)(x.b * p.Hq + x.h) * p.L + qt) * kHD;
       if (x.n > 0) {
-        ltot = l + exchange(x.n, l);  // use n: the parity the last iteration did not touch
         tc::tc_fence_after();
-        const float inv = ltot > 0.f ? 1.f / ltot : 0.f;
+        const float inv = l > 0.f ? 1.f / l : 0.f;
 #pragma unroll
-        for (int c = 0; c < 2; ++c) {
+        for (int c = 0; c < 4; ++c) {
           uint32_t v[32];
           tc::tmem_ld32(tO + c * 32, v);
           tc::tmem_wait_ld();
@@ -569,11 +540,11 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
         }
       } else {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) reinterpret_cast<uint4*>(orow)[q] = make_uint4(0, 0, 0, 0);
+        for (int q = 0; q < 16; ++q) reinterpret_cast<uint4*>(orow)[q] = make_uint4(0, 0, 0, 0);
       }
-      if (p.lse != nullptr && hf == 0)
+      if (p.lse != nullptr)
         p.lse[(size_t)(x.b * p.Hq + x.h) * p.L + qt] =
-            (x.n > 0 && ltot > 0.f) ? (m + log2f(ltot)) * 0.6931471805599453f : -INFINITY;
+            (x.n > 0 && l > 0.f) ? (m + log2f(l)) * 0.6931471805599453f : -INFINITY;
     }
   }
 
