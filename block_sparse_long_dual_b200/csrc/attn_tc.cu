@@ -17,8 +17,9 @@
 //                    row maximum with no exchange, rescales O_t lazily, computes
 //                    P_t from the same registers and writes it (bf16) back into
 //                    the S_t columns of TMEM; final O_t / l epilogue.
-//   warp 4 KT        producer: TMA loads of Q_t and of K_t(j), V_t(j) for every
-//                    kept block j of each tile (one K and one V slot per tile).
+//   warp 4 KT        producer: TMA loads of Q_t (started at entry, while warps 0
+//                    and 4 validate the index lists) and of K_t(j), V_t(j) for
+//                    every kept block j of each tile (one K and one V slot per tile).
 //   warp 4 KT + 1    MMA issuer: S_t = Q_t K_t^T (A, B from shared memory) and
 //                    O_t += P_t V_t (A = P_t from TMEM, B = V_t from shared
 //                    memory), M = N = 128, K = 16 steps; completion tracked with
@@ -239,6 +240,7 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
   tl[0] = decode_tile(p, KT * blockIdx.x);
   tl[1] = decode_tile(p, KT == 2 ? 2 * blockIdx.x + 1 : KT * blockIdx.x);
   if (KT == 1) tl[1].valid = false;
+  bool qearly[2] = {false, false};  // producer: Q copy started before the lists were validated
 
   if (warp == 0 || (KT == 2 && warp == 4)) {
     // Validate one tile's index list: count in [0, kmax], entries ascending in [0, nb), <= i if causal.
@@ -247,13 +249,24 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
     int n = 0;
     if (x.valid) {
       const size_t rowid = (size_t)(x.b * p.Hq + x.h) * p.nb + x.i;
+      // The count and the list's first 32 slots are loaded together (a row holds kmax slots), so a
+      // list of up to 32 entries costs one round trip; each entry is compared with its predecessor
+      // through a shuffle.
+      int j0 = lane < p.kmax ? x.list[lane] : 0;
       n = p.counts[rowid];
       bool ok = n >= 0 && n <= p.kmax;
       if (ok) {
-        for (int u = lane; u < n; u += 32) {
-          const int j = x.list[u];
-          if (j < 0 || j >= p.nb || (p.causal && j > x.i) || (u > 0 && x.list[u - 1] >= j)) ok = false;
-          if (u < kMaxList) slist[t * kMaxList + u] = j;
+        int prev = -1;  // last entry of the previous 32
+        for (int u0 = 0; u0 < n; u0 += 32) {
+          const int u = u0 + lane;
+          const int j = u0 == 0 ? j0 : (u < n ? x.list[u] : 0);
+          const int up = __shfl_up_sync(0xffffffffu, j, 1);
+          const int before = lane == 0 ? prev : up;
+          if (u < n) {
+            if (j < 0 || j >= p.nb || (p.causal && j > x.i) || (u > 0 && before >= j)) ok = false;
+            if (u < kMaxList) slist[t * kMaxList + u] = j;
+          }
+          prev = __shfl_sync(0xffffffffu, j, 31);
         }
       }
       ok = __all_sync(0xffffffffu, ok);
@@ -263,17 +276,27 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
       }
     }
     if (lane == 0) nsh[t] = n;
-    if (warp == 0 && lane == 0) {
-      *cx.abort_flag = 0;
-      for (int k = 0; k < NBAR; ++k)
-        tc::mbar_init(cx.bar(k), k == B_QR ? L::kSoftmaxThreads
-                                 : (k == B_PF || k == B_PF + 1 || k == B_PH || k == B_PH + 1) ? 128 : 1);
-      tc::fence_mbar_init();
-    }
   } else if (warp == L::kProducerWarp && lane == 0) {
+    *cx.abort_flag = 0;
+    for (int k = 0; k < NBAR; ++k)
+      tc::mbar_init(cx.bar(k), k == B_QR ? L::kSoftmaxThreads
+                               : (k == B_PF || k == B_PF + 1 || k == B_PH || k == B_PH + 1) ? 128 : 1);
+    tc::fence_mbar_init();
     tc::prefetch_tmap(&tmQ);
     tc::prefetch_tmap(&tmK);
     tc::prefetch_tmap(&tmV);
+    // A Q tile depends only on the tile, not on its list: its copy starts while the lists are
+    // being validated.
+#pragma unroll
+    for (int t = 0; t < KT; ++t) {
+      if (!tl[t].valid) continue;
+      const int qrow = (tl[t].b * p.Hq + tl[t].h) * p.L + tl[t].i * 128;
+      const uint32_t sQ = cx.sbase + L::off_q(t);
+      tc::mbar_arrive_expect_tx(cx.bar(B_Q + t), kTile);
+      tc::tma_load_2d(sQ, &tmQ, cx.bar(B_Q + t), 0, qrow);
+      tc::tma_load_2d(sQ + kSub, &tmQ, cx.bar(B_Q + t), 64, qrow);
+      qearly[t] = true;
+    }
   } else if (warp == L::kMmaWarp) {
     tc::tmem_alloc(tc::smem_u32(tmem_slot), L::TMEM_COLS);
     tc::tmem_relinquish();
@@ -290,17 +313,6 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
     // ------------------------------ producer ------------------------------
     if (lane == 0 && nmax > 0) {
       int kissued[2] = {0, 0}, vissued[2] = {0, 0};
-      bool qissued[2] = {false, false};
-#pragma unroll
-      for (int t = 0; t < KT; ++t) {
-        if (tl[t].n == 0) continue;
-        const int qrow = (tl[t].b * p.Hq + tl[t].h) * p.L + tl[t].i * 128;
-        const uint32_t sQ = cx.sbase + L::off_q(t);
-        tc::mbar_arrive_expect_tx(cx.bar(B_Q + t), kTile);
-        tc::tma_load_2d(sQ, &tmQ, cx.bar(B_Q + t), 0, qrow);
-        tc::tma_load_2d(sQ + kSub, &tmQ, cx.bar(B_Q + t), 64, qrow);
-        qissued[t] = true;
-      }
       bool ok = true;
       for (int it = 0; ok && it < nmax; ++it) {
 #pragma unroll
@@ -329,12 +341,16 @@ __global__ void __launch_bounds__(Layout<KT>::kThreads, 3 - KT)
       if (*cx.abort_flag) {
         // Let every copy this CTA started land before the CTA exits.
         for (int t = 0; t < KT; ++t) {
-          if (qissued[t]) drain_wait(cx.bar(B_Q + t), 0);
           if (kissued[t] > 0) drain_wait(cx.bar(B_KF + t), (kissued[t] - 1) & 1);
           if (vissued[t] > 0) drain_wait(cx.bar(B_VF + t), (vissued[t] - 1) & 1);
         }
       }
     }
+    // Every Q copy lands before the CTA exits, including a tile whose list came out empty (no MMA
+    // waits for it); for the others the phase has completed already.
+    if (lane == 0)
+      for (int t = 0; t < KT; ++t)
+        if (qearly[t]) drain_wait(cx.bar(B_Q + t), 0);
   } else if (warp == L::kMmaWarp) {
     // ------------------------------ MMA issuer ----------------------------
     if (lane == 0 && nmax > 0) {
