@@ -334,7 +334,8 @@ def run_decode(args, w: wl.DecodeWorkload, rank, world):
         torch.cuda.synchronize(dev)
         return g0.elapsed_time(g1) / reps
 
-    K_ = max(args.steps, 50)
+    # at least 500 step replays (~50 ms at 128K x 4), so that the clock sampler sees the timed region
+    K_ = max(args.steps, 500)
     t_app = graph_ms(lambda: m.refresh_keys(Kd, pos0=w.seq_len - 1, npos=1), K_)
     t_sel = graph_ms(lambda: m.select(qd), K_)
     t_att = graph_ms(lambda: m.attend(qd, Kd, Vd), K_)
