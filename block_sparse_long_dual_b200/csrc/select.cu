@@ -19,8 +19,18 @@ __global__ void __launch_bounds__(kWarps * 32) select_kernel(SelectParams p) {
   if (row >= nrows) return;
   const int i = (int)(row % p.nb);
   const float* prow = p.probs + row * p.nb;
-  const int n = select_row_warp<NPL>([&](int j) { return __ldg(prow + j); }, i, p.k, p.mass, p.flags,
-                                     p.idx + row * p.kmax, p.kmax);
+  auto prob = [&](int j) { return __ldg(prow + j); };
+  int* out = p.idx + row * p.kmax;
+  // A row's causal prefix (blocks 0 .. i) fills i / 32 + 1 register slots: rows in the first
+  // quarter (half) of the range run the routine with a quarter (half) of the slots, so their
+  // bisection steps scan only those.
+  int n;
+  if (NPL >= 16 && i < NPL * 8)
+    n = select_row_warp<(NPL >= 16 ? NPL / 4 : 1)>(prob, i, p.k, p.mass, p.flags, out, p.kmax);
+  else if (NPL >= 16 && i < NPL * 16)
+    n = select_row_warp<(NPL >= 16 ? NPL / 2 : 1)>(prob, i, p.k, p.mass, p.flags, out, p.kmax);
+  else
+    n = select_row_warp<NPL>(prob, i, p.k, p.mass, p.flags, out, p.kmax);
   if (lane == 0) p.counts[row] = n;
 }
 
