@@ -34,7 +34,7 @@ namespace sfa {
 // float64 to the block mean and the per-band energies.
 // ---------------------------------------------------------------------------
 template <typename T, int D, int PASSES, int NS>
-__global__ void __launch_bounds__(256, 1) rope_pool_energy_kernel(RopePoolParams p, int heads_per_cta) {
+__global__ void __launch_bounds__(256, (sizeof(T) == 2 ? 2 : 1)) rope_pool_energy_kernel(RopePoolParams p, int heads_per_cta) {
   constexpr int CH = D / 16;
   constexpr int TPP = 256 / CH;  // tokens per pass
   constexpr int NW = 8;
@@ -486,15 +486,18 @@ __global__ void __launch_bounds__(256, 1) block_score_softmax_kernel(ScoreParams
 // ---------------------------------------------------------------------------
 template <typename T, int D, int PASSES>
 static cudaError_t launch_rope_pool_tdp(const RopePoolParams& p, cudaStream_t st) {
-  constexpr int NS = sizeof(T) == 2 ? 3 : 2;  // ring stages of one head's block rows
+  constexpr int NS = 2;  // ring stages of one head's block rows
   const size_t smem = (size_t)NS * (256 / (D / 16)) * PASSES * D * sizeof(T);
   auto kern = rope_pool_energy_kernel<T, D, PASSES, NS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  // Enough CTAs for about four waves of 148 SMs; each CTA reads the table slice once for its heads.
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  if (e != cudaSuccess) return e;
+  // Enough CTAs for about four waves of two CTAs on each of 148 SMs (bf16: two CTAs of a two-stage
+  // ring share an SM); each CTA reads the table slice once for its heads.
   const int heads = p.Hq + p.Hkv;
   const long long blocks = (long long)p.B * p.nb;
-  int groups = (int)((4LL * 148 + blocks - 1) / blocks);
+  int groups = (int)((8LL * 148 + blocks - 1) / blocks);
   groups = groups < 1 ? 1 : (groups > heads ? heads : groups);
   const int per = (heads + groups - 1) / groups;
   groups = (heads + per - 1) / per;
