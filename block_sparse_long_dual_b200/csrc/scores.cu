@@ -486,7 +486,7 @@ __global__ void __launch_bounds__(256, 1) block_score_softmax_kernel(ScoreParams
 // ---------------------------------------------------------------------------
 template <typename T, int D, int PASSES>
 static cudaError_t launch_rope_pool_tdp(const RopePoolParams& p, cudaStream_t st) {
-  constexpr int NS = 2;  // ring stages of one head's block rows
+  constexpr int NS = sizeof(T) == 2 ? 3 : 2;  // ring stages of one head's block rows
   const size_t smem = (size_t)NS * (256 / (D / 16)) * PASSES * D * sizeof(T);
   auto kern = rope_pool_energy_kernel<T, D, PASSES, NS>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
