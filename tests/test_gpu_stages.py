@@ -138,3 +138,43 @@ def test_attention_rejects_bad_index_lists(dt, block, d):
     torch.cuda.synchronize()
     assert int(status.item()) == 8
     assert torch.all(O.float() == 0).item()
+
+
+def test_attention_bad_list_beside_a_good_one_two_tile_layout():
+    """kmax above the short-list cut: two query tiles per CTA (two Q heads of a GQA group at one
+    query block).  A tile whose list is invalid is zeroed and flagged while its CTA partner is
+    computed exactly as in a call where the bad list is simply empty."""
+    B, Hq, Hkv, nb, block, d = 1, 2, 1, 4, 128, 128
+    L = nb * block
+    dev = torch.device("cuda")
+    g = torch.Generator().manual_seed(11)
+    Q = torch.randn((B, Hq, L, d), generator=g).to(torch.bfloat16).to(dev)
+    K, V = (torch.randn((B, Hkv, L, d), generator=g).to(torch.bfloat16).to(dev) for _ in range(2))
+    kmax = 16
+    idx = torch.full((B, Hq, nb, kmax), -1, dtype=torch.int32)
+    counts = torch.zeros((B, Hq, nb), dtype=torch.int32)
+    for h in range(Hq):
+        for i in range(nb):
+            idx[0, h, i, :i + 1] = torch.arange(i + 1, dtype=torch.int32)
+            counts[0, h, i] = i + 1
+    bad_idx, bad_counts = idx.clone(), counts.clone()
+    bad_idx[0, 0, 2, :3] = torch.tensor([1, 0, 2], dtype=torch.int32)  # head 0, block 2: not ascending
+    bad_idx[0, 1, 3, 1] = 7                                             # head 1, block 3: out of range
+    good_counts = counts.clone()
+    good_counts[0, 0, 2] = 0
+    good_counts[0, 1, 3] = 0
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    O_bad = sfa.block_sparse_attn(Q, K, V, bad_counts.to(dev), bad_idx.to(dev), block=block, causal=True,
+                                  status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 8
+    status.zero_()
+    O_good = sfa.block_sparse_attn(Q, K, V, good_counts.to(dev), idx.to(dev), block=block, causal=True,
+                                   status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == 0
+    rows = lambda i: slice(i * block, (i + 1) * block)
+    assert torch.all(O_bad[0, 0, rows(2)].float() == 0).item()
+    assert torch.all(O_bad[0, 1, rows(3)].float() == 0).item()
+    assert torch.equal(O_bad, O_good)
+    assert O_good[0, 0, rows(3)].float().abs().sum().item() > 0  # a partner tile was computed
