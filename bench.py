@@ -60,6 +60,8 @@ def parse():
     ap.add_argument("--e2e-steps", type=int, default=None)
     ap.add_argument("--fused", action="store_true",
                     help="estimate and selection in one call (sfa_block_scores_select; probabilities not stored)")
+    ap.add_argument("--rope-on-load", action="store_true",
+                    help="the attention rotates Q as it loads it (sfa_block_sparse_attn_rope; Q_rot not stored)")
     return ap.parse_args()
 
 
@@ -79,16 +81,17 @@ def attention_flops(counts: np.ndarray, block: int, d: int) -> float:
     return float(4.0 * d * (block * block * (n - diag) + block * (block + 1) / 2.0 * diag).sum())
 
 
-def scoring_bytes(w: wl.Workload, store_probs: bool = True) -> float:
-    """Algorithmic HBM bytes of sfa_block_scores: read Q, K; write Q_r, K_r; read the cos/sin
-    table once; write the float64 block means; write probs [B, Hq, nb, nb] (unless the selection
-    is fused and the probabilities are not stored)."""
+def scoring_bytes(w: wl.Workload, store_probs: bool = True, store_q_rot: bool = True) -> float:
+    """Algorithmic HBM bytes of sfa_block_scores: read Q, K; write Q_r (unless the attention
+    rotates Q on load), K_r; read the cos/sin table once; write the float64 block means; write
+    probs [B, Hq, nb, nb] (unless the selection is fused and the probabilities are not stored)."""
     e = 2 if w.dtype == "bf16" else 4
     qk = w.batch * (w.heads_q + w.heads_kv) * w.seq_len * w.head_dim * e
+    k_only = w.batch * w.heads_kv * w.seq_len * w.head_dim * e
     table = 2 * w.seq_len * (w.head_dim // 2) * 4
     means = w.batch * (w.heads_q + w.heads_kv) * w.nb * w.head_dim * 8
     probs = w.batch * w.heads_q * w.nb * w.nb * 4 if store_probs else 0
-    return float(2 * qk + table + means + probs)
+    return float(qk + (qk if store_q_rot else k_only) + table + means + probs)
 
 
 def select_bytes(w: wl.Workload, kmax: int, read_probs: bool = True) -> float:
@@ -469,7 +472,7 @@ def main():
     model = sfa.PrismAttention(batch=w.batch, heads_q=w.heads_q, heads_kv=w.heads_kv, seq_len=w.seq_len,
                                head_dim=w.head_dim, dtype=w.dtype, block=w.block, rope_base=w.rope_base,
                                band_split=w.band_split, k=w.k, mass=w.mass, flags=w.flags, device=dev,
-                               fused=args.fused)
+                               fused=args.fused, rope_on_load=args.rope_on_load)
     Qd, Kd, Vd = Q.to(dev), K.to(dev), V.to(dev)
     stream = torch.cuda.current_stream(dev)
     for _ in range(args.warmup):
@@ -496,7 +499,7 @@ def main():
             if not args.fused:
                 model.select()
             ev[s][2].record(stream)
-            model.attend(Vd)
+            model.attend(Vd, Qd)
             ev[s][3].record(stream)
         stop.record(stream)
         torch.cuda.synchronize(dev)
@@ -575,7 +578,8 @@ def main():
         achieved = flops_step / (attn_ms * 1e-3) / 1e12
         peak = float(pk["bf16_tflops"])
         tr = traffic_record("block_sparse_long_dual_b200/csrc/attn_tc.cu")
-        sb, selb = scoring_bytes(w, not args.fused), select_bytes(w, model.kmax, not args.fused)
+        sb = scoring_bytes(w, not args.fused, not args.rope_on_load)
+        selb = select_bytes(w, model.kmax, not args.fused)
         line = {
             "metric": "prefill attention effective TFLOP/s over kept blocks (whole path)",
             "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": K_, "warmup": args.warmup,
@@ -584,11 +588,14 @@ def main():
             "config": {**layer_config(w, world), "kept_fraction": round(kept_frac, 5),
                        "estimate": ("fused with the selection (sfa_block_scores_select, probabilities not stored)"
                                     if args.fused else "sfa_block_scores then sfa_select"),
+                       "attention": ("RoPE on load (sfa_block_sparse_attn_rope: Q rotated in the attention kernel, "
+                                     "Q_rot not stored)" if args.rope_on_load else "sfa_block_sparse_attn on Q_rot"),
                        "l2": "inputs larger than L2 (Q 1.07 GB, K 0.27 GB, V 0.27 GB at 128K); no flush"},
             "stages_ms": {"block_scores": scores_ms, "select": select_ms, "attention": attn_ms},
             "scoring": {"bytes": sb + selb, "GB_s": (sb + selb) / ((scores_ms + select_ms) * 1e-3) / 1e9,
                         "frac_hbm": (sb + selb) / ((scores_ms + select_ms) * 1e-3) / 1e9 / float(pk["hbm_gbs"])},
-            "roofline": {"kernel": "attn_tc_kernel (sfa_block_sparse_attn)", "bound": "tensor",
+            "roofline": {"kernel": ("attn_tc_kernel (sfa_block_sparse_attn_rope)" if args.rope_on_load
+                                    else "attn_tc_kernel (sfa_block_sparse_attn)"), "bound": "tensor",
                          "achieved": achieved, "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
                          "peak_source": f"{pk_src} bf16 burst",
                          "frac_of_sustained": achieved / float(pk.get("bf16_tflops_sustained", peak)),
