@@ -55,3 +55,17 @@ def test_scoring_and_decode_bytes(bench):
     assert sel == 4 * 8 * 131072 * 24 * 2 + 4 * 32 * 128 * 2       # compact keys + q
     assert att == 4 * 32 * (256 * 2 * 128 * 2 + 2 * 128 * 2 + 256 * 4)
     assert total > sel + att
+
+
+def test_scoring_bytes_without_stored_q_rot_or_probs(bench):
+    """RoPE on load drops the Q_rot write (K_rot is still written); a fused selection drops the
+    probabilities; counted directly for the 128K layer."""
+    w = wl.LLAMA_128K
+    q = 32 * 131072 * 128 * 2
+    k = 8 * 131072 * 128 * 2
+    table = 2 * 131072 * 64 * 4
+    means = (32 + 8) * 1024 * 128 * 8
+    probs = 32 * 1024 * 1024 * 4
+    assert bench.scoring_bytes(w, True, False) == (q + k) + k + table + means + probs
+    assert bench.scoring_bytes(w, False, True) == 2 * (q + k) + table + means
+    assert bench.scoring_bytes(w, False, False) == (q + k) + k + table + means
